@@ -1,0 +1,197 @@
+/*
+ * libmsa -- C ABI of the Memory Sparse Attention (MSA) hot path on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The path, as the pages describing MSA define it:
+ *   1. encode:  document-wise RoPE on token K, then 64-token chunk means of
+ *               K, V and the routing key K_r  (msa_encode_pool);
+ *   2. route:   cosine of Q_r against each pooled K̄_r, mean over heads, max
+ *               over query tokens, max over a document's chunks
+ *               (msa_route_scores), then the top-k documents (msa_topk_docs);
+ *   3. attend:  gather the selected documents' pooled K̄/V̄ in rank order
+ *               (msa_gather_kv) and run GQA attention over [memory ; local
+ *               causal context] with global RoPE starting at offset k
+ *               (msa_sparse_attn).
+ *
+ * Sources, cited by page title and section:
+ *   [DEEP]  "深度分析MSA:把超长文档组织成可检索内部记忆的工程路径"
+ *           (yeyulingfeng.com), §"三、文档如何变成 memory" and
+ *           §"五、推理阶段：memory 的使用方式".
+ *   [HYSEN] "EverMind-AI/MSA: routing top-k compressed documents inside
+ *           attention, and where the 100M-token claim stops"
+ *           (hysenlabs.com), §"Routing happens inside attention, not in a
+ *           retrieval service in front of the model", §"Document-wise RoPE
+ *           resets every document to position zero", §"Memory must be
+ *           encoded offline before a query can reach it".
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers owned by the caller, row-major
+ *     and contiguous, in the layouts stated per function.  Integer
+ *     arguments are host values.  The library keeps no pointer after a call
+ *     returns and allocates no device memory: scratch comes from the
+ *     caller's workspace (sizes from the *_workspace_size functions).
+ *   - `dt` selects the element type of every floating-point tensor of the
+ *     call (MSA_F32 = float, MSA_BF16 = __nv_bfloat16); arithmetic is fp32.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and never synchronises the host.
+ *   - Errors the host can see (bad sizes, NULL or misaligned pointers,
+ *     unsupported shapes) are returned before anything is launched; a
+ *     failing CUDA launch returns MSA_ERR_CUDA and msa_last_cuda_error()
+ *     gives the cudaError_t.  Errors only the device can see (a gather that
+ *     overflows its capacity, a bounded wait that ran out) are recorded in a
+ *     per-device status word read with msa_device_status().
+ *   - Tensors read with 16-byte vector loads must be 16-byte aligned; this
+ *     is checked and reported as MSA_ERR_INVALID_ARG.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* msa_stream_t;
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = -1,  /* NULL/misaligned pointer, bad size, k > n_docs, ... */
+  MSA_ERR_UNSUPPORTED = -2,  /* shape outside what the kernels implement          */
+  MSA_ERR_CAPACITY = -3,     /* gather: selected rows exceed m_cap (device word)  */
+  MSA_ERR_CUDA = -4,         /* a CUDA call failed; see msa_last_cuda_error()     */
+  MSA_ERR_TIMEOUT = -5,      /* a bounded device wait ran out (device word)       */
+  MSA_ERR_WORKSPACE = -6     /* workspace NULL or smaller than required           */
+} msa_status;
+
+typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype;
+
+/* Static, NUL-terminated description of a status code. Never NULL. */
+const char* msa_status_string(int status);
+
+/* cudaError_t of the last CUDA failure seen by a libmsa call on the calling
+ * host thread (0 if none). */
+int msa_last_cuda_error(void);
+
+/* Library version string, e.g. "libmsa 0.1.0 sm_100a". */
+const char* msa_version(void);
+
+/* Reads (and, if clear != 0, resets) the status word of the current device:
+ * MSA_OK or the first device-detected error (MSA_ERR_CAPACITY,
+ * MSA_ERR_TIMEOUT) since the last reset.  Ordered after the work already
+ * queued on `stream`; blocks the host until that work is done. */
+int msa_device_status(int32_t* host_out, int clear, msa_stream_t stream);
+
+/* Chunk offsets of the bank -- [DEEP] §"三、文档如何变成 memory",
+ * "2. chunk 压缩": every `chunk` (64) tokens of a document form one chunk and
+ * a trailing partial chunk is kept (180 tokens -> 3 chunks).
+ *   tok_offsets   [n_docs+1] int64, device: document d owns token rows
+ *                 [tok_offsets[d], tok_offsets[d+1]).
+ *   chunk_offsets [n_docs+1] int64, device, written: exclusive prefix sum of
+ *                 ceil(len_d / chunk); document d owns chunk rows
+ *                 [chunk_offsets[d], chunk_offsets[d+1]).
+ * An empty document (len <= 0) gets no chunk and records
+ * MSA_ERR_INVALID_ARG in the device status word.  1 <= chunk <= 64. */
+int msa_chunk_offsets(int n_docs, const int64_t* tok_offsets, int chunk,
+                      int64_t* chunk_offsets, msa_stream_t stream);
+
+/* Memory encoding -- [HYSEN] §"Document-wise RoPE resets every document to
+ * position zero" and §"Memory must be encoded offline before a query can
+ * reach it"; [DEEP] "2. chunk 压缩".
+ *   k_tok, v_tok, kr_tok   [L][n_tok][H][D] (dt): token-level K, V, K_r of
+ *                          L routed layers, laid out contiguously.
+ *   tok_offsets, chunk_offsets  [n_docs+1] int64 (device), as above;
+ *                          n_chunks = chunk_offsets[n_docs].
+ *   k_bar, v_bar, kr_bar   [L][n_chunks][H][D] (dt), written.
+ * K row t of document d is rotated to position t - tok_offsets[d] (RoPE,
+ * pairs (i, i+D/2), inverse frequency rope_base^(-2i/D)); K, V and K_r are
+ * then averaged over each chunk's tokens (fp32 sums, one rounding to dt).
+ * Supported: D in {64,128}, 1 <= H <= 16, 1 <= chunk <= 64. */
+int msa_encode_pool(msa_dtype dt, int L, int64_t n_tok, int n_docs, int H,
+                    int D, const void* k_tok, const void* v_tok,
+                    const void* kr_tok, const int64_t* tok_offsets,
+                    const int64_t* chunk_offsets, int64_t n_chunks,
+                    float rope_base, int chunk, void* k_bar, void* v_bar,
+                    void* kr_bar, msa_stream_t stream);
+
+/* Routing -- [HYSEN] §"Routing happens inside attention ...": relevance is
+ * the cosine similarity of Q_r and K̄_r, averaged over heads, then the
+ * maximum over query tokens; [DEEP] §"五、推理阶段" Step 2.  A document's
+ * score is the maximum over its chunks (the pages leave this aggregation
+ * open).
+ *   q_r          [B][T][H][D] (dt): routing queries, B independent queries
+ *                of T tokens.
+ *   kr_bar       [n_chunks][H][D] (dt): one layer of the pooled bank.
+ *   chunk_offsets [n_docs+1] int64 (device).
+ *   doc_scores   [B][n_docs] float, written (-inf for an empty document).
+ *   chunk_scores [B][n_chunks] float, written when not NULL.
+ *   ws           workspace of >= msa_route_workspace_size(...) bytes.
+ * cos(q,k) = q.k / (max(|q|,1e-12) max(|k|,1e-12)).  MSA_BF16 runs the
+ * contraction on the tcgen05 tensor cores (bf16 operands, fp32 accumulate);
+ * MSA_F32 runs it on the CUDA cores in fp32.
+ * Supported: D in {64,128}, 1 <= H <= 8 (bf16) or 16 (fp32), B*T >= 1. */
+size_t msa_route_workspace_size(msa_dtype dt, int B, int T, int H, int D);
+int msa_route_scores(msa_dtype dt, int B, int T, int H, int D,
+                     const void* q_r, const void* kr_bar, int64_t n_chunks,
+                     const int64_t* chunk_offsets, int n_docs,
+                     float* doc_scores, float* chunk_scores, void* ws,
+                     size_t ws_bytes, msa_stream_t stream);
+
+/* Top-k documents -- [HYSEN] §"Routing happens inside attention ...": the
+ * router selects the top-k documents.  Ties go to the lower document index.
+ *   scores      [B][n_docs] float (device).
+ *   idx         [B][k] int32, written, in rank order (best first).
+ *   top_scores  [B][k] float, written when not NULL.
+ * NaN scores rank below every number.  1 <= k <= min(n_docs, 1024). */
+size_t msa_topk_workspace_size(int B, int n_docs, int k);
+int msa_topk_docs(int B, int n_docs, int k, const float* scores,
+                  int32_t* idx, float* top_scores, void* ws, size_t ws_bytes,
+                  msa_stream_t stream);
+
+/* Context assembly -- [HYSEN] §"Memory must be encoded offline ...": only
+ * the selected documents' K/V are loaded and joined with the local context.
+ *   idx          [B][k] int32 (device), document ids in rank order.
+ *   k_bar, v_bar [n_chunks][H][D] (dt), one layer of the pooled bank.
+ *   k_mem, v_mem [B][m_cap][H][D] (dt), written: rows 0..mem_len[b]-1 are
+ *                the chunk rows of idx[b][0], idx[b][1], ... concatenated.
+ *   mem_len      [B] int32, written: min(total rows, m_cap).
+ * If a query's rows exceed m_cap, rows past m_cap are dropped and
+ * MSA_ERR_CAPACITY is recorded in the device status word.  An index outside
+ * [0, n_docs) contributes no rows and records MSA_ERR_INVALID_ARG there. */
+int msa_gather_kv(msa_dtype dt, int B, int k, int H, int D,
+                  const int32_t* idx, const int64_t* chunk_offsets,
+                  int n_docs, const void* k_bar, const void* v_bar,
+                  int m_cap, void* k_mem, void* v_mem, int32_t* mem_len,
+                  msa_stream_t stream);
+
+/* Sparse attention, prefill (T > 1) and decode (T = 1) -- [HYSEN]
+ * §"Routing happens inside attention ..." (the selected compressed K/V are
+ * concatenated with the query's local K/V) and §"Document-wise RoPE ..."
+ * (global RoPE: the query's start index is offset by k).
+ *   q            [B][T][Hq][D] (dt): the last T of the T_loc local tokens.
+ *   k_mem, v_mem [B][m_cap][H][D] (dt) with mem_len [B] int32 (device):
+ *                memory rows, used as stored (they keep their
+ *                document-wise rotation).
+ *   k_loc, v_loc [B][T_loc][H][D] (dt): local context, unrotated.
+ *   out          [B][T][Hq][D] (dt), written.
+ * Local key j is rotated to position pos0 + j, query token i to
+ * pos0 + T_loc - T + i; query i sees every memory row and local keys
+ * j <= T_loc - T + i.  Query head h reads KV head floor(h*H/Hq).  scale <= 0
+ * selects 1/sqrt(D).  Softmax and accumulation in fp32.
+ * Supported: D in {64,128}, Hq % H == 0, Hq/H <= 16, 1 <= T <= T_loc. */
+size_t msa_sparse_attn_workspace_size(msa_dtype dt, int B, int T, int T_loc,
+                                      int Hq, int H, int D, int m_cap);
+int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, int H,
+                    int D, const void* q, const void* k_mem,
+                    const void* v_mem, const int32_t* mem_len, int m_cap,
+                    const void* k_loc, const void* v_loc, int pos0,
+                    float rope_base, float scale, void* out, void* ws,
+                    size_t ws_bytes, msa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */

@@ -1,0 +1,18 @@
+// bf16 prefill attention on the tcgen05 tensor cores (attn_tc.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace msa {
+
+// True when the tensor-core prefill kernel takes this shape.
+bool attn_tc_supported(int B, int T, int T_loc, int Hq, int H, int D, int m_cap);
+size_t attn_tc_workspace_size(int B, int T, int T_loc, int Hq, int H, int D, int m_cap);
+int attn_tc_launch(int B, int T, int T_loc, int Hq, int H, int D, const void* q,
+                   const void* k_mem, const void* v_mem, const int32_t* mem_len, int m_cap,
+                   const void* k_loc, const void* v_loc, int pos0, float rope_base, float qscale,
+                   void* out, void* ws, cudaStream_t s);
+
+}  // namespace msa

@@ -1,0 +1,23 @@
+// bf16 routing scan on the tcgen05 tensor cores (route_tc.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace msa {
+
+// Query columns of one pass over the bank and the padded column count of
+// the normalised-query workspace: B*T <= 256 is padded to 64, 128 or 256
+// columns (one pass); larger B*T to a multiple of 256 (one pass per 256).
+int64_t route_tc_columns(int64_t n_queries_tokens);
+
+// Scans the whole bank once per pass.  qhat: [H][n_pad][D] bf16, each row
+// Q_r / max(|Q_r|, eps) / H (rows >= B*T zero).  kr: [C][H][D] bf16.
+// doc_u / chunk_u: order-preserving uint32 maxima, pre-set to -inf.
+int route_tc_launch(int B, int T, int H, int D, const __nv_bfloat16* qhat, int n_pad,
+                    const __nv_bfloat16* kr, int64_t C, const int64_t* chunk_off,
+                    int n_docs, uint32_t* doc_u, uint32_t* chunk_u, int* status,
+                    cudaStream_t s);
+
+}  // namespace msa

@@ -1,0 +1,222 @@
+"""ctypes binding of libmsa (include/msa.h), with the same names.
+
+Argument marshalling only: every step of the MSA hot path runs in the CUDA
+kernels of ``libmsa.so``.  Tensor arguments may be torch tensors (their
+device pointer is passed; shapes are checked against the sizes given) or raw
+integer device addresses.  ``stream`` defaults to torch's current stream on
+the current device.  A non-zero status raises ``MsaError``; the library must
+have been built (``python -m latent_memory_routing_b200.build``) -- there is
+no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmsa.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "msa.h")
+
+MSA_F32 = 0
+MSA_BF16 = 1
+
+_STATUS = {0: "MSA_OK", -1: "MSA_ERR_INVALID_ARG", -2: "MSA_ERR_UNSUPPORTED",
+           -3: "MSA_ERR_CAPACITY", -4: "MSA_ERR_CUDA", -5: "MSA_ERR_TIMEOUT",
+           -6: "MSA_ERR_WORKSPACE"}
+
+
+class MsaError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        super().__init__(f"{fn} -> {_STATUS.get(status, status)}"
+                         + (f" ({detail})" if detail else ""))
+
+
+_lib = None
+
+c_i = ctypes.c_int
+c_i64 = ctypes.c_int64
+c_f = ctypes.c_float
+c_sz = ctypes.c_size_t
+c_p = ctypes.c_void_p
+
+_SIGS = {
+    "msa_status_string": (ctypes.c_char_p, [c_i]),
+    "msa_last_cuda_error": (c_i, []),
+    "msa_version": (ctypes.c_char_p, []),
+    "msa_device_status": (c_i, [c_p, c_i, c_p]),
+    "msa_chunk_offsets": (c_i, [c_i, c_p, c_i, c_p, c_p]),
+    "msa_encode_pool": (c_i, [c_i, c_i, c_i64, c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_p,
+                              c_i64, c_f, c_i, c_p, c_p, c_p, c_p]),
+    "msa_route_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i]),
+    "msa_route_scores": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i64, c_p, c_i, c_p, c_p,
+                               c_p, c_sz, c_p]),
+    "msa_topk_workspace_size": (c_sz, [c_i, c_i, c_i]),
+    "msa_topk_docs": (c_i, [c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_sz, c_p]),
+    "msa_gather_kv": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i, c_p, c_p, c_i, c_p, c_p,
+                            c_p, c_p]),
+    "msa_sparse_attn_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_i]),
+    "msa_sparse_attn": (c_i, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_i, c_p,
+                              c_p, c_i, c_f, c_f, c_p, c_p, c_sz, c_p]),
+}
+
+
+def header_symbols(path: str = HEADER) -> list[str]:
+    """Function names declared in include/msa.h."""
+    with open(path, encoding="utf-8") as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z0-9_]+)\s*\(", text)))
+
+
+def lib(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libmsa.so (once) and declares every signature."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with "
+                              "`python -m latent_memory_routing_b200.build`")
+        handle = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def dtype_code(t) -> int:
+    import torch
+    if t == torch.float32:
+        return MSA_F32
+    if t == torch.bfloat16:
+        return MSA_BF16
+    raise ValueError(f"unsupported dtype {t}")
+
+
+def _check(name: str, rc: int):
+    if rc != 0:
+        detail = ""
+        if rc == -4:
+            detail = f"cudaError {lib().msa_last_cuda_error()}"
+        raise MsaError(name, rc, detail)
+
+
+def _numel_ok(t, n, what):
+    if t is not None and not isinstance(t, int):
+        if not t.is_contiguous():
+            raise ValueError(f"{what} must be contiguous")
+        if t.numel() < n:
+            raise ValueError(f"{what} holds {t.numel()} elements, needs {n}")
+
+
+# ---------------------------------------------------------------- entry points
+
+def msa_status_string(status: int) -> str:
+    return lib().msa_status_string(status).decode()
+
+
+def msa_version() -> str:
+    return lib().msa_version().decode()
+
+
+def msa_last_cuda_error() -> int:
+    return lib().msa_last_cuda_error()
+
+
+def msa_device_status(clear: bool = True, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _check("msa_device_status",
+           lib().msa_device_status(ctypes.addressof(out), int(clear), _stream(stream)))
+    return out.value
+
+
+def msa_chunk_offsets(n_docs, tok_offsets, chunk, chunk_offsets, stream=None):
+    _numel_ok(tok_offsets, n_docs + 1, "tok_offsets")
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets")
+    _check("msa_chunk_offsets", lib().msa_chunk_offsets(
+        n_docs, _ptr(tok_offsets), chunk, _ptr(chunk_offsets), _stream(stream)))
+
+
+def msa_encode_pool(dt, L, n_tok, n_docs, H, D, k_tok, v_tok, kr_tok, tok_offsets,
+                    chunk_offsets, n_chunks, rope_base, chunk, k_bar, v_bar, kr_bar,
+                    stream=None):
+    for t, what in ((k_tok, "k_tok"), (v_tok, "v_tok"), (kr_tok, "kr_tok")):
+        _numel_ok(t, L * n_tok * H * D, what)
+    for t, what in ((k_bar, "k_bar"), (v_bar, "v_bar"), (kr_bar, "kr_bar")):
+        _numel_ok(t, L * n_chunks * H * D, what)
+    _check("msa_encode_pool", lib().msa_encode_pool(
+        dt, L, n_tok, n_docs, H, D, _ptr(k_tok), _ptr(v_tok), _ptr(kr_tok),
+        _ptr(tok_offsets), _ptr(chunk_offsets), n_chunks, rope_base, chunk,
+        _ptr(k_bar), _ptr(v_bar), _ptr(kr_bar), _stream(stream)))
+
+
+def msa_route_workspace_size(dt, B, T, H, D) -> int:
+    return lib().msa_route_workspace_size(dt, B, T, H, D)
+
+
+def msa_route_scores(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_docs,
+                     doc_scores, chunk_scores, ws, ws_bytes, stream=None):
+    _numel_ok(q_r, B * T * H * D, "q_r")
+    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
+    _numel_ok(doc_scores, B * n_docs, "doc_scores")
+    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores")
+    _check("msa_route_scores", lib().msa_route_scores(
+        dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
+        _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def msa_topk_workspace_size(B, n_docs, k) -> int:
+    return lib().msa_topk_workspace_size(B, n_docs, k)
+
+
+def msa_topk_docs(B, n_docs, k, scores, idx, top_scores, ws, ws_bytes, stream=None):
+    _numel_ok(scores, B * n_docs, "scores")
+    _numel_ok(idx, B * k, "idx")
+    _check("msa_topk_docs", lib().msa_topk_docs(
+        B, n_docs, k, _ptr(scores), _ptr(idx), _ptr(top_scores), _ptr(ws), ws_bytes,
+        _stream(stream)))
+
+
+def msa_gather_kv(dt, B, k, H, D, idx, chunk_offsets, n_docs, k_bar, v_bar, m_cap, k_mem,
+                  v_mem, mem_len, stream=None):
+    _numel_ok(idx, B * k, "idx")
+    _numel_ok(k_mem, B * m_cap * H * D, "k_mem")
+    _numel_ok(v_mem, B * m_cap * H * D, "v_mem")
+    _check("msa_gather_kv", lib().msa_gather_kv(
+        dt, B, k, H, D, _ptr(idx), _ptr(chunk_offsets), n_docs, _ptr(k_bar), _ptr(v_bar),
+        m_cap, _ptr(k_mem), _ptr(v_mem), _ptr(mem_len), _stream(stream)))
+
+
+def msa_sparse_attn_workspace_size(dt, B, T, T_loc, Hq, H, D, m_cap) -> int:
+    return lib().msa_sparse_attn_workspace_size(dt, B, T, T_loc, Hq, H, D, m_cap)
+
+
+def msa_sparse_attn(dt, B, T, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc,
+                    pos0, rope_base, scale, out, ws, ws_bytes, stream=None):
+    _numel_ok(q, B * T * Hq * D, "q")
+    _numel_ok(k_loc, B * T_loc * H * D, "k_loc")
+    _numel_ok(v_loc, B * T_loc * H * D, "v_loc")
+    _numel_ok(out, B * T * Hq * D, "out")
+    _check("msa_sparse_attn", lib().msa_sparse_attn(
+        dt, B, T, T_loc, Hq, H, D, _ptr(q), _ptr(k_mem), _ptr(v_mem), _ptr(mem_len), m_cap,
+        _ptr(k_loc), _ptr(v_loc), pos0, rope_base, scale, _ptr(out), _ptr(ws), ws_bytes,
+        _stream(stream)))

@@ -1,0 +1,134 @@
+"""Buffer management around the libmsa C ABI: allocates device tensors with
+torch and chains the entry points encode -> route -> top-k -> gather ->
+attend.  No arithmetic of the method happens here; every step is one call
+into libmsa.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import msa as _m
+
+
+def dt_code(t: torch.Tensor) -> int:
+    return _m.dtype_code(t.dtype)
+
+
+def chunk_offsets(tok_offsets: torch.Tensor, chunk: int = 64, stream=None) -> torch.Tensor:
+    """Device chunk offsets [n_docs+1] (int64) from device token offsets."""
+    n_docs = tok_offsets.numel() - 1
+    out = torch.empty(n_docs + 1, dtype=torch.int64, device=tok_offsets.device)
+    _m.msa_chunk_offsets(n_docs, tok_offsets, chunk, out, stream)
+    return out
+
+
+def encode_pool(k_tok, v_tok, kr_tok, tok_offsets, chunk_offs, n_chunks: int,
+                rope_base: float = 10000.0, chunk: int = 64, out=None, stream=None):
+    """Token-level [L][N][H][D] -> pooled banks [L][C][H][D] (same dtype)."""
+    L, N, H, D = k_tok.shape
+    n_docs = tok_offsets.numel() - 1
+    if out is None:
+        out = tuple(torch.empty((L, n_chunks, H, D), dtype=k_tok.dtype, device=k_tok.device)
+                    for _ in range(3))
+    kb, vb, rb = out
+    _m.msa_encode_pool(dt_code(k_tok), L, N, n_docs, H, D, k_tok, v_tok, kr_tok, tok_offsets,
+                       chunk_offs, n_chunks, rope_base, chunk, kb, vb, rb, stream)
+    return kb, vb, rb
+
+
+class Router:
+    """Holds the workspace of msa_route_scores for fixed (dtype, B, T, H, D)."""
+
+    def __init__(self, dtype: torch.dtype, B: int, T: int, H: int, D: int, device):
+        self.dt = _m.dtype_code(dtype)
+        self.B, self.T, self.H, self.D = B, T, H, D
+        n = _m.msa_route_workspace_size(self.dt, B, T, H, D)
+        self.ws = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+    def __call__(self, q_r, kr_bar, chunk_offs, n_docs, doc_scores=None, chunk_scores=None,
+                 stream=None):
+        C = kr_bar.shape[0]
+        if doc_scores is None:
+            doc_scores = torch.empty((self.B, n_docs), dtype=torch.float32, device=q_r.device)
+        _m.msa_route_scores(self.dt, self.B, self.T, self.H, self.D, q_r, kr_bar, C, chunk_offs,
+                            n_docs, doc_scores, chunk_scores, self.ws, self.ws.numel(), stream)
+        return doc_scores
+
+
+def topk_docs(scores: torch.Tensor, k: int, idx=None, top=None, stream=None):
+    B, n = scores.shape
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+    _m.msa_topk_docs(B, n, k, scores, idx, top, None, 0, stream)
+    return idx, top
+
+
+def gather_kv(idx, chunk_offs, k_bar, v_bar, m_cap: int, k_mem=None, v_mem=None, mem_len=None,
+              stream=None):
+    B, k = idx.shape
+    C, H, D = k_bar.shape
+    n_docs = chunk_offs.numel() - 1
+    dev = k_bar.device
+    if k_mem is None:
+        k_mem = torch.empty((B, m_cap, H, D), dtype=k_bar.dtype, device=dev)
+        v_mem = torch.empty((B, m_cap, H, D), dtype=k_bar.dtype, device=dev)
+    if mem_len is None:
+        mem_len = torch.empty(B, dtype=torch.int32, device=dev)
+    _m.msa_gather_kv(dt_code(k_bar), B, k, H, D, idx, chunk_offs, n_docs, k_bar, v_bar, m_cap,
+                     k_mem, v_mem, mem_len, stream)
+    return k_mem, v_mem, mem_len
+
+
+class Attention:
+    """Holds the workspace of msa_sparse_attn for fixed shapes."""
+
+    def __init__(self, dtype, B, T, T_loc, Hq, H, D, m_cap, device):
+        self.dt = _m.dtype_code(dtype)
+        self.shape = (B, T, T_loc, Hq, H, D, m_cap)
+        n = _m.msa_sparse_attn_workspace_size(self.dt, B, T, T_loc, Hq, H, D, m_cap)
+        self.ws = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+    def __call__(self, q, k_mem, v_mem, mem_len, k_loc, v_loc, pos0: int,
+                 rope_base: float = 10000.0, scale: float = 0.0, out=None, stream=None):
+        B, T, T_loc, Hq, H, D, m_cap = self.shape
+        if out is None:
+            out = torch.empty((B, T, Hq, D), dtype=q.dtype, device=q.device)
+        _m.msa_sparse_attn(self.dt, B, T, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len, m_cap,
+                           k_loc, v_loc, pos0, rope_base, scale, out, self.ws, self.ws.numel(),
+                           stream)
+        return out
+
+
+class Pipeline:
+    """route -> top-k -> gather -> attend over a resident pooled bank (one
+    layer), with every buffer allocated once."""
+
+    def __init__(self, kr_bar, k_bar, v_bar, chunk_offs, *, B, T, T_loc, Hq, k, m_cap,
+                 pos0=None, rope_base=10000.0):
+        C, H, D = kr_bar.shape
+        dev = kr_bar.device
+        self.kr_bar, self.k_bar, self.v_bar, self.coff = kr_bar, k_bar, v_bar, chunk_offs
+        self.n_docs = chunk_offs.numel() - 1
+        self.B, self.T, self.T_loc, self.Hq, self.H, self.D = B, T, T_loc, Hq, H, D
+        self.k, self.m_cap = k, m_cap
+        self.pos0 = k if pos0 is None else pos0
+        self.rope_base = rope_base
+        self.router = Router(kr_bar.dtype, B, T, H, D, dev)
+        self.attn = Attention(kr_bar.dtype, B, T, T_loc, Hq, H, D, m_cap, dev)
+        self.doc_scores = torch.empty((B, self.n_docs), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+        self.top = torch.empty((B, k), dtype=torch.float32, device=dev)
+        self.k_mem = torch.empty((B, max(m_cap, 1), H, D), dtype=kr_bar.dtype, device=dev)
+        self.v_mem = torch.empty_like(self.k_mem)
+        self.mem_len = torch.empty(B, dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, T, Hq, D), dtype=kr_bar.dtype, device=dev)
+
+    def __call__(self, q_r, q, k_loc, v_loc, stream=None):
+        self.router(q_r, self.kr_bar, self.coff, self.n_docs, self.doc_scores, None, stream)
+        topk_docs(self.doc_scores, self.k, self.idx, self.top, stream)
+        gather_kv(self.idx, self.coff, self.k_bar, self.v_bar, self.m_cap, self.k_mem,
+                  self.v_mem, self.mem_len, stream)
+        self.attn(q, self.k_mem, self.v_mem, self.mem_len, k_loc, v_loc, self.pos0,
+                  self.rope_base, 0.0, self.out, stream)
+        return self.out

@@ -1,0 +1,78 @@
+"""CPU checks of the C ABI boundary: libmsa.so loads, exports every function
+include/msa.h declares, and rejects bad arguments on the host before any
+CUDA work (no GPU needed for these paths)."""
+
+import ctypes
+
+import pytest
+
+from latent_memory_routing_b200 import msa
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return msa.lib()
+
+
+def test_header_declares_the_hot_path(lib):
+    names = msa.header_symbols()
+    for required in ("msa_encode_pool", "msa_route_scores", "msa_topk_docs",
+                     "msa_gather_kv", "msa_sparse_attn"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in msa.header_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_header():
+    assert set(msa.header_symbols()) == set(msa._SIGS)
+
+
+def test_status_strings(lib):
+    for code in range(-6, 1):
+        assert msa.msa_status_string(code)
+    assert msa.msa_status_string(12345) == "unknown status"
+    assert "sm_100a" in msa.msa_version()
+
+
+NULL = None
+
+
+def test_host_validation_topk(lib):
+    f = lib.msa_topk_docs
+    assert f(1, 10, 11, 16, 16, NULL, NULL, 0, NULL) == -1      # k > n_docs
+    assert f(1, 10, 0, 16, 16, NULL, NULL, 0, NULL) == -1       # k == 0
+    assert f(1, 10, 2, NULL, 16, NULL, NULL, 0, NULL) == -1     # NULL scores
+
+
+def test_host_validation_route(lib):
+    f = lib.msa_route_scores
+    p = 256
+    assert f(1, 1, 4, 0, 128, p, p, 10, p, 2, p, NULL, p, 1 << 20, NULL) == -1   # H == 0
+    assert f(1, 1, 4, 8, 96, p, p, 10, p, 2, p, NULL, p, 1 << 20, NULL) == -2    # D == 96
+    assert f(1, 1, 4, 9, 128, p, p, 10, p, 2, p, NULL, p, 1 << 20, NULL) == -2   # bf16 H > 8
+    assert f(1, 1, 4, 8, 128, p + 4, p, 10, p, 2, p, NULL, p, 1 << 20, NULL) == -1  # misaligned
+    assert f(1, 1, 4, 8, 128, p, p, 10, p, 2, p, NULL, NULL, 0, NULL) == -6      # no workspace
+
+
+def test_host_validation_encode_gather_attn(lib):
+    p = 256
+    assert lib.msa_encode_pool(1, 1, 100, 2, 8, 128, p, p, p, p, p, 4, 1e4, 65,
+                               p, p, p, NULL) == -1                              # chunk > 64
+    assert lib.msa_encode_pool(1, 1, 100, 2, 8, 100, p, p, p, p, p, 4, 1e4, 64,
+                               p, p, p, NULL) == -2                              # D == 100
+    assert lib.msa_gather_kv(1, 1, 3, 8, 128, p, p, 2, p, p, 16, p, p, p, NULL) == -1  # k > n
+    assert lib.msa_sparse_attn(1, 1, 5, 4, 32, 8, 128, p, p, p, p, 16, p, p, 16, 1e4, 0.0,
+                               p, p, 1 << 20, NULL) == -1                        # T > T_loc
+    assert lib.msa_sparse_attn(1, 1, 1, 4, 30, 8, 128, p, p, p, p, 16, p, p, 16, 1e4, 0.0,
+                               p, p, 1 << 20, NULL) == -2                        # Hq % H
+    assert lib.msa_device_status(NULL, 0, NULL) == -1
+
+
+def test_workspace_sizes_are_monotone(lib):
+    a = msa.msa_route_workspace_size(1, 1, 256, 8, 128)
+    b = msa.msa_route_workspace_size(1, 2, 256, 8, 128)
+    assert 0 < a < b
+    assert msa.msa_route_workspace_size(1, 0, 256, 8, 128) == 0

@@ -1,0 +1,454 @@
+"""GPU parity of every libmsa entry point against the float64 oracle.
+
+Inputs come from ``latent_memory_routing_b200.synth`` (seeded); both sides
+consume the same bytes (the GPU tensor, and its copy upcast to float64 for
+the oracle).  No expected value comes from the CUDA path.  Tolerances:
+
+* pooled K̄/V̄/K̄_r: normwise relative error (max |gpu-oracle| / max |oracle|
+  per tensor) <= 1e-5 in fp32, <= 1e-2 in bf16;
+* routing scores: <= 2e-3 absolute;
+* top-k: identical to the oracle on identical scores; on routed scores,
+  identical wherever the oracle's gap between consecutive ranks exceeds
+  4e-3;
+* attention: <= 2e-2 max-abs in bf16; <= 1e-4 in fp32 (fp32 sums over at
+  most a few thousand keys plus a 2e-7 RoPE angle error stay below 1e-5;
+  1e-4 leaves a 10x margin).
+
+Full-size workloads are checked on sampled outputs that the oracle computes
+one by one.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from latent_memory_routing_b200 import msa, pipeline, synth
+
+pytestmark = pytest.mark.gpu
+
+RTOL_F32 = 1e-5
+RTOL_BF16 = 1e-2
+ROUTE_ATOL = 2e-3
+GAP = 4e-3
+ATTN_BF16 = 2e-2
+ATTN_F32 = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    from latent_memory_routing_b200 import build
+    build.build()
+    msa.lib()
+    msa.msa_device_status(clear=True)
+    yield
+    torch.cuda.synchronize()
+
+
+def f64(t):
+    return t.detach().double().cpu().numpy()
+
+
+def normwise(gpu, ref):
+    ref = np.asarray(ref)
+    return float(np.max(np.abs(np.asarray(gpu) - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+def status_ok():
+    torch.cuda.synchronize()
+    assert msa.msa_device_status(clear=True) == 0
+
+
+# ------------------------------------------------------------------ chunking
+
+@pytest.mark.parametrize("lengths", [
+    [180] * 16, [1], [64], [65], [1, 2, 3, 64, 128, 129, 8192],
+    list(synth.bank_10m_lengths().numpy()), list(synth.bank_100m_lengths().numpy()),
+])
+def test_chunk_offsets_bit_exact(lengths):
+    toff = synth.tok_offsets(torch.tensor(lengths)).cuda()
+    got = pipeline.chunk_offsets(toff).cpu().numpy()
+    want = oracle.chunk_offsets_from_lengths(lengths)
+    np.testing.assert_array_equal(got, want)
+    status_ok()
+
+
+# ------------------------------------------------------------------ encoding
+
+def _encode_case(dtype, L, lengths, H, D, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    toff_c = synth.tok_offsets(torch.tensor(lengths))
+    N = int(toff_c[-1])
+    k, v, r = (synth.randn((L, N, H, D), dtype, "cuda", g) for _ in range(3))
+    toff = toff_c.cuda()
+    coff = pipeline.chunk_offsets(toff)
+    C = int(coff[-1])
+    kb, vb, rb = pipeline.encode_pool(k, v, r, toff, coff, C)
+    torch.cuda.synchronize()
+    return k, v, r, toff_c, coff.cpu().numpy(), (kb, vb, rb)
+
+
+@pytest.mark.parametrize("dtype,L,H,D,tol", [
+    (torch.float32, 1, 2, 64, RTOL_F32),
+    (torch.float32, 2, 8, 128, RTOL_F32),
+    (torch.bfloat16, 2, 8, 128, RTOL_BF16),
+    (torch.bfloat16, 1, 4, 64, RTOL_BF16),
+    (torch.bfloat16, 3, 16, 128, RTOL_BF16),
+])
+def test_encode_ragged(dtype, L, H, D, tol):
+    lengths = [1, 5, 63, 64, 65, 127, 128, 129, 180, 300, 777, 2, 4000]
+    k, v, r, toff, coff, (kb, vb, rb) = _encode_case(dtype, L, lengths, H, D, 7)
+    ok, ov, orr, ocoff = oracle.encode_pool(f64(k), f64(v), f64(r), toff.numpy(), 10000.0)
+    np.testing.assert_array_equal(coff, ocoff)
+    assert normwise(f64(kb), ok) <= tol
+    assert normwise(f64(vb), ov) <= tol
+    assert normwise(f64(rb), orr) <= tol
+    status_ok()
+
+
+def test_encode_tiny_workload_fp32():
+    w = synth.tiny("cuda")
+    toff = w["tok_offsets"].cuda()
+    coff = pipeline.chunk_offsets(toff)
+    kb, vb, rb = pipeline.encode_pool(w["k_tok"], w["v_tok"], w["kr_tok"], toff, coff, 48)
+    ok, ov, orr, _ = oracle.encode_pool(f64(w["k_tok"]), f64(w["v_tok"]), f64(w["kr_tok"]),
+                                        w["tok_offsets"].numpy(), 10000.0)
+    for got, want in ((kb, ok), (vb, ov), (rb, orr)):
+        assert normwise(f64(got), want) <= RTOL_F32
+    status_ok()
+
+
+def test_encode_4_layers_1m_tokens_sampled():
+    w = synth.encode_4l("cuda")
+    toff = w["tok_offsets"].cuda()
+    coff = pipeline.chunk_offsets(toff)
+    C = int(coff[-1])
+    kb, vb, rb = pipeline.encode_pool(w["k_tok"], w["v_tok"], w["kr_tok"], toff, coff, C)
+    torch.cuda.synchronize()
+    coff_h = coff.cpu().numpy()
+    toff_h = w["tok_offsets"].numpy()
+    n_docs = len(toff_h) - 1
+    rng = np.random.default_rng(5)
+    docs = sorted(set(rng.choice(n_docs, 24, replace=False).tolist()) | {0, n_docs - 1})
+    for d in docs:
+        t0, t1 = int(toff_h[d]), int(toff_h[d + 1])
+        c0, c1 = int(coff_h[d]), int(coff_h[d + 1])
+        for l in range(w["L"]):
+            want = oracle.encode_pool_doc(f64(w["k_tok"][l, t0:t1]), f64(w["v_tok"][l, t0:t1]),
+                                          f64(w["kr_tok"][l, t0:t1]), 10000.0)
+            for got, ref in zip((kb, vb, rb), want):
+                assert normwise(f64(got[l, c0:c1]), ref) <= RTOL_BF16, (d, l)
+    status_ok()
+
+
+# ------------------------------------------------------------------- routing
+
+def _pooled_bank(n_docs, lo, hi, H, D, dtype, seed, needle_q=None):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    gc = torch.Generator().manual_seed(seed)
+    lengths = torch.randint(lo, hi + 1, (n_docs,), generator=gc)
+    coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
+    C = int(coff_h[-1])
+    kr = synth.randn((C, H, D), dtype, "cuda", g)
+    if needle_q is not None:
+        synth.plant_pooled_needles(kr, coff_h, [n_docs // 3], needle_q, g)
+    return kr, torch.from_numpy(coff_h).cuda(), coff_h
+
+
+def _route(q_r, kr, coff, n_docs, with_chunks=True):
+    B, T, H, D = q_r.shape
+    router = pipeline.Router(q_r.dtype, B, T, H, D, "cuda")
+    cs = torch.empty((B, kr.shape[0]), dtype=torch.float32, device="cuda") if with_chunks else None
+    ds = router(q_r, kr, coff, n_docs, chunk_scores=cs)
+    torch.cuda.synchronize()
+    return ds, cs
+
+
+@pytest.mark.parametrize("B,T,H,D,n_docs", [
+    (1, 256, 8, 128, 150),    # one pass, N = 256 (the 100M prefill shape)
+    (1, 128, 8, 128, 90),     # N = 128
+    (64, 1, 8, 128, 60),      # N = 64, one column per query (decode shape)
+    (3, 7, 8, 128, 40),       # N = 64 with 21 live columns
+    (3, 48, 8, 128, 40),      # N = 256, query 2 straddles the column halves
+    (2, 150, 8, 128, 40),     # 300 columns: two passes over the bank
+    (1, 64, 2, 64, 70),       # D = 64, H = 2
+    (5, 3, 1, 128, 33),       # H = 1
+])
+def test_route_bf16_vs_oracle(B, T, H, D, n_docs):
+    g = torch.Generator(device="cuda").manual_seed(100 + B * T)
+    q_r = synth.randn((B, T, H, D), torch.bfloat16, "cuda", g)
+    kr, coff, coff_h = _pooled_bank(n_docs, 1, 900, H, D, torch.bfloat16, 11 + T,
+                                    needle_q=q_r[0])
+    ds, cs = _route(q_r, kr, coff, n_docs)
+    ods, ocs = oracle.route_scores(f64(q_r), f64(kr), coff_h)
+    assert np.max(np.abs(f64(cs) - ocs)) <= ROUTE_ATOL
+    assert np.max(np.abs(f64(ds) - ods)) <= ROUTE_ATOL
+    status_ok()
+
+
+def test_route_fp32_tiny():
+    w = synth.tiny("cuda")
+    ok, ov, orr, coff_h = oracle.encode_pool(f64(w["k_tok"]), f64(w["v_tok"]), f64(w["kr_tok"]),
+                                             w["tok_offsets"].numpy(), 10000.0)
+    kr = torch.from_numpy(orr[0]).float().cuda()  # oracle bank as the common input
+    ds, cs = _route(w["q_r"], kr, torch.from_numpy(coff_h).cuda(), 16)
+    ods, ocs = oracle.route_scores(f64(w["q_r"]), f64(kr), coff_h)
+    assert np.max(np.abs(f64(cs) - ocs)) <= 1e-5
+    assert np.max(np.abs(f64(ds) - ods)) <= 1e-5
+    assert int(torch.argmax(ds[0])) == 5
+    status_ok()
+
+
+def test_route_zero_key_scores_zero():
+    H, D = 8, 128
+    kr = torch.zeros((130, H, D), dtype=torch.bfloat16, device="cuda")
+    kr[:65] = 1.0
+    coff_h = np.array([0, 65, 130])
+    q = torch.ones((1, 4, H, D), dtype=torch.bfloat16, device="cuda")
+    ds, cs = _route(q, kr, torch.from_numpy(coff_h).cuda(), 2)
+    assert abs(float(ds[0, 0]) - 1.0) <= ROUTE_ATOL
+    assert float(ds[0, 1]) == 0.0
+    status_ok()
+
+
+def _check_topk_on_routed(idx, oracle_scores, k):
+    """Indices must match the oracle wherever the oracle ranking is
+    unambiguous by more than GAP."""
+    idx = np.asarray(idx)
+    for b in range(oracle_scores.shape[0]):
+        s = oracle_scores[b]
+        order = np.lexsort((np.arange(s.shape[0]), -s))
+        srt = s[order]
+        if srt[k - 1] - srt[k] > GAP:
+            assert set(idx[b].tolist()) == set(order[:k].tolist()), b
+        for r in range(k):
+            left = srt[r - 1] - srt[r] if r > 0 else np.inf
+            right = srt[r] - srt[r + 1]
+            if left > GAP and right > GAP:
+                assert idx[b, r] == order[r], (b, r)
+
+
+def test_route_topk_10m_decode_full():
+    lengths = synth.bank_10m_lengths()
+    coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
+    w = synth.bank_10m(coff_h, "cuda")
+    coff = torch.from_numpy(coff_h).cuda()
+    ds, _ = _route(w["q_r"], w["kr_bar"], coff, len(lengths), with_chunks=False)
+    ods, _ = oracle.route_scores(f64(w["q_r"]), f64(w["kr_bar"]), coff_h)
+    assert np.max(np.abs(f64(ds) - ods)) <= ROUTE_ATOL
+    idx, _ = pipeline.topk_docs(ds, 16)
+    _check_topk_on_routed(idx.cpu().numpy(), ods, 16)
+    status_ok()
+
+
+def test_route_100m_prefill_sampled():
+    lengths = synth.bank_100m_lengths()
+    coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
+    w = synth.bank_100m(coff_h, "cuda")
+    coff = torch.from_numpy(coff_h).cuda()
+    n_docs = len(lengths)
+    ds, cs = _route(w["q_r"], w["kr_bar"], coff, n_docs)
+    idx, _ = pipeline.topk_docs(ds, 16)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(3)
+    C = int(coff_h[-1])
+    q = f64(w["q_r"])
+    chunks = np.unique(np.concatenate([rng.choice(C, 6000, replace=False),
+                                       np.arange(C - 300, C), np.arange(0, 300)]))
+    ocs = oracle.route_chunk_scores(q, f64(w["kr_bar"][torch.from_numpy(chunks).cuda()]))
+    assert np.max(np.abs(f64(cs)[0, chunks] - ocs[0])) <= ROUTE_ATOL
+    docs = np.unique(np.concatenate([rng.choice(n_docs, 300, replace=False), w["needles"],
+                                     idx[0].cpu().numpy()]))
+    for d in docs:
+        rows = torch.arange(int(coff_h[d]), int(coff_h[d + 1]), device="cuda")
+        od = oracle.route_chunk_scores(q, f64(w["kr_bar"][rows])).max()
+        assert abs(float(ds[0, d]) - od) <= ROUTE_ATOL, d
+    # top-k is exact on the GPU's own scores: every unselected score is below
+    # the k-th (or equal with a higher index), selection is in rank order
+    s = ds[0].cpu().numpy()
+    sel = idx[0].cpu().numpy()
+    kth = s[sel[-1]]
+    assert np.all(np.diff(s[sel]) <= 0)
+    rest = np.setdiff1d(np.arange(n_docs), sel)
+    assert np.all((s[rest] < kth) | ((s[rest] == kth) & (rest > sel[-1])))
+    status_ok()
+
+
+# --------------------------------------------------------------------- top-k
+
+@pytest.mark.parametrize("B,n,k,quant", [
+    (1, 16, 2, None), (4, 1000, 16, None), (64, 10000, 16, None), (1, 100000, 16, None),
+    (3, 5000, 1024, None), (2, 300, 300, None), (2, 5000, 16, 8.0), (1, 4096, 64, 1.0),
+])
+def test_topk_identical_to_oracle(B, n, k, quant):
+    g = torch.Generator(device="cuda").manual_seed(n + k)
+    s = torch.randn((B, n), device="cuda", generator=g)
+    if quant is not None:  # many exact ties
+        s = torch.round(s * quant) / quant
+    idx, top = torch.empty((B, k), dtype=torch.int32, device="cuda"), \
+        torch.empty((B, k), device="cuda")
+    pipeline.topk_docs(s, k, idx, top)
+    oi, ot = oracle.topk_docs(f64(s), k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), oi)
+    np.testing.assert_array_equal(f64(top), ot)
+    status_ok()
+
+
+def test_topk_special_values():
+    s = torch.tensor([[0.5, float("nan"), -float("inf"), 0.5, float("inf"), -0.0, 0.0]],
+                     device="cuda")
+    idx, _ = pipeline.topk_docs(s, 7)
+    # +inf, the two 0.5 by index, -0.0 and 0.0 as equal scores by index,
+    # -inf, NaN last
+    assert idx[0].tolist() == [4, 0, 3, 5, 6, 2, 1]
+    oi, _ = oracle.topk_docs(f64(s), 7)
+    assert oi[0].tolist() == idx[0].tolist()
+    status_ok()
+
+
+# -------------------------------------------------------------------- gather
+
+def test_gather_bit_exact_and_capacity():
+    H, D = 8, 128
+    kr, coff, coff_h = _pooled_bank(50, 1, 700, H, D, torch.bfloat16, 21)
+    g = torch.Generator(device="cuda").manual_seed(22)
+    kb = synth.randn(kr.shape, torch.bfloat16, "cuda", g)
+    vb = synth.randn(kr.shape, torch.bfloat16, "cuda", g)
+    idx = torch.tensor([[7, 3, 49, 0], [12, 12, 5, 30]], dtype=torch.int32, device="cuda")
+    counts = np.diff(coff_h)
+    need = [int(counts[r].sum()) for r in idx.cpu().numpy()]
+    m_cap = max(need) + 3
+    km, vm, ml = pipeline.gather_kv(idx, coff, kb, vb, m_cap)
+    okm, ovm, oml = oracle.gather_kv(idx.cpu().numpy(), coff_h, f64(kb), f64(vb))
+    assert ml.cpu().tolist() == oml.tolist()
+    for b in range(2):
+        np.testing.assert_array_equal(f64(km[b, :oml[b]]), okm[b])
+        np.testing.assert_array_equal(f64(vm[b, :oml[b]]), ovm[b])
+    status_ok()
+    # capacity overflow: rows past m_cap dropped, status word set
+    small = min(need) - 1
+    km2, vm2, ml2 = pipeline.gather_kv(idx, coff, kb, vb, small)
+    torch.cuda.synchronize()
+    assert ml2.cpu().tolist() == [small, small]
+    np.testing.assert_array_equal(f64(km2[0]), okm[0][:small])
+    assert msa.msa_device_status(clear=True) == -3
+
+
+def test_gather_fp32_tiny():
+    w = synth.tiny("cuda")
+    ok, ov, orr, coff_h = oracle.encode_pool(f64(w["k_tok"]), f64(w["v_tok"]), f64(w["kr_tok"]),
+                                             w["tok_offsets"].numpy(), 10000.0)
+    kb = torch.from_numpy(ok[0]).float().cuda()
+    vb = torch.from_numpy(ov[0]).float().cuda()
+    idx = torch.tensor([[5, 0]], dtype=torch.int32, device="cuda")
+    km, vm, ml = pipeline.gather_kv(idx, torch.from_numpy(coff_h).cuda(), kb, vb, 6)
+    okm, ovm, oml = oracle.gather_kv([[5, 0]], coff_h, f64(kb), f64(vb))
+    assert int(ml[0]) == 6
+    np.testing.assert_array_equal(f64(km[0]), okm[0])
+    np.testing.assert_array_equal(f64(vm[0]), ovm[0])
+    status_ok()
+
+
+# ----------------------------------------------------------------- attention
+
+def _attn_case(dtype, B, T, T_loc, Hq, H, D, m_cap, mem_lens, pos0, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q = synth.randn((B, T, Hq, D), dtype, "cuda", g)
+    km = synth.randn((B, max(m_cap, 1), H, D), dtype, "cuda", g)
+    vm = synth.randn((B, max(m_cap, 1), H, D), dtype, "cuda", g)
+    kl = synth.randn((B, T_loc, H, D), dtype, "cuda", g)
+    vl = synth.randn((B, T_loc, H, D), dtype, "cuda", g)
+    ml = torch.tensor(mem_lens, dtype=torch.int32, device="cuda")
+    att = pipeline.Attention(dtype, B, T, T_loc, Hq, H, D, m_cap, "cuda")
+    out = att(q, km, vm, ml, kl, vl, pos0)
+    torch.cuda.synchronize()
+    okm = [f64(km[b, :mem_lens[b]]) for b in range(B)]
+    ovm = [f64(vm[b, :mem_lens[b]]) for b in range(B)]
+    want = oracle.sparse_attn(f64(q), okm, ovm, f64(kl), f64(vl), pos0, 10000.0)
+    return f64(out), want
+
+
+@pytest.mark.parametrize("dtype,B,T,T_loc,Hq,H,D,m_cap,mem_lens,pos0,tol", [
+    (torch.float32, 1, 16, 16, 4, 2, 64, 6, [6], 2, ATTN_F32),          # tiny workload shape
+    (torch.float32, 2, 5, 9, 8, 2, 128, 40, [33, 0], 16, ATTN_F32),     # chunked prefill, empty mem
+    (torch.float32, 3, 1, 300, 32, 8, 128, 100, [100, 7, 64], 16, ATTN_F32),  # decode
+    (torch.bfloat16, 1, 128, 128, 32, 8, 128, 300, [257], 16, ATTN_BF16),
+    (torch.bfloat16, 1, 256, 256, 32, 8, 128, 384, [371], 16, ATTN_BF16),
+    (torch.bfloat16, 2, 40, 100, 16, 2, 64, 50, [50, 0], 3, ATTN_BF16),
+    (torch.bfloat16, 8, 1, 2048, 32, 8, 128, 2048, [250, 0, 2048, 1, 100, 300, 17, 64], 16,
+     ATTN_BF16),
+    (torch.bfloat16, 2, 3, 7, 8, 8, 128, 5, [5, 2], 0, ATTN_BF16),      # G = 1
+])
+def test_attention_vs_oracle(dtype, B, T, T_loc, Hq, H, D, m_cap, mem_lens, pos0, tol):
+    got, want = _attn_case(dtype, B, T, T_loc, Hq, H, D, m_cap, mem_lens, pos0, 31 + T)
+    assert np.max(np.abs(got - want)) <= tol
+    status_ok()
+
+
+def test_attention_decode_10m_workload_full():
+    lengths = synth.bank_10m_lengths()
+    coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
+    w = synth.bank_10m(coff_h, "cuda")
+    B = w["B"]
+    rng = np.random.default_rng(9)
+    # 16 documents per query, as the router would select
+    idx = np.stack([rng.choice(len(lengths), 16, replace=False) for _ in range(B)])
+    counts = np.diff(coff_h)
+    m_cap = int(max(counts[r].sum() for r in idx))
+    km, vm, ml = pipeline.gather_kv(torch.from_numpy(idx).int().cuda(),
+                                    torch.from_numpy(coff_h).cuda(), w["k_bar"], w["v_bar"], m_cap)
+    att = pipeline.Attention(torch.bfloat16, B, 1, 2048, 32, 8, 128, m_cap, "cuda")
+    out = att(w["q"], km, vm, ml, w["k_loc"], w["v_loc"], 16)
+    torch.cuda.synchronize()
+    okm, ovm, _ = oracle.gather_kv(idx, coff_h, f64(w["k_bar"]), f64(w["v_bar"]))
+    want = oracle.sparse_attn(f64(w["q"]), okm, ovm, f64(w["k_loc"]), f64(w["v_loc"]), 16)
+    assert np.max(np.abs(f64(out) - want)) <= ATTN_BF16
+    status_ok()
+
+
+# ------------------------------------------------------------ whole pipeline
+
+def test_tiny_pipeline_end_to_end_fp32():
+    w = synth.tiny("cuda")
+    toff = w["tok_offsets"].cuda()
+    coff = pipeline.chunk_offsets(toff)
+    kb, vb, rb = pipeline.encode_pool(w["k_tok"], w["v_tok"], w["kr_tok"], toff, coff, 48)
+    p = pipeline.Pipeline(rb[0], kb[0], vb[0], coff, B=1, T=16, T_loc=16, Hq=4, k=2, m_cap=6)
+    out = p(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    torch.cuda.synchronize()
+    ref = oracle.msa_forward(f64(w["k_tok"]), f64(w["v_tok"]), f64(w["kr_tok"]),
+                             w["tok_offsets"].numpy(), f64(w["q_r"]), f64(w["q"]),
+                             f64(w["k_loc"]), f64(w["v_loc"]), k=2)
+    assert p.idx[0].tolist() == ref["topk_idx"][0].tolist() == [5, p.idx[0, 1].item()]
+    assert int(p.mem_len[0]) == 6
+    assert np.max(np.abs(f64(p.doc_scores) - ref["doc_scores"])) <= 1e-5
+    assert np.max(np.abs(f64(out) - ref["out"])) <= ATTN_F32
+    status_ok()
+
+
+def test_1m_bank_chain_sampled():
+    """Token-level 1M bank: encode on the GPU, route, top-k; compared with the
+    oracle encoding + routing of the sampled documents."""
+    w = synth.bank_1m("cuda")
+    toff = w["tok_offsets"].cuda()
+    coff = pipeline.chunk_offsets(toff)
+    C = int(coff[-1])
+    kb, vb, rb = pipeline.encode_pool(w["k_tok"], w["v_tok"], w["kr_tok"], toff, coff, C)
+    ds, _ = _route(w["q_r"], rb[0], coff, 1000, with_chunks=False)
+    idx, _ = pipeline.topk_docs(ds, 16)
+    torch.cuda.synchronize()
+    toff_h = w["tok_offsets"].numpy()
+    q = f64(w["q_r"])
+    rng = np.random.default_rng(1)
+    docs = np.unique(np.concatenate([rng.choice(1000, 40, replace=False), w["needles"],
+                                     idx[0].cpu().numpy()]))
+    for d in docs:
+        t0, t1 = int(toff_h[d]), int(toff_h[d + 1])
+        _, _, orb = oracle.encode_pool_doc(f64(w["k_tok"][0, t0:t1]), f64(w["v_tok"][0, t0:t1]),
+                                           f64(w["kr_tok"][0, t0:t1]), 10000.0)
+        od = oracle.route_chunk_scores(q, orb).max()
+        # the GPU routes its own bf16-rounded bank: allow the bank rounding
+        assert abs(float(ds[0, d]) - od) <= ROUTE_ATOL + 2e-3, d
+    status_ok()
