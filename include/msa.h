@@ -139,6 +139,27 @@ int msa_route_scores(msa_dtype dt, int B, int T, int H, int D,
                      float* doc_scores, float* chunk_scores, void* ws,
                      size_t ws_bytes, msa_stream_t stream);
 
+/* Routing over a prepared bank.  The per-row normalisation of K̄_r depends
+ * only on the bank, so it can be done once when the bank is built (the
+ * pages encode the memory offline, [HYSEN] §"Memory must be encoded offline
+ * before a query can reach it") instead of on every query:
+ *   msa_route_prepare_bank writes kr_hat[c][h] = K̄_r[c][h] /
+ *     max(|K̄_r[c][h]|, 1e-12), rounded to bf16 ([n_chunks][H][D], may not
+ *     alias kr_bar);
+ *   msa_route_scores_prepared takes kr_hat in place of kr_bar and returns
+ *     the same scores as msa_route_scores (identical rounding: the raw scan
+ *     normalises the rows the same way in shared memory).
+ * bf16 only (MSA_ERR_UNSUPPORTED otherwise).  Same workspace, layouts and
+ * errors as msa_route_scores. */
+int msa_route_prepare_bank(msa_dtype dt, int64_t n_chunks, int H, int D,
+                           const void* kr_bar, void* kr_hat, msa_stream_t stream);
+int msa_route_scores_prepared(msa_dtype dt, int B, int T, int H, int D,
+                              const void* q_r, const void* kr_hat,
+                              int64_t n_chunks, const int64_t* chunk_offsets,
+                              int n_docs, float* doc_scores,
+                              float* chunk_scores, void* ws, size_t ws_bytes,
+                              msa_stream_t stream);
+
 /* Top-k documents -- [HYSEN] §"Routing happens inside attention ...": the
  * router selects the top-k documents.  Ties go to the lower document index.
  *   scores      [B][n_docs] float (device).

@@ -20,7 +20,9 @@ from .msa import (  # noqa: F401
     msa_encode_pool,
     msa_gather_kv,
     msa_last_cuda_error,
+    msa_route_prepare_bank,
     msa_route_scores,
+    msa_route_scores_prepared,
     msa_route_workspace_size,
     msa_sparse_attn,
     msa_sparse_attn_workspace_size,

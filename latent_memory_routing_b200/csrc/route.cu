@@ -12,6 +12,8 @@
 // fold in 1/H), the fp32 CUDA-core scan, the final conversion of the
 // order-preserving integer maxima to floats, and the C entry point.  The bf16
 // scan on the tcgen05 tensor cores lives in route_tc.cu.
+#include <algorithm>
+
 #include "msa_common.cuh"
 #include "route_tc.cuh"
 
@@ -148,23 +150,23 @@ extern "C" size_t msa_route_workspace_size(msa_dtype dt, int B, int T, int H,
   return msa::qhat_bytes(dt, B, T, H, D);
 }
 
-extern "C" int msa_route_scores(msa_dtype dt, int B, int T, int H, int D,
-                                const void* q_r, const void* kr_bar,
-                                int64_t n_chunks, const int64_t* chunk_offsets,
-                                int n_docs, float* doc_scores,
-                                float* chunk_scores, void* ws, size_t ws_bytes,
-                                msa_stream_t stream) {
-  using namespace msa;
+namespace msa {
+namespace {
+
+int route_scores_impl(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
+                      const void* kr, int64_t n_chunks, const int64_t* chunk_offsets, int n_docs,
+                      float* doc_scores, float* chunk_scores, void* ws, size_t ws_bytes,
+                      bool prepared, cudaStream_t s) {
   if (B <= 0 || T <= 0 || H <= 0 || n_docs <= 0 || n_chunks <= 0) return MSA_ERR_INVALID_ARG;
-  if (!q_r || !kr_bar || !chunk_offsets || !doc_scores) return MSA_ERR_INVALID_ARG;
-  if (!aligned16(kr_bar) || !aligned16(q_r)) return MSA_ERR_INVALID_ARG;
+  if (!q_r || !kr || !chunk_offsets || !doc_scores) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(kr) || !aligned16(q_r)) return MSA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return MSA_ERR_UNSUPPORTED;
   if (dt != MSA_F32 && dt != MSA_BF16) return MSA_ERR_INVALID_ARG;
-  if (H < 1 || H > (dt == MSA_BF16 ? 8 : 16)) return MSA_ERR_UNSUPPORTED;
+  if (prepared && dt != MSA_BF16) return MSA_ERR_UNSUPPORTED;
+  if (H > (dt == MSA_BF16 ? 8 : 16)) return MSA_ERR_UNSUPPORTED;
   if ((int64_t)B * T > (1LL << 24)) return MSA_ERR_UNSUPPORTED;
   const size_t need = qhat_bytes(dt, B, T, H, D);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int NT = B * T;
   uint32_t* doc_u = reinterpret_cast<uint32_t*>(doc_scores);
   uint32_t* chunk_u = reinterpret_cast<uint32_t*>(chunk_scores);
@@ -182,11 +184,11 @@ extern "C" int msa_route_scores(msa_dtype dt, int B, int T, int H, int D,
     const dim3 grid((unsigned)((n_chunks + 7) / 8), (unsigned)B);
     if (D == 64)
       route_simt_kernel<64><<<grid, 256, 0, s>>>(T, H, static_cast<const float*>(ws),
-                                                 static_cast<const float*>(kr_bar), n_chunks,
+                                                 static_cast<const float*>(kr), n_chunks,
                                                  chunk_offsets, n_docs, doc_u, chunk_u);
     else
       route_simt_kernel<128><<<grid, 256, 0, s>>>(T, H, static_cast<const float*>(ws),
-                                                  static_cast<const float*>(kr_bar), n_chunks,
+                                                  static_cast<const float*>(kr), n_chunks,
                                                   chunk_offsets, n_docs, doc_u, chunk_u);
     if ((rc = check_launch())) return rc;
   } else {
@@ -199,10 +201,44 @@ extern "C" int msa_route_scores(msa_dtype dt, int B, int T, int H, int D,
             static_cast<__nv_bfloat16*>(ws), doc_u, n_doc_u, chunk_u, n_chunk_u);
     if ((rc = check_launch())) return rc;
     rc = route_tc_launch(B, T, H, D, static_cast<const __nv_bfloat16*>(ws), n_pad,
-                         static_cast<const __nv_bfloat16*>(kr_bar), n_chunks,
-                         chunk_offsets, n_docs, doc_u, chunk_u, device_status_ptr(), s);
+                         static_cast<const __nv_bfloat16*>(kr), n_chunks, chunk_offsets, n_docs,
+                         doc_u, chunk_u, device_status_ptr(), prepared, s);
     if (rc) return rc;
   }
   route_finalize_kernel<<<(unsigned)sms * 4, 256, 0, s>>>(doc_u, n_doc_u, chunk_u, n_chunk_u);
   return check_launch();
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" int msa_route_scores(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
+                                const void* kr_bar, int64_t n_chunks,
+                                const int64_t* chunk_offsets, int n_docs, float* doc_scores,
+                                float* chunk_scores, void* ws, size_t ws_bytes,
+                                msa_stream_t stream) {
+  return msa::route_scores_impl(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_docs,
+                                doc_scores, chunk_scores, ws, ws_bytes, false,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int msa_route_scores_prepared(msa_dtype dt, int B, int T, int H, int D,
+                                         const void* q_r, const void* kr_hat, int64_t n_chunks,
+                                         const int64_t* chunk_offsets, int n_docs,
+                                         float* doc_scores, float* chunk_scores, void* ws,
+                                         size_t ws_bytes, msa_stream_t stream) {
+  return msa::route_scores_impl(dt, B, T, H, D, q_r, kr_hat, n_chunks, chunk_offsets, n_docs,
+                                doc_scores, chunk_scores, ws, ws_bytes, true,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int msa_route_prepare_bank(msa_dtype dt, int64_t n_chunks, int H, int D,
+                                      const void* kr_bar, void* kr_hat, msa_stream_t stream) {
+  using namespace msa;
+  if (n_chunks <= 0 || H <= 0 || !kr_bar || !kr_hat) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(kr_bar) || !aligned16(kr_hat)) return MSA_ERR_INVALID_ARG;
+  if (dt != MSA_BF16 || (D != 64 && D != 128)) return MSA_ERR_UNSUPPORTED;
+  return route_prepare_bank_launch(n_chunks * H, D, static_cast<const __nv_bfloat16*>(kr_bar),
+                                   static_cast<__nv_bfloat16*>(kr_hat),
+                                   reinterpret_cast<cudaStream_t>(stream));
 }

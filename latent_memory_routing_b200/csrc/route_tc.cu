@@ -9,23 +9,32 @@
 // a document's chunks is this library's reading of the document score.
 //
 // Design.  The bank is streamed once per pass (<= 256 query columns):
-//   * persistent CTAs, one per SM, walk 128-chunk tiles round-robin;
-//   * warp 0 (one lane) TMA-loads, per (tile, head), the tile's K̄_r rows of
-//     that head (128 x D bf16, 128B-swizzled) and the head's normalised
-//     query columns (N x D) into a multi-stage shared-memory ring;
+//   * persistent CTAs, one per SM, each owning a contiguous range of
+//     128-chunk tiles (so a tile's documents follow the previous tile's);
+//   * warp 0 (one lane) TMA-loads the tile's K̄_r rows of one head (128 x 64
+//     bf16 per K block, 128B-swizzled) and that head's normalised query
+//     columns (N x 64) into a multi-stage shared-memory ring;
+//   * raw bank: warps 2..5 (the transform, one thread per chunk row)
+//     normalise each row in place -- |K̄_r[c,h]| from the row's 16-byte
+//     pieces read in swizzled order (bank-conflict free), then
+//     K̄_r / max(|K̄_r|, 1e-12) rounded to bf16 -- so a stage holds a whole
+//     head.  Prepared bank (rows already unit-normalised by
+//     msa_route_prepare_bank when the bank was built): no transform, and a
+//     stage is one 64-wide K block, so twice as many stages fit;
 //   * warp 1 (one lane) issues tcgen05.mma M=128 (chunks) x N (query
-//     columns) x K=D per head into one of two TMEM accumulators, so the
-//     next head's MMAs overlap the epilogue of this one;
-//   * warps 2..9 (the epilogue) compute |K̄_r[c,h]| from the same shared
-//     tile, read the head's 128 x N scores from TMEM (one chunk row per
-//     thread, half of the columns per warpgroup), and accumulate
-//     inv|k| * score in registers -- the query side is pre-normalised with
-//     1/H folded in, so after the last head the registers hold the
-//     head-mean cosine;
-//   * the tile's row values go back to TMEM once, are reduced over each
-//     query's tokens (max), then over the rows of each document inside the
-//     warp (segmented shuffle max), and only one order-preserving atomicMax
-//     per (query, document segment) reaches global memory.
+//     columns) x K=16 for every head and K block of the tile into ONE TMEM
+//     accumulator: with unit rows on both sides (the query pre-normalised
+//     with 1/H folded in) the sum over heads is the head-mean cosine; two
+//     accumulators alternate between tiles so the next tile's MMAs overlap
+//     this tile's epilogue;
+//   * warps 6..9 (the epilogue, one thread per chunk row) find the row's
+//     document from a window of chunk offsets prefetched during the previous
+//     tile, read the 128 x N cosines from TMEM 32 columns at a time (the
+//     next load in flight while one is reduced), take the maximum over each
+//     query's tokens (a tree maximum when 32 columns belong to one query),
+//     then over the rows of each document inside the warp (segmented
+//     shuffle maximum), and issue one order-preserving atomicMax per
+//     (query, document segment).
 // Scores never round-trip through HBM.  No cluster multicast is used.
 #include <cudaTypedefs.h>
 
@@ -39,34 +48,35 @@ namespace msa {
 namespace {
 
 constexpr int kTile = 128;  // chunks per tile = MMA M = TMEM lanes
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kXWarps = 4;   // transform warps (raw bank)
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * (kXWarps + kEpiWarps);
 constexpr int kWindow = 256;  // documents cached per tile for chunk -> doc
 constexpr int kEpiBar = 1;    // named barrier of the epilogue warps
+constexpr int kMaxStages = 8;
 
-template <int N, int D>
+template <int N, int D, bool kPrep>
 struct Cfg {
-  static constexpr int KB = D / 64;                   // 64-element K blocks
-  static constexpr int A_BYTES = KB * kTile * 128;    // one head of a tile
-  static constexpr int B_BYTES = KB * N * 128;        // one head of the queries
+  static constexpr int KB = D / 64;                   // 64-element K blocks per head
+  static constexpr int SKB = kPrep ? 1 : KB;          // K blocks per stage
+  static constexpr int SPH = KB / SKB;                // stages per head
+  static constexpr int A_BYTES = SKB * kTile * 128;
+  static constexpr int B_BYTES = SKB * N * 128;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES_FIT = (196 * 1024) / STAGE;
-  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
-  static constexpr int TMEM_COLS = 2 * N < 32 ? 32 : 2 * N;
-  static constexpr int HALF_N = N / 2;
+  static constexpr int STAGES_FIT = (200 * 1024) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > kMaxStages ? kMaxStages : STAGES_FIT;
+  static constexpr int TMEM_COLS = 2 * N;
   static constexpr uint32_t IDESC = tc::idesc_bf16_f32(kTile, N);
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE;
   static_assert(STAGES >= 2, "need a double-buffered ring");
-  static_assert(N % 64 == 0 && N >= 64 && N <= 256, "N: whole 32-column TMEM loads per half");
+  static_assert(N % 64 == 0 && N >= 64 && N <= 256, "N");
 };
 
 struct Aux {
-  uint64_t full[4], empty[4], accf[2], acce[2];
+  uint64_t full[kMaxStages], ready[kMaxStages], empty[kMaxStages], accf[2], acce[2];
   uint32_t tmem_base;
   int abort_flag;
   int d0;
-  int doc_row[kTile];
-  float npart[2][2][kTile];
   int64_t win[kWindow + 1];
 };
 
@@ -74,38 +84,109 @@ __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync %0, %1;" ::"n"(kEpiBar), "n"(32 * kEpiWarps) : "memory");
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
-      "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]),
-      "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]),
-      "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]),
-      "f"(v[29]), "f"(v[30]), "f"(v[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+// x*x summed over the 8 bf16 of a 16-byte piece, in packed fp32 pairs.
+__device__ __forceinline__ void sumsq8(const uint4& v, unsigned long long& acc) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const unsigned long long x =
+        ((unsigned long long)(w[i] & 0xffff0000u) << 32) | (unsigned long long)(w[i] << 16);
+    asm("fma.rn.f32x2 %0, %1, %1, %0;" : "+l"(acc) : "l"(x));
+  }
 }
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ float sumsq8(const uint4& v) {
-  float a = bf16lo(v.x), b = bf16hi(v.x), c = bf16lo(v.y), d = bf16hi(v.y);
-  float e = bf16lo(v.z), f = bf16hi(v.z), g = bf16lo(v.w), h = bf16hi(v.w);
-  return a * a + b * b + c * c + d * d + e * e + f * f + g * g + h * h;
+__device__ __forceinline__ uint4 scale8(const uint4& v, unsigned long long k2) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const unsigned long long x =
+        ((unsigned long long)(w[i] & 0xffff0000u) << 32) | (unsigned long long)(w[i] << 16);
+    unsigned long long y;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(x), "l"(k2));
+    const float lo = __uint_as_float((uint32_t)y), hi = __uint_as_float((uint32_t)(y >> 32));
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    o[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <int N, int D>
+// largest d in [0, n) with off[d] <= x, by bisection of a global array
+__device__ __forceinline__ int bisect_global(const int64_t* off, int lo, int hi, int64_t x) {
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(off + mid) <= x) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Per-row epilogue state shared by the reduction helpers.
+struct Emit {
+  const int64_t c;
+  const int dd;
+  const bool valid, head;
+  const unsigned same;
+  const int64_t C;
+  const int n_docs;
+  uint32_t* doc_u;
+  uint32_t* chunk_u;
+  __device__ __forceinline__ void operator()(float m, int b) const {
+    const uint32_t o = valid ? f2o(m) : 0u;
+    if (chunk_u && valid) atomicMax(chunk_u + (int64_t)b * C + c, o);
+    uint32_t x = o;
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, x, 1 << k);
+      if (same & (1u << k)) x = max(x, y);
+    }
+    if (head) atomicMax(doc_u + (int64_t)b * n_docs + dd, x);
+  }
+};
+
+// Folds 32 consecutive columns [cs, cs+32) of this row into the running
+// token maximum m of query b (token t), emitting at each query's last
+// column, at the last column of the pass (last_chunk) and at NT.
+__device__ __forceinline__ void reduce32(const uint32_t (&r)[32], int cs, int NT, int T,
+                                         bool last_chunk, float& m, int& b, int& t,
+                                         const Emit& emit) {
+  if (cs + 31 < NT && t + 32 <= T) {  // one query owns all 32 columns
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      v[i] = fmaxf(__uint_as_float(r[i]), __uint_as_float(r[i + 16]));
+#pragma unroll
+    for (int w = 8; w; w >>= 1)
+#pragma unroll
+      for (int i = 0; i < w; ++i) v[i] = fmaxf(v[i], v[i + w]);
+    m = fmaxf(m, v[0]);
+    t += 32;
+    if (t == T || last_chunk || cs + 32 >= NT) {
+      emit(m, b);
+      m = -INFINITY;
+      if (t == T) { t = 0; ++b; }
+    }
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int col = cs + i;
+    if (col >= NT) break;  // warp-uniform
+    m = fmaxf(m, __uint_as_float(r[i]));
+    if ((last_chunk && i == 31) || col + 1 >= NT || t + 1 == T) {
+      emit(m, b);
+      m = -INFINITY;
+    }
+    if (++t == T) { t = 0; ++b; }
+  }
+}
+
+template <int N, int D, bool kPrep>
 __global__ void __launch_bounds__(kThreads, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 int H, int NT, int T, int n_pass, int64_t C, int64_t n_tiles,
                 const int64_t* __restrict__ coff, int n_docs, uint32_t* __restrict__ doc_u,
                 uint32_t* __restrict__ chunk_u, int* __restrict__ status) {
-  using K = Cfg<N, D>;
+  using K = Cfg<N, D, kPrep>;
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ Aux aux;
   unsigned char* ring = reinterpret_cast<unsigned char*>(
@@ -113,11 +194,15 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // contiguous tile range of this CTA
+  const int64_t tb = (int64_t)blockIdx.x * n_tiles / gridDim.x;
+  const int64_t te = (int64_t)(blockIdx.x + 1) * n_tiles / gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < K::STAGES; ++i) {
       tc::mbar_init(&aux.full[i], 1);
-      tc::mbar_init(&aux.empty[i], 1 + kEpiWarps);
+      tc::mbar_init(&aux.ready[i], kXWarps);
+      tc::mbar_init(&aux.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&aux.accf[i], 1);
@@ -142,27 +227,30 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
       tc::tma_prefetch_desc(&tm_k);
       tc::tma_prefetch_desc(&tm_q);
       uint32_t u = 0;
-      for (int p = 0; p < n_pass && !*abort_flag; ++p)
-        for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x)
-          for (int h = 0; h < H; ++h, ++u) {
-            const int st = u % K::STAGES;
-            const uint32_t ph = (u / K::STAGES) & 1u;
-            if (!tc::mbar_wait(&aux.empty[st], ph ^ 1u)) {
-              record_error(status, MSA_ERR_TIMEOUT);
-              *abort_flag = 1;
-              break;
+      bool stop = false;
+      for (int p = 0; p < n_pass && !stop; ++p)
+        for (int64_t tile = tb; tile < te && !stop; ++tile)
+          for (int h = 0; h < H && !stop; ++h)
+            for (int s = 0; s < K::SPH; ++s, ++u) {
+              const int st = u % K::STAGES;
+              const uint32_t ph = (u / K::STAGES) & 1u;
+              if (*abort_flag || !tc::mbar_wait(&aux.empty[st], ph ^ 1u)) {
+                record_error(status, MSA_ERR_TIMEOUT);
+                *abort_flag = 1;
+                stop = true;
+                break;
+              }
+              unsigned char* a = ring + st * K::STAGE;
+              unsigned char* b = a + K::A_BYTES;
+              tc::mbar_arrive_expect_tx(&aux.full[st], K::STAGE);
+#pragma unroll
+              for (int kb = 0; kb < K::SKB; ++kb) {
+                const int x = (s * K::SKB + kb) * 64;
+                tc::tma_load_3d(a + kb * kTile * 128, &tm_k, &aux.full[st], x, h,
+                                (int32_t)(tile * kTile));
+                tc::tma_load_3d(b + kb * N * 128, &tm_q, &aux.full[st], x, p * N, h);
+              }
             }
-            unsigned char* a = ring + st * K::STAGE;
-            unsigned char* b = a + K::A_BYTES;
-            tc::mbar_arrive_expect_tx(&aux.full[st], K::STAGE);
-#pragma unroll
-            for (int kb = 0; kb < K::KB; ++kb)
-              tc::tma_load_3d(a + kb * kTile * 128, &tm_k, &aux.full[st], kb * 64, h,
-                              (int32_t)(tile * kTile));
-#pragma unroll
-            for (int kb = 0; kb < K::KB; ++kb)
-              tc::tma_load_3d(b + kb * N * 128, &tm_q, &aux.full[st], kb * 64, p * N, h);
-          }
       // Drain: every load issued must have landed before the CTA exits.
       const uint32_t issued = u;
       for (uint32_t v = issued > (uint32_t)K::STAGES ? issued - K::STAGES : 0; v < issued; ++v)
@@ -171,52 +259,103 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
+      uint32_t u = 0, it = 0;
+      bool stop = false;
+      for (int p = 0; p < n_pass && !stop; ++p)
+        for (int64_t tile = tb; tile < te && !stop; ++tile, ++it) {
+          const int ab = it & 1;
+          const uint32_t aph = (it >> 1) & 1u;
+          const uint32_t d_tmem = tmem + ab * N;
+          if (*abort_flag || !tc::mbar_wait(&aux.acce[ab], aph ^ 1u)) {
+            record_error(status, MSA_ERR_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+          for (int h = 0; h < H && !stop; ++h)
+            for (int s = 0; s < K::SPH; ++s, ++u) {
+              const int st = u % K::STAGES;
+              const uint32_t ph = (u / K::STAGES) & 1u;
+              if (*abort_flag ||
+                  !tc::mbar_wait(kPrep ? &aux.full[st] : &aux.ready[st], ph)) {
+                record_error(status, MSA_ERR_TIMEOUT);
+                *abort_flag = 1;
+                stop = true;
+                break;
+              }
+              tc::tc_fence_after();
+              const uint32_t a0 = tc::smem_u32(ring + st * K::STAGE);
+              const uint32_t b0 = a0 + K::A_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < K::SKB * 4; ++kk) {
+                const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside the swizzle atom
+                const uint64_t ad = tc::sdesc_kmajor_sw128(a0 + (kk >> 2) * (kTile * 128) + koff);
+                const uint64_t bd = tc::sdesc_kmajor_sw128(b0 + (kk >> 2) * (N * 128) + koff);
+                tc::mma_bf16_ss(d_tmem, ad, bd, K::IDESC, (h > 0 || s > 0 || kk > 0) ? 1u : 0u);
+              }
+              tc::mma_commit(&aux.empty[st]);
+            }
+          if (!stop) tc::mma_commit(&aux.accf[ab]);
+        }
+    }
+  } else if (warp < 2 + kXWarps) {
+    // ------------------------------------------------ transform (raw bank)
+    if (!kPrep) {
+      const int row = (warp - 2) * 32 + lane;
       uint32_t u = 0;
-      for (int p = 0; p < n_pass && !*abort_flag; ++p)
-        for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x)
+      for (int p = 0; p < n_pass; ++p)
+        for (int64_t tile = tb; tile < te; ++tile)
           for (int h = 0; h < H; ++h, ++u) {
             const int st = u % K::STAGES;
             const uint32_t ph = (u / K::STAGES) & 1u;
-            const int ab = u & 1;
-            const uint32_t aph = (u >> 1) & 1u;
-            if (!tc::mbar_wait(&aux.full[st], ph) || !tc::mbar_wait(&aux.acce[ab], aph ^ 1u)) {
+            // After a timeout every role keeps walking its loop without
+            // waiting, so nobody blocks on a barrier that will not complete.
+            if (!*abort_flag && !tc::mbar_wait(&aux.full[st], ph)) {
               record_error(status, MSA_ERR_TIMEOUT);
               *abort_flag = 1;
-              break;
             }
-            tc::tc_fence_after();
-            const uint32_t a0 = tc::smem_u32(ring + st * K::STAGE);
-            const uint32_t b0 = a0 + K::A_BYTES;
-            const uint32_t d_tmem = tmem + ab * N;
+            unsigned char* arow = ring + st * K::STAGE + row * 128;
+            uint4 v[K::KB][8];
+            unsigned long long ss2 = 0ull;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside the swizzle atom
-              const uint64_t ad = tc::sdesc_kmajor_sw128(a0 + (kk >> 2) * (kTile * 128) + koff);
-              const uint64_t bd = tc::sdesc_kmajor_sw128(b0 + (kk >> 2) * (N * 128) + koff);
-              tc::mma_bf16_ss(d_tmem, ad, bd, K::IDESC, kk > 0 ? 1u : 0u);
-            }
-            tc::mma_commit(&aux.empty[st]);
-            tc::mma_commit(&aux.accf[ab]);
+            for (int kb = 0; kb < K::KB; ++kb)
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                // piece j of the swizzled row sits at 16 * (j ^ row % 8); any
+                // order serves a sum, and this one keeps the warp's 8-row
+                // groups on distinct banks
+                v[kb][j] = *reinterpret_cast<const uint4*>(arow + kb * (kTile * 128) +
+                                                          ((j ^ (row & 7)) << 4));
+                sumsq8(v[kb][j], ss2);
+              }
+            const float ss = __uint_as_float((uint32_t)ss2) + __uint_as_float((uint32_t)(ss2 >> 32));
+            const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+            const unsigned long long inv2 =
+                ((unsigned long long)__float_as_uint(inv) << 32) | __float_as_uint(inv);
+#pragma unroll
+            for (int kb = 0; kb < K::KB; ++kb)
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(arow + kb * (kTile * 128) + ((j ^ (row & 7)) << 4)) =
+                    scale8(v[kb][j], inv2);
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&aux.ready[st]);
           }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;
+    const int ew = warp - 2 - kXWarps;
     const int quad = warp & 3;  // TMEM lane quarter this warp may access
-    const int half = ew >> 2;   // which half of the query columns
     const int row = quad * 32 + lane;
     const int et = ew * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    float acc[K::HALF_N];
-    uint32_t u = 0;
+    uint32_t it = 0;
     for (int p = 0; p < n_pass; ++p) {
-      const int col_begin = p * N + half * K::HALF_N;  // first global column of this half
-      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t c0 = tile * kTile;
-        const int64_t c = c0 + row;
-        // chunk -> document for the tile's rows
+      const int col0 = p * N;
+      // first tile of the pass: look its document window up synchronously
+      if (tb < te) {
         if (ew == 0) {
-          const int64_t d0 = warp_find_segment(coff, n_docs, c0);
+          const int64_t d0 = warp_find_segment(coff, n_docs, tb * kTile);
           if (lane == 0) aux.d0 = (int)d0;
         }
         epi_bar();
@@ -226,136 +365,96 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
           aux.win[i] = di <= n_docs ? __ldg(coff + di) : INT64_MAX;
         }
         epi_bar();
-        if (half == 0) {
-          int dd = -1;
-          if (c < C) {
-            if (c < aux.win[kWindow]) {
-              int lo = 0, hi = kWindow;  // win[lo] <= c < win[hi]
-              while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (aux.win[mid] <= c) lo = mid; else hi = mid;
-              }
-              dd = d0 + lo;
-            } else {  // more than kWindow documents in one tile (empty documents)
-              int lo = d0, hi = n_docs;
-              while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (__ldg(coff + mid) <= c) lo = mid; else hi = mid;
-              }
-              dd = lo;
+      }
+      for (int64_t tile = tb; tile < te; ++tile, ++it) {
+        const int ab = it & 1;
+        const uint32_t aph = (it >> 1) & 1u;
+        const int64_t c0 = tile * kTile;
+        const int64_t c = c0 + row;
+        const int d0 = aux.d0;
+        const int64_t wend = aux.win[kWindow];
+        // this row's document
+        int dd = -1;
+        if (c < C) {
+          if (c < wend) {
+            int lo = 0, hi = kWindow;  // win[lo] <= c < win[hi]
+            while (hi - lo > 1) {
+              const int mid = (lo + hi) >> 1;
+              if (aux.win[mid] <= c) lo = mid; else hi = mid;
             }
+            dd = d0 + lo;
+          } else {  // more than kWindow documents in one tile (empty documents)
+            dd = bisect_global(coff, d0, n_docs, c);
           }
-          aux.doc_row[row] = dd;
         }
+        // next tile's window: base document and prefetch into registers
+        const bool has_next = tile + 1 < te;
+        int d0n = d0;
+        int64_t w0 = INT64_MAX, w1 = INT64_MAX, w2 = INT64_MAX;
+        if (has_next) {
+          const int64_t cn = c0 + kTile;
+          if (cn < wend) {
+            int lo = 0, hi = kWindow;
+            while (hi - lo > 1) {
+              const int mid = (lo + hi) >> 1;
+              if (aux.win[mid] <= cn) lo = mid; else hi = mid;
+            }
+            d0n = d0 + lo;
+          } else {
+            d0n = bisect_global(coff, d0, n_docs, cn);
+          }
+          if ((int64_t)d0n + et <= n_docs) w0 = __ldg(coff + d0n + et);
+          if ((int64_t)d0n + et + 128 <= n_docs) w1 = __ldg(coff + d0n + et + 128);
+          if (et == 0 && (int64_t)d0n + kWindow <= n_docs) w2 = __ldg(coff + d0n + kWindow);
+        }
+        const bool valid = dd >= 0;
+        unsigned same = 0;  // segment structure of the warp's rows
 #pragma unroll
-        for (int j = 0; j < K::HALF_N; ++j) acc[j] = 0.f;
+        for (int k = 0; k < 5; ++k) {
+          const int off = 1 << k;
+          const int od = __shfl_down_sync(0xffffffffu, dd, off);
+          if (lane + off < 32 && od == dd) same |= 1u << k;
+        }
+        const int up = __shfl_up_sync(0xffffffffu, dd, 1);
+        const Emit emit{c, dd, valid, valid && (lane == 0 || up != dd), same, C, n_docs,
+                        doc_u, chunk_u};
 
-        for (int h = 0; h < H; ++h, ++u) {
-          const int st = u % K::STAGES;
-          const uint32_t ph = (u / K::STAGES) & 1u;
-          const int ab = u & 1;
-          const uint32_t aph = (u >> 1) & 1u;
-          // After a timeout the epilogue keeps walking its loop (skipping the
-          // waits) so that every epilogue warp reaches every named barrier.
-          if (!*abort_flag && !tc::mbar_wait(&aux.full[st], ph)) {
-            record_error(status, MSA_ERR_TIMEOUT);
-            *abort_flag = 1;
-          }
-          // |K̄_r[c, h]|^2 from this head's shared tile (swizzle only permutes
-          // 16-byte pieces inside a row, which a sum of squares ignores)
-          const unsigned char* arow = ring + st * K::STAGE + row * 128;
-          float ss = 0.f;
-          if (D == 128) {
-            const unsigned char* base = arow + half * (kTile * 128);
+        if (!*abort_flag && !tc::mbar_wait(&aux.accf[ab], aph)) {
+          record_error(status, MSA_ERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+        tc::tc_fence_after();
+        const uint32_t tbase = tmem + lane_addr + ab * N;
+        int b = col0 / T;
+        int t = col0 - b * T;
+        float m = -INFINITY;
+        uint32_t r0[32], r1[32];
+        tc::tmem_ld32(tbase, r0);
+        tc::tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              ss += sumsq8(*reinterpret_cast<const uint4*>(base + j * 16));
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              ss += sumsq8(*reinterpret_cast<const uint4*>(arow + (half * 4 + j) * 16));
-          }
-          aux.npart[u & 1][half][row] = ss;
-          epi_bar();
-          const float tot = aux.npart[u & 1][0][row] + aux.npart[u & 1][1][row];
-          const float inv = 1.0f / fmaxf(sqrtf(tot), 1e-12f);
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&aux.empty[st]);
-          if (!*abort_flag && !tc::mbar_wait(&aux.accf[ab], aph)) {
-            record_error(status, MSA_ERR_TIMEOUT);
-            *abort_flag = 1;
-          }
-          tc::tc_fence_after();
-          const uint32_t tbase = tmem + lane_addr + ab * N + half * K::HALF_N;
-#pragma unroll
-          for (int j = 0; j < K::HALF_N / 32; ++j) {
-            uint32_t r[32];
-            tc::tmem_ld32(tbase + j * 32, r);
+        for (int j = 0; j < N / 32; j += 2) {
+          if (j + 1 < N / 32) tc::tmem_ld32(tbase + (j + 1) * 32, r1);
+          reduce32(r0, col0 + j * 32, NT, T, j + 1 == N / 32, m, b, t, emit);
+          tc::tmem_ld_wait();
+          if (j + 1 < N / 32) {
+            if (j + 2 < N / 32) tc::tmem_ld32(tbase + (j + 2) * 32, r0);
+            reduce32(r1, col0 + (j + 1) * 32, NT, T, j + 2 == N / 32, m, b, t, emit);
             tc::tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[j * 32 + i] = fmaf(inv, __uint_as_float(r[i]), acc[j * 32 + i]);
-          }
-          if (h + 1 < H) {
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&aux.acce[ab]);
-          } else {
-            // last head: park the head-mean cosines in the TMEM buffer just
-            // read, then reduce them over tokens and documents
-#pragma unroll
-            for (int j = 0; j < K::HALF_N / 32; ++j) {
-              float v[32];
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = acc[j * 32 + i];
-              tmem_st32(tbase + j * 32, v);
-            }
-            tmem_st_wait();
-            const int dd = aux.doc_row[row];
-            const bool valid = dd >= 0;
-            // segment structure of the warp's rows (rows ascend with lanes)
-            unsigned same = 0;
-#pragma unroll
-            for (int k = 0; k < 5; ++k) {
-              const int off = 1 << k;
-              const int od = __shfl_down_sync(0xffffffffu, dd, off);
-              if (lane + off < 32 && od == dd) same |= 1u << k;
-            }
-            const int up = __shfl_up_sync(0xffffffffu, dd, 1);
-            const bool head = valid && (lane == 0 || up != dd);
-            int b = col_begin / T;
-            int t = col_begin - b * T;
-            float m = -INFINITY;
-            for (int j = 0; j < K::HALF_N / 32; ++j) {
-              uint32_t r[32];
-              tc::tmem_ld32(tbase + j * 32, r);
-              tc::tmem_ld_wait();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int col = col_begin + j * 32 + i;
-                if (col >= NT) break;  // warp-uniform
-                m = fmaxf(m, __uint_as_float(r[i]));
-                const bool last_col = (j * 32 + i == K::HALF_N - 1) || (col + 1 >= NT) || (t + 1 == T);
-                if (last_col) {
-                  const uint32_t o = valid ? f2o(m) : 0u;
-                  if (chunk_u && valid) atomicMax(chunk_u + (int64_t)b * C + c, o);
-                  uint32_t x = o;
-#pragma unroll
-                  for (int k = 0; k < 5; ++k) {
-                    const uint32_t y = __shfl_down_sync(0xffffffffu, x, 1 << k);
-                    if (same & (1u << k)) x = max(x, y);
-                  }
-                  if (head) atomicMax(doc_u + (int64_t)b * n_docs + dd, x);
-                  m = -INFINITY;
-                }
-                if (++t == T) { t = 0; ++b; }
-              }
-            }
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&aux.acce[ab]);
           }
         }
-        epi_bar();  // doc_row / win are rewritten by the next tile
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&aux.acce[ab]);
+        epi_bar();  // everyone is done with this tile's window
+        if (has_next) {
+          aux.win[et] = w0;
+          aux.win[et + 128] = w1;
+          if (et == 0) {
+            aux.win[kWindow] = w2;
+            aux.d0 = d0n;
+          }
+        }
+        epi_bar();
       }
     }
   }
@@ -366,6 +465,32 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, K::TMEM_COLS);
   }
+}
+
+// Prepared routing bank: each (chunk, head) row divided by max(|row|, 1e-12)
+// and rounded to bf16.  Two rows per warp, 16 lanes x 16 bytes per row.
+template <int D>
+__global__ void __launch_bounds__(256)
+prepare_bank_kernel(int64_t n_rows, const __nv_bfloat16* __restrict__ src,
+                    __nv_bfloat16* __restrict__ dst) {
+  constexpr int LPR = D / 8;  // lanes per row
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = gt / LPR;
+  const int sub = (int)(gt % LPR);
+  const bool live = row < n_rows;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (live) v = ld_stream16(src + row * D + sub * 8);
+  float f[8];
+  Vec16<__nv_bfloat16>::unpack(v, f);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
+#pragma unroll
+  for (int o = LPR / 2; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] *= inv;
+  if (live) st16(dst + row * D + sub * 8, Vec16<__nv_bfloat16>::pack(f));
 }
 
 // ----------------------------------------------------------------- host
@@ -400,17 +525,17 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N, int D>
+template <int N, int D, bool kPrep>
 int launch(int B, int T, int H, const __nv_bfloat16* qhat, int n_pad, const __nv_bfloat16* kr,
            int64_t C, const int64_t* coff, int n_docs, uint32_t* doc_u, uint32_t* chunk_u,
            int* status, cudaStream_t s) {
-  using K = Cfg<N, D>;
+  using K = Cfg<N, D, kPrep>;
   CUtensorMap tm_k, tm_q;
   if (!make_map(&tm_k, kr, D, H, C, (uint64_t)D * 2, (uint64_t)H * D * 2, 1, kTile))
     return note_cuda(cudaErrorInvalidValue);
   if (!make_map(&tm_q, qhat, D, n_pad, H, (uint64_t)D * 2, (uint64_t)n_pad * D * 2, N, 1))
     return note_cuda(cudaErrorInvalidValue);
-  auto kern = route_tc_kernel<N, D>;
+  auto kern = route_tc_kernel<N, D, kPrep>;
   int rc = note_cuda(
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM));
   if (rc) return rc;
@@ -433,20 +558,40 @@ int64_t route_tc_columns(int64_t nt) {
 
 int route_tc_launch(int B, int T, int H, int D, const __nv_bfloat16* qhat, int n_pad,
                     const __nv_bfloat16* kr, int64_t C, const int64_t* coff, int n_docs,
-                    uint32_t* doc_u, uint32_t* chunk_u, int* status, cudaStream_t s) {
+                    uint32_t* doc_u, uint32_t* chunk_u, int* status, bool prepared,
+                    cudaStream_t s) {
   const int N = n_pad <= 128 ? n_pad : 256;
   if (!aligned16(qhat) || !aligned16(kr)) return MSA_ERR_INVALID_ARG;
-#define MSA_ROUTE_CASE(NN)                                                                      \
-  if (N == NN)                                                                                  \
-    return D == 64 ? launch<NN, 64>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u, chunk_u,  \
-                                    status, s)                                                  \
-                   : launch<NN, 128>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u, chunk_u, \
-                                     status, s);
-  MSA_ROUTE_CASE(64)
-  MSA_ROUTE_CASE(128)
-  MSA_ROUTE_CASE(256)
+#define MSA_ROUTE_CASE(NN, DD, PP)                                                        \
+  if (N == NN && D == DD && prepared == PP)                                                \
+    return launch<NN, DD, PP>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u, chunk_u, \
+                              status, s);
+  MSA_ROUTE_CASE(64, 64, false)
+  MSA_ROUTE_CASE(64, 128, false)
+  MSA_ROUTE_CASE(128, 64, false)
+  MSA_ROUTE_CASE(128, 128, false)
+  MSA_ROUTE_CASE(256, 64, false)
+  MSA_ROUTE_CASE(256, 128, false)
+  MSA_ROUTE_CASE(64, 64, true)
+  MSA_ROUTE_CASE(64, 128, true)
+  MSA_ROUTE_CASE(128, 64, true)
+  MSA_ROUTE_CASE(128, 128, true)
+  MSA_ROUTE_CASE(256, 64, true)
+  MSA_ROUTE_CASE(256, 128, true)
 #undef MSA_ROUTE_CASE
   return MSA_ERR_UNSUPPORTED;
+}
+
+int route_prepare_bank_launch(int64_t n_rows, int D, const __nv_bfloat16* src,
+                              __nv_bfloat16* dst, cudaStream_t s) {
+  const int64_t threads = n_rows * (D / 8);
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
+  if (D == 64)
+    prepare_bank_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(n_rows, src, dst);
+  else
+    prepare_bank_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(n_rows, src, dst);
+  return check_launch();
 }
 
 }  // namespace msa

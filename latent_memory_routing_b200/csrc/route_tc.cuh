@@ -15,9 +15,15 @@ int64_t route_tc_columns(int64_t n_queries_tokens);
 // Scans the whole bank once per pass.  qhat: [H][n_pad][D] bf16, each row
 // Q_r / max(|Q_r|, eps) / H (rows >= B*T zero).  kr: [C][H][D] bf16.
 // doc_u / chunk_u: order-preserving uint32 maxima, pre-set to -inf.
+// `prepared`: kr rows are already unit-normalised (msa_route_prepare_bank);
+// otherwise the kernel normalises them in shared memory.
 int route_tc_launch(int B, int T, int H, int D, const __nv_bfloat16* qhat, int n_pad,
                     const __nv_bfloat16* kr, int64_t C, const int64_t* chunk_off,
                     int n_docs, uint32_t* doc_u, uint32_t* chunk_u, int* status,
-                    cudaStream_t s);
+                    bool prepared, cudaStream_t s);
+
+// dst[r] = src[r] / max(|src[r]|, 1e-12) for n_rows rows of D bf16.
+int route_prepare_bank_launch(int64_t n_rows, int D, const __nv_bfloat16* src,
+                              __nv_bfloat16* dst, cudaStream_t s);
 
 }  // namespace msa

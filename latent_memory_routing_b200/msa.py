@@ -53,6 +53,9 @@ _SIGS = {
     "msa_route_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i]),
     "msa_route_scores": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i64, c_p, c_i, c_p, c_p,
                                c_p, c_sz, c_p]),
+    "msa_route_prepare_bank": (c_i, [c_i, c_i64, c_i, c_i, c_p, c_p, c_p]),
+    "msa_route_scores_prepared": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i64, c_p, c_i, c_p,
+                                        c_p, c_p, c_sz, c_p]),
     "msa_topk_workspace_size": (c_sz, [c_i, c_i, c_i]),
     "msa_topk_docs": (c_i, [c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_sz, c_p]),
     "msa_gather_kv": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i, c_p, c_p, c_i, c_p, c_p,
@@ -181,6 +184,24 @@ def msa_route_scores(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_doc
     _numel_ok(chunk_scores, B * n_chunks, "chunk_scores")
     _check("msa_route_scores", lib().msa_route_scores(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
+        _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def msa_route_prepare_bank(dt, n_chunks, H, D, kr_bar, kr_hat, stream=None):
+    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
+    _numel_ok(kr_hat, n_chunks * H * D, "kr_hat")
+    _check("msa_route_prepare_bank", lib().msa_route_prepare_bank(
+        dt, n_chunks, H, D, _ptr(kr_bar), _ptr(kr_hat), _stream(stream)))
+
+
+def msa_route_scores_prepared(dt, B, T, H, D, q_r, kr_hat, n_chunks, chunk_offsets, n_docs,
+                              doc_scores, chunk_scores, ws, ws_bytes, stream=None):
+    _numel_ok(q_r, B * T * H * D, "q_r")
+    _numel_ok(kr_hat, n_chunks * H * D, "kr_hat")
+    _numel_ok(doc_scores, B * n_docs, "doc_scores")
+    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores")
+    _check("msa_route_scores_prepared", lib().msa_route_scores_prepared(
+        dt, B, T, H, D, _ptr(q_r), _ptr(kr_hat), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws_bytes, _stream(stream)))
 
 

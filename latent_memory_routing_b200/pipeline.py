@@ -37,12 +37,25 @@ def encode_pool(k_tok, v_tok, kr_tok, tok_offsets, chunk_offs, n_chunks: int,
     return kb, vb, rb
 
 
-class Router:
-    """Holds the workspace of msa_route_scores for fixed (dtype, B, T, H, D)."""
+def prepare_bank(kr_bar, out=None, stream=None):
+    """Unit-normalised copy of a bf16 routing bank [C][H][D] (built once per
+    bank; see msa_route_prepare_bank)."""
+    C, H, D = kr_bar.shape
+    if out is None:
+        out = torch.empty_like(kr_bar)
+    _m.msa_route_prepare_bank(dt_code(kr_bar), C, H, D, kr_bar, out, stream)
+    return out
 
-    def __init__(self, dtype: torch.dtype, B: int, T: int, H: int, D: int, device):
+
+class Router:
+    """Holds the workspace of msa_route_scores for fixed (dtype, B, T, H, D).
+    ``prepared=True`` routes over a bank made by ``prepare_bank``."""
+
+    def __init__(self, dtype: torch.dtype, B: int, T: int, H: int, D: int, device,
+                 prepared: bool = False):
         self.dt = _m.dtype_code(dtype)
         self.B, self.T, self.H, self.D = B, T, H, D
+        self.fn = _m.msa_route_scores_prepared if prepared else _m.msa_route_scores
         n = _m.msa_route_workspace_size(self.dt, B, T, H, D)
         self.ws = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
 
@@ -51,8 +64,8 @@ class Router:
         C = kr_bar.shape[0]
         if doc_scores is None:
             doc_scores = torch.empty((self.B, n_docs), dtype=torch.float32, device=q_r.device)
-        _m.msa_route_scores(self.dt, self.B, self.T, self.H, self.D, q_r, kr_bar, C, chunk_offs,
-                            n_docs, doc_scores, chunk_scores, self.ws, self.ws.numel(), stream)
+        self.fn(self.dt, self.B, self.T, self.H, self.D, q_r, kr_bar, C, chunk_offs, n_docs,
+                doc_scores, chunk_scores, self.ws, self.ws.numel(), stream)
         return doc_scores
 
 
@@ -102,10 +115,11 @@ class Attention:
 
 class Pipeline:
     """route -> top-k -> gather -> attend over a resident pooled bank (one
-    layer), with every buffer allocated once."""
+    layer), with every buffer allocated once.  With ``prepared=True``,
+    ``kr_bar`` is a bank made by ``prepare_bank``."""
 
     def __init__(self, kr_bar, k_bar, v_bar, chunk_offs, *, B, T, T_loc, Hq, k, m_cap,
-                 pos0=None, rope_base=10000.0):
+                 pos0=None, rope_base=10000.0, prepared=False):
         C, H, D = kr_bar.shape
         dev = kr_bar.device
         self.kr_bar, self.k_bar, self.v_bar, self.coff = kr_bar, k_bar, v_bar, chunk_offs
@@ -114,7 +128,7 @@ class Pipeline:
         self.k, self.m_cap = k, m_cap
         self.pos0 = k if pos0 is None else pos0
         self.rope_base = rope_base
-        self.router = Router(kr_bar.dtype, B, T, H, D, dev)
+        self.router = Router(kr_bar.dtype, B, T, H, D, dev, prepared=prepared)
         self.attn = Attention(kr_bar.dtype, B, T, T_loc, Hq, H, D, m_cap, dev)
         self.doc_scores = torch.empty((B, self.n_docs), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, k), dtype=torch.int32, device=dev)

@@ -157,15 +157,19 @@ def _pooled_bank(n_docs, lo, hi, H, D, dtype, seed, needle_q=None):
     return kr, torch.from_numpy(coff_h).cuda(), coff_h
 
 
-def _route(q_r, kr, coff, n_docs, with_chunks=True):
+def _route(q_r, kr, coff, n_docs, with_chunks=True, prepared=False):
+    """Routes q_r over the raw bank kr, or over its prepared (unit-row) copy
+    made by msa_route_prepare_bank."""
     B, T, H, D = q_r.shape
-    router = pipeline.Router(q_r.dtype, B, T, H, D, "cuda")
+    router = pipeline.Router(q_r.dtype, B, T, H, D, "cuda", prepared=prepared)
+    bank = pipeline.prepare_bank(kr) if prepared else kr
     cs = torch.empty((B, kr.shape[0]), dtype=torch.float32, device="cuda") if with_chunks else None
-    ds = router(q_r, kr, coff, n_docs, chunk_scores=cs)
+    ds = router(q_r, bank, coff, n_docs, chunk_scores=cs)
     torch.cuda.synchronize()
     return ds, cs
 
 
+@pytest.mark.parametrize("prepared", [False, True])
 @pytest.mark.parametrize("B,T,H,D,n_docs", [
     (1, 256, 8, 128, 150),    # one pass, N = 256 (the 100M prefill shape)
     (1, 128, 8, 128, 90),     # N = 128
@@ -176,12 +180,12 @@ def _route(q_r, kr, coff, n_docs, with_chunks=True):
     (1, 64, 2, 64, 70),       # D = 64, H = 2
     (5, 3, 1, 128, 33),       # H = 1
 ])
-def test_route_bf16_vs_oracle(B, T, H, D, n_docs):
+def test_route_bf16_vs_oracle(B, T, H, D, n_docs, prepared):
     g = torch.Generator(device="cuda").manual_seed(100 + B * T)
     q_r = synth.randn((B, T, H, D), torch.bfloat16, "cuda", g)
     kr, coff, coff_h = _pooled_bank(n_docs, 1, 900, H, D, torch.bfloat16, 11 + T,
                                     needle_q=q_r[0])
-    ds, cs = _route(q_r, kr, coff, n_docs)
+    ds, cs = _route(q_r, kr, coff, n_docs, prepared=prepared)
     ods, ocs = oracle.route_scores(f64(q_r), f64(kr), coff_h)
     assert np.max(np.abs(f64(cs) - ocs)) <= ROUTE_ATOL
     assert np.max(np.abs(f64(ds) - ods)) <= ROUTE_ATOL
@@ -198,6 +202,24 @@ def test_route_fp32_tiny():
     assert np.max(np.abs(f64(cs) - ocs)) <= 1e-5
     assert np.max(np.abs(f64(ds) - ods)) <= 1e-5
     assert int(torch.argmax(ds[0])) == 5
+    status_ok()
+
+
+def test_prepared_bank_rows_are_unit_and_scores_agree():
+    H, D = 8, 128
+    g = torch.Generator(device="cuda").manual_seed(77)
+    kr = synth.randn((3000, H, D), torch.bfloat16, "cuda", g) * 3.0
+    kr[5] = 0.0
+    hat = pipeline.prepare_bank(kr)
+    n = hat.float().norm(dim=-1).cpu().numpy()
+    assert np.all(np.abs(n[np.arange(3000) != 5] - 1.0) <= 4e-3)
+    assert np.all(n[5] == 0.0)
+    q = synth.randn((2, 40, H, D), torch.bfloat16, "cuda", g)
+    coff_h = np.arange(0, 3001, 30)
+    coff = torch.from_numpy(coff_h).cuda()
+    a, _ = _route(q, kr, coff, 100)
+    b, _ = _route(q, kr, coff, 100, prepared=True)
+    assert np.max(np.abs(f64(a) - f64(b))) <= 1e-4
     status_ok()
 
 
@@ -230,12 +252,14 @@ def _check_topk_on_routed(idx, oracle_scores, k):
                 assert idx[b, r] == order[r], (b, r)
 
 
-def test_route_topk_10m_decode_full():
+@pytest.mark.parametrize("prepared", [False, True])
+def test_route_topk_10m_decode_full(prepared):
     lengths = synth.bank_10m_lengths()
     coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
     w = synth.bank_10m(coff_h, "cuda")
     coff = torch.from_numpy(coff_h).cuda()
-    ds, _ = _route(w["q_r"], w["kr_bar"], coff, len(lengths), with_chunks=False)
+    ds, _ = _route(w["q_r"], w["kr_bar"], coff, len(lengths), with_chunks=False,
+                   prepared=prepared)
     ods, _ = oracle.route_scores(f64(w["q_r"]), f64(w["kr_bar"]), coff_h)
     assert np.max(np.abs(f64(ds) - ods)) <= ROUTE_ATOL
     idx, _ = pipeline.topk_docs(ds, 16)
@@ -243,13 +267,14 @@ def test_route_topk_10m_decode_full():
     status_ok()
 
 
-def test_route_100m_prefill_sampled():
+@pytest.mark.parametrize("prepared", [False, True])
+def test_route_100m_prefill_sampled(prepared):
     lengths = synth.bank_100m_lengths()
     coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
     w = synth.bank_100m(coff_h, "cuda")
     coff = torch.from_numpy(coff_h).cuda()
     n_docs = len(lengths)
-    ds, cs = _route(w["q_r"], w["kr_bar"], coff, n_docs)
+    ds, cs = _route(w["q_r"], w["kr_bar"], coff, n_docs, prepared=prepared)
     idx, _ = pipeline.topk_docs(ds, 16)
     torch.cuda.synchronize()
     rng = np.random.default_rng(3)
