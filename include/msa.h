@@ -160,6 +160,32 @@ int msa_route_scores_prepared(msa_dtype dt, int B, int T, int H, int D,
                               float* chunk_scores, void* ws, size_t ws_bytes,
                               msa_stream_t stream);
 
+/* Routing without any device allocation.  The paper has no counterpart: this
+ * is a deployment variant of msa_route_scores for callers that cannot call
+ * cudaMalloc -- an engine whose device memory is all owned by its own pool
+ * allocator, or a latency-critical loop where an allocation (which may
+ * synchronise the device) is not acceptable.  It computes exactly what
+ * msa_route_scores computes, with the same arguments minus the workspace:
+ * the scratch is a fixed array of msa_route_noalloc_scratch_bytes() bytes
+ * (512 KiB) compiled into the library, one per device, held by every GPU
+ * that loads the library until the process exits.  The caller still owns
+ * and passes every input and output.
+ *   - A shape whose workspace (msa_route_workspace_size) exceeds the array
+ *     -- e.g. more than 256 query columns at 8 x 128 in bf16 -- returns
+ *     MSA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture begins.
+ *   - All calls on a device share the array: calls that overlap on the GPU
+ *     race on it and must be ordered (one stream, or events).  Each call
+ *     rewrites every byte it reads, so nothing carries over between calls. */
+size_t msa_route_noalloc_scratch_bytes(void);
+int msa_route_scores_noalloc(msa_dtype dt, int B, int T, int H, int D,
+                             const void* q_r, const void* kr_bar,
+                             int64_t n_chunks, const int64_t* chunk_offsets,
+                             int n_docs, float* doc_scores, float* chunk_scores,
+                             msa_stream_t stream);
+
 /* Top-k documents -- [HYSEN] §"Routing happens inside attention ...": the
  * router selects the top-k documents.  Ties go to the lower document index.
  *   scores      [B][n_docs] float (device).

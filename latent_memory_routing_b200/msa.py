@@ -56,6 +56,9 @@ _SIGS = {
     "msa_route_prepare_bank": (c_i, [c_i, c_i64, c_i, c_i, c_p, c_p, c_p]),
     "msa_route_scores_prepared": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i64, c_p, c_i, c_p,
                                         c_p, c_p, c_sz, c_p]),
+    "msa_route_noalloc_scratch_bytes": (c_sz, []),
+    "msa_route_scores_noalloc": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i64, c_p, c_i, c_p,
+                                       c_p, c_p]),
     "msa_topk_workspace_size": (c_sz, [c_i, c_i, c_i]),
     "msa_topk_docs": (c_i, [c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_sz, c_p]),
     "msa_gather_kv": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i, c_p, c_p, c_i, c_p, c_p,
@@ -203,6 +206,23 @@ def msa_route_scores_prepared(dt, B, T, H, D, q_r, kr_hat, n_chunks, chunk_offse
     _check("msa_route_scores_prepared", lib().msa_route_scores_prepared(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_hat), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def msa_route_noalloc_scratch_bytes() -> int:
+    return lib().msa_route_noalloc_scratch_bytes()
+
+
+def msa_route_scores_noalloc(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_docs,
+                             doc_scores, chunk_scores, stream=None):
+    """msa_route_scores with the library's fixed scratch array instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    _numel_ok(q_r, B * T * H * D, "q_r")
+    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
+    _numel_ok(doc_scores, B * n_docs, "doc_scores")
+    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores")
+    _check("msa_route_scores_noalloc", lib().msa_route_scores_noalloc(
+        dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
+        _ptr(doc_scores), _ptr(chunk_scores), _stream(stream)))
 
 
 def msa_topk_workspace_size(B, n_docs, k) -> int:
