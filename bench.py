@@ -164,7 +164,7 @@ def timed_step(p, w, ev):
     ev[0].record()
     p.router(w["q_r"], p.kr_bar, p.coff, p.n_docs, p.doc_scores, None)
     ev[1].record()
-    pipeline.topk_docs(p.doc_scores, p.k, p.idx, p.top)
+    pipeline.topk_docs(p.doc_scores, p.k, p.idx, p.top, p.topk_ws)
     ev[2].record()
     pipeline.gather_kv(p.idx, p.coff, p.k_bar, p.v_bar, p.m_cap, p.k_mem, p.v_mem, p.mem_len)
     ev[3].record()
@@ -189,7 +189,7 @@ def run_libmsa(args, world, rank, local):
     import torch
 
     from latent_memory_routing_b200 import build as _b
-    from latent_memory_routing_b200 import msa
+    from latent_memory_routing_b200 import msa, pipeline
     _b.build()
     msa.lib()
     w, p, C = build_workload(rank)

@@ -1,15 +1,504 @@
-// bf16 prefill attention on the tcgen05 tensor cores.
+// bf16 prefill attention over [gathered memory ; local causal context] on the
+// sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Method: "EverMind-AI/MSA: routing top-k compressed documents inside
+// attention ..." (hysenlabs.com), §"Routing happens inside attention ..."
+// (the selected documents' compressed K/V are concatenated ahead of the
+// query's local K/V) and §"Document-wise RoPE resets every document to
+// position zero" (global RoPE whose query start is offset by k).  Memory rows
+// keep their document-wise rotation; local keys are causal.
+//
+// Design.
+//   * rope_rows_kernel rotates Q (to pos0 + T_loc - T + i) and the local K
+//     (to pos0 + j) once per call into bf16 workspace copies, from a per-call
+//     cos/sin table (angles reduced in double).
+//   * attn_tc_kernel: one CTA per (128 query rows, KV head, batch).  GQA rows
+//     are packed as (token, head of the group): a TMA box of
+//     {64 d, G heads, 128/G tokens} lands as 128 rows of 128 B -- the Q tile
+//     of all G query heads sharing one KV head.  Key tiles of 128 rows come
+//     first from the memory (mem_len rows) then from the local context
+//     (up to the block's last visible key), each as K and V TMA boxes.
+//     - warp 0 (one lane): TMA producer, 2-stage K/V ring;
+//     - warp 1 (one lane): tcgen05.mma S = Q K^T (M=128, N=128 keys, K=D)
+//       into one of two TMEM buffers, and O_tile = P V (M=128, N=D, K=128
+//       keys, V read MN-major straight from its TMA tile) into a third; the
+//       S of tile j+1 is issued before the P V of tile j;
+//     - warps 2..5 (one thread per row): online softmax in fp32 -- masked
+//       row maximum, p = 2^(s - m) written as bf16 into a double-buffered
+//       shared P tile (128B-swizzled, the MMA's A operand), row sum -- and
+//       the running output O = O * 2^(m_old - m_new) + O_tile in registers,
+//       consuming tile j's O_tile after computing tile j+1's P.
+//   * Every mbarrier wait is bounded; a timeout records MSA_ERR_TIMEOUT and
+//     all roles finish their loops without waiting.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
 #include "attn_tc.cuh"
 #include "msa_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace msa {
+namespace {
 
-bool attn_tc_supported(int, int, int, int, int, int, int) { return false; }
-size_t attn_tc_workspace_size(int, int, int, int, int, int, int) { return 0; }
-int attn_tc_launch(int, int, int, int, int, int, const void*, const void*, const void*,
-                   const int32_t*, int, const void*, const void*, int, float, float, void*, void*,
-                   cudaStream_t) {
-  return MSA_ERR_UNSUPPORTED;
+constexpr int kRows = 128;   // query rows per CTA (MMA M)
+constexpr int kKeys = 128;   // keys per tile (MMA N of S, K of P V)
+constexpr int kSoftWarps = 4;
+constexpr int kThreads = 64 + 32 * kSoftWarps;
+constexpr int kStages = 2;
+
+template <int D>
+struct ACfg {
+  static constexpr int KB = D / 64;
+  static constexpr int Q_BYTES = KB * kRows * 128;
+  static constexpr int K_BYTES = KB * kKeys * 128;
+  static constexpr int V_BYTES = KB * kKeys * 128;
+  static constexpr int STAGE = K_BYTES + V_BYTES;
+  static constexpr int P_BYTES = 2 * kRows * 128;  // 128 keys x bf16 = 2 K blocks
+  static constexpr size_t SMEM = 1024 + Q_BYTES + kStages * STAGE + 2 * P_BYTES;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // S: M=128, N=128 keys, A (Q) and B (K) K-major
+  static constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(kRows, kKeys);
+  // O: M=128, N=D, A (P) K-major, B (V) MN-major (bit 16)
+  static constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(kRows, D) | (1u << 16);
+};
+
+struct AAux {
+  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
+      o_full, o_empty;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// UMMA descriptor of an MN-major, 128B-swizzled operand whose MN extent is
+// split in 64-element (128 B) column blocks `lbo` bytes apart and whose K
+// rows are 128 B apart (8-row swizzle atoms 1024 B apart): the layout of a
+// TMA box {64 MN, rows K} stored block after block.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo) {
+  return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_km,
+               const __grid_constant__ CUtensorMap tm_vm, const __grid_constant__ CUtensorMap tm_kl,
+               const __grid_constant__ CUtensorMap tm_vl, int T, int T_loc, int Hq, int H, int G,
+               const int32_t* __restrict__ mem_len, int m_cap, float qscale,
+               __nv_bfloat16* __restrict__ out, int* __restrict__ status) {
+  using K = ACfg<D>;
+  extern __shared__ __align__(1024) unsigned char smem_dyn[];
+  __shared__ AAux aux;
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = base;
+  unsigned char* sKV = sQ + K::Q_BYTES;
+  unsigned char* sP = sKV + kStages * K::STAGE;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int TQ = kRows / G;  // tokens per CTA
+  const int tok0 = mt * TQ;
+  const int n_tok = min(TQ, T - tok0);
+  const int M = min(max(mem_len[b], 0), m_cap);
+  const int lim_max = T_loc - T + tok0 + n_tok - 1;  // last local key any row sees
+  const int n_mt = (M + kKeys - 1) / kKeys;
+  const int n_lt = (lim_max + 1 + kKeys - 1) / kKeys;
+  const int nt = n_mt + n_lt;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&aux.q_full, 1);
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&aux.kv_full[i], 1);
+      tc::mbar_init(&aux.kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&aux.s_full[i], 1);
+      tc::mbar_init(&aux.s_empty[i], kSoftWarps);
+      tc::mbar_init(&aux.p_full[i], kSoftWarps);
+    }
+    tc::mbar_init(&aux.o_full, 1);
+    tc::mbar_init(&aux.o_empty, kSoftWarps);
+    aux.abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&aux.tmem_base, K::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = aux.tmem_base;
+  const uint32_t tS[2] = {tmem, tmem + kKeys};
+  const uint32_t tO = tmem + 2 * kKeys;
+  volatile int* abort_flag = &aux.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0;
+      tc::mbar_arrive_expect_tx(&aux.q_full, K::Q_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < K::KB; ++kb)
+        tc::tma_load_3d(sQ + kb * kRows * 128, &tm_q, &aux.q_full, kb * 64, g * G,
+                        b * T + tok0);
+      for (int j = 0; j < nt; ++j) {
+        const int st = j % kStages;
+        if (*abort_flag || !tc::mbar_wait(&aux.kv_empty[st], ((j / kStages) & 1) ^ 1)) {
+          record_error(status, MSA_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        unsigned char* k_dst = sKV + st * K::STAGE;
+        unsigned char* v_dst = k_dst + K::K_BYTES;
+        tc::mbar_arrive_expect_tx(&aux.kv_full[st], K::STAGE);
+        const bool mem = j < n_mt;
+        const CUtensorMap* mk = mem ? &tm_km : &tm_kl;
+        const CUtensorMap* mv = mem ? &tm_vm : &tm_vl;
+        const int row = mem ? b * m_cap + j * kKeys : b * T_loc + (j - n_mt) * kKeys;
+#pragma unroll
+        for (int kb = 0; kb < K::KB; ++kb) {
+          tc::tma_load_3d(k_dst + kb * kKeys * 128, mk, &aux.kv_full[st], kb * 64, g, row);
+          tc::tma_load_3d(v_dst + kb * kKeys * 128, mv, &aux.kv_full[st], kb * 64, g, row);
+        }
+        ++issued;
+      }
+      // every load issued must land before the CTA exits
+      tc::mbar_wait(&aux.q_full, 0);
+      for (uint32_t v = issued > (uint32_t)kStages ? issued - kStages : 0; v < issued; ++v)
+        tc::mbar_wait(&aux.kv_full[v % kStages], (v / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t q0 = tc::smem_u32(sQ);
+      auto fail = [&]() {
+        record_error(status, MSA_ERR_TIMEOUT);
+        *abort_flag = 1;
+      };
+      auto issue_s = [&](int j) -> bool {
+        const int st = j % kStages, sb = j & 1;
+        if (*abort_flag || !tc::mbar_wait(&aux.kv_full[st], (j / kStages) & 1) ||
+            !tc::mbar_wait(&aux.s_empty[sb], ((j >> 1) & 1) ^ 1))
+          return false;
+        tc::tc_fence_after();
+        const uint32_t k0 = tc::smem_u32(sKV + st * K::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+          const uint32_t koff = (kk >> 2) * (kKeys * 128) + (kk & 3) * 32;
+          tc::mma_bf16_ss(tS[sb], tc::sdesc_kmajor_sw128(q0 + off),
+                          tc::sdesc_kmajor_sw128(k0 + koff), K::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&aux.s_full[sb]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int st = j % kStages, pb = j & 1;
+        if (*abort_flag || !tc::mbar_wait(&aux.p_full[pb], (j >> 1) & 1) ||
+            !tc::mbar_wait(&aux.o_empty, (j & 1) ^ 1))
+          return false;
+        tc::tc_fence_after();
+        const uint32_t p0 = tc::smem_u32(sP + pb * K::P_BYTES);
+        const uint32_t v0 = tc::smem_u32(sKV + st * K::STAGE + K::K_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          // A = P (rows x keys, K-major, 64-key blocks); B = V (keys x d,
+          // MN-major: 64-d column blocks 128*128 B apart, 16 keys = 2048 B)
+          const uint32_t poff = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+          tc::mma_bf16_ss(tO, tc::sdesc_kmajor_sw128(p0 + poff),
+                          sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kKeys * 128), K::IDESC_O,
+                          kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&aux.o_full);
+        tc::mma_commit(&aux.kv_empty[st]);
+        return true;
+      };
+      if (!tc::mbar_wait(&aux.q_full, 0)) fail();
+      else if (nt > 0) {
+        bool ok = issue_s(0);
+        for (int j = 0; ok && j < nt; ++j) {
+          if (j + 1 < nt) ok = issue_s(j + 1);
+          if (ok) ok = issue_pv(j);
+        }
+        if (!ok) fail();
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // this thread's query row (TMEM lane)
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const int tok = tok0 + r / G;
+    const int lim = T_loc - T + tok;  // last visible local key
+    float m_run = -INFINITY, l_run = 0.f, alpha_prev = 1.f;
+    float o[D];
+#pragma unroll
+    for (int d = 0; d < D; ++d) o[d] = 0.f;
+    auto consume_o = [&](int j, float alpha) {
+      if (!*abort_flag && !tc::mbar_wait(&aux.o_full, j & 1)) {
+        record_error(status, MSA_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      tc::tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tc::tmem_ld32(tO + lane_addr + c * 32, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha, __uint_as_float(v[i]));
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&aux.o_empty);
+    };
+    for (int j = 0; j < nt; ++j) {
+      const int sb = j & 1;
+      if (!*abort_flag && !tc::mbar_wait(&aux.s_full[sb], (j >> 1) & 1)) {
+        record_error(status, MSA_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      tc::tc_fence_after();
+      // visible keys of this tile: memory rows < M, local rows <= lim
+      const bool mem = j < n_mt;
+      const int key0 = mem ? j * kKeys : (j - n_mt) * kKeys;
+      const int n_vis = mem ? min(kKeys, M - key0) : max(0, min(kKeys, lim - key0 + 1));
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c) {
+        uint32_t v[32];
+        tc::tmem_ld32(tS[sb] + lane_addr + c * 32, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c * 32 + i < n_vis) mt = fmaxf(mt, __uint_as_float(v[i]) * qscale);
+      }
+      const float m_new = fmaxf(m_run, mt);
+      const float alpha = m_new == -INFINITY ? 1.f : exp2f(m_run - m_new);
+      float ls = 0.f;
+      unsigned char* prow = sP + sb * K::P_BYTES + r * 128;
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c) {
+        uint32_t v[32];
+        tc::tmem_ld32(tS[sb] + lane_addr + c * 32, v);
+        tc::tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = (c * 32 + i < n_vis) ? exp2f(__uint_as_float(v[i]) * qscale - m_new) : 0.f;
+          const float p1 =
+              (c * 32 + i + 1 < n_vis) ? exp2f(__uint_as_float(v[i + 1]) * qscale - m_new) : 0.f;
+          ls += p0 + p1;
+          w[i / 2] = pack_bf16(p0, p1);
+        }
+        // keys c*32 .. c*32+31 are 16-byte pieces 4(c%2) .. 4(c%2)+3 of K
+        // block c/2 of row r, stored at their 128B-swizzled positions
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int piece = (c & 1) * 4 + q;
+          *reinterpret_cast<uint4*>(prow + (c >> 1) * (kRows * 128) + ((piece ^ (r & 7)) << 4)) =
+              make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+      }
+      l_run = l_run * alpha + ls;
+      m_run = m_new;
+      if (mem && M - key0 < kKeys && r >= M - key0) {
+        // rows past mem_len in the last memory tile hold whatever the
+        // caller's buffer holds there; zero their V so that 0 * V stays 0
+        unsigned char* vrow = sKV + (j % kStages) * K::STAGE + K::K_BYTES + r * 128;
+#pragma unroll
+        for (int kb = 0; kb < K::KB; ++kb)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4*>(vrow + kb * (kKeys * 128) + q * 16) = make_uint4(0, 0, 0, 0);
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(&aux.p_full[sb]);
+        tc::mbar_arrive(&aux.s_empty[sb]);
+      }
+      if (j > 0) consume_o(j - 1, alpha_prev);
+      alpha_prev = alpha;
+    }
+    if (nt > 0) consume_o(nt - 1, alpha_prev);
+    // normalise and store this row (token tok, head g*G + r%G)
+    if (r / G < n_tok) {
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      __nv_bfloat16* op = out + (((int64_t)b * T + tok) * Hq + g * G + r % G) * D;
+#pragma unroll
+      for (int d = 0; d < D; d += 8) {
+        const uint4 pk = make_uint4(pack_bf16(o[d] * inv, o[d + 1] * inv),
+                                    pack_bf16(o[d + 2] * inv, o[d + 3] * inv),
+                                    pack_bf16(o[d + 4] * inv, o[d + 5] * inv),
+                                    pack_bf16(o[d + 6] * inv, o[d + 7] * inv));
+        *reinterpret_cast<uint4*>(op + d) = pk;
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, K::TMEM_COLS);
+  }
+}
+
+// Rotates rows of x [n_rows][heads][D] (bf16) whose position is
+// pos_base + (row % rows_per_seq) + pos_shift into y, from cs[pos][D/2].
+__global__ void rope_rows_kernel(int64_t n_rows, int heads, int D, int rows_per_seq,
+                                 int pos_shift, const __nv_bfloat16* __restrict__ x,
+                                 const float2* __restrict__ cs, __nv_bfloat16* __restrict__ y) {
+  const int half = D / 2;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // one pair each
+  const int64_t per_row = (int64_t)heads * half;
+  if (e >= n_rows * per_row) return;
+  const int64_t row = e / per_row;
+  const int rem = (int)(e % per_row);
+  const int h = rem / half, i = rem % half;
+  const int p = (int)(row % rows_per_seq) + pos_shift;
+  const __nv_bfloat16* xr = x + (row * heads + h) * D;
+  const float a = __bfloat162float(xr[i]), c = __bfloat162float(xr[i + half]);
+  const float2 t = cs[(int64_t)p * half + i];
+  __nv_bfloat16* yr = y + (row * heads + h) * D;
+  yr[i] = __float2bfloat16_rn(a * t.x - c * t.y);
+  yr[i + half] = __float2bfloat16_rn(c * t.x + a * t.y);
+}
+
+__global__ void rope_table_kernel2(int n_pos, int half, int D, int64_t pos0, double base,
+                                   float2* __restrict__ cs) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)n_pos * half) return;
+  const int j = (int)(e / half), i = (int)(e % half);
+  cs[e] = rope_cs(pos0 + j, rope_inv_freq(base, i, D));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// bf16 [rows][heads][D] viewed as dims {D, heads, rows}; box {64, bh, br}.
+bool map3(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int bh, int br) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)bh, (cuuint32_t)br};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct TcPlan {
+  size_t cs_bytes, q_bytes, k_bytes, total;
+};
+
+TcPlan tc_plan(int B, int T, int T_loc, int Hq, int H, int D) {
+  TcPlan p{};
+  p.cs_bytes = round_up((size_t)T_loc * (D / 2) * sizeof(float2), 256);
+  p.q_bytes = round_up((size_t)B * T * Hq * D * 2, 256);
+  p.k_bytes = round_up((size_t)B * T_loc * H * D * 2, 256);
+  p.total = p.cs_bytes + p.q_bytes + p.k_bytes;
+  return p;
+}
+
+template <int D>
+int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void* k_mem,
+              const void* v_mem, const int32_t* mem_len, int m_cap, const void* k_loc,
+              const void* v_loc, int pos0, float rope_base, float qscale, void* out, void* ws,
+              cudaStream_t s) {
+  using K = ACfg<D>;
+  const int G = Hq / H;
+  const TcPlan p = tc_plan(B, T, T_loc, Hq, H, D);
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  float2* cs = reinterpret_cast<float2*>(w);
+  __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(w + p.cs_bytes);
+  __nv_bfloat16* k_rot = reinterpret_cast<__nv_bfloat16*>(w + p.cs_bytes + p.q_bytes);
+  const int64_t n_cs = (int64_t)T_loc * (D / 2);
+  rope_table_kernel2<<<(unsigned)((n_cs + 255) / 256), 256, 0, s>>>(T_loc, D / 2, D, pos0,
+                                                                   (double)rope_base, cs);
+  int rc = check_launch();
+  if (rc) return rc;
+  const int64_t nq = (int64_t)B * T * Hq * (D / 2);
+  rope_rows_kernel<<<(unsigned)((nq + 255) / 256), 256, 0, s>>>(
+      (int64_t)B * T, Hq, D, T, T_loc - T, static_cast<const __nv_bfloat16*>(q), cs, q_rot);
+  if ((rc = check_launch())) return rc;
+  const int64_t nk = (int64_t)B * T_loc * H * (D / 2);
+  rope_rows_kernel<<<(unsigned)((nk + 255) / 256), 256, 0, s>>>(
+      (int64_t)B * T_loc, H, D, T_loc, 0, static_cast<const __nv_bfloat16*>(k_loc), cs, k_rot);
+  if ((rc = check_launch())) return rc;
+
+  CUtensorMap tq, tkm, tvm, tkl, tvl;
+  const int TQ = kRows / G;
+  const int64_t mem_rows = std::max<int64_t>((int64_t)B * m_cap, 1);
+  const void* km = m_cap > 0 ? k_mem : k_rot;  // any valid address when there is no memory
+  const void* vm = m_cap > 0 ? v_mem : v_loc;
+  if (!map3(&tq, q_rot, D, Hq, (int64_t)B * T, G, TQ) ||
+      !map3(&tkm, km, D, H, m_cap > 0 ? mem_rows : (int64_t)B * T_loc, 1, kKeys) ||
+      !map3(&tvm, vm, D, H, m_cap > 0 ? mem_rows : (int64_t)B * T_loc, 1, kKeys) ||
+      !map3(&tkl, k_rot, D, H, (int64_t)B * T_loc, 1, kKeys) ||
+      !map3(&tvl, v_loc, D, H, (int64_t)B * T_loc, 1, kKeys))
+    return note_cuda(cudaErrorInvalidValue);
+  auto kern = attn_tc_kernel<D>;
+  rc = note_cuda(
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM));
+  if (rc) return rc;
+  const dim3 grid((unsigned)((T + TQ - 1) / TQ), (unsigned)H, (unsigned)B);
+  kern<<<grid, kThreads, K::SMEM, s>>>(tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G, mem_len,
+                                       m_cap, qscale, static_cast<__nv_bfloat16*>(out),
+                                       device_status_ptr());
+  return check_launch();
+}
+
+}  // namespace
+
+bool attn_tc_supported(int B, int T, int T_loc, int Hq, int H, int D, int m_cap) {
+  if (T < 2 || (D != 64 && D != 128) || H <= 0 || Hq % H) return false;
+  const int G = Hq / H;
+  if (G > 16 || (G & (G - 1))) return false;
+  if ((int64_t)B * T > (1LL << 30) || (int64_t)B * T_loc > (1LL << 30) ||
+      (int64_t)B * m_cap > (1LL << 30) || B > 65535 || H > 65535)
+    return false;
+  return true;
+}
+
+size_t attn_tc_workspace_size(int B, int T, int T_loc, int Hq, int H, int D, int) {
+  return tc_plan(B, T, T_loc, Hq, H, D).total;
+}
+
+int attn_tc_launch(int B, int T, int T_loc, int Hq, int H, int D, const void* q,
+                   const void* k_mem, const void* v_mem, const int32_t* mem_len, int m_cap,
+                   const void* k_loc, const void* v_loc, int pos0, float rope_base, float qscale,
+                   void* out, void* ws, cudaStream_t s) {
+  if (!aligned16(q) || !aligned16(k_loc) || !aligned16(v_loc) || !aligned16(out) ||
+      (m_cap > 0 && (!aligned16(k_mem) || !aligned16(v_mem))))
+    return MSA_ERR_INVALID_ARG;
+  if (D == 64)
+    return launch_tc<64>(B, T, T_loc, Hq, H, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc, pos0,
+                         rope_base, qscale, out, ws, s);
+  return launch_tc<128>(B, T, T_loc, Hq, H, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc, pos0,
+                        rope_base, qscale, out, ws, s);
 }
 
 }  // namespace msa

@@ -6,20 +6,31 @@
 // Step 2 (score -> top-k memory).  Equal scores are broken by the lower
 // document index, and the output is in rank order.
 //
-// Design: one 1024-thread CTA per query runs an exact radix select on the
-// 32-bit order-preserving key of each score (4 passes of 8 bits, histograms
-// in shared memory), which yields the k-th largest key K* and how many of
-// the k are strictly above it.  A compaction pass collects the keys > K*,
-// an index-ordered pass appends the lowest-index keys == K*, and a bitonic
-// sort of the k (score, ~index) 64-bit keys gives rank order.  Scores are
-// read from L2 (the whole vector of a 100K-document bank is 400 KB).
+// Design.  A score becomes a 32-bit order-preserving key (NaN lowest,
+// -0 == +0), and a candidate a 64-bit key (key << 32 | ~index), so that
+// "larger 64-bit key" is exactly "better rank" and all candidates differ.
+//   * select: one 1024-thread CTA per (segment, query).  The segment's keys
+//     are loaded once into shared memory; an exact 4-pass radix select
+//     (8 bits per pass, warp-aggregated shared histograms) finds the
+//     segment's k-th key; a compaction pass takes the keys above it and an
+//     index-ordered pass the lowest-index ties.  With one segment per query
+//     the k candidates are bitonic-sorted and written as the result;
+//     otherwise they go to the workspace.
+//   * merge: one CTA per query bitonic-sorts the segments' candidates and
+//     writes the first k.
+// Very large score vectors whose segments would not fit in shared memory
+// keep their keys in global memory (L2) with the same select.
+#include <algorithm>
+
 #include "msa_common.cuh"
 
 namespace msa {
 namespace {
 
-constexpr int kTopkThreads = 1024;
+constexpr int kThreads = 1024;
 constexpr int kMaxK = 1024;
+constexpr int kSegSmem = 16384;      // keys per segment held in shared memory
+constexpr int kMaxCand = 8192;       // candidates one merge CTA sorts
 
 // NaN ranks below every number; -0.0 and +0.0 are the same score (so their
 // tie goes to the lower index, like every other tie).
@@ -27,53 +38,82 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return isnan(s) ? 0u : f2o(s + 0.0f);
 }
 
-__global__ void __launch_bounds__(kTopkThreads)
-topk_kernel(int n, int k, const float* __restrict__ scores, int32_t* __restrict__ idx_out,
-            float* __restrict__ top_out) {
-  __shared__ uint32_t hist[256];
-  __shared__ unsigned long long cand[kMaxK];
-  __shared__ uint32_t s_sel, s_above;
-  __shared__ int s_n_gt, s_warp_cnt[32], s_running;
-  const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const float* s = scores + (int64_t)blockIdx.x * n;
+__device__ __forceinline__ unsigned long long cand_key(uint32_t key, uint32_t idx) {
+  return ((unsigned long long)key << 32) | (0xffffffffu - idx);
+}
 
+// Descending bitonic sort of c[0..P) (P a power of two) by the whole block.
+__device__ void bitonic_desc(unsigned long long* c, int P) {
+  for (int size = 2; size <= P; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < P; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0;
+          const unsigned long long a = c[i], b = c[j];
+          if (desc ? (a < b) : (a > b)) { c[i] = b; c[j] = a; }
+        }
+      }
+      __syncthreads();
+    }
+}
+
+struct SmemKeys {
+  const uint32_t* k;
+  __device__ __forceinline__ uint32_t operator()(int i) const { return k[i]; }
+};
+struct GlobalKeys {
+  const float* s;
+  __device__ __forceinline__ uint32_t operator()(int i) const { return score_key(__ldg(s + i)); }
+};
+
+struct SelectShared {
+  uint32_t hist[256];
+  uint32_t sel, above;
+  int n_gt, running, warp_cnt[32];
+};
+
+// Exact top-kk of keys(0..len) into cand[0..kk) (unordered), ties to the
+// lower index; indices are offset by base.  Whole block.
+template <class Keys>
+__device__ void select_topk(const Keys& keys, int len, int kk, uint32_t base,
+                            unsigned long long* cand, SelectShared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0, mask = 0;
-  int krem = k;
+  int krem = kk;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
+    for (int i = tid; i < 256; i += blockDim.x) sh.hist[i] = 0;
     __syncthreads();
     // warp-aggregated histogram: scores cluster in few bins, so lanes that
     // share a bin add their count with one shared-memory atomic
-    for (int base = 0; base < n; base += kTopkThreads) {
-      const int i = base + tid;
-      const uint32_t u = i < n ? score_key(__ldg(s + i)) : 0u;
-      const bool act = i < n && (u & mask) == prefix;
+    for (int i0 = 0; i0 < len; i0 += blockDim.x) {
+      const int i = i0 + tid;
+      const uint32_t u = i < len ? keys(i) : 0u;
+      const bool act = i < len && (u & mask) == prefix;
       const unsigned dig = act ? ((u >> shift) & 255u) : 256u;
       const unsigned peers = __match_any_sync(0xffffffffu, dig);
-      if (act && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (uint32_t)__popc(peers));
+      if (act && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
       // lane l owns digits [8l, 8l+8); suffix sums from the top digit down
       uint32_t own = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) own += hist[8 * lane + j];
-      uint32_t suf = own;  // inclusive suffix sum over lanes >= lane
+      for (int j = 0; j < 8; ++j) own += sh.hist[8 * lane + j];
+      uint32_t suf = own;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const uint32_t o = __shfl_down_sync(0xffffffffu, suf, off);
         if (lane + off < 32) suf += o;
       }
-      const uint32_t above_lane = suf - own;  // count in lanes > lane
-      const bool here = above_lane < (uint32_t)krem && suf >= (uint32_t)krem;
-      if (here) {
+      const uint32_t above_lane = suf - own;
+      if (above_lane < (uint32_t)krem && suf >= (uint32_t)krem) {
         uint32_t cum = above_lane;
         for (int j = 7; j >= 0; --j) {
-          const uint32_t hj = hist[8 * lane + j];
+          const uint32_t hj = sh.hist[8 * lane + j];
           if (cum + hj >= (uint32_t)krem) {
-            s_sel = 8 * lane + j;
-            s_above = cum;
+            sh.sel = 8 * lane + j;
+            sh.above = cum;
             break;
           }
           cum += hj;
@@ -81,85 +121,173 @@ topk_kernel(int n, int k, const float* __restrict__ scores, int32_t* __restrict_
       }
     }
     __syncthreads();
-    prefix |= s_sel << shift;
+    prefix |= sh.sel << shift;
     mask |= 0xffu << shift;
-    krem -= (int)s_above;
+    krem -= (int)sh.above;
     __syncthreads();
   }
-  // prefix = key of the k-th best; k - krem keys are strictly greater
-  if (tid == 0) { s_n_gt = 0; s_running = 0; }
+  // prefix = the kk-th best key; kk - krem keys are strictly greater
+  if (tid == 0) { sh.n_gt = 0; sh.running = 0; }
   __syncthreads();
-  for (int i = tid; i < n; i += kTopkThreads) {
-    const uint32_t u = score_key(__ldg(s + i));
-    if (u > prefix) {
-      const int pos = atomicAdd(&s_n_gt, 1);
-      cand[pos] = ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)i);
-    }
+  for (int i = tid; i < len; i += blockDim.x) {
+    const uint32_t u = keys(i);
+    if (u > prefix) cand[atomicAdd(&sh.n_gt, 1)] = cand_key(u, base + (uint32_t)i);
   }
   __syncthreads();
-  const int n_gt = s_n_gt;  // == k - krem
+  const int n_gt = sh.n_gt;
   // lowest-index keys equal to the threshold, in index order
-  for (int base = 0; base < n; base += kTopkThreads) {
-    if (s_running >= krem) break;  // uniform: read after a barrier
-    const int i = base + tid;
-    const bool eq = i < n && score_key(__ldg(s + i)) == prefix;
+  for (int i0 = 0; i0 < len; i0 += blockDim.x) {
+    if (sh.running >= krem) break;  // uniform: read after a barrier
+    const int i = i0 + tid;
+    const bool eq = i < len && keys(i) == prefix;
     const unsigned bal = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) s_warp_cnt[warp] = __popc(bal);
+    if (lane == 0) sh.warp_cnt[warp] = __popc(bal);
     __syncthreads();
-    int before = s_running;
-    for (int w = 0; w < warp; ++w) before += s_warp_cnt[w];
+    int before = sh.running;
+    for (int w = 0; w < warp; ++w) before += sh.warp_cnt[w];
     const int pos = before + __popc(bal & ((1u << lane) - 1u));
-    if (eq && pos < krem)
-      cand[n_gt + pos] = ((unsigned long long)prefix << 32) | (0xffffffffu - (uint32_t)i);
+    if (eq && pos < krem) cand[n_gt + pos] = cand_key(prefix, base + (uint32_t)i);
     __syncthreads();
     if (tid == 0) {
       int tot = 0;
-      for (int w = 0; w < 32; ++w) tot += s_warp_cnt[w];
-      s_running += tot;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += sh.warp_cnt[w];
+      sh.running += tot;
     }
     __syncthreads();
   }
-  // bitonic sort of cand[0..P) descending, P = next power of two >= k
-  int P = 1;
-  while (P < k) P <<= 1;
-  for (int i = k + tid; i < P; i += kTopkThreads) cand[i] = 0ull;
-  __syncthreads();
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < P; i += kTopkThreads) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool desc = (i & size) == 0;
-          const unsigned long long a = cand[i], b = cand[j];
-          if (desc ? (a < b) : (a > b)) { cand[i] = b; cand[j] = a; }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  for (int r = tid; r < k; r += kTopkThreads) {
+}
+
+__device__ void write_result(const unsigned long long* cand, int k, const float* s,
+                             int32_t* idx_out, float* top_out) {
+  for (int r = threadIdx.x; r < k; r += blockDim.x) {
     const uint32_t i = 0xffffffffu - (uint32_t)(cand[r] & 0xffffffffull);
-    idx_out[(int64_t)blockIdx.x * k + r] = (int32_t)i;
-    if (top_out) top_out[(int64_t)blockIdx.x * k + r] = s[i];
+    idx_out[r] = (int32_t)i;
+    if (top_out) top_out[r] = s[i];
   }
+}
+
+// grid (n_seg, B).  cand_ws == nullptr: one segment per query, write result.
+template <bool kSmemKeys>
+__global__ void __launch_bounds__(kThreads)
+topk_select_kernel(int n, int k, int seg_len, const float* __restrict__ scores,
+                   int32_t* __restrict__ idx_out, float* __restrict__ top_out,
+                   unsigned long long* __restrict__ cand_ws) {
+  extern __shared__ __align__(16) unsigned char dyn[];
+  __shared__ unsigned long long cand[kMaxK];
+  __shared__ SelectShared sh;
+  const int seg = blockIdx.x, b = blockIdx.y;
+  const int s0 = seg * seg_len;
+  const int len = min(seg_len, n - s0);
+  const int kk = min(k, len);
+  const float* s = scores + (int64_t)b * n;
+  if (kSmemKeys) {
+    uint32_t* keys = reinterpret_cast<uint32_t*>(dyn);
+    for (int i = threadIdx.x; i < len; i += blockDim.x) keys[i] = score_key(__ldg(s + s0 + i));
+    __syncthreads();
+    select_topk(SmemKeys{keys}, len, kk, (uint32_t)s0, cand, sh);
+  } else {
+    select_topk(GlobalKeys{s + s0}, len, kk, (uint32_t)s0, cand, sh);
+  }
+  __syncthreads();
+  if (cand_ws == nullptr) {
+    int P = 1;
+    while (P < kk) P <<= 1;
+    for (int i = kk + threadIdx.x; i < P; i += blockDim.x) cand[i] = 0ull;
+    __syncthreads();
+    bitonic_desc(cand, P);
+    write_result(cand, k, s, idx_out + (int64_t)b * k, top_out ? top_out + (int64_t)b * k : nullptr);
+  } else {
+    unsigned long long* dst = cand_ws + ((int64_t)b * gridDim.x + seg) * k;
+    for (int r = threadIdx.x; r < k; r += blockDim.x) dst[r] = r < kk ? cand[r] : 0ull;
+  }
+}
+
+// grid (B): the n_seg * k candidates of one query -> its top-k in rank order.
+__global__ void __launch_bounds__(kThreads)
+topk_merge_kernel(int n, int k, int n_cand, const unsigned long long* __restrict__ cand_ws,
+                  const float* __restrict__ scores, int32_t* __restrict__ idx_out,
+                  float* __restrict__ top_out) {
+  extern __shared__ __align__(16) unsigned char dyn[];
+  unsigned long long* c = reinterpret_cast<unsigned long long*>(dyn);
+  const int b = blockIdx.x;
+  int P = 1;
+  while (P < n_cand) P <<= 1;
+  const unsigned long long* src = cand_ws + (int64_t)b * n_cand;
+  for (int i = threadIdx.x; i < P; i += blockDim.x) c[i] = i < n_cand ? src[i] : 0ull;
+  __syncthreads();
+  bitonic_desc(c, P);
+  write_result(c, k, scores + (int64_t)b * n, idx_out + (int64_t)b * k,
+               top_out ? top_out + (int64_t)b * k : nullptr);
+}
+
+struct TopkPlan {
+  int seg_len, n_seg;
+  bool smem_keys;
+  size_t ws_bytes;
+};
+
+TopkPlan plan(int B, int n, int k) {
+  TopkPlan p{};
+  if (n <= kSegSmem) {
+    p.seg_len = n;
+    p.n_seg = 1;
+    p.smem_keys = true;
+    return p;
+  }
+  // about 4096 keys per segment, fewer segments when k is large
+  int seg = 4096;
+  const int max_seg_count = std::max(1, kMaxCand / k);
+  if ((n + seg - 1) / seg > max_seg_count) seg = (n + max_seg_count - 1) / max_seg_count;
+  seg = (seg + 1023) / 1024 * 1024;
+  p.seg_len = seg;
+  p.n_seg = (n + seg - 1) / seg;
+  p.smem_keys = seg <= kSegSmem;
+  if (p.n_seg == 1) return p;
+  p.ws_bytes = (size_t)B * p.n_seg * k * sizeof(unsigned long long);
+  return p;
 }
 
 }  // namespace
 }  // namespace msa
 
 extern "C" size_t msa_topk_workspace_size(int B, int n_docs, int k) {
-  (void)B; (void)n_docs; (void)k;
-  return 0;
+  if (B <= 0 || n_docs <= 0 || k <= 0 || k > n_docs || k > msa::kMaxK) return 0;
+  return msa::plan(B, n_docs, k).ws_bytes;
 }
 
 extern "C" int msa_topk_docs(int B, int n_docs, int k, const float* scores, int32_t* idx,
                              float* top_scores, void* ws, size_t ws_bytes,
                              msa_stream_t stream) {
-  (void)ws; (void)ws_bytes;
-  if (B <= 0 || n_docs <= 0 || k <= 0 || k > n_docs || k > msa::kMaxK) return MSA_ERR_INVALID_ARG;
+  using namespace msa;
+  if (B <= 0 || n_docs <= 0 || k <= 0 || k > n_docs || k > kMaxK) return MSA_ERR_INVALID_ARG;
   if (!scores || !idx) return MSA_ERR_INVALID_ARG;
-  if (B > 65535 * 1024) return MSA_ERR_UNSUPPORTED;
+  if (B > 65535) return MSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  msa::topk_kernel<<<B, msa::kTopkThreads, 0, s>>>(n_docs, k, scores, idx, top_scores);
-  return msa::check_launch();
+  const TopkPlan p = plan(B, n_docs, k);
+  if (p.ws_bytes && (!ws || ws_bytes < p.ws_bytes || !aligned16(ws))) return MSA_ERR_WORKSPACE;
+  unsigned long long* cand = p.n_seg > 1 ? static_cast<unsigned long long*>(ws) : nullptr;
+  const dim3 grid((unsigned)p.n_seg, (unsigned)B);
+  int rc;
+  if (p.smem_keys) {
+    const size_t smem = (size_t)p.seg_len * sizeof(uint32_t);
+    rc = note_cuda(cudaFuncSetAttribute(topk_select_kernel<true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    if (rc) return rc;
+    topk_select_kernel<true><<<grid, kThreads, smem, s>>>(n_docs, k, p.seg_len, scores, idx,
+                                                           top_scores, cand);
+  } else {
+    topk_select_kernel<false><<<grid, kThreads, 0, s>>>(n_docs, k, p.seg_len, scores, idx,
+                                                         top_scores, cand);
+  }
+  if ((rc = check_launch())) return rc;
+  if (p.n_seg == 1) return MSA_OK;
+  const int n_cand = p.n_seg * k;
+  int P = 1;
+  while (P < n_cand) P <<= 1;
+  const size_t smem = (size_t)P * sizeof(unsigned long long);
+  rc = note_cuda(cudaFuncSetAttribute(topk_merge_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (rc) return rc;
+  topk_merge_kernel<<<B, kThreads, smem, s>>>(n_docs, k, n_cand, cand, scores, idx, top_scores);
+  return check_launch();
 }

@@ -69,11 +69,18 @@ class Router:
         return doc_scores
 
 
-def topk_docs(scores: torch.Tensor, k: int, idx=None, top=None, stream=None):
+def topk_workspace(B: int, n: int, k: int, device):
+    n_ws = _m.msa_topk_workspace_size(B, n, k)
+    return torch.empty(max(n_ws, 16), dtype=torch.uint8, device=device)
+
+
+def topk_docs(scores: torch.Tensor, k: int, idx=None, top=None, ws=None, stream=None):
     B, n = scores.shape
     if idx is None:
         idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
-    _m.msa_topk_docs(B, n, k, scores, idx, top, None, 0, stream)
+    if ws is None:
+        ws = topk_workspace(B, n, k, scores.device)
+    _m.msa_topk_docs(B, n, k, scores, idx, top, ws, ws.numel(), stream)
     return idx, top
 
 
@@ -133,6 +140,7 @@ class Pipeline:
         self.doc_scores = torch.empty((B, self.n_docs), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, k), dtype=torch.int32, device=dev)
         self.top = torch.empty((B, k), dtype=torch.float32, device=dev)
+        self.topk_ws = topk_workspace(B, self.n_docs, k, dev)
         self.k_mem = torch.empty((B, max(m_cap, 1), H, D), dtype=kr_bar.dtype, device=dev)
         self.v_mem = torch.empty_like(self.k_mem)
         self.mem_len = torch.empty(B, dtype=torch.int32, device=dev)
@@ -140,7 +148,7 @@ class Pipeline:
 
     def __call__(self, q_r, q, k_loc, v_loc, stream=None):
         self.router(q_r, self.kr_bar, self.coff, self.n_docs, self.doc_scores, None, stream)
-        topk_docs(self.doc_scores, self.k, self.idx, self.top, stream)
+        topk_docs(self.doc_scores, self.k, self.idx, self.top, self.topk_ws, stream)
         gather_kv(self.idx, self.coff, self.k_bar, self.v_bar, self.m_cap, self.k_mem,
                   self.v_mem, self.mem_len, stream)
         self.attn(q, self.k_mem, self.v_mem, self.mem_len, k_loc, v_loc, self.pos0,

@@ -306,6 +306,9 @@ def test_route_100m_prefill_sampled(prepared):
 @pytest.mark.parametrize("B,n,k,quant", [
     (1, 16, 2, None), (4, 1000, 16, None), (64, 10000, 16, None), (1, 100000, 16, None),
     (3, 5000, 1024, None), (2, 300, 300, None), (2, 5000, 16, 8.0), (1, 4096, 64, 1.0),
+    (2, 16384, 16, None), (2, 16385, 16, 64.0),          # one segment / two segments
+    (1, 200000, 1024, None),                              # 8 segments of 25K keys (L2 keys)
+    (3, 70000, 100, 16.0), (1, 1000000, 16, None),        # many ties; 1M documents
 ])
 def test_topk_identical_to_oracle(B, n, k, quant):
     g = torch.Generator(device="cuda").manual_seed(n + k)
@@ -409,6 +412,37 @@ def _attn_case(dtype, B, T, T_loc, Hq, H, D, m_cap, mem_lens, pos0, seed):
 def test_attention_vs_oracle(dtype, B, T, T_loc, Hq, H, D, m_cap, mem_lens, pos0, tol):
     got, want = _attn_case(dtype, B, T, T_loc, Hq, H, D, m_cap, mem_lens, pos0, 31 + T)
     assert np.max(np.abs(got - want)) <= tol
+    status_ok()
+
+
+@pytest.mark.parametrize("B,T,T_loc,Hq,H,D,m_cap,mem_lens", [
+    (2, 300, 700, 32, 8, 128, 500, [500, 129]),   # several key tiles each side
+    (3, 64, 64, 8, 8, 64, 130, [128, 0, 1]),       # G = 1, empty and 1-row memory
+    (1, 17, 1000, 16, 1, 128, 256, [256]),         # G = 16, chunked prefill
+])
+def test_attention_prefill_tensor_core_shapes(B, T, T_loc, Hq, H, D, m_cap, mem_lens):
+    """Rows past mem_len are filled with NaN: they must not reach the
+    output (the kernel loads whole 128-key tiles)."""
+    g = torch.Generator(device="cuda").manual_seed(T + T_loc)
+    dt = torch.bfloat16
+    q = synth.randn((B, T, Hq, D), dt, "cuda", g)
+    km = synth.randn((B, m_cap, H, D), dt, "cuda", g)
+    vm = synth.randn((B, m_cap, H, D), dt, "cuda", g)
+    for b, n in enumerate(mem_lens):
+        km[b, n:] = float("nan")
+        vm[b, n:] = float("nan")
+    kl = synth.randn((B, T_loc, H, D), dt, "cuda", g)
+    vl = synth.randn((B, T_loc, H, D), dt, "cuda", g)
+    ml = torch.tensor(mem_lens, dtype=torch.int32, device="cuda")
+    att = pipeline.Attention(dt, B, T, T_loc, Hq, H, D, m_cap, "cuda")
+    out = att(q, km, vm, ml, kl, vl, 16)
+    torch.cuda.synchronize()
+    want = oracle.sparse_attn(f64(q), [f64(km[b, :n]) for b, n in enumerate(mem_lens)],
+                              [f64(vm[b, :n]) for b, n in enumerate(mem_lens)],
+                              f64(kl), f64(vl), 16, 10000.0)
+    got = f64(out)
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got - want)) <= ATTN_BF16
     status_ok()
 
 
