@@ -135,15 +135,15 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
-def build_workload(rank: int):
+def build_workload(rank: int, n_docs: int = 100000):
     import torch
 
     from latent_memory_routing_b200 import pipeline, synth
-    lengths = synth.bank_100m_lengths()
+    lengths = synth.bank_100m_lengths(n_docs)
     toff = synth.tok_offsets(lengths).cuda()
     coff = pipeline.chunk_offsets(toff)
     coff_h = coff.cpu()
-    w = synth.bank_100m(coff_h, "cuda")
+    w = synth.bank_100m(coff_h, "cuda", n_docs=n_docs)
     if rank:  # independent replica per rank: different query draws
         g = torch.Generator(device="cuda").manual_seed(7919 * rank)
         for key in ("q", "q_r", "k_loc", "v_loc"):
@@ -192,7 +192,7 @@ def run_libmsa(args, world, rank, local):
     from latent_memory_routing_b200 import msa, pipeline
     _b.build()
     msa.lib()
-    w, p, C = build_workload(rank)
+    w, p, C = build_workload(rank, args.n_docs)
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
     for _ in range(max(args.warmup, 3)):
@@ -284,7 +284,9 @@ def run_libmsa(args, world, rank, local):
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) pooled bank drawn at chunk level + planted needles)",
-        "config": {"workload": WORKLOAD, "n_chunks": C, "n_docs": p.n_docs, "global_batch": world,
+        "config": {"workload": WORKLOAD if args.n_docs == 100000 else
+                   f"bank_100m recipe cut to {args.n_docs} docs (profiling case)",
+                   "n_chunks": C, "n_docs": p.n_docs, "global_batch": world,
                    "seq_len": w["T"], "top_k": w["k"], "m_cap": p.m_cap,
                    "parallelism": f"replica x{world}",
                    "l2": "the 3.2 GB routing bank streams through the 126 MB L2 every step"},
@@ -423,6 +425,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--n-docs", type=int, default=100000,
+                    help="documents in the bank (fewer only to profile a small case)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args.gpus)
