@@ -1,6 +1,8 @@
 // Library-wide entry points of libmsa: status strings, CUDA error capture,
 // the per-device status word.
 #include <mutex>
+#include <map>
+#include <utility>
 
 #include "msa_common.cuh"
 
@@ -61,6 +63,22 @@ int num_sms() {
     g_sms[dev] = n;
   }
   return g_sms[dev];
+}
+
+int ensure_smem_attr(const void* func, int bytes) {
+  // The attribute is one value per (kernel, device): keep the largest value
+  // set so far and only ever raise it.
+  const int dev = current_device();
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> limit;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_pair(func, dev);
+  const auto it = limit.find(key);
+  if (it != limit.end() && it->second >= bytes) return MSA_OK;
+  const int rc = note_cuda(
+      cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  if (rc == MSA_OK) limit[key] = bytes;
+  return rc;
 }
 
 }  // namespace msa

@@ -9,9 +9,9 @@
 // keep their document-wise rotation; local keys are causal.
 //
 // Design.
-//   * rope_rows_kernel rotates Q (to pos0 + T_loc - T + i) and the local K
-//     (to pos0 + j) once per call into bf16 workspace copies, from a per-call
-//     cos/sin table (angles reduced in double).
+//   * rope_prep_kernel rotates Q (to pos0 + T_loc - T + i) and the local K
+//     (to pos0 + j) once per call into bf16 workspace copies, one launch,
+//     cos/sin per position built in shared memory (angles reduced in double).
 //   * attn_tc_kernel: one CTA per (128 query rows, KV head, batch).  GQA rows
 //     are packed as (token, head of the group): a TMA box of
 //     {64 d, G heads, 128/G tokens} lands as 128 rows of 128 B -- the Q tile
@@ -353,33 +353,69 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
 }
 
-// Rotates rows of x [n_rows][heads][D] (bf16) whose position is
-// pos_base + (row % rows_per_seq) + pos_shift into y, from cs[pos][D/2].
-__global__ void rope_rows_kernel(int64_t n_rows, int heads, int D, int rows_per_seq,
-                                 int pos_shift, const __nv_bfloat16* __restrict__ x,
-                                 const float2* __restrict__ cs, __nv_bfloat16* __restrict__ y) {
-  const int half = D / 2;
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // one pair each
-  const int64_t per_row = (int64_t)heads * half;
-  if (e >= n_rows * per_row) return;
-  const int64_t row = e / per_row;
-  const int rem = (int)(e % per_row);
-  const int h = rem / half, i = rem % half;
-  const int p = (int)(row % rows_per_seq) + pos_shift;
-  const __nv_bfloat16* xr = x + (row * heads + h) * D;
-  const float a = __bfloat162float(xr[i]), c = __bfloat162float(xr[i + half]);
-  const float2 t = cs[(int64_t)p * half + i];
-  __nv_bfloat16* yr = y + (row * heads + h) * D;
-  yr[i] = __float2bfloat16_rn(a * t.x - c * t.y);
-  yr[i + half] = __float2bfloat16_rn(c * t.x + a * t.y);
-}
+// Global RoPE of the query and the local keys, one launch: CTA i owns local
+// positions [i*kPosPerCta, ...): it builds their (cos, sin) in shared memory
+// (angles reduced in double), then rotates every local K row and every query
+// row at those positions (query token t sits at local position T_loc - T + t)
+// with 16-byte loads of an element group and its rotate-half partner.
+constexpr int kPosPerCta = 4;
 
-__global__ void rope_table_kernel2(int n_pos, int half, int D, int64_t pos0, double base,
-                                   float2* __restrict__ cs) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= (int64_t)n_pos * half) return;
-  const int j = (int)(e / half), i = (int)(e % half);
-  cs[e] = rope_cs(pos0 + j, rope_inv_freq(base, i, D));
+template <int D>
+__global__ void __launch_bounds__(256)
+rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0, double base,
+                 const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_loc,
+                 __nv_bfloat16* __restrict__ q_rot, __nv_bfloat16* __restrict__ k_rot) {
+  constexpr int HALF = D / 2;
+  constexpr int UPH = HALF / 8;  // 16-byte pair units per head
+  __shared__ float2 cs[kPosPerCta][HALF];
+  const int p0 = blockIdx.x * kPosPerCta;
+  const int np = min(kPosPerCta, T_loc - p0);
+  for (int e = threadIdx.x; e < np * HALF; e += blockDim.x) {
+    const int j = e / HALF, i = e % HALF;
+    cs[j][i] = rope_cs(pos0 + p0 + j, rope_inv_freq(base, i, D));
+  }
+  __syncthreads();
+  // local keys: B x np positions x H heads x UPH units
+  const int nk = B * np * H * UPH;
+  for (int e = threadIdx.x; e < nk; e += blockDim.x) {
+    const int u = e % UPH, h = (e / UPH) % H, j = (e / (UPH * H)) % np, b = e / (UPH * H * np);
+    const int64_t off = (((int64_t)b * T_loc + p0 + j) * H + h) * D + u * 8;
+    float x1[8], x2[8], y1[8], y2[8];
+    Vec16<__nv_bfloat16>::unpack(ldg16(k_loc + off), x1);
+    Vec16<__nv_bfloat16>::unpack(ldg16(k_loc + off + HALF), x2);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const float2 c = cs[j][u * 8 + t];
+      y1[t] = x1[t] * c.x - x2[t] * c.y;
+      y2[t] = x2[t] * c.x + x1[t] * c.y;
+    }
+    st16(k_rot + off, Vec16<__nv_bfloat16>::pack(y1));
+    st16(k_rot + off + HALF, Vec16<__nv_bfloat16>::pack(y2));
+  }
+  // query tokens at these positions
+  const int first_q = T_loc - T;  // local position of query token 0
+  const int t_lo = max(p0, first_q) - first_q, t_hi = p0 + np - first_q;
+  if (t_hi <= t_lo) return;
+  const int nt = t_hi - t_lo;
+  const int nq = B * nt * Hq * UPH;
+  for (int e = threadIdx.x; e < nq; e += blockDim.x) {
+    const int u = e % UPH, h = (e / UPH) % Hq, tt = (e / (UPH * Hq)) % nt,
+              b = e / (UPH * Hq * nt);
+    const int t = t_lo + tt;
+    const int j = first_q + t - p0;
+    const int64_t off = (((int64_t)b * T + t) * Hq + h) * D + u * 8;
+    float x1[8], x2[8], y1[8], y2[8];
+    Vec16<__nv_bfloat16>::unpack(ldg16(q + off), x1);
+    Vec16<__nv_bfloat16>::unpack(ldg16(q + off + HALF), x2);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 c = cs[j][u * 8 + i];
+      y1[i] = x1[i] * c.x - x2[i] * c.y;
+      y2[i] = x2[i] * c.x + x1[i] * c.y;
+    }
+    st16(q_rot + off, Vec16<__nv_bfloat16>::pack(y1));
+    st16(q_rot + off + HALF, Vec16<__nv_bfloat16>::pack(y2));
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -416,7 +452,7 @@ struct TcPlan {
 
 TcPlan tc_plan(int B, int T, int T_loc, int Hq, int H, int D) {
   TcPlan p{};
-  p.cs_bytes = round_up((size_t)T_loc * (D / 2) * sizeof(float2), 256);
+  p.cs_bytes = 0;
   p.q_bytes = round_up((size_t)B * T * Hq * D * 2, 256);
   p.k_bytes = round_up((size_t)B * T_loc * H * D * 2, 256);
   p.total = p.cs_bytes + p.q_bytes + p.k_bytes;
@@ -432,22 +468,13 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   const int G = Hq / H;
   const TcPlan p = tc_plan(B, T, T_loc, Hq, H, D);
   unsigned char* w = static_cast<unsigned char*>(ws);
-  float2* cs = reinterpret_cast<float2*>(w);
   __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(w + p.cs_bytes);
   __nv_bfloat16* k_rot = reinterpret_cast<__nv_bfloat16*>(w + p.cs_bytes + p.q_bytes);
-  const int64_t n_cs = (int64_t)T_loc * (D / 2);
-  rope_table_kernel2<<<(unsigned)((n_cs + 255) / 256), 256, 0, s>>>(T_loc, D / 2, D, pos0,
-                                                                   (double)rope_base, cs);
+  rope_prep_kernel<D><<<(unsigned)((T_loc + kPosPerCta - 1) / kPosPerCta), 256, 0, s>>>(
+      B, T, T_loc, Hq, H, pos0, (double)rope_base, static_cast<const __nv_bfloat16*>(q),
+      static_cast<const __nv_bfloat16*>(k_loc), q_rot, k_rot);
   int rc = check_launch();
   if (rc) return rc;
-  const int64_t nq = (int64_t)B * T * Hq * (D / 2);
-  rope_rows_kernel<<<(unsigned)((nq + 255) / 256), 256, 0, s>>>(
-      (int64_t)B * T, Hq, D, T, T_loc - T, static_cast<const __nv_bfloat16*>(q), cs, q_rot);
-  if ((rc = check_launch())) return rc;
-  const int64_t nk = (int64_t)B * T_loc * H * (D / 2);
-  rope_rows_kernel<<<(unsigned)((nk + 255) / 256), 256, 0, s>>>(
-      (int64_t)B * T_loc, H, D, T_loc, 0, static_cast<const __nv_bfloat16*>(k_loc), cs, k_rot);
-  if ((rc = check_launch())) return rc;
 
   CUtensorMap tq, tkm, tvm, tkl, tvl;
   const int TQ = kRows / G;
@@ -461,8 +488,7 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
       !map3(&tvl, v_loc, D, H, (int64_t)B * T_loc, 1, kKeys))
     return note_cuda(cudaErrorInvalidValue);
   auto kern = attn_tc_kernel<D>;
-  rc = note_cuda(
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM));
+  rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
   const dim3 grid((unsigned)((T + TQ - 1) / TQ), (unsigned)H, (unsigned)B);
   kern<<<grid, kThreads, K::SMEM, s>>>(tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G, mem_len,

@@ -184,8 +184,7 @@ int launch_encode(int L, int64_t n_tok, int n_docs, int H, const void* k,
   const size_t smem = sizeof(float2) * kMaxChunk * (D / 2) +
                       sizeof(float) * (size_t)R * 3 * H * D;
   auto kern = encode_pool_kernel<T, D>;
-  int rc = note_cuda(cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem);
   if (rc) return rc;
   if (n_chunks == 0) return MSA_OK;
   kern<<<(unsigned)n_chunks, threads, smem, s>>>(

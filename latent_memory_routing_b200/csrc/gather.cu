@@ -7,15 +7,18 @@
 // local context) and §"Routing happens inside attention ..." (their
 // compressed K/V are concatenated with the query's local K/V).
 //
-// Design: one CTA per (rank, query).  Each CTA finds its destination offset
+// Design: kSplit CTAs per (rank, query).  Each finds its destination offset
 // from the chunk counts of the higher-ranked documents (k <= 1024 small
-// reads), then streams the document's contiguous chunk rows of K̄ and V̄ with
-// 16-byte loads and stores.  HBM-bound; rows past m_cap are dropped and the
+// reads), then streams its share of the document's contiguous chunk rows of
+// K̄ and V̄ with 16-byte loads and stores -- enough CTAs in flight to cover
+// memory latency even for one query.  Rows past m_cap are dropped and the
 // overflow is recorded in the device status word.
 #include "msa_common.cuh"
 
 namespace msa {
 namespace {
+
+constexpr int kSplit = 4;
 
 __global__ void __launch_bounds__(256)
 gather_kernel(int k, int n_docs, int row_vecs, const int32_t* __restrict__ idx,
@@ -23,7 +26,7 @@ gather_kernel(int k, int n_docs, int row_vecs, const int32_t* __restrict__ idx,
               const uint4* __restrict__ vb, int m_cap, uint4* __restrict__ km,
               uint4* __restrict__ vm, int32_t* __restrict__ mem_len, int* status) {
   __shared__ int64_t s_off, s_src, s_rows;
-  const int r = blockIdx.x, b = blockIdx.y;
+  const int r = blockIdx.x / kSplit, part = blockIdx.x % kSplit, b = blockIdx.y;
   const int32_t* ib = idx + (int64_t)b * k;
   if (threadIdx.x < 32) {
     // destination offset = rows of ranks < r (warp-strided sum)
@@ -43,7 +46,7 @@ gather_kernel(int k, int n_docs, int row_vecs, const int32_t* __restrict__ idx,
       } else {
         record_error(status, MSA_ERR_INVALID_ARG);
       }
-      if (r == k - 1) {
+      if (r == k - 1 && part == 0) {
         const int64_t total = off + rows;
         mem_len[b] = (int32_t)(total < m_cap ? total : m_cap);
         if (total > m_cap) record_error(status, MSA_ERR_CAPACITY);
@@ -54,13 +57,17 @@ gather_kernel(int k, int n_docs, int row_vecs, const int32_t* __restrict__ idx,
     }
   }
   __syncthreads();
-  const int64_t off = s_off;
   int64_t rows = s_rows;
-  if (off >= m_cap) return;
-  if (off + rows > m_cap) rows = m_cap - off;
-  const int64_t n_vec = rows * row_vecs;
-  const uint4* ks = kb + s_src * row_vecs;
-  const uint4* vs = vb + s_src * row_vecs;
+  if (s_off >= m_cap) return;
+  if (s_off + rows > m_cap) rows = m_cap - s_off;
+  // this CTA's share of the rows
+  const int64_t per = (rows + kSplit - 1) / kSplit;
+  const int64_t r0 = rows < part * per ? rows : part * per;
+  const int64_t r1 = rows < r0 + per ? rows : r0 + per;
+  const int64_t n_vec = (r1 - r0) * row_vecs;
+  const int64_t off = s_off + r0;
+  const uint4* ks = kb + (s_src + r0) * row_vecs;
+  const uint4* vs = vb + (s_src + r0) * row_vecs;
   uint4* kd = km + ((int64_t)b * m_cap + off) * row_vecs;
   uint4* vd = vm + ((int64_t)b * m_cap + off) * row_vecs;
   for (int64_t i = threadIdx.x; i < n_vec; i += blockDim.x) {
@@ -91,7 +98,7 @@ extern "C" int msa_gather_kv(msa_dtype dt, int B, int k, int H, int D, const int
   if (row_bytes % 16) return MSA_ERR_UNSUPPORTED;
   if (B > 65535) return MSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const dim3 grid((unsigned)k, (unsigned)B);
+  const dim3 grid((unsigned)(k * kSplit), (unsigned)B);
   gather_kernel<<<grid, 256, 0, s>>>(k, n_docs, (int)(row_bytes / 16), idx, chunk_offsets,
                                      static_cast<const uint4*>(k_bar),
                                      static_cast<const uint4*>(v_bar), m_cap,

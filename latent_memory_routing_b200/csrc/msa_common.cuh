@@ -26,6 +26,11 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// Sets a kernel's dynamic shared-memory limit once per (kernel, device), so
+// that later calls -- including calls made while a stream is being captured
+// into a CUDA graph -- only launch.
+int ensure_smem_attr(const void* func, int bytes);
+
 // ---------------------------------------------------------- device status
 
 // Device address of the current device's status word (first

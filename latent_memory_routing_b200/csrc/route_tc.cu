@@ -536,8 +536,7 @@ int launch(int B, int T, int H, const __nv_bfloat16* qhat, int n_pad, const __nv
   if (!make_map(&tm_q, qhat, D, n_pad, H, (uint64_t)D * 2, (uint64_t)n_pad * D * 2, N, 1))
     return note_cuda(cudaErrorInvalidValue);
   auto kern = route_tc_kernel<N, D, kPrep>;
-  int rc = note_cuda(
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM));
+  int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
   const int64_t n_tiles = (C + kTile - 1) / kTile;
   const int grid = (int)std::min<int64_t>(n_tiles, num_sms());

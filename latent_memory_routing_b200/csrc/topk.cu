@@ -10,14 +10,15 @@
 // -0 == +0), and a candidate a 64-bit key (key << 32 | ~index), so that
 // "larger 64-bit key" is exactly "better rank" and all candidates differ.
 //   * select: one 1024-thread CTA per (segment, query).  The segment's keys
-//     are loaded once into shared memory; an exact 4-pass radix select
-//     (8 bits per pass, warp-aggregated shared histograms) finds the
+//     are loaded once into shared memory; an exact 3-pass radix select
+//     (11, 11 and 10 bits, warp-aggregated shared histograms) finds the
 //     segment's k-th key; a compaction pass takes the keys above it and an
 //     index-ordered pass the lowest-index ties.  With one segment per query
-//     the k candidates are bitonic-sorted and written as the result;
+//     the k candidates are placed in rank order by counting (each key's rank
+//     = number of larger keys; all keys differ) and written as the result;
 //     otherwise they go to the workspace.
-//   * merge: one CTA per query bitonic-sorts the segments' candidates and
-//     writes the first k.
+//   * merge: one CTA per query ranks the segments' candidates the same way
+//     (a bitonic sort above 2048 candidates) and writes the first k.
 // Very large score vectors whose segments would not fit in shared memory
 // keep their keys in global memory (L2) with the same select.
 #include <algorithm>
@@ -31,6 +32,7 @@ constexpr int kThreads = 1024;
 constexpr int kMaxK = 1024;
 constexpr int kSegSmem = 16384;      // keys per segment held in shared memory
 constexpr int kMaxCand = 8192;       // candidates one merge CTA sorts
+constexpr int kRankMax = 2048;       // up to this many, merge by counting ranks
 
 // NaN ranks below every number; -0.0 and +0.0 are the same score (so their
 // tie goes to the lower index, like every other tie).
@@ -67,8 +69,10 @@ struct GlobalKeys {
   __device__ __forceinline__ uint32_t operator()(int i) const { return score_key(__ldg(s + i)); }
 };
 
+constexpr int kBins = 2048;  // 11-bit digits: passes over bits 31..21, 20..10, 9..0
+
 struct SelectShared {
-  uint32_t hist[256];
+  uint32_t hist[kBins];
   uint32_t sel, above;
   int n_gt, running, warp_cnt[32];
 };
@@ -81,8 +85,12 @@ __device__ void select_topk(const Keys& keys, int len, int kk, uint32_t base,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0, mask = 0;
   int krem = kk;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += blockDim.x) sh.hist[i] = 0;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+    const int nb = (int)dmask + 1;
+    for (int i = tid; i < nb; i += blockDim.x) sh.hist[i] = 0;
     __syncthreads();
     // warp-aggregated histogram: scores cluster in few bins, so lanes that
     // share a bin add their count with one shared-memory atomic
@@ -90,16 +98,16 @@ __device__ void select_topk(const Keys& keys, int len, int kk, uint32_t base,
       const int i = i0 + tid;
       const uint32_t u = i < len ? keys(i) : 0u;
       const bool act = i < len && (u & mask) == prefix;
-      const unsigned dig = act ? ((u >> shift) & 255u) : 256u;
+      const unsigned dig = act ? ((u >> shift) & dmask) : 0xffffffffu;
       const unsigned peers = __match_any_sync(0xffffffffu, dig);
       if (act && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
-      // lane l owns digits [8l, 8l+8); suffix sums from the top digit down
+      // lane l owns digits [l*per, (l+1)*per); suffix sums from the top down
+      const int per = nb / 32;
       uint32_t own = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) own += sh.hist[8 * lane + j];
+      for (int j = 0; j < per; ++j) own += sh.hist[per * lane + j];
       uint32_t suf = own;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -109,10 +117,10 @@ __device__ void select_topk(const Keys& keys, int len, int kk, uint32_t base,
       const uint32_t above_lane = suf - own;
       if (above_lane < (uint32_t)krem && suf >= (uint32_t)krem) {
         uint32_t cum = above_lane;
-        for (int j = 7; j >= 0; --j) {
-          const uint32_t hj = sh.hist[8 * lane + j];
+        for (int j = per - 1; j >= 0; --j) {
+          const uint32_t hj = sh.hist[per * lane + j];
           if (cum + hj >= (uint32_t)krem) {
-            sh.sel = 8 * lane + j;
+            sh.sel = per * lane + j;
             sh.above = cum;
             break;
           }
@@ -122,7 +130,7 @@ __device__ void select_topk(const Keys& keys, int len, int kk, uint32_t base,
     }
     __syncthreads();
     prefix |= sh.sel << shift;
-    mask |= 0xffu << shift;
+    mask |= dmask << shift;
     krem -= (int)sh.above;
     __syncthreads();
   }
@@ -157,6 +165,19 @@ __device__ void select_topk(const Keys& keys, int len, int kk, uint32_t base,
   }
 }
 
+// Places the n distinct keys c[0..n) in descending order into o[0..min(n,k))
+// by counting, for each key, how many keys are larger (its rank): one
+// barrier instead of a sorting network.  n <= a few thousand.
+__device__ void rank_place(const unsigned long long* c, int n, int k, unsigned long long* o) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const unsigned long long x = c[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) rank += c[j] > x;
+    if (rank < k) o[rank] = x;
+  }
+  __syncthreads();
+}
+
 __device__ void write_result(const unsigned long long* cand, int k, const float* s,
                              int32_t* idx_out, float* top_out) {
   for (int r = threadIdx.x; r < k; r += blockDim.x) {
@@ -174,6 +195,7 @@ topk_select_kernel(int n, int k, int seg_len, const float* __restrict__ scores,
                    unsigned long long* __restrict__ cand_ws) {
   extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ unsigned long long cand[kMaxK];
+  __shared__ unsigned long long ranked[kMaxK];
   __shared__ SelectShared sh;
   const int seg = blockIdx.x, b = blockIdx.y;
   const int s0 = seg * seg_len;
@@ -190,12 +212,9 @@ topk_select_kernel(int n, int k, int seg_len, const float* __restrict__ scores,
   }
   __syncthreads();
   if (cand_ws == nullptr) {
-    int P = 1;
-    while (P < kk) P <<= 1;
-    for (int i = kk + threadIdx.x; i < P; i += blockDim.x) cand[i] = 0ull;
-    __syncthreads();
-    bitonic_desc(cand, P);
-    write_result(cand, k, s, idx_out + (int64_t)b * k, top_out ? top_out + (int64_t)b * k : nullptr);
+    rank_place(cand, kk, k, ranked);
+    write_result(ranked, k, s, idx_out + (int64_t)b * k,
+                 top_out ? top_out + (int64_t)b * k : nullptr);
   } else {
     unsigned long long* dst = cand_ws + ((int64_t)b * gridDim.x + seg) * k;
     for (int r = threadIdx.x; r < k; r += blockDim.x) dst[r] = r < kk ? cand[r] : 0ull;
@@ -210,9 +229,19 @@ topk_merge_kernel(int n, int k, int n_cand, const unsigned long long* __restrict
   extern __shared__ __align__(16) unsigned char dyn[];
   unsigned long long* c = reinterpret_cast<unsigned long long*>(dyn);
   const int b = blockIdx.x;
+  const unsigned long long* src = cand_ws + (int64_t)b * n_cand;
+  if (n_cand <= kRankMax) {
+    // the segments' pads (key 0) rank last and never reach the first k
+    unsigned long long* ranked = c + n_cand;
+    for (int i = threadIdx.x; i < n_cand; i += blockDim.x) c[i] = src[i];
+    __syncthreads();
+    rank_place(c, n_cand, k, ranked);
+    write_result(ranked, k, scores + (int64_t)b * n, idx_out + (int64_t)b * k,
+                 top_out ? top_out + (int64_t)b * k : nullptr);
+    return;
+  }
   int P = 1;
   while (P < n_cand) P <<= 1;
-  const unsigned long long* src = cand_ws + (int64_t)b * n_cand;
   for (int i = threadIdx.x; i < P; i += blockDim.x) c[i] = i < n_cand ? src[i] : 0ull;
   __syncthreads();
   bitonic_desc(c, P);
@@ -270,8 +299,7 @@ extern "C" int msa_topk_docs(int B, int n_docs, int k, const float* scores, int3
   int rc;
   if (p.smem_keys) {
     const size_t smem = (size_t)p.seg_len * sizeof(uint32_t);
-    rc = note_cuda(cudaFuncSetAttribute(topk_select_kernel<true>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    rc = ensure_smem_attr(reinterpret_cast<const void*>(topk_select_kernel<true>), (int)smem);
     if (rc) return rc;
     topk_select_kernel<true><<<grid, kThreads, smem, s>>>(n_docs, k, p.seg_len, scores, idx,
                                                            top_scores, cand);
@@ -284,9 +312,9 @@ extern "C" int msa_topk_docs(int B, int n_docs, int k, const float* scores, int3
   const int n_cand = p.n_seg * k;
   int P = 1;
   while (P < n_cand) P <<= 1;
-  const size_t smem = (size_t)P * sizeof(unsigned long long);
-  rc = note_cuda(cudaFuncSetAttribute(topk_merge_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const size_t smem = (size_t)std::max(P, n_cand <= kRankMax ? n_cand + k : 0) *
+                      sizeof(unsigned long long);
+  rc = ensure_smem_attr(reinterpret_cast<const void*>(topk_merge_kernel), (int)smem);
   if (rc) return rc;
   topk_merge_kernel<<<B, kThreads, smem, s>>>(n_docs, k, n_cand, cand, scores, idx, top_scores);
   return check_launch();
