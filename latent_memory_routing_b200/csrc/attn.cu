@@ -224,6 +224,17 @@ __global__ void attn_combine_kernel(int Tq, int Hq, int D, int n_split,
   }
 }
 
+}  // namespace
+
+int attn_combine_bf16(int B, int T, int Hq, int D, int n_split, const float* part_o,
+                      const float2* part_ml, void* out, cudaStream_t s) {
+  attn_combine_kernel<__nv_bfloat16><<<(unsigned)((int64_t)B * Hq * T), 128, 0, s>>>(
+      T, Hq, D, n_split, part_o, part_ml, static_cast<__nv_bfloat16*>(out));
+  return check_launch();
+}
+
+namespace {
+
 template <typename T, int D>
 int launch_simt(int B, int Tq, int T_loc, int Hq, int H, const void* q, const void* k_mem,
                 const void* v_mem, const int32_t* mem_len, int m_cap, const void* k_loc,

@@ -12,7 +12,9 @@
 //   * rope_prep_kernel rotates Q (to pos0 + T_loc - T + i) and the local K
 //     (to pos0 + j) once per call into bf16 workspace copies, one launch,
 //     cos/sin per position built in shared memory (angles reduced in double).
-//   * attn_tc_kernel: one CTA per (128 query rows, KV head, batch).  GQA rows
+//   * attn_tc_kernel: one CTA per (128 query rows, KV head, batch, key split;
+//     up to 3 splits of the key tiles, merged by the split-KV combine
+//     kernel, when there are too few row tiles to fill the SMs).  GQA rows
 //     are packed as (token, head of the group): a TMA box of
 //     {64 d, G heads, 128/G tokens} lands as 128 rows of 128 B -- the Q tile
 //     of all G query heads sharing one KV head.  Key tiles of 128 rows come
@@ -20,14 +22,16 @@
 //     (up to the block's last visible key), each as K and V TMA boxes.
 //     - warp 0 (one lane): TMA producer, 2-stage K/V ring;
 //     - warp 1 (one lane): tcgen05.mma S = Q K^T (M=128, N=128 keys, K=D)
-//       into one of two TMEM buffers, and O_tile = P V (M=128, N=D, K=128
-//       keys, V read MN-major straight from its TMA tile) into a third; the
-//       S of tile j+1 is issued before the P V of tile j;
-//     - warps 2..5 (one thread per row): online softmax in fp32 -- masked
-//       row maximum, p = 2^(s - m) written as bf16 into a double-buffered
-//       shared P tile (128B-swizzled, the MMA's A operand), row sum -- and
-//       the running output O = O * 2^(m_old - m_new) + O_tile in registers,
-//       consuming tile j's O_tile after computing tile j+1's P.
+//       into one of two TMEM buffers, and O += P V (M=128, N=D, K=128 keys,
+//       V read MN-major straight from its TMA tile) into the TMEM output
+//       accumulator; the S of tile j+1 is issued before the P V of tile j;
+//     - warps 2..5 (one thread per row): online softmax in fp32 -- the
+//       tile's scores read once from TMEM, masked row maximum, p = 2^(s - m)
+//       (SFU ex2) written as bf16 into a double-buffered shared P tile
+//       (128B-swizzled, the MMA's A operand), row sum.  O accumulates in
+//       TMEM; a row rescales O and its sum only when its maximum grows by
+//       more than 2^8 (then p <= 256 meanwhile), which after the first tiles
+//       is rare.
 //   * Every mbarrier wait is bounded; a timeout records MSA_ERR_TIMEOUT and
 //     all roles finish their loops without waiting.
 #include <cudaTypedefs.h>
@@ -65,7 +69,7 @@ struct ACfg {
 
 struct AAux {
   uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
-      o_full, o_empty;
+      o_full;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -79,6 +83,29 @@ __device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t smem_addr, uint
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// 2^x by the SFU (ex2.approx, ~2 ulp); its result feeds a bf16 P tile.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -89,8 +116,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_km,
                const __grid_constant__ CUtensorMap tm_vm, const __grid_constant__ CUtensorMap tm_kl,
                const __grid_constant__ CUtensorMap tm_vl, int T, int T_loc, int Hq, int H, int G,
-               const int32_t* __restrict__ mem_len, int m_cap, float qscale,
-               __nv_bfloat16* __restrict__ out, int* __restrict__ status) {
+               const int32_t* __restrict__ mem_len, int m_cap, float qscale, int n_split,
+               __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
+               float2* __restrict__ part_ml, int* __restrict__ status) {
   using K = ACfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ AAux aux;
@@ -101,7 +129,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   unsigned char* sP = sKV + kStages * K::STAGE;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int mt = blockIdx.x / n_split, sp = blockIdx.x % n_split;
+  const int g = blockIdx.y, b = blockIdx.z;
   const int TQ = kRows / G;  // tokens per CTA
   const int tok0 = mt * TQ;
   const int n_tok = min(TQ, T - tok0);
@@ -109,7 +138,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int lim_max = T_loc - T + tok0 + n_tok - 1;  // last local key any row sees
   const int n_mt = (M + kKeys - 1) / kKeys;
   const int n_lt = (lim_max + 1 + kKeys - 1) / kKeys;
-  const int nt = n_mt + n_lt;
+  const int nt_all = n_mt + n_lt;
+  // this CTA's share [j_lo, j_hi) of the key tiles
+  const int j_lo = (int)((int64_t)sp * nt_all / n_split);
+  const int j_hi = (int)((int64_t)(sp + 1) * nt_all / n_split);
+  if (j_lo == j_hi) {  // nothing to attend: an empty partial (uniform exit)
+    for (int r = threadIdx.x; r < kRows; r += blockDim.x) {
+      if (r / G >= n_tok) continue;
+      const int64_t row_id = ((int64_t)b * Hq + g * G + r % G) * T + tok0 + r / G;
+      float* po = part_o + (row_id * n_split + sp) * D;
+      for (int d = 0; d < D; ++d) po[d] = 0.f;
+      part_ml[row_id * n_split + sp] = make_float2(-INFINITY, 0.f);
+    }
+    return;
+  }
+  const int nt = j_hi - j_lo;  // tiles j_lo + 0 .. j_lo + nt - 1
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&aux.q_full, 1);
@@ -123,7 +166,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_init(&aux.p_full[i], kSoftWarps);
     }
     tc::mbar_init(&aux.o_full, 1);
-    tc::mbar_init(&aux.o_empty, kSoftWarps);
     aux.abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -158,10 +200,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         unsigned char* k_dst = sKV + st * K::STAGE;
         unsigned char* v_dst = k_dst + K::K_BYTES;
         tc::mbar_arrive_expect_tx(&aux.kv_full[st], K::STAGE);
-        const bool mem = j < n_mt;
+        const int jj = j_lo + j;
+        const bool mem = jj < n_mt;
         const CUtensorMap* mk = mem ? &tm_km : &tm_kl;
         const CUtensorMap* mv = mem ? &tm_vm : &tm_vl;
-        const int row = mem ? b * m_cap + j * kKeys : b * T_loc + (j - n_mt) * kKeys;
+        const int row = mem ? b * m_cap + jj * kKeys : b * T_loc + (jj - n_mt) * kKeys;
 #pragma unroll
         for (int kb = 0; kb < K::KB; ++kb) {
           tc::tma_load_3d(k_dst + kb * kKeys * 128, mk, &aux.kv_full[st], kb * 64, g, row);
@@ -201,9 +244,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       };
       auto issue_pv = [&](int j) -> bool {
         const int st = j % kStages, pb = j & 1;
-        if (*abort_flag || !tc::mbar_wait(&aux.p_full[pb], (j >> 1) & 1) ||
-            !tc::mbar_wait(&aux.o_empty, (j & 1) ^ 1))
-          return false;
+        // P of tile j written (and any rescale of O done) by the softmax
+        if (*abort_flag || !tc::mbar_wait(&aux.p_full[pb], (j >> 1) & 1)) return false;
         tc::tc_fence_after();
         const uint32_t p0 = tc::smem_u32(sP + pb * K::P_BYTES);
         const uint32_t v0 = tc::smem_u32(sKV + st * K::STAGE + K::K_BYTES);
@@ -214,7 +256,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint32_t poff = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
           tc::mma_bf16_ss(tO, tc::sdesc_kmajor_sw128(p0 + poff),
                           sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kKeys * 128), K::IDESC_O,
-                          kk > 0 ? 1u : 0u);
+                          (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(&aux.o_full);
         tc::mma_commit(&aux.kv_empty[st]);
@@ -232,32 +274,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------- softmax
+    // One thread per query row.  O accumulates in TMEM across key tiles;
+    // the row's reference maximum m_run only moves when a tile's maximum
+    // exceeds it by more than 2^kRescaleLog2 -- then O (in TMEM) and l are
+    // rescaled once, after the previous P V has landed -- so p = 2^(s - m_run)
+    // stays <= 2^kRescaleLog2 and most tiles need no rescale at all.
+    constexpr float kRescaleLog2 = 8.f;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // this thread's query row (TMEM lane)
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const int tok = tok0 + r / G;
     const int lim = T_loc - T + tok;  // last visible local key
-    float m_run = -INFINITY, l_run = 0.f, alpha_prev = 1.f;
-    float o[D];
-#pragma unroll
-    for (int d = 0; d < D; ++d) o[d] = 0.f;
-    auto consume_o = [&](int j, float alpha) {
+    float m_run = -INFINITY, l_run = 0.f;
+    auto wait_o = [&](int j) {  // the P V of tile j has completed
       if (!*abort_flag && !tc::mbar_wait(&aux.o_full, j & 1)) {
         record_error(status, MSA_ERR_TIMEOUT);
         *abort_flag = 1;
       }
       tc::tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tc::tmem_ld32(tO + lane_addr + c * 32, v);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha, __uint_as_float(v[i]));
-      }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&aux.o_empty);
     };
     for (int j = 0; j < nt; ++j) {
       const int sb = j & 1;
@@ -267,34 +301,54 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       tc::tc_fence_after();
       // visible keys of this tile: memory rows < M, local rows <= lim
-      const bool mem = j < n_mt;
-      const int key0 = mem ? j * kKeys : (j - n_mt) * kKeys;
+      const int jj = j_lo + j;
+      const bool mem = jj < n_mt;
+      const int key0 = mem ? jj * kKeys : (jj - n_mt) * kKeys;
       const int n_vis = mem ? min(kKeys, M - key0) : max(0, min(kKeys, lim - key0 + 1));
-      float mt = -INFINITY;
+      uint32_t sv[kKeys];
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        uint32_t v[32];
-        tc::tmem_ld32(tS[sb] + lane_addr + c * 32, v);
-        tc::tmem_ld_wait();
+      for (int c = 0; c < kKeys / 32; ++c)
+        tc::tmem_ld32(tS[sb] + lane_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
+      tc::tmem_ld_wait();
+      float mraw = -INFINITY;  // raw (unscaled) maximum of the visible scores
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (c * 32 + i < n_vis) mt = fmaxf(mt, __uint_as_float(v[i]) * qscale);
+      for (int i = 0; i < kKeys; ++i)
+        if (i < n_vis) mraw = fmaxf(mraw, __uint_as_float(sv[i]));
+      const float mt = mraw * qscale;  // qscale > 0 keeps the order
+      // rows whose maximum grew too much rescale O and l (warp-collective)
+      const bool grow = mt > m_run + kRescaleLog2;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = m_run == -INFINITY ? 0.f : ex2_approx(m_run - mt);
+        m_run = mt;
       }
-      const float m_new = fmaxf(m_run, mt);
-      const float alpha = m_new == -INFINITY ? 1.f : exp2f(m_run - m_new);
-      float ls = 0.f;
+      if (__any_sync(0xffffffffu, grow && alpha != 0.f) && j > 0) {
+        wait_o(j - 1);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tc::tmem_ld32(tO + lane_addr + c * 32, v);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+          tmem_st32(tO + lane_addr + c * 32, v);
+        }
+        tmem_st_wait();
+      }
+      l_run *= alpha;
+      // p = 2^(s*qscale - m_run) as bf16 into the swizzled P tile
       unsigned char* prow = sP + sb * K::P_BYTES + r * 128;
+      const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+      float ls = 0.f;
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) {
-        uint32_t v[32];
-        tc::tmem_ld32(tS[sb] + lane_addr + c * 32, v);
-        tc::tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = (c * 32 + i < n_vis) ? exp2f(__uint_as_float(v[i]) * qscale - m_new) : 0.f;
+          const int k0 = c * 32 + i;
+          const float p0 = k0 < n_vis ? ex2_approx(fmaf(__uint_as_float(sv[k0]), qscale, neg_m)) : 0.f;
           const float p1 =
-              (c * 32 + i + 1 < n_vis) ? exp2f(__uint_as_float(v[i + 1]) * qscale - m_new) : 0.f;
+              k0 + 1 < n_vis ? ex2_approx(fmaf(__uint_as_float(sv[k0 + 1]), qscale, neg_m)) : 0.f;
           ls += p0 + p1;
           w[i / 2] = pack_bf16(p0, p1);
         }
@@ -307,8 +361,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
       }
-      l_run = l_run * alpha + ls;
-      m_run = m_new;
+      l_run += ls;
       if (mem && M - key0 < kKeys && r >= M - key0) {
         // rows past mem_len in the last memory tile hold whatever the
         // caller's buffer holds there; zero their V so that 0 * V stays 0
@@ -326,23 +379,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::mbar_arrive(&aux.p_full[sb]);
         tc::mbar_arrive(&aux.s_empty[sb]);
       }
-      if (j > 0) consume_o(j - 1, alpha_prev);
-      alpha_prev = alpha;
     }
-    if (nt > 0) consume_o(nt - 1, alpha_prev);
-    // normalise and store this row (token tok, head g*G + r%G)
-    if (r / G < n_tok) {
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      __nv_bfloat16* op = out + (((int64_t)b * T + tok) * Hq + g * G + r % G) * D;
+    // the last P V, then this row's output.  s_full of tile nt-1 implied
+    // that P V nt-3 had completed; wait for nt-2 and nt-1 in turn, so that
+    // each parity wait is at most one phase behind.
+    if (nt >= 2) wait_o(nt - 2);
+    wait_o(nt - 1);
+    const bool row_ok = r / G < n_tok;
+    const int64_t row_id = ((int64_t)b * Hq + g * G + r % G) * T + tok;
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
-      for (int d = 0; d < D; d += 8) {
-        const uint4 pk = make_uint4(pack_bf16(o[d] * inv, o[d + 1] * inv),
-                                    pack_bf16(o[d + 2] * inv, o[d + 3] * inv),
-                                    pack_bf16(o[d + 4] * inv, o[d + 5] * inv),
-                                    pack_bf16(o[d + 6] * inv, o[d + 7] * inv));
-        *reinterpret_cast<uint4*>(op + d) = pk;
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t v[32];
+      tc::tmem_ld32(tO + lane_addr + c * 32, v);
+      tc::tmem_ld_wait();
+      if (!row_ok) continue;
+      if (n_split > 1) {
+        float* po = part_o + (row_id * n_split + sp) * D + c * 32;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(po + i) =
+              make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                          __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+      } else {
+        __nv_bfloat16* op = out + (((int64_t)b * T + tok) * Hq + g * G + r % G) * D + c * 32;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          *reinterpret_cast<uint4*>(op + i) = make_uint4(
+              pack_bf16(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv),
+              pack_bf16(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv),
+              pack_bf16(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
+              pack_bf16(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
       }
     }
+    if (row_ok && n_split > 1) part_ml[row_id * n_split + sp] = make_float2(m_run, l_run);
   }
 
   tc::tc_fence_before();
@@ -447,15 +517,29 @@ bool map3(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int b
 }
 
 struct TcPlan {
-  size_t cs_bytes, q_bytes, k_bytes, total;
+  int n_split;
+  size_t q_bytes, k_bytes, po_bytes, ml_bytes, total;
 };
 
-TcPlan tc_plan(int B, int T, int T_loc, int Hq, int H, int D) {
+// Key-tile splits: enough CTAs to cover the SMs twice, at most 3 (each split
+// re-reads the query tile and writes an fp32 partial) and at most the
+// number of key tiles.
+TcPlan tc_plan(int B, int T, int T_loc, int Hq, int H, int D, int m_cap) {
   TcPlan p{};
-  p.cs_bytes = 0;
+  const int G = Hq / H;
+  const int TQ = kRows / G;
+  const int64_t base = (int64_t)((T + TQ - 1) / TQ) * H * B;
+  const int64_t max_tiles = (m_cap + kKeys - 1) / kKeys + (T_loc + kKeys - 1) / kKeys;
+  int64_t ns = (2LL * num_sms() + base - 1) / base;
+  ns = std::min<int64_t>(ns, 3);
+  ns = std::min<int64_t>(ns, max_tiles);
+  p.n_split = (int)std::max<int64_t>(ns, 1);
   p.q_bytes = round_up((size_t)B * T * Hq * D * 2, 256);
   p.k_bytes = round_up((size_t)B * T_loc * H * D * 2, 256);
-  p.total = p.cs_bytes + p.q_bytes + p.k_bytes;
+  const size_t rows = (size_t)B * Hq * T;
+  p.po_bytes = p.n_split > 1 ? round_up(rows * p.n_split * D * sizeof(float), 256) : 0;
+  p.ml_bytes = p.n_split > 1 ? round_up(rows * p.n_split * sizeof(float2), 256) : 0;
+  p.total = p.q_bytes + p.k_bytes + p.po_bytes + p.ml_bytes;
   return p;
 }
 
@@ -466,10 +550,12 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
               cudaStream_t s) {
   using K = ACfg<D>;
   const int G = Hq / H;
-  const TcPlan p = tc_plan(B, T, T_loc, Hq, H, D);
+  const TcPlan p = tc_plan(B, T, T_loc, Hq, H, D, m_cap);
   unsigned char* w = static_cast<unsigned char*>(ws);
-  __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(w + p.cs_bytes);
-  __nv_bfloat16* k_rot = reinterpret_cast<__nv_bfloat16*>(w + p.cs_bytes + p.q_bytes);
+  __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(w);
+  __nv_bfloat16* k_rot = reinterpret_cast<__nv_bfloat16*>(w + p.q_bytes);
+  float* part_o = reinterpret_cast<float*>(w + p.q_bytes + p.k_bytes);
+  float2* part_ml = reinterpret_cast<float2*>(w + p.q_bytes + p.k_bytes + p.po_bytes);
   rope_prep_kernel<D><<<(unsigned)((T_loc + kPosPerCta - 1) / kPosPerCta), 256, 0, s>>>(
       B, T, T_loc, Hq, H, pos0, (double)rope_base, static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k_loc), q_rot, k_rot);
@@ -490,11 +576,13 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   auto kern = attn_tc_kernel<D>;
   rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
-  const dim3 grid((unsigned)((T + TQ - 1) / TQ), (unsigned)H, (unsigned)B);
+  const dim3 grid((unsigned)((T + TQ - 1) / TQ * p.n_split), (unsigned)H, (unsigned)B);
   kern<<<grid, kThreads, K::SMEM, s>>>(tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G, mem_len,
-                                       m_cap, qscale, static_cast<__nv_bfloat16*>(out),
-                                       device_status_ptr());
-  return check_launch();
+                                       m_cap, qscale, p.n_split, static_cast<__nv_bfloat16*>(out),
+                                       part_o, part_ml, device_status_ptr());
+  rc = check_launch();
+  if (rc || p.n_split == 1) return rc;
+  return attn_combine_bf16(B, T, Hq, D, p.n_split, part_o, part_ml, out, s);
 }
 
 }  // namespace
@@ -509,8 +597,8 @@ bool attn_tc_supported(int B, int T, int T_loc, int Hq, int H, int D, int m_cap)
   return true;
 }
 
-size_t attn_tc_workspace_size(int B, int T, int T_loc, int Hq, int H, int D, int) {
-  return tc_plan(B, T, T_loc, Hq, H, D).total;
+size_t attn_tc_workspace_size(int B, int T, int T_loc, int Hq, int H, int D, int m_cap) {
+  return tc_plan(B, T, T_loc, Hq, H, D, m_cap).total;
 }
 
 int attn_tc_launch(int B, int T, int T_loc, int Hq, int H, int D, const void* q,

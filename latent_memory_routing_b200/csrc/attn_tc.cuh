@@ -15,4 +15,9 @@ int attn_tc_launch(int B, int T, int T_loc, int Hq, int H, int D, const void* q,
                    const void* k_loc, const void* v_loc, int pos0, float rope_base, float qscale,
                    void* out, void* ws, cudaStream_t s);
 
+// Merges n_split partial results (unnormalised O in fp32, (max, sum) in the
+// base-2 exponent domain) of each (query, head, token) row into bf16 out.
+int attn_combine_bf16(int B, int T, int Hq, int D, int n_split, const float* part_o,
+                      const float2* part_ml, void* out, cudaStream_t s);
+
 }  // namespace msa
