@@ -10,8 +10,10 @@
 // keep their document-wise rotation and are visible to every query token;
 // local keys are causal; softmax scale 1/sqrt(D).
 //
-// This file holds the CUDA-core path (every fp32 call, bf16 decode and the
-// bf16 shapes the tensor-core prefill does not take): a split-KV flash
+// This file holds the CUDA-core path for every fp32 call and the bf16 shapes
+// the tensor-core prefill (attn_tc.cu) and the decode kernel
+// (attn_decode.cu) do not take, and the entry point that picks among them
+// by shape: a split-KV flash
 // kernel -- one CTA per (query block, KV head, key split), 32-key tiles
 // staged in shared memory in fp32 with local keys rotated on the way in,
 // online softmax in fp32 per query row -- and the kernel that merges the
@@ -260,6 +262,8 @@ extern "C" size_t msa_sparse_attn_workspace_size(msa_dtype dt, int B, int T, int
                                                  int H, int D, int m_cap) {
   using namespace msa;
   if (B <= 0 || T <= 0 || T_loc < T || H <= 0 || Hq % H || D <= 0 || m_cap < 0) return 0;
+  if (dt == MSA_BF16 && attn_decode_supported(T, Hq, H, D))
+    return std::max<size_t>(attn_decode_workspace_size(B, T_loc, Hq, H, D, m_cap), 256);
   if (dt == MSA_BF16 && attn_tc_supported(B, T, T_loc, Hq, H, D, m_cap))
     return attn_tc_workspace_size(B, T, T_loc, Hq, H, D, m_cap);
   return plan(B, T, T_loc, Hq, H, D, m_cap, num_sms()).total;
@@ -282,6 +286,12 @@ extern "C" int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
   const float qscale = sc * kLog2e;
+  if (dt == MSA_BF16 && attn_decode_supported(T, Hq, H, D)) {
+    const size_t need = attn_decode_workspace_size(B, T_loc, Hq, H, D, m_cap);
+    if (need && (!ws || ws_bytes < need || !aligned16(ws))) return MSA_ERR_WORKSPACE;
+    return attn_decode_launch(B, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc,
+                              pos0, rope_base, qscale, out, ws, s);
+  }
   if (dt == MSA_BF16 && attn_tc_supported(B, T, T_loc, Hq, H, D, m_cap)) {
     const size_t need = attn_tc_workspace_size(B, T, T_loc, Hq, H, D, m_cap);
     if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;

@@ -15,6 +15,14 @@ int attn_tc_launch(int B, int T, int T_loc, int Hq, int H, int D, const void* q,
                    const void* k_loc, const void* v_loc, int pos0, float rope_base, float qscale,
                    void* out, void* ws, cudaStream_t s);
 
+// bf16 decode (T = 1) on the CUDA cores, streaming K/V once (attn_decode.cu).
+bool attn_decode_supported(int T, int Hq, int H, int D);
+size_t attn_decode_workspace_size(int B, int T_loc, int Hq, int H, int D, int m_cap);
+int attn_decode_launch(int B, int T_loc, int Hq, int H, int D, const void* q, const void* k_mem,
+                       const void* v_mem, const int32_t* mem_len, int m_cap, const void* k_loc,
+                       const void* v_loc, int pos0, float rope_base, float qscale, void* out,
+                       void* ws, cudaStream_t s);
+
 // Merges n_split partial results (unnormalised O in fp32, (max, sum) in the
 // base-2 exponent domain) of each (query, head, token) row into bf16 out.
 int attn_combine_bf16(int B, int T, int Hq, int D, int n_split, const float* part_o,
