@@ -330,7 +330,97 @@ def run_libmsa(args, world, rank, local):
     }
     if args.cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, p, C)
+    if args.extra and world == 1:
+        del p, w
+        torch.cuda.empty_cache()
+        line["workloads"] = {"encode_4l": bench_encode(max(args.steps // 4, 3), pk["hbm"]),
+                             "bank_10m_decode": bench_decode(args.steps, pk["hbm"])}
     return line
+
+
+def time_device(fn, steps: int) -> float:
+    """Mean device milliseconds per call over `steps` back-to-back calls
+    (CUDA events on the launching stream, after warm-up)."""
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def bench_encode(steps: int, peak_hbm: float) -> dict:
+    """4 routed layers x 1M tokens: doc-wise RoPE + 64-token chunk means."""
+    import torch
+
+    from latent_memory_routing_b200 import pipeline, synth
+    w = synth.encode_4l("cuda")
+    toff = w["tok_offsets"].cuda()
+    coff = pipeline.chunk_offsets(toff)
+    C = int(coff[-1])
+    L, N, H, D = w["k_tok"].shape
+    out = tuple(torch.empty((L, C, H, D), dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    ms = time_device(lambda: pipeline.encode_pool(w["k_tok"], w["v_tok"], w["kr_tok"], toff,
+                                                  coff, C, out=out), steps)
+    algo = 3 * L * N * H * D * 2 + 3 * L * C * H * D * 2
+    gbs = algo / (ms * 1e-3) / 1e9
+    res = {"workload": "encode_4l: 4 layers x 1,000,000 tokens, docs U[100,4000], K/V/K_r "
+                       "bf16 [4][1M][8][128] -> pooled [4][C][8][128]",
+           "ms": round(ms, 4), "token_layers_per_s": round(L * N / (ms * 1e-3), 1),
+           "n_chunks_per_layer": C, "algorithmic_bytes": algo,
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_hbm,
+                        "unit": "GB/s", "frac": round(gbs / peak_hbm, 4)}}
+    del w, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode(steps: int, peak_hbm: float) -> dict:
+    """10M-token bank, 64 single-token decode queries: route (prepared bank)
+    -> top-16 -> gather -> decode attention over memory + 2,048 local tokens."""
+    import torch
+
+    from latent_memory_routing_b200 import pipeline, synth
+    lengths = synth.bank_10m_lengths()
+    toff = synth.tok_offsets(lengths).cuda()
+    coff = pipeline.chunk_offsets(toff)
+    coff_h = coff.cpu()
+    w = synth.bank_10m(coff_h, "cuda")
+    C = int(coff_h[-1])
+    m_cap = w["k"] * int((coff_h[1:] - coff_h[:-1]).max())
+    hat = pipeline.prepare_bank(w["kr_bar"])
+    p = pipeline.Pipeline(hat, w["k_bar"], w["v_bar"], coff, B=w["B"], T=1, T_loc=w["T_loc"],
+                          Hq=w["Hq"], k=w["k"], m_cap=m_cap, pos0=w["pos0"], prepared=True)
+    p(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    graph = p.capture(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    ms = time_device(graph.replay, steps)
+    ms_route = time_device(lambda: p.router(w["q_r"], p.kr_bar, p.coff, p.n_docs,
+                                            p.doc_scores, None), steps)
+    ms_attn = time_device(lambda: p.attn(w["q"], p.k_mem, p.v_mem, p.mem_len, w["k_loc"],
+                                         w["v_loc"], p.pos0, p.rope_base, 0.0, p.out), steps)
+    H, D = p.H, p.D
+    rows = int(p.mem_len.sum()) + w["B"] * w["T_loc"]
+    attn_bytes = rows * H * D * 2 * 2 + 2 * w["q"].numel() * 2
+    gbs = attn_bytes / (ms_attn * 1e-3) / 1e9
+    res = {"workload": "bank_10m: 10,000 docs, lengths LogNormal(ln 800, 0.65) in [64, 8192], "
+                       "pooled bf16 bank; 64 single-token decode queries, 2,048 local tokens, top-16",
+           "ms_per_step": round(ms, 4), "decode_tok_s": round(w["B"] / (ms * 1e-3), 1),
+           "route_ms": round(ms_route, 4),
+           "route_gchunks_s": round(C / (ms_route * 1e-3) / 1e9, 4),
+           "route_hbm_frac": round(C * BYTES_PER_CHUNK / (ms_route * 1e-3) / 1e9 / peak_hbm, 4),
+           "attn_ms": round(ms_attn, 4),
+           "attn_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_hbm,
+                             "unit": "GB/s", "frac": round(gbs / peak_hbm, 4)},
+           "n_chunks": C}
+    del w, p, graph, hat
+    torch.cuda.empty_cache()
+    return res
 
 
 def attn_flops_per_step(p) -> float:
@@ -439,6 +529,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-extra", dest="extra", action="store_false",
+                    help="skip the encode and decode workloads reported beside the step")
     ap.add_argument("--n-docs", type=int, default=100000,
                     help="documents in the bank (fewer only to profile a small case)")
     args = ap.parse_args()

@@ -10,17 +10,20 @@
 //
 // Design (HBM-bound: every K/V byte is read once).  One CTA of 128 threads
 // per (key split, batch element, KV head), serving the G query heads that
-// share the KV head:
-//   * 64-key tiles of K and V are streamed with 16-byte cp.async into a
-//     2-stage shared ring (64 KB + 32 KB of RoPE state: two CTAs per SM);
-//   * two threads per key row each own half of the rotate-half pairs; a
-//     local row is rotated in registers with (cos, sin) of its position held
-//     in shared memory for the tile's 64 rows -- anchored exactly (angles
-//     reduced in double) at the CTA's first local tile and advanced by one
-//     complex multiply per tile (the rows move 64 positions), so drift stays
-//     at a few 1e-7 over a split -- then dotted with the G rotated queries;
-//   * one warp per query head runs the online softmax over the tile and
-//     accumulates O (4 dims per lane) from the V tile;
+// share the KV head; about 40 KB of shared memory, so four CTAs per SM:
+//   * 32-key tiles of K and V stream with 16-byte cp.async through a 3-stage
+//     shared ring;
+//   * four threads per key row, each owning 16 of the 64 rotate-half pairs.
+//     A local row is rotated in registers with the (cos, sin) of its
+//     position, also in registers: computed exactly (angle reduced in double)
+//     at the CTA's first tile holding a local row, then advanced by one
+//     complex multiply per tile (the row moves 32 positions), so the drift
+//     over a split stays at a few 1e-7.  The rotated quarter-row is dotted
+//     with the G rotated queries (shared memory) and the four partial dots
+//     are summed with two shuffles;
+//   * one warp per query head runs the online softmax over the tile's 32
+//     scores (one per lane) and accumulates O, 4 dims per lane, from the V
+//     tile with packed fp32 FMAs;
 //   * splits write (max, sum, O) partials that the split-KV combine kernel
 //     merges; a single split writes the normalised output directly.
 #include <algorithm>
@@ -32,8 +35,8 @@ namespace msa {
 namespace {
 
 constexpr int kDThreads = 128;
-constexpr int kDKeys = 64;  // keys per tile
-constexpr int kDStages = 2;
+constexpr int kDKeys = 32;   // keys per tile
+constexpr int kDStages = 3;
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -55,8 +58,17 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
+// o += p * (lo, hi) on a packed fp32 pair.
+__device__ __forceinline__ void fma2(unsigned long long& o, unsigned long long p2,
+                                     unsigned long long v2) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(o) : "l"(p2), "l"(v2));
+}
+__device__ __forceinline__ unsigned long long bf2_to_f2(uint32_t w) {
+  return ((unsigned long long)(w & 0xffff0000u) << 32) | (unsigned long long)(w << 16);
+}
+
 template <int D, int G>
-__global__ void __launch_bounds__(kDThreads, 2)
+__global__ void __launch_bounds__(kDThreads, 4)
 attn_decode_kernel(int T_loc, int Hq, int H, const __nv_bfloat16* __restrict__ q,
                    const __nv_bfloat16* __restrict__ k_mem,
                    const __nv_bfloat16* __restrict__ v_mem, const int32_t* __restrict__ mem_len,
@@ -64,19 +76,17 @@ attn_decode_kernel(int T_loc, int Hq, int H, const __nv_bfloat16* __restrict__ q
                    const __nv_bfloat16* __restrict__ v_loc, int64_t pos0, double base,
                    float qscale, int n_split, __nv_bfloat16* __restrict__ out,
                    float* __restrict__ part_o, float2* __restrict__ part_ml) {
+  static_assert(D == 128, "four output dims per lane, 16 pairs per thread");
   constexpr int HALF = D / 2;
-  constexpr int QP = HALF / 2;            // pairs per thread (two threads per row)
-  constexpr int ROW_B = D * 2;            // bytes per K/V row
-  constexpr int VPL = D / 32;             // output dims per lane
-  extern __shared__ __align__(16) unsigned char smem[];
-  unsigned char* sK = smem;                                        // [stage][64][D] bf16
-  unsigned char* sV = sK + kDStages * kDKeys * ROW_B;              // [stage][64][D] bf16
-  float2* cs = reinterpret_cast<float2*>(sV + kDStages * kDKeys * ROW_B);  // [64][HALF]
-  static_assert(D == 128, "four output dims per lane");
-  __shared__ float2 step[HALF];                   // e^{i 64 w_i}
-  __shared__ __align__(16) float qs[G][D];        // rotated, scaled queries
-  __shared__ float sc[G][kDKeys];                 // tile scores, then probabilities
-  __shared__ double wf[HALF];                     // inverse frequencies
+  constexpr int QP = 16;       // pairs per thread (four threads per row)
+  constexpr int ROW_B = D * 2;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  unsigned char* sK = dsm;                                 // [stage][32 rows][D] bf16
+  unsigned char* sV = dsm + kDStages * kDKeys * ROW_B;     // [stage][32 rows][D] bf16
+  __shared__ __align__(16) float qs[G][D];   // rotated, scaled queries
+  __shared__ float sc[G][kDKeys];            // tile scores
+  __shared__ double wf[HALF];                // inverse frequencies
+  __shared__ float2 stepw[HALF];             // e^{i 32 w_i}: one tile forward
 
   const int split = blockIdx.x;
   const int b = blockIdx.y / H, g = blockIdx.y % H;
@@ -87,7 +97,10 @@ attn_decode_kernel(int T_loc, int Hq, int H, const __nv_bfloat16* __restrict__ q
   const int k_lo = min(n_keys, split * per), k_hi = min(n_keys, k_lo + per);
   const int n_tiles = (k_hi - k_lo + kDKeys - 1) / kDKeys;
 
-  for (int i = tid; i < HALF; i += kDThreads) wf[i] = rope_inv_freq(base, i, D);
+  for (int i = tid; i < HALF; i += kDThreads) {
+    wf[i] = rope_inv_freq(base, i, D);
+    stepw[i] = rope_cs(kDKeys, wf[i]);
+  }
   __syncthreads();
   // queries of the group, rotated to pos0 + T_loc - 1 and scaled
   for (int e = tid; e < G * HALF; e += kDThreads) {
@@ -98,7 +111,6 @@ attn_decode_kernel(int T_loc, int Hq, int H, const __nv_bfloat16* __restrict__ q
     qs[h][i] = (x1 * c.x - x2 * c.y) * qscale;
     qs[h][i + HALF] = (x2 * c.x + x1 * c.y) * qscale;
   }
-  for (int i = tid; i < HALF; i += kDThreads) step[i] = rope_cs(kDKeys, wf[i]);
 
   auto load_tile = [&](int t, int st) {
     const int key0 = k_lo + t * kDKeys;
@@ -128,152 +140,165 @@ attn_decode_kernel(int T_loc, int Hq, int H, const __nv_bfloat16* __restrict__ q
     cp_async_commit();
   };
 
-  // running softmax state: warp w owns heads w, w+4, ...
-  constexpr int HPW = (G + 3) / 4;
-  float m_run[HPW], l_run[HPW], o[HPW][VPL];
+  constexpr int HPW = (G + 3) / 4;  // heads per warp in the softmax
+  float m_run[HPW], l_run[HPW];
+  unsigned long long o2[HPW][2];    // 4 output dims per lane, packed pairs
 #pragma unroll
   for (int a = 0; a < HPW; ++a) {
     m_run[a] = -INFINITY;
     l_run[a] = 0.f;
-#pragma unroll
-    for (int x = 0; x < VPL; ++x) o[a][x] = 0.f;
+    o2[a][0] = o2[a][1] = 0ull;
   }
 
-  const int row = tid >> 1, hp = tid & 1;  // key row and pair half of this thread
-  bool cs_ready = false;
-  if (n_tiles > 0) load_tile(0, 0);
+  const int row = tid >> 2, qq = tid & 3;  // key row and pair quarter
+  const int i0 = qq * QP;                  // first pair of this thread
+  float cr[QP], sr[QP];                    // rotation of this row
+  bool anchored = false;
+#pragma unroll
+  for (int e = 0; e < QP; ++e) {
+    cr[e] = 1.f;
+    sr[e] = 0.f;
+  }
+  __syncthreads();
+
+#pragma unroll 1
+  for (int t = 0; t < kDStages - 1; ++t)
+    if (t < n_tiles) load_tile(t, t);
+    else cp_async_commit();
+
+#pragma unroll 1
   for (int t = 0; t < n_tiles; ++t) {
-    const int st = t & 1;
+    const int st = t % kDStages;
     const int key0 = k_lo + t * kDKeys;
-    if (t + 1 < n_tiles) {
-      load_tile(t + 1, st ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    // (cos, sin) of this tile's rows: anchored at the first tile holding a
-    // local row, then advanced by 64 positions per tile
-    const bool any_local = key0 + kDKeys > M;
-    if (any_local && !cs_ready) {
-      for (int e = tid; e < kDKeys * HALF; e += kDThreads) {
-        const int r = e / HALF, i = e % HALF;
-        cs[e] = rope_cs(pos0 + (int64_t)(key0 + r - M), wf[i]);
-      }
-      cs_ready = true;
-    } else if (any_local) {
-      for (int e = tid; e < kDKeys * HALF; e += kDThreads) {
-        const float2 a = cs[e], w = step[e % HALF];
-        cs[e] = make_float2(a.x * w.x - a.y * w.y, a.x * w.y + a.y * w.x);
-      }
-    }
+    if (t + kDStages - 1 < n_tiles) load_tile(t + kDStages - 1, (t + kDStages - 1) % kDStages);
+    else cp_async_commit();
+    cp_async_wait<kDStages - 1>();
     __syncthreads();
 
-    // scores of (row, head) -- two threads per row, HALF/2 pairs each
+    // this row's rotation: exact at the first tile holding a local row, then
+    // one complex multiply per tile
+    const bool tile_local = key0 + kDKeys > M;
+    if (tile_local) {
+      if (!anchored) {
+        const int64_t p = pos0 + (int64_t)(key0 + row - M);
+#pragma unroll
+        for (int e = 0; e < QP; ++e) {
+          const float2 c = rope_cs(p, wf[i0 + e]);
+          cr[e] = c.x;
+          sr[e] = c.y;
+        }
+        anchored = true;
+      } else {
+#pragma unroll
+        for (int e = 0; e < QP; ++e) {
+          const float2 w = stepw[i0 + e];
+          const float c = cr[e] * w.x - sr[e] * w.y;
+          sr[e] = cr[e] * w.y + sr[e] * w.x;
+          cr[e] = c;
+        }
+      }
+    }
+
+    // partial dot of this quarter-row with each query head
     {
       const unsigned char* kr = sK + (st * kDKeys + row) * ROW_B;
-      const bool local = key0 + row >= M;
-      float acc[G];
+      float x1[QP], x2[QP];
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = 0.f;
+      for (int v = 0; v < QP / 8; ++v) {
+        Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(kr + (i0 + 8 * v) * 2),
+                                     x1 + 8 * v);
+        Vec16<__nv_bfloat16>::unpack(
+            *reinterpret_cast<const uint4*>(kr + (i0 + 8 * v + HALF) * 2), x2 + 8 * v);
+      }
+      if (key0 + row >= M) {
 #pragma unroll
-      for (int v8 = 0; v8 < QP / 8; ++v8) {
-        const int i0 = hp * QP + v8 * 8;  // first pair index of this 8-group
-        float x1[8], x2[8];
-        Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(kr + i0 * 2), x1);
-        Vec16<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(kr + (i0 + HALF) * 2), x2);
-        if (local) {
-          const float2* c = cs + row * HALF + i0;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 w = c[e];
-            const float a = x1[e], bb = x2[e];
-            x1[e] = a * w.x - bb * w.y;
-            x2[e] = bb * w.x + a * w.y;
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float4 q1a = *reinterpret_cast<const float4*>(&qs[h][i0]);
-          const float4 q1b = *reinterpret_cast<const float4*>(&qs[h][i0 + 4]);
-          const float4 q2a = *reinterpret_cast<const float4*>(&qs[h][i0 + HALF]);
-          const float4 q2b = *reinterpret_cast<const float4*>(&qs[h][i0 + HALF + 4]);
-          float s = acc[h];
-          s = fmaf(q1a.x, x1[0], s); s = fmaf(q1a.y, x1[1], s);
-          s = fmaf(q1a.z, x1[2], s); s = fmaf(q1a.w, x1[3], s);
-          s = fmaf(q1b.x, x1[4], s); s = fmaf(q1b.y, x1[5], s);
-          s = fmaf(q1b.z, x1[6], s); s = fmaf(q1b.w, x1[7], s);
-          s = fmaf(q2a.x, x2[0], s); s = fmaf(q2a.y, x2[1], s);
-          s = fmaf(q2a.z, x2[2], s); s = fmaf(q2a.w, x2[3], s);
-          s = fmaf(q2b.x, x2[4], s); s = fmaf(q2b.y, x2[5], s);
-          s = fmaf(q2b.z, x2[6], s); s = fmaf(q2b.w, x2[7], s);
-          acc[h] = s;
+        for (int e = 0; e < QP; ++e) {
+          const float a = x1[e], bb = x2[e];
+          x1[e] = a * cr[e] - bb * sr[e];
+          x2[e] = bb * cr[e] + a * sr[e];
         }
       }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float s = acc[h] + __shfl_xor_sync(0xffffffffu, acc[h], 1);
-        if (hp == 0) sc[h][row] = key0 + row < k_hi ? s : -INFINITY;
+        float s = 0.f;
+#pragma unroll
+        for (int v = 0; v < QP / 4; ++v) {
+          const float4 a = *reinterpret_cast<const float4*>(&qs[h][i0 + 4 * v]);
+          const float4 c = *reinterpret_cast<const float4*>(&qs[h][i0 + 4 * v + HALF]);
+          s = fmaf(a.x, x1[4 * v], s);
+          s = fmaf(a.y, x1[4 * v + 1], s);
+          s = fmaf(a.z, x1[4 * v + 2], s);
+          s = fmaf(a.w, x1[4 * v + 3], s);
+          s = fmaf(c.x, x2[4 * v], s);
+          s = fmaf(c.y, x2[4 * v + 1], s);
+          s = fmaf(c.z, x2[4 * v + 2], s);
+          s = fmaf(c.w, x2[4 * v + 3], s);
+        }
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        if (qq == 0) sc[h][row] = key0 + row < k_hi ? s : -INFINITY;
       }
     }
     __syncthreads();
 
-    // softmax and P V: warp w handles heads w, w+4, ...
+    // softmax and P V: warp w handles heads w, w+4, ...; lane = key row
 #pragma unroll
     for (int a = 0; a < HPW; ++a) {
       const int h = warp + 4 * a;
       if (h >= G) break;
-      const float s0 = sc[h][lane], s1 = sc[h][lane + 32];
-      float mt = fmaxf(s0, s1);
+      const float s = sc[h][lane];
+      float mt = s;
 #pragma unroll
       for (int off = 16; off; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
       const float m_new = fmaxf(m_run[a], mt);
       if (m_new == -INFINITY) continue;  // warp-uniform: nothing visible yet
       const float alpha = ex2f(m_run[a] - m_new);
-      const float p0 = ex2f(s0 - m_new), p1 = ex2f(s1 - m_new);
-      float ps = p0 + p1;
+      const float p = ex2f(s - m_new);
+      float ps = p;
 #pragma unroll
       for (int off = 16; off; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
       l_run[a] = l_run[a] * alpha + ps;
       m_run[a] = m_new;
-      __syncwarp();
-      sc[h][lane] = p0;
-      sc[h][lane + 32] = p1;
-      __syncwarp();
-#pragma unroll
-      for (int x = 0; x < VPL; ++x) o[a][x] *= alpha;
-      const unsigned char* vt = sV + st * kDKeys * ROW_B + lane * VPL * 2;
+      const unsigned long long al2 =
+          ((unsigned long long)__float_as_uint(alpha) << 32) | __float_as_uint(alpha);
+      unsigned long long z = 0ull;
+      asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(o2[a][0]), "l"(al2));
+      o2[a][0] = z;
+      asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(o2[a][1]), "l"(al2));
+      o2[a][1] = z;
+      const unsigned char* vt = sV + st * kDKeys * ROW_B + lane * 8;
 #pragma unroll 8
       for (int r = 0; r < kDKeys; ++r) {
-        const float p = sc[h][r];
+        const float pr = __shfl_sync(0xffffffffu, p, r);
+        const unsigned long long p2 =
+            ((unsigned long long)__float_as_uint(pr) << 32) | __float_as_uint(pr);
         const uint2 w = *reinterpret_cast<const uint2*>(vt + r * ROW_B);
-        o[a][0] = fmaf(p, __uint_as_float(w.x << 16), o[a][0]);
-        o[a][1] = fmaf(p, __uint_as_float(w.x & 0xffff0000u), o[a][1]);
-        o[a][2] = fmaf(p, __uint_as_float(w.y << 16), o[a][2]);
-        o[a][3] = fmaf(p, __uint_as_float(w.y & 0xffff0000u), o[a][3]);
+        fma2(o2[a][0], p2, bf2_to_f2(w.x));
+        fma2(o2[a][1], p2, bf2_to_f2(w.y));
       }
     }
     __syncthreads();  // the stage and sc are rewritten next
   }
+  cp_async_wait<0>();
 
 #pragma unroll
   for (int a = 0; a < HPW; ++a) {
     const int h = warp + 4 * a;
     if (h >= G) break;
-    const int hq = g * G + h;
-    const int64_t row_id = (int64_t)b * Hq + hq;  // T == 1
+    const int64_t row_id = (int64_t)b * Hq + g * G + h;  // T == 1
+    const float o0 = __uint_as_float((uint32_t)o2[a][0]), o1 = __uint_as_float((uint32_t)(o2[a][0] >> 32));
+    const float o2v = __uint_as_float((uint32_t)o2[a][1]), o3 = __uint_as_float((uint32_t)(o2[a][1] >> 32));
     if (n_split == 1) {
       const float inv = l_run[a] > 0.f ? 1.f / l_run[a] : 0.f;
-      float f[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) f[x] = o[a][x] * inv;
-      __nv_bfloat162 lo = __floats2bfloat162_rn(f[0], f[1]), hi = __floats2bfloat162_rn(f[2], f[3]);
+      __nv_bfloat162 lo = __floats2bfloat162_rn(o0 * inv, o1 * inv);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(o2v * inv, o3 * inv);
       uint2 pk;
       pk.x = *reinterpret_cast<uint32_t*>(&lo);
       pk.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(out + row_id * D + lane * VPL) = pk;
+      *reinterpret_cast<uint2*>(out + row_id * D + lane * 4) = pk;
     } else {
-      float* po = part_o + (row_id * n_split + split) * D + lane * VPL;
-      *reinterpret_cast<float4*>(po) = make_float4(o[a][0], o[a][1], o[a][2], o[a][3]);
+      float* po = part_o + (row_id * n_split + split) * D + lane * 4;
+      *reinterpret_cast<float4*>(po) = make_float4(o0, o1, o2v, o3);
       if (lane == 0) part_ml[row_id * n_split + split] = make_float2(m_run[a], l_run[a]);
     }
   }
@@ -288,7 +313,7 @@ DecPlan dec_plan(int B, int Hq, int H, int D, int T_loc, int m_cap) {
   DecPlan p{};
   const int64_t base = (int64_t)B * H;
   const int64_t keys = (int64_t)m_cap + T_loc;
-  int64_t ns = (4LL * num_sms() + base - 1) / base;  // two resident CTAs per SM, twice over
+  int64_t ns = (8LL * num_sms() + base - 1) / base;  // four resident CTAs per SM, twice over
   ns = std::min<int64_t>(ns, std::max<int64_t>(1, keys / 256));
   ns = std::min<int64_t>(ns, 64);
   p.n_split = (int)std::max<int64_t>(ns, 1);
@@ -308,8 +333,8 @@ int launch_dec(int B, int T_loc, int Hq, int H, const void* q, const void* k_mem
   unsigned char* w = static_cast<unsigned char*>(ws);
   float* part_o = reinterpret_cast<float*>(w);
   float2* part_ml = reinterpret_cast<float2*>(w + p.po_bytes);
-  const size_t smem = (size_t)2 * kDStages * kDKeys * D * 2 + (size_t)kDKeys * (D / 2) * 8;
   auto kern = attn_decode_kernel<D, G>;
+  const size_t smem = (size_t)2 * kDStages * kDKeys * D * 2;
   int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem);
   if (rc) return rc;
   const dim3 grid((unsigned)p.n_split, (unsigned)(B * H));

@@ -73,7 +73,7 @@ constexpr int kBins = 2048;  // 11-bit digits: passes over bits 31..21, 20..10, 
 
 struct SelectShared {
   uint32_t hist[kBins];
-  uint32_t sel, above;
+  uint32_t sel, above, warp_tot[32];
   int n_gt, running, warp_cnt[32];
 };
 
@@ -103,24 +103,32 @@ __device__ void select_topk(const Keys& keys, int len, int kk, uint32_t base,
       if (act && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (warp == 0) {
-      // lane l owns digits [l*per, (l+1)*per); suffix sums from the top down
-      const int per = nb / 32;
+    {
+      // the whole block finds the digit: thread t owns bins [bpt*t, bpt*t+bpt);
+      // a block suffix sum (warp shuffles, then the 32 warp totals) gives
+      // the count above each thread's bins
+      const int bpt = (nb + blockDim.x - 1) / blockDim.x;
+      const int b0 = tid * bpt;
       uint32_t own = 0;
-      for (int j = 0; j < per; ++j) own += sh.hist[per * lane + j];
-      uint32_t suf = own;
+      for (int j = 0; j < bpt; ++j)
+        if (b0 + j < nb) own += sh.hist[b0 + j];
+      uint32_t suf = own;  // inclusive suffix sum over lanes >= lane
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const uint32_t o = __shfl_down_sync(0xffffffffu, suf, off);
         if (lane + off < 32) suf += o;
       }
-      const uint32_t above_lane = suf - own;
-      if (above_lane < (uint32_t)krem && suf >= (uint32_t)krem) {
-        uint32_t cum = above_lane;
-        for (int j = per - 1; j >= 0; --j) {
-          const uint32_t hj = sh.hist[per * lane + j];
+      if (lane == 0) sh.warp_tot[warp] = suf;
+      __syncthreads();
+      uint32_t above_warps = 0;
+      for (int w = warp + 1; w < (int)(blockDim.x >> 5); ++w) above_warps += sh.warp_tot[w];
+      const uint32_t above_me = above_warps + suf - own;  // count in bins above mine
+      if (above_me < (uint32_t)krem && above_me + own >= (uint32_t)krem) {
+        uint32_t cum = above_me;
+        for (int j = bpt - 1; j >= 0; --j) {
+          const uint32_t hj = b0 + j < nb ? sh.hist[b0 + j] : 0u;
           if (cum + hj >= (uint32_t)krem) {
-            sh.sel = per * lane + j;
+            sh.sel = b0 + j;
             sh.above = cum;
             break;
           }
