@@ -45,34 +45,55 @@
 namespace msa {
 namespace {
 
-constexpr int kRows = 128;   // query rows per CTA (MMA M)
+constexpr int kRows = 128;   // query rows per Q tile (MMA M)
+constexpr int kQT = 2;       // Q tiles per CTA, one softmax warpgroup each
 constexpr int kKeys = 128;   // keys per tile (MMA N of S, K of P V)
-constexpr int kSoftWarps = 4;
-constexpr int kThreads = 64 + 32 * kSoftWarps;
+constexpr int kSoftWarps = 4 * kQT;
+// warpgroup 0: TMA producer (warp 0), MMA issuer (warp 1), two idle warps;
+// warpgroups 1 .. kQT: softmax.  Registers move from warpgroup 0 to the
+// softmax warpgroups: 128 x kRegLow + 256 x kRegHigh = 384 x 168, the
+// block's launch allocation under __launch_bounds__(384, 1).
+constexpr int kThreads = 128 + 32 * kSoftWarps;
+constexpr int kRegLow = 56;
+constexpr int kRegHigh = 224;
+static_assert(kQT == 2 && 128 * kRegLow + 256 * kRegHigh == 384 * 168, "register split");
 constexpr int kStages = 2;
 
 template <int D>
 struct ACfg {
   static constexpr int KB = D / 64;
-  static constexpr int Q_BYTES = KB * kRows * 128;
+  static constexpr int Q_BYTES = KB * kRows * 128;   // one Q tile
   static constexpr int K_BYTES = KB * kKeys * 128;
   static constexpr int V_BYTES = KB * kKeys * 128;
   static constexpr int STAGE = K_BYTES + V_BYTES;
-  static constexpr int P_BYTES = 2 * kRows * 128;  // 128 keys x bf16 = 2 K blocks
-  static constexpr size_t SMEM = 1024 + Q_BYTES + kStages * STAGE + 2 * P_BYTES;
+  static constexpr size_t SMEM = 1024 + kQT * Q_BYTES + kStages * STAGE;
+  // TMEM: per Q tile an S tile (128 fp32 columns, whose first 64 columns
+  // then hold P as packed bf16) and an O tile (D fp32 columns)
   static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(kQT * (kKeys + D) <= 512, "TMEM budget");
   // S: M=128, N=128 keys, A (Q) and B (K) K-major
   static constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(kRows, kKeys);
-  // O: M=128, N=D, A (P) K-major, B (V) MN-major (bit 16)
+  // O: M=128, N=D, A (P, TMEM) K-major, B (V) MN-major (bit 16)
   static constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(kRows, D) | (1u << 16);
 };
 
 struct AAux {
-  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], p_full[2],
-      o_full;
+  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[kQT], p_full[kQT], o_full[kQT];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16; A is M x K bf16 in TMEM,
+// row m in lane m, elements 2c and 2c+1 of K packed in column c.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 // UMMA descriptor of an MN-major, 128B-swizzled operand whose MN extent is
 // split in 64-element (128 B) column blocks `lbo` bytes apart and whose K
@@ -124,16 +145,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __shared__ AAux aux;
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-  unsigned char* sQ = base;
-  unsigned char* sKV = sQ + K::Q_BYTES;
-  unsigned char* sP = sKV + kStages * K::STAGE;
+  unsigned char* sQ = base;                        // kQT Q tiles
+  unsigned char* sKV = sQ + kQT * K::Q_BYTES;      // kStages x (K tile, V tile)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mt = blockIdx.x / n_split, sp = blockIdx.x % n_split;
   const int g = blockIdx.y, b = blockIdx.z;
-  const int TQ = kRows / G;  // tokens per CTA
-  const int tok0 = mt * TQ;
-  const int n_tok = min(TQ, T - tok0);
+  const int TQ = kRows / G;          // tokens per Q tile
+  const int tok0 = mt * kQT * TQ;    // first token of the CTA
+  const int n_tok = min(kQT * TQ, T - tok0);
   const int M = min(max(mem_len[b], 0), m_cap);
   const int lim_max = T_loc - T + tok0 + n_tok - 1;  // last local key any row sees
   const int n_mt = (M + kKeys - 1) / kKeys;
@@ -143,7 +163,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int j_lo = (int)((int64_t)sp * nt_all / n_split);
   const int j_hi = (int)((int64_t)(sp + 1) * nt_all / n_split);
   if (j_lo == j_hi) {  // nothing to attend: an empty partial (uniform exit)
-    for (int r = threadIdx.x; r < kRows; r += blockDim.x) {
+    for (int r = threadIdx.x; r < kQT * kRows; r += blockDim.x) {
       if (r / G >= n_tok) continue;
       const int64_t row_id = ((int64_t)b * Hq + g * G + r % G) * T + tok0 + r / G;
       float* po = part_o + (row_id * n_split + sp) * D;
@@ -160,12 +180,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_init(&aux.kv_full[i], 1);
       tc::mbar_init(&aux.kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kQT; ++i) {
       tc::mbar_init(&aux.s_full[i], 1);
-      tc::mbar_init(&aux.s_empty[i], kSoftWarps);
-      tc::mbar_init(&aux.p_full[i], kSoftWarps);
+      tc::mbar_init(&aux.p_full[i], 4);
+      tc::mbar_init(&aux.o_full[i], 1);
     }
-    tc::mbar_init(&aux.o_full, 1);
     aux.abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -177,19 +196,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = aux.tmem_base;
-  const uint32_t tS[2] = {tmem, tmem + kKeys};
-  const uint32_t tO = tmem + 2 * kKeys;
+  // TMEM columns: S/P of tile i at i*kKeys, O of tile i at kQT*kKeys + i*D
   volatile int* abort_flag = &aux.abort_flag;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegLow));
+   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t issued = 0;
-      tc::mbar_arrive_expect_tx(&aux.q_full, K::Q_BYTES);
+      tc::mbar_arrive_expect_tx(&aux.q_full, kQT * K::Q_BYTES);
 #pragma unroll
-      for (int kb = 0; kb < K::KB; ++kb)
-        tc::tma_load_3d(sQ + kb * kRows * 128, &tm_q, &aux.q_full, kb * 64, g * G,
-                        b * T + tok0);
+      for (int i = 0; i < kQT; ++i)
+#pragma unroll
+        for (int kb = 0; kb < K::KB; ++kb)
+          tc::tma_load_3d(sQ + i * K::Q_BYTES + kb * kRows * 128, &tm_q, &aux.q_full, kb * 64,
+                          g * G, b * T + tok0 + i * TQ);
       for (int j = 0; j < nt; ++j) {
         const int st = j % kStages;
         if (*abort_flag || !tc::mbar_wait(&aux.kv_empty[st], ((j / kStages) & 1) ^ 1)) {
@@ -217,90 +239,88 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (uint32_t v = issued > (uint32_t)kStages ? issued - kStages : 0; v < issued; ++v)
         tc::mbar_wait(&aux.kv_full[v % kStages], (v / kStages) & 1);
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
+    // order: S_0(0) S_1(0) | P_0V(0) S_0(1) P_1V(0) S_1(1) | ... so each
+    // softmax warpgroup works while the tensor core serves the other one;
+    // S_i(j) is issued after P_iV(j-1), which makes the TMEM columns that
+    // held P_i(j-1) safe to overwrite and lets s_full_i(j) imply that
+    // P_iV(j-1) has completed.
     if (lane == 0) {
-      const uint32_t q0 = tc::smem_u32(sQ);
-      auto fail = [&]() {
-        record_error(status, MSA_ERR_TIMEOUT);
-        *abort_flag = 1;
-      };
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kStages, sb = j & 1;
-        if (*abort_flag || !tc::mbar_wait(&aux.kv_full[st], (j / kStages) & 1) ||
-            !tc::mbar_wait(&aux.s_empty[sb], ((j >> 1) & 1) ^ 1))
-          return false;
+      bool ok = tc::mbar_wait(&aux.q_full, 0);
+      auto issue_s = [&](int i, int j) -> bool {
+        const int st = j % kStages;
+        if (*abort_flag || !tc::mbar_wait(&aux.kv_full[st], (j / kStages) & 1)) return false;
+        // S_i(j) overwrites P_i(j-1); the P V that reads it was issued
+        // (after its p_full wait) before this MMA, and the tensor core runs
+        // one thread's MMAs in issue order
         tc::tc_fence_after();
+        const uint32_t q0 = tc::smem_u32(sQ + i * K::Q_BYTES);
         const uint32_t k0 = tc::smem_u32(sKV + st * K::STAGE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * (kKeys * 128) + (kk & 3) * 32;
-          tc::mma_bf16_ss(tS[sb], tc::sdesc_kmajor_sw128(q0 + off),
+          tc::mma_bf16_ss(tmem + i * kKeys, tc::sdesc_kmajor_sw128(q0 + off),
                           tc::sdesc_kmajor_sw128(k0 + koff), K::IDESC_S, kk > 0 ? 1u : 0u);
         }
-        tc::mma_commit(&aux.s_full[sb]);
+        tc::mma_commit(&aux.s_full[i]);
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j % kStages, pb = j & 1;
-        // P of tile j written (and any rescale of O done) by the softmax
-        if (*abort_flag || !tc::mbar_wait(&aux.p_full[pb], (j >> 1) & 1)) return false;
+      auto issue_pv = [&](int i, int j) -> bool {
+        const int st = j % kStages;
+        // P_i(j) written (and any rescale of O_i done) by softmax group i
+        if (*abort_flag || !tc::mbar_wait(&aux.p_full[i], j & 1)) return false;
         tc::tc_fence_after();
-        const uint32_t p0 = tc::smem_u32(sP + pb * K::P_BYTES);
         const uint32_t v0 = tc::smem_u32(sKV + st * K::STAGE + K::K_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          // A = P (rows x keys, K-major, 64-key blocks); B = V (keys x d,
-          // MN-major: 64-d column blocks 128*128 B apart, 16 keys = 2048 B)
-          const uint32_t poff = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
-          tc::mma_bf16_ss(tO, tc::sdesc_kmajor_sw128(p0 + poff),
-                          sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kKeys * 128), K::IDESC_O,
-                          (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc::mma_commit(&aux.o_full);
-        tc::mma_commit(&aux.kv_empty[st]);
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          mma_bf16_ts(tmem + kQT * kKeys + i * D, tmem + i * kKeys + kk * 8,
+                      sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kKeys * 128), K::IDESC_O,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        if (j == nt - 1) tc::mma_commit(&aux.o_full[i]);  // one phase: O_i final
+        if (i == kQT - 1) tc::mma_commit(&aux.kv_empty[st]);
         return true;
       };
-      if (!tc::mbar_wait(&aux.q_full, 0)) fail();
-      else if (nt > 0) {
-        bool ok = issue_s(0);
-        for (int j = 0; ok && j < nt; ++j) {
-          if (j + 1 < nt) ok = issue_s(j + 1);
-          if (ok) ok = issue_pv(j);
+      for (int i = 0; ok && i < kQT; ++i) ok = issue_s(i, 0);
+      for (int j = 0; ok && j < nt; ++j)
+        for (int i = 0; ok && i < kQT; ++i) {
+          ok = issue_pv(i, j);
+          if (ok && j + 1 < nt) ok = issue_s(i, j + 1);
         }
-        if (!ok) fail();
+      if (!ok) {
+        record_error(status, MSA_ERR_TIMEOUT);
+        *abort_flag = 1;
       }
     }
+   }
   } else {
     // ------------------------------------------------------------- softmax
-    // One thread per query row.  O accumulates in TMEM across key tiles;
-    // the row's reference maximum m_run only moves when a tile's maximum
-    // exceeds it by more than 2^kRescaleLog2 -- then O (in TMEM) and l are
-    // rescaled once, after the previous P V has landed -- so p = 2^(s - m_run)
-    // stays <= 2^kRescaleLog2 and most tiles need no rescale at all.
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegHigh));
+    // Warpgroup i owns Q tile i, one thread per query row.  O_i accumulates
+    // in TMEM; the row's reference maximum m_run only moves when a tile's
+    // maximum exceeds it by more than 2^kRescaleLog2 -- then O_i (in TMEM)
+    // and l are rescaled once (s_full_i(j) implies P_iV(j-1) is done) -- so
+    // p = 2^(s - m_run) stays <= 2^kRescaleLog2 and most tiles need no
+    // rescale.  P goes back into the S tile's first 64 TMEM columns as
+    // packed bf16, the A operand of the P V MMA.
     constexpr float kRescaleLog2 = 8.f;
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // this thread's query row (TMEM lane)
+    const int qt = (warp - 4) >> 2;   // Q tile of this warpgroup
+    const int quad = warp & 3;        // TMEM lane quarter
+    const int r = quad * 32 + lane;   // row within the Q tile
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const int tok = tok0 + r / G;
+    const uint32_t tSP = tmem + qt * kKeys + lane_addr;
+    const uint32_t tOi = tmem + kQT * kKeys + qt * D + lane_addr;
+    const int tok_local = qt * TQ + r / G;
+    const int tok = tok0 + tok_local;
     const int lim = T_loc - T + tok;  // last visible local key
     float m_run = -INFINITY, l_run = 0.f;
-    auto wait_o = [&](int j) {  // the P V of tile j has completed
-      if (!*abort_flag && !tc::mbar_wait(&aux.o_full, j & 1)) {
-        record_error(status, MSA_ERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      tc::tc_fence_after();
-    };
     for (int j = 0; j < nt; ++j) {
-      const int sb = j & 1;
-      if (!*abort_flag && !tc::mbar_wait(&aux.s_full[sb], (j >> 1) & 1)) {
+      if (!*abort_flag && !tc::mbar_wait(&aux.s_full[qt], j & 1)) {
         record_error(status, MSA_ERR_TIMEOUT);
         *abort_flag = 1;
       }
       tc::tc_fence_after();
-      // visible keys of this tile: memory rows < M, local rows <= lim
       const int jj = j_lo + j;
       const bool mem = jj < n_mt;
       const int key0 = mem ? jj * kKeys : (jj - n_mt) * kKeys;
@@ -308,14 +328,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       uint32_t sv[kKeys];
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c)
-        tc::tmem_ld32(tS[sb] + lane_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
+        tc::tmem_ld32(tSP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
       tc::tmem_ld_wait();
-      float mraw = -INFINITY;  // raw (unscaled) maximum of the visible scores
+      float mraw = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < kKeys; ++i)
-        if (i < n_vis) mraw = fmaxf(mraw, __uint_as_float(sv[i]));
+      for (int c = 0; c < kKeys; ++c)
+        if (c < n_vis) mraw = fmaxf(mraw, __uint_as_float(sv[c]));
       const float mt = mraw * qscale;  // qscale > 0 keeps the order
-      // rows whose maximum grew too much rescale O and l (warp-collective)
       const bool grow = mt > m_run + kRescaleLog2;
       float alpha = 1.f;
       if (grow) {
@@ -323,93 +342,84 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         m_run = mt;
       }
       if (__any_sync(0xffffffffu, grow && alpha != 0.f) && j > 0) {
-        wait_o(j - 1);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
-          tc::tmem_ld32(tO + lane_addr + c * 32, v);
+          tc::tmem_ld32(tOi + c * 32, v);
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-          tmem_st32(tO + lane_addr + c * 32, v);
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+          tmem_st32(tOi + c * 32, v);
         }
-        tmem_st_wait();
       }
       l_run *= alpha;
-      // p = 2^(s*qscale - m_run) as bf16 into the swizzled P tile
-      unsigned char* prow = sP + sb * K::P_BYTES + r * 128;
       const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
       float ls = 0.f;
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        uint32_t w[16];
+      for (int c = 0; c < kKeys / 64; ++c) {
+        uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int k0 = c * 32 + i;
+        for (int e = 0; e < 32; ++e) {
+          const int k0 = c * 64 + 2 * e;
           const float p0 = k0 < n_vis ? ex2_approx(fmaf(__uint_as_float(sv[k0]), qscale, neg_m)) : 0.f;
           const float p1 =
               k0 + 1 < n_vis ? ex2_approx(fmaf(__uint_as_float(sv[k0 + 1]), qscale, neg_m)) : 0.f;
           ls += p0 + p1;
-          w[i / 2] = pack_bf16(p0, p1);
+          w[e] = pack_bf16(p0, p1);
         }
-        // keys c*32 .. c*32+31 are 16-byte pieces 4(c%2) .. 4(c%2)+3 of K
-        // block c/2 of row r, stored at their 128B-swizzled positions
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int piece = (c & 1) * 4 + q;
-          *reinterpret_cast<uint4*>(prow + (c >> 1) * (kRows * 128) + ((piece ^ (r & 7)) << 4)) =
-              make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        }
+        tmem_st32(tSP + c * 32, w);  // keys 64c .. 64c+63 -> columns 32c .. 32c+31
       }
       l_run += ls;
-      if (mem && M - key0 < kKeys && r >= M - key0) {
+      if (mem && M - key0 < kKeys) {
         // rows past mem_len in the last memory tile hold whatever the
         // caller's buffer holds there; zero their V so that 0 * V stays 0
-        unsigned char* vrow = sKV + (j % kStages) * K::STAGE + K::K_BYTES + r * 128;
+        const int vrow = quad * 32 + lane;  // one V row per thread of group 0
+        if (qt == 0 && vrow >= M - key0) {
+          unsigned char* vp = sKV + (j % kStages) * K::STAGE + K::K_BYTES + vrow * 128;
 #pragma unroll
-        for (int kb = 0; kb < K::KB; ++kb)
+          for (int kb = 0; kb < K::KB; ++kb)
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<uint4*>(vrow + kb * (kKeys * 128) + q * 16) = make_uint4(0, 0, 0, 0);
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<uint4*>(vp + kb * (kKeys * 128) + q * 16) = make_uint4(0, 0, 0, 0);
+        }
+        tc::fence_proxy_async_smem();
       }
-      tc::fence_proxy_async_smem();
+      tmem_st_wait();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        tc::mbar_arrive(&aux.p_full[sb]);
-        tc::mbar_arrive(&aux.s_empty[sb]);
-      }
+      if (lane == 0) tc::mbar_arrive(&aux.p_full[qt]);
     }
-    // the last P V, then this row's output.  s_full of tile nt-1 implied
-    // that P V nt-3 had completed; wait for nt-2 and nt-1 in turn, so that
-    // each parity wait is at most one phase behind.
-    if (nt >= 2) wait_o(nt - 2);
-    wait_o(nt - 1);
-    const bool row_ok = r / G < n_tok;
+    // O_i is final once the last P V completes (o_full has one phase)
+    if (!*abort_flag && !tc::mbar_wait(&aux.o_full[qt], 0)) {
+      record_error(status, MSA_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    tc::tc_fence_after();
+    const bool row_ok = tok_local < n_tok;
     const int64_t row_id = ((int64_t)b * Hq + g * G + r % G) * T + tok;
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t v[32];
-      tc::tmem_ld32(tO + lane_addr + c * 32, v);
+      tc::tmem_ld32(tOi + c * 32, v);
       tc::tmem_ld_wait();
       if (!row_ok) continue;
       if (n_split > 1) {
         float* po = part_o + (row_id * n_split + sp) * D + c * 32;
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(po + i) =
-              make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                          __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(po + e) =
+              make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                          __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
       } else {
         __nv_bfloat16* op = out + (((int64_t)b * T + tok) * Hq + g * G + r % G) * D + c * 32;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          *reinterpret_cast<uint4*>(op + i) = make_uint4(
-              pack_bf16(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv),
-              pack_bf16(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv),
-              pack_bf16(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
-              pack_bf16(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
+        for (int e = 0; e < 32; e += 8)
+          *reinterpret_cast<uint4*>(op + e) = make_uint4(
+              pack_bf16(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv),
+              pack_bf16(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv),
+              pack_bf16(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv),
+              pack_bf16(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv));
       }
     }
     if (row_ok && n_split > 1) part_ml[row_id * n_split + sp] = make_float2(m_run, l_run);
@@ -527,7 +537,7 @@ struct TcPlan {
 TcPlan tc_plan(int B, int T, int T_loc, int Hq, int H, int D, int m_cap) {
   TcPlan p{};
   const int G = Hq / H;
-  const int TQ = kRows / G;
+  const int TQ = kQT * kRows / G;  // tokens per CTA
   const int64_t base = (int64_t)((T + TQ - 1) / TQ) * H * B;
   const int64_t max_tiles = (m_cap + kKeys - 1) / kKeys + (T_loc + kKeys - 1) / kKeys;
   int64_t ns = (2LL * num_sms() + base - 1) / base;
@@ -563,7 +573,7 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   if (rc) return rc;
 
   CUtensorMap tq, tkm, tvm, tkl, tvl;
-  const int TQ = kRows / G;
+  const int TQ = kRows / G;  // tokens per Q tile (the TMA box)
   const int64_t mem_rows = std::max<int64_t>((int64_t)B * m_cap, 1);
   const void* km = m_cap > 0 ? k_mem : k_rot;  // any valid address when there is no memory
   const void* vm = m_cap > 0 ? v_mem : v_loc;
@@ -576,7 +586,8 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   auto kern = attn_tc_kernel<D>;
   rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
-  const dim3 grid((unsigned)((T + TQ - 1) / TQ * p.n_split), (unsigned)H, (unsigned)B);
+  const dim3 grid((unsigned)((T + kQT * TQ - 1) / (kQT * TQ) * p.n_split), (unsigned)H,
+                  (unsigned)B);
   kern<<<grid, kThreads, K::SMEM, s>>>(tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G, mem_len,
                                        m_cap, qscale, p.n_split, static_cast<__nv_bfloat16*>(out),
                                        part_o, part_ml, device_status_ptr());
