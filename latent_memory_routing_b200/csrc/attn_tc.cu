@@ -54,8 +54,8 @@ constexpr int kSoftWarps = 4 * kQT;
 // softmax warpgroups: 128 x kRegLow + 256 x kRegHigh = 384 x 168, the
 // block's launch allocation under __launch_bounds__(384, 1).
 constexpr int kThreads = 128 + 32 * kSoftWarps;
-constexpr int kRegLow = 56;
-constexpr int kRegHigh = 224;
+constexpr int kRegLow = 40;
+constexpr int kRegHigh = 232;
 static_assert(kQT == 2 && 128 * kRegLow + 256 * kRegHigh == 384 * 168, "register split");
 constexpr int kStages = 2;
 
@@ -127,6 +127,15 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  return (unsigned long long)__float_as_uint(lo) | ((unsigned long long)__float_as_uint(hi) << 32);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -149,8 +158,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   unsigned char* sKV = sQ + kQT * K::Q_BYTES;      // kStages x (K tile, V tile)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x / n_split, sp = blockIdx.x % n_split;
-  const int g = blockIdx.y, b = blockIdx.z;
+  // grid (split x head, batch, query block): z is dispatched slowest and
+  // runs the query blocks in descending order -- under a causal mask later
+  // blocks see more key tiles, so the longest CTAs start first
+  const int mt = (int)(gridDim.z - 1 - blockIdx.z);
+  const int b = blockIdx.y;
+  const int g = blockIdx.x / n_split, sp = blockIdx.x % n_split;
   const int TQ = kRows / G;          // tokens per Q tile
   const int tok0 = mt * kQT * TQ;    // first token of the CTA
   const int n_tok = min(kQT * TQ, T - tok0);
@@ -330,10 +343,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int c = 0; c < kKeys / 32; ++c)
         tc::tmem_ld32(tSP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
       tc::tmem_ld_wait();
-      float mraw = -INFINITY;
+      // keys a row may not see read as -inf (also hides whatever S holds
+      // there: rows past mem_len, keys past the causal limit)
+      if (!__all_sync(0xffffffffu, n_vis == kKeys)) {
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c)
-        if (c < n_vis) mraw = fmaxf(mraw, __uint_as_float(sv[c]));
+        for (int c = 0; c < kKeys; ++c)
+          if (c >= n_vis) sv[c] = 0xff800000u;
+      }
+      // row maximum: 8 independent chains of 3-input max
+      float mx[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(sv[c]);
+#pragma unroll
+      for (int c = 8; c < kKeys; c += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          mx[u] = fmax3(mx[u], __uint_as_float(sv[c + u]), __uint_as_float(sv[c + 8 + u]));
+      const float mraw = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                               fmaxf(mx[6], mx[7]));
       const float mt = mraw * qscale;  // qscale > 0 keeps the order
       const bool grow = mt > m_run + kRescaleLog2;
       float alpha = 1.f;
@@ -354,21 +381,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       l_run *= alpha;
       const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-      float ls = 0.f;
+      // p = 2^(s * qscale - m_run): the affine step on pairs (f32x2), one
+      // ex2 per key, packed to bf16 pairs; the row sum in pairs too
+      const unsigned long long sc2 = f2_pack(qscale, qscale), nm2 = f2_pack(neg_m, neg_m);
+      unsigned long long ls2[2] = {0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < kKeys / 64; ++c) {
         uint32_t w[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int k0 = c * 64 + 2 * e;
-          const float p0 = k0 < n_vis ? ex2_approx(fmaf(__uint_as_float(sv[k0]), qscale, neg_m)) : 0.f;
-          const float p1 =
-              k0 + 1 < n_vis ? ex2_approx(fmaf(__uint_as_float(sv[k0 + 1]), qscale, neg_m)) : 0.f;
-          ls += p0 + p1;
+          unsigned long long x2 = (unsigned long long)sv[k0] | ((unsigned long long)sv[k0 + 1] << 32);
+          asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(x2) : "l"(sc2), "l"(nm2));
+          const float p0 = ex2_approx(__uint_as_float((uint32_t)x2));
+          const float p1 = ex2_approx(__uint_as_float((uint32_t)(x2 >> 32)));
+          const unsigned long long p2 = f2_pack(p0, p1);
+          asm("add.rn.f32x2 %0, %0, %1;" : "+l"(ls2[e & 1]) : "l"(p2));
           w[e] = pack_bf16(p0, p1);
         }
         tmem_st32(tSP + c * 32, w);  // keys 64c .. 64c+63 -> columns 32c .. 32c+31
       }
+      asm("add.rn.f32x2 %0, %0, %1;" : "+l"(ls2[0]) : "l"(ls2[1]));
+      const float ls = __uint_as_float((uint32_t)ls2[0]) + __uint_as_float((uint32_t)(ls2[0] >> 32));
       l_run += ls;
       if (mem && M - key0 < kKeys) {
         // rows past mem_len in the last memory tile hold whatever the
@@ -586,8 +620,9 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   auto kern = attn_tc_kernel<D>;
   rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
-  const dim3 grid((unsigned)((T + kQT * TQ - 1) / (kQT * TQ) * p.n_split), (unsigned)H,
-                  (unsigned)B);
+  const int n_qb = (T + kQT * TQ - 1) / (kQT * TQ);
+  if (n_qb > 65535 || B > 65535) return MSA_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)(p.n_split * H), (unsigned)B, (unsigned)n_qb);
   kern<<<grid, kThreads, K::SMEM, s>>>(tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G, mem_len,
                                        m_cap, qscale, p.n_split, static_cast<__nv_bfloat16*>(out),
                                        part_o, part_ml, device_status_ptr());
@@ -604,6 +639,9 @@ bool attn_tc_supported(int B, int T, int T_loc, int Hq, int H, int D, int m_cap)
   if (G > 16 || (G & (G - 1))) return false;
   if ((int64_t)B * T > (1LL << 30) || (int64_t)B * T_loc > (1LL << 30) ||
       (int64_t)B * m_cap > (1LL << 30) || B > 65535 || H > 65535)
+    return false;
+  // grid (3 splits x H, B, query blocks of kQT * 128 / G tokens)
+  if ((int64_t)3 * H > INT32_MAX || (T + kQT * (kRows / G) - 1) / (kQT * (kRows / G)) > 65535)
     return false;
   return true;
 }
