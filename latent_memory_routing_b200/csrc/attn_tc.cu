@@ -152,8 +152,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   using K = ACfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ AAux aux;
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  unsigned char* base = tc::smem_align<1024>(smem_dyn);
   unsigned char* sQ = base;                        // kQT Q tiles
   unsigned char* sKV = sQ + kQT * K::Q_BYTES;      // kStages x (K tile, V tile)
 
@@ -559,6 +558,22 @@ bool map3(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int b
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+}  // namespace
+
+bool tma_map_rows_bf16(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int br) {
+  auto fn = encode_fn();
+  if (!fn || D > 256 || br > 256) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)br};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
 
 struct TcPlan {
   int n_split;

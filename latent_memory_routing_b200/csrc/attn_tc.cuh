@@ -1,6 +1,7 @@
 // bf16 prefill attention on the tcgen05 tensor cores (attn_tc.cu).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -22,6 +23,12 @@ int attn_decode_launch(int B, int T_loc, int Hq, int H, int D, const void* q, co
                        const void* v_mem, const int32_t* mem_len, int m_cap, const void* k_loc,
                        const void* v_loc, int pos0, float rope_base, float qscale, void* out,
                        void* ws, cudaStream_t s);
+
+// Tensor map of a bf16 [rows][heads][D] array viewed as dims {D, heads,
+// rows}, no swizzle, box {D, 1, br}: one head's D-vector of br consecutive
+// rows, stored densely (D * 2 bytes per row).  False if the driver's encoder
+// is unavailable or rejects the shape.
+bool tma_map_rows_bf16(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int br);
 
 // Merges n_split partial results (unnormalised O in fp32, (max, sum) in the
 // base-2 exponent domain) of each (query, head, token) row into bf16 out.

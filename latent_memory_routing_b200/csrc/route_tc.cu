@@ -189,8 +189,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   using K = Cfg<N, D, kPrep>;
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ Aux aux;
-  unsigned char* ring = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  unsigned char* ring = tc::smem_align<1024>(smem_dyn);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;

@@ -15,6 +15,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// p advanced to the next multiple of A bytes in the shared window.  The
+// offset is added to p itself (no integer round trip of the pointer), so the
+// compiler still knows the result points to shared memory and emits
+// shared-memory loads and stores through it.
+template <uint32_t A>
+__device__ __forceinline__ unsigned char* smem_align(unsigned char* p) {
+  return p + ((A - (smem_u32(p) & (A - 1))) & (A - 1));
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

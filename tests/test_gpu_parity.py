@@ -446,6 +446,43 @@ def test_attention_prefill_tensor_core_shapes(B, T, T_loc, Hq, H, D, m_cap, mem_
     status_ok()
 
 
+@pytest.mark.parametrize("B,T_loc,Hq,H,m_cap,mem_lens", [
+    (3, 1, 32, 8, 70, [70, 0, 65]),         # one local token, ragged memory tile
+    (2, 65, 8, 8, 64, [64, 1]),             # G = 1, local tail of one key
+    (2, 200, 16, 8, 130, [129, 3]),         # G = 2
+    (2, 129, 64, 8, 200, [200, 77]),        # G = 8
+    (1, 100, 16, 1, 500, [500]),            # G = 16, one KV head
+    (2, 90, 32, 8, 64, [0, 0]),             # no memory rows at all
+    (4, 4096, 32, 8, 1024, [1000, 0, 1024, 513]),  # long context, several splits
+])
+def test_attention_decode_shapes(B, T_loc, Hq, H, m_cap, mem_lens):
+    """bf16 decode over 64-key tiles: rows past mem_len hold NaN and must not
+    reach the output; the relative-RoPE local tiles must match absolute
+    positions."""
+    D = 128
+    g = torch.Generator(device="cuda").manual_seed(T_loc + m_cap)
+    dt = torch.bfloat16
+    q = synth.randn((B, 1, Hq, D), dt, "cuda", g)
+    km = synth.randn((B, m_cap, H, D), dt, "cuda", g)
+    vm = synth.randn((B, m_cap, H, D), dt, "cuda", g)
+    for b, n in enumerate(mem_lens):
+        km[b, n:] = float("nan")
+        vm[b, n:] = float("nan")
+    kl = synth.randn((B, T_loc, H, D), dt, "cuda", g)
+    vl = synth.randn((B, T_loc, H, D), dt, "cuda", g)
+    ml = torch.tensor(mem_lens, dtype=torch.int32, device="cuda")
+    att = pipeline.Attention(dt, B, 1, T_loc, Hq, H, D, m_cap, "cuda")
+    out = att(q, km, vm, ml, kl, vl, 16)
+    torch.cuda.synchronize()
+    want = oracle.sparse_attn(f64(q), [f64(km[b, :n]) for b, n in enumerate(mem_lens)],
+                              [f64(vm[b, :n]) for b, n in enumerate(mem_lens)],
+                              f64(kl), f64(vl), 16, 10000.0)
+    got = f64(out)
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got - want)) <= ATTN_BF16
+    status_ok()
+
+
 def test_attention_decode_10m_workload_full():
     lengths = synth.bank_10m_lengths()
     coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
