@@ -331,11 +331,47 @@ def run_libmsa(args, world, rank, local):
     if args.cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, p, C)
     if args.extra and world == 1:
+        tiered = bench_tiered(w, p, args.steps, ms_step)
         del p, w
         torch.cuda.empty_cache()
         line["workloads"] = {"encode_4l": bench_encode(max(args.steps // 4, 3), pk["hbm"]),
-                             "bank_10m_decode": bench_decode(args.steps, pk["hbm"])}
+                             "bank_10m_decode": bench_decode(args.steps, pk["hbm"]),
+                             "bank_100m_tiered": tiered}
     return line
+
+
+def bench_tiered(w, p, steps: int, resident_ms: float) -> dict:
+    """The headline step with the content K̄/V̄ in pinned host memory (the
+    routing keys stay in HBM): the gather reads the 16 selected documents'
+    rows over the host link."""
+    import torch
+
+    from latent_memory_routing_b200 import pipeline
+    try:
+        kh = pipeline.to_host_tier(w["k_bar"])
+        vh = pipeline.to_host_tier(w["v_bar"])
+    except RuntimeError as e:  # host memory too small to pin the bank
+        return {"unavailable": f"pinning the 6.6 GB K/V bank failed: {str(e)[:120]}"}
+    pt = pipeline.Pipeline(w["kr_hat"], kh, vh, p.coff, B=1, T=w["T"], T_loc=w["T_loc"],
+                           Hq=w["Hq"], k=w["k"], m_cap=p.m_cap, pos0=w["pos0"], prepared=True)
+    out_t = pt(w["q_r"], w["q"], w["k_loc"], w["v_loc"]).clone()
+    out_r = p(w["q_r"], w["q"], w["k_loc"], w["v_loc"]).clone()
+    graph = pt.capture(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    ms = time_device(graph.replay, steps)
+    ms_g = time_device(lambda: pipeline.gather_kv(pt.idx, pt.coff, kh, vh, pt.m_cap, pt.k_mem,
+                                                  pt.v_mem, pt.mem_len), steps)
+    rows = int(pt.mem_len.sum())
+    gbytes = 2 * rows * pt.H * pt.D * 2
+    C = int(p.coff[-1])
+    res = {"workload": "bank_100m with K̄/V̄ (2 x 3.3 GB) in pinned, device-mapped host memory; "
+                       "K̄_r (prepared) in HBM",
+           "ms_per_step": round(ms, 4), "gchunks_s": round(C / (ms * 1e-3) / 1e9, 4),
+           "resident_ms_per_step": round(resident_ms, 4),
+           "gather_ms": round(ms_g, 4), "gather_rows": rows, "gather_bytes": gbytes,
+           "gather_gbs_over_host_link": round(gbytes / (ms_g * 1e-3) / 1e9, 2),
+           "same_output_as_resident": bool(torch.equal(out_t, out_r))}
+    del graph, pt, kh, vh
+    return res
 
 
 def time_device(fn, steps: int) -> float:

@@ -206,7 +206,14 @@ int msa_topk_docs(int B, int n_docs, int k, const float* scores,
  *   mem_len      [B] int32, written: min(total rows, m_cap).
  * If a query's rows exceed m_cap, rows past m_cap are dropped and
  * MSA_ERR_CAPACITY is recorded in the device status word.  An index outside
- * [0, n_docs) contributes no rows and records MSA_ERR_INVALID_ARG there. */
+ * [0, n_docs) contributes no rows and records MSA_ERR_INVALID_ARG there.
+ * Tiered storage -- [HYSEN] §"The 100M-token setup depends on host memory as
+ * well as two GPUs" and [WIKI] §6 (routing keys on the GPU, content K/V in
+ * host memory): k_bar and v_bar may instead point into pinned host memory
+ * that is mapped into the device's address space (cudaHostAlloc, or
+ * cudaHostRegister with mapping; the unified address is passed).  The same
+ * kernel then reads only the selected rows over the host link; idx,
+ * chunk_offsets and the outputs stay in device memory. */
 int msa_gather_kv(msa_dtype dt, int B, int k, int H, int D,
                   const int32_t* idx, const int64_t* chunk_offsets,
                   int n_docs, const void* k_bar, const void* v_bar,

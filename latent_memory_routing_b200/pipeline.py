@@ -89,7 +89,7 @@ def gather_kv(idx, chunk_offs, k_bar, v_bar, m_cap: int, k_mem=None, v_mem=None,
     B, k = idx.shape
     C, H, D = k_bar.shape
     n_docs = chunk_offs.numel() - 1
-    dev = k_bar.device
+    dev = idx.device  # the bank may sit in (pinned, mapped) host memory
     if k_mem is None:
         k_mem = torch.empty((B, m_cap, H, D), dtype=k_bar.dtype, device=dev)
         v_mem = torch.empty((B, m_cap, H, D), dtype=k_bar.dtype, device=dev)
@@ -98,6 +98,17 @@ def gather_kv(idx, chunk_offs, k_bar, v_bar, m_cap: int, k_mem=None, v_mem=None,
     _m.msa_gather_kv(dt_code(k_bar), B, k, H, D, idx, chunk_offs, n_docs, k_bar, v_bar, m_cap,
                      k_mem, v_mem, mem_len, stream)
     return k_mem, v_mem, mem_len
+
+
+def to_host_tier(t):
+    """A copy of a bank tensor in pinned host memory.  Pinned allocations are
+    mapped into every device's address space, so msa_gather_kv reads the
+    selected rows straight from it over the host link (tiered storage: the
+    routing keys stay in HBM, the content K/V in host DRAM)."""
+    import torch
+    h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    h.copy_(t)
+    return h
 
 
 class Attention:

@@ -364,6 +364,33 @@ def test_gather_bit_exact_and_capacity():
     assert msa.msa_device_status(clear=True) == -3
 
 
+def test_gather_tiered_host_bank():
+    """Tiered storage: K̄/V̄ in pinned host memory, read by the same gather
+    kernel over the host link; bit-identical to the device-resident gather."""
+    H, D = 8, 128
+    kr, coff, coff_h = _pooled_bank(300, 1, 700, H, D, torch.bfloat16, 23)
+    g = torch.Generator(device="cuda").manual_seed(24)
+    kb = synth.randn(kr.shape, torch.bfloat16, "cuda", g)
+    vb = synth.randn(kr.shape, torch.bfloat16, "cuda", g)
+    kh, vh = pipeline.to_host_tier(kb), pipeline.to_host_tier(vb)
+    assert kh.is_pinned() and not kh.is_cuda
+    idx = torch.stack([torch.randperm(300, generator=torch.Generator().manual_seed(s))[:16]
+                       for s in range(3)]).int().cuda()
+    counts = np.diff(coff_h)
+    m_cap = max(int(counts[r].sum()) for r in idx.cpu().numpy())
+    km, vm, ml = pipeline.gather_kv(idx, coff, kh, vh, m_cap)
+    kd, vd, mld = pipeline.gather_kv(idx, coff, kb, vb, m_cap)
+    torch.cuda.synchronize()
+    assert km.is_cuda and ml.tolist() == mld.tolist()
+    okm, ovm, oml = oracle.gather_kv(idx.cpu().numpy(), coff_h, f64(kb), f64(vb))
+    for b in range(3):
+        n = int(oml[b])
+        assert torch.equal(km[b, :n], kd[b, :n]) and torch.equal(vm[b, :n], vd[b, :n])
+        np.testing.assert_array_equal(f64(km[b, :n]), okm[b])
+        np.testing.assert_array_equal(f64(vm[b, :n]), ovm[b])
+    status_ok()
+
+
 def test_gather_fp32_tiny():
     w = synth.tiny("cuda")
     ok, ov, orr, coff_h = oracle.encode_pool(f64(w["k_tok"]), f64(w["v_tok"]), f64(w["kr_tok"]),
@@ -521,6 +548,35 @@ def test_tiny_pipeline_end_to_end_fp32():
     assert int(p.mem_len[0]) == 6
     assert np.max(np.abs(f64(p.doc_scores) - ref["doc_scores"])) <= 1e-5
     assert np.max(np.abs(f64(out) - ref["out"])) <= ATTN_F32
+    status_ok()
+
+
+def test_pipeline_tiered_matches_resident():
+    """Routing keys in HBM, content K̄/V̄ in pinned host memory: the whole
+    step (route, top-k, gather over the host link, prefill attention) gives
+    the same bytes as the all-HBM pipeline, and matches the oracle."""
+    H, D, Hq, T, k = 8, 128, 32, 64, 8
+    kr, coff, coff_h = _pooled_bank(400, 1, 600, H, D, torch.bfloat16, 25)
+    g = torch.Generator(device="cuda").manual_seed(26)
+    kb = synth.randn(kr.shape, torch.bfloat16, "cuda", g)
+    vb = synth.randn(kr.shape, torch.bfloat16, "cuda", g)
+    q_r = synth.randn((1, T, H, D), torch.bfloat16, "cuda", g)
+    q = synth.randn((1, T, Hq, D), torch.bfloat16, "cuda", g)
+    kl = synth.randn((1, T, H, D), torch.bfloat16, "cuda", g)
+    vl = synth.randn((1, T, H, D), torch.bfloat16, "cuda", g)
+    m_cap = k * int(np.diff(coff_h).max())
+    outs = []
+    for kk, vv in ((kb, vb), (pipeline.to_host_tier(kb), pipeline.to_host_tier(vb))):
+        p = pipeline.Pipeline(kr, kk, vv, coff, B=1, T=T, T_loc=T, Hq=Hq, k=k, m_cap=m_cap,
+                              pos0=k)
+        outs.append((p(q_r, q, kl, vl).clone(), p.idx.clone(), p.mem_len.clone()))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0][1], outs[1][1]) and torch.equal(outs[0][2], outs[1][2])
+    assert torch.equal(outs[0][0], outs[1][0])
+    idx = outs[1][1].cpu().numpy()
+    okm, ovm, _ = oracle.gather_kv(idx, coff_h, f64(kb), f64(vb))
+    want = oracle.sparse_attn(f64(q), okm, ovm, f64(kl), f64(vl), k, 10000.0)
+    assert np.max(np.abs(f64(outs[1][0]) - want)) <= ATTN_BF16
     status_ok()
 
 
