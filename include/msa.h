@@ -197,6 +197,26 @@ int msa_topk_docs(int B, int n_docs, int k, const float* scores,
                   int32_t* idx, float* top_scores, void* ws, size_t ws_bytes,
                   msa_stream_t stream);
 
+/* Memory Parallel merge -- [HYSEN] §"The 100M-token setup depends on host
+ * memory as well as two GPUs": the routing keys are split across GPUs, each
+ * scores the query against its part, and the partial results are reduced
+ * into one selection.  A shard is a contiguous document range; shard r's
+ * local top-k (msa_topk_docs over its own documents) has been all-gathered.
+ *   cand_scores [world][B][k] float (device), shard r's scores in rank order.
+ *   cand_idx    [world][B][k] int32 (device), the matching shard-local ids.
+ *   doc_base    [world] int32 (device): global id of shard r's document 0;
+ *               shards hold disjoint, increasing document ranges.
+ *   idx         [B][k] int32, written: the global top-k ids in rank order.
+ *   top_scores  [B][k] float, written when not NULL.
+ * Same order as msa_topk_docs: score descending, lower global id first,
+ * NaN last, -0 == +0.  Candidate ids must be distinct (they are, when each
+ * shard returns each of its documents at most once).  world * k <= 4096,
+ * else MSA_ERR_UNSUPPORTED; a global id outside int32 records
+ * MSA_ERR_INVALID_ARG in the device status word. */
+int msa_topk_merge_shards(int B, int world, int k, const float* cand_scores,
+                          const int32_t* cand_idx, const int32_t* doc_base,
+                          int32_t* idx, float* top_scores, msa_stream_t stream);
+
 /* Context assembly -- [HYSEN] §"Memory must be encoded offline ...": only
  * the selected documents' K/V are loaded and joined with the local context.
  *   idx          [B][k] int32 (device), document ids in rank order.

@@ -61,6 +61,7 @@ _SIGS = {
                                        c_p, c_p]),
     "msa_topk_workspace_size": (c_sz, [c_i, c_i, c_i]),
     "msa_topk_docs": (c_i, [c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_sz, c_p]),
+    "msa_topk_merge_shards": (c_i, [c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_p, c_p]),
     "msa_gather_kv": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i, c_p, c_p, c_i, c_p, c_p,
                             c_p, c_p]),
     "msa_sparse_attn_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_i]),
@@ -227,6 +228,17 @@ def msa_route_scores_noalloc(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offset
 
 def msa_topk_workspace_size(B, n_docs, k) -> int:
     return lib().msa_topk_workspace_size(B, n_docs, k)
+
+
+def msa_topk_merge_shards(B, world, k, cand_scores, cand_idx, doc_base, idx, top_scores,
+                          stream=None):
+    _numel_ok(cand_scores, world * B * k, "cand_scores")
+    _numel_ok(cand_idx, world * B * k, "cand_idx")
+    _numel_ok(doc_base, world, "doc_base")
+    _numel_ok(idx, B * k, "idx")
+    _check("msa_topk_merge_shards", lib().msa_topk_merge_shards(
+        B, world, k, _ptr(cand_scores), _ptr(cand_idx), _ptr(doc_base), _ptr(idx),
+        _ptr(top_scores), _stream(stream)))
 
 
 def msa_topk_docs(B, n_docs, k, scores, idx, top_scores, ws, ws_bytes, stream=None):

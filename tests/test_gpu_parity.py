@@ -25,6 +25,7 @@ import pytest
 import torch
 
 import oracle
+from latent_memory_routing_b200 import memory_parallel as mpar
 from latent_memory_routing_b200 import msa, pipeline, synth
 
 pytestmark = pytest.mark.gpu
@@ -333,6 +334,75 @@ def test_topk_special_values():
     assert idx[0].tolist() == [4, 0, 3, 5, 6, 2, 1]
     oi, _ = oracle.topk_docs(f64(s), 7)
     assert oi[0].tolist() == idx[0].tolist()
+    status_ok()
+
+
+# ----------------------------------------------------- Memory Parallel merge
+
+def test_merge_shards_vs_oracle_special_values():
+    """msa_topk_merge_shards over hand-made candidates: ties across shards go
+    to the lower global id, -0 == +0, NaN last; compared with the oracle's
+    top-k over the dense score vector the candidates describe."""
+    world, B, k = 3, 2, 5
+    base = [0, 100, 200]
+    rng = np.random.default_rng(5)
+    cs = np.zeros((world, B, k), np.float32)
+    ci = np.zeros((world, B, k), np.int32)
+    for r in range(world):
+        for b in range(B):
+            ci[r, b] = rng.choice(100, k, replace=False)
+            cs[r, b] = np.round(rng.standard_normal(k), 1)  # coarse: many ties
+    cs[1, 0, 0], cs[2, 0, 1] = 0.0, -0.0
+    cs[0, 1, 2] = np.nan
+    dense = np.full((B, 300), np.nan)
+    for r in range(world):
+        for b in range(B):
+            dense[b, ci[r, b] + base[r]] = cs[r, b]
+    want, wscore = oracle.topk_docs(dense, k)
+    idx, top = mpar.merge_shards(torch.from_numpy(cs).cuda(), torch.from_numpy(ci).cuda(),
+                                 torch.tensor(base, dtype=torch.int32, device="cuda"), k,
+                                 top=torch.empty((B, k), device="cuda"))
+    torch.cuda.synchronize()
+    assert idx.cpu().tolist() == want.tolist()
+    np.testing.assert_array_equal(top.cpu().numpy(), wscore.astype(np.float32))
+    status_ok()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_memory_parallel_emulated_matches_single_gpu(world):
+    """Memory Parallel with its shards emulated in one process: each shard's
+    prepared routing + local top-k, the stacked candidates merged by
+    msa_topk_merge_shards, equal bit for bit to the unsharded route + top-k
+    (each chunk's score does not depend on the shard it sits in).  Two
+    identical best documents in the first and last shard: the lower id wins."""
+    H, D, B, T, k = 8, 128, 3, 32, 16
+    kr, coff, coff_h = _pooled_bank(1500, 1, 900, H, D, torch.bfloat16, 41)
+    g = torch.Generator(device="cuda").manual_seed(42)
+    q_r = synth.randn((B, T, H, D), torch.bfloat16, "cuda", g)
+    plan = mpar.shard_plan(coff_h, world, k)
+    counts = np.diff(coff_h)
+    da = plan[0][0] + 5
+    db = next(d for d in range(plan[-1][0], plan[-1][1]) if counts[d] == counts[da])
+    kr[coff_h[da]:coff_h[da + 1]] = q_r[0, 0]  # cosine 1 with query 0's first token
+    kr[coff_h[db]:coff_h[db + 1]] = kr[coff_h[da]:coff_h[da + 1]]
+    hat = pipeline.prepare_bank(kr)
+    n_docs = len(counts)
+    router = pipeline.Router(torch.bfloat16, B, T, H, D, "cuda", prepared=True)
+    ds = torch.empty((B, n_docs), dtype=torch.float32, device="cuda")
+    router(q_r, hat, coff, n_docs, ds)
+    gi, gt = pipeline.topk_docs(ds, k, top=torch.empty((B, k), device="cuda"))
+    cs = torch.empty((world, B, k), dtype=torch.float32, device="cuda")
+    ci = torch.empty((world, B, k), dtype=torch.int32, device="cuda")
+    for r, (d0, d1, c0, c1) in enumerate(plan):
+        lc = torch.from_numpy(mpar.local_offsets(coff_h, plan, r)).cuda()
+        dsr = torch.empty((B, d1 - d0), dtype=torch.float32, device="cuda")
+        router(q_r, hat[c0:c1], lc, d1 - d0, dsr)
+        pipeline.topk_docs(dsr, k, ci[r], cs[r])
+    base = torch.tensor([p[0] for p in plan], dtype=torch.int32, device="cuda")
+    idx, top = mpar.merge_shards(cs, ci, base, k, top=torch.empty((B, k), device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(idx, gi) and torch.equal(top, gt)
+    assert idx[0, :2].tolist() == [da, db]
     status_ok()
 
 
