@@ -40,6 +40,13 @@ WORKLOAD = ("bank_100m: 100,000 docs of U[500,1500] tokens (~1.56M chunks of 64)
 BYTES_PER_CHUNK = 8 * 128 * 2  # algorithmic routing bytes: one pooled K̄_r row
 
 
+# DRAM bytes per routed chunk of route_tc_kernel (prepared bank, 256 query
+# columns), read + written, from one ncu capture of the current kernel on a
+# 192,961-chunk bank (400 MB, beyond L2): 396.09 MB + 3.75 MB.  Traffic grows
+# with the chunks scanned, so a full launch is this times C.
+ROUTE_DRAM_BYTES_PER_CHUNK = (396.093952e6 + 3.748096e6) / 192961
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -305,7 +312,12 @@ def run_libmsa(args, world, rank, local):
         "roofline": {"bound": "hbm",
                      "kernel": "route_tc_kernel, prepared bank (msa_route_scores_prepared call)",
                      "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": round(achieved / pk["hbm"], 4), "traffic": None,
+                     "frac": round(achieved / pk["hbm"], 4),
+                     "traffic": round(ROUTE_DRAM_BYTES_PER_CHUNK * C / 1e9, 3),
+                     "traffic_unit": "GB per launch",
+                     "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of this "
+                                     "kernel on a 192,961-chunk bank (2072 B per chunk), scaled "
+                                     "by chunks to this bank",
                      "peak_source": pk["src"]},
         "stages_ms": {"route": round(seg[0], 4), "topk": round(seg[1], 4),
                       "gather": round(seg[2], 4), "attn": round(seg[3], 4),
@@ -558,6 +570,40 @@ def run_reference(args, world, rank):
     }
 
 
+# Single-kernel shapes for profiling (three calls each, no timing): the
+# tensor-core prefill at a mid-size causal shape and the decode kernel at the
+# bank_10m decode shape (memory rows as the router selects them there).
+CASES = {
+    "prefill_b1_t4096": dict(B=1, T=4096, T_loc=4096, M=384),
+    "prefill_b2_t8192": dict(B=2, T=8192, T_loc=8192, M=384),
+    "decode_b64_t2048": dict(B=64, T=1, T_loc=2048, M=250),
+}
+
+
+def run_case(name: str):
+    import torch
+
+    from latent_memory_routing_b200 import build as _b
+    from latent_memory_routing_b200 import pipeline, synth
+    _b.build()
+    c = CASES[name]
+    B, T, T_loc, M, Hq, H, D = c["B"], c["T"], c["T_loc"], c["M"], 32, 8, 128
+    g = torch.Generator(device="cuda").manual_seed(1)
+    dt = torch.bfloat16
+    q = synth.randn((B, T, Hq, D), dt, "cuda", g)
+    km = synth.randn((B, M, H, D), dt, "cuda", g)
+    vm = synth.randn((B, M, H, D), dt, "cuda", g)
+    kl = synth.randn((B, T_loc, H, D), dt, "cuda", g)
+    vl = synth.randn((B, T_loc, H, D), dt, "cuda", g)
+    ml = torch.full((B,), M, dtype=torch.int32, device="cuda")
+    att = pipeline.Attention(dt, B, T, T_loc, Hq, H, D, M, "cuda")
+    out = torch.empty((B, T, Hq, D), dtype=dt, device="cuda")
+    for _ in range(3):
+        att(q, km, vm, ml, kl, vl, 16, out=out)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": name, **c, "out_abs_mean": float(out.float().abs().mean())}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -569,7 +615,12 @@ def main():
                     help="skip the encode and decode workloads reported beside the step")
     ap.add_argument("--n-docs", type=int, default=100000,
                     help="documents in the bank (fewer only to profile a small case)")
+    ap.add_argument("--case", choices=sorted(CASES),
+                    help="run one attention kernel shape three times (for profiling) and exit")
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case)
+        return
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args.gpus)
     try:
