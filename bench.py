@@ -40,11 +40,12 @@ WORKLOAD = ("bank_100m: 100,000 docs of U[500,1500] tokens (~1.56M chunks of 64)
 BYTES_PER_CHUNK = 8 * 128 * 2  # algorithmic routing bytes: one pooled K̄_r row
 
 
-# DRAM bytes per routed chunk of route_tc_kernel (prepared bank, 256 query
-# columns), read + written, from one ncu capture of the current kernel on a
-# 192,961-chunk bank (400 MB, beyond L2): 396.09 MB + 3.75 MB.  Traffic grows
-# with the chunks scanned, so a full launch is this times C.
-ROUTE_DRAM_BYTES_PER_CHUNK = (396.093952e6 + 3.748096e6) / 192961
+def ROUTE_DRAM_TRAFFIC(C):
+    """DRAM bytes (GB) of one route_tc_kernel launch over C chunks, from the
+    ncu dram__bytes_read.sum + dram__bytes_write.sum of the current kernel on
+    a smaller bank, scaled by chunks (the kernel's traffic grows with the
+    chunks it scans); None until the current kernel has been captured."""
+    return None
 
 
 def peaks():
@@ -297,6 +298,10 @@ def run_libmsa(args, world, rank, local):
     pk = peaks()
     route_ms = seg[0]
     achieved = C * BYTES_PER_CHUNK / (route_ms * 1e-3) / 1e9
+    nt = p.B * w["T"]  # query columns the scan multiplies (padded as the library pads them)
+    n_cols = 64 if nt <= 64 else 128 if nt <= 128 else (nt + 255) // 256 * 256
+    route_flops = 2.0 * p.H * p.D * n_cols * C
+    route_tf = route_flops / (route_ms * 1e-3) / 1e12
     attn_flops = attn_flops_per_step(p)
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
@@ -309,15 +314,22 @@ def run_libmsa(args, world, rank, local):
                    "seq_len": w["T"], "top_k": w["k"], "m_cap": p.m_cap,
                    "parallelism": f"replica x{world}",
                    "l2": "the 3.2 GB routing bank streams through the 126 MB L2 every step"},
-        "roofline": {"bound": "hbm",
-                     "kernel": "route_tc_kernel, prepared bank (msa_route_scores_prepared call)",
-                     "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": round(achieved / pk["hbm"], 4),
-                     "traffic": round(ROUTE_DRAM_BYTES_PER_CHUNK * C / 1e9, 3),
+        # 256 query columns: 2*H*D*256 = 524,288 FLOP per 2,048-byte chunk row
+        # = 256 FLOP/B, above the measured ridge (sustained 210, burst 249):
+        # the scan is bound by the tensor pipe, with HBM just below it
+        "roofline": {"bound": "tensor",
+                     "kernel": "route_tc_kernel on CTA pairs, prepared bank "
+                               "(msa_route_scores_prepared call)",
+                     "achieved": round(route_tf, 1), "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                     "frac": round(route_tf / pk["bf16_sus"], 4),
+                     "peak_kind": "sustained bf16 (the kernel runs back to back for seconds "
+                                  "under the power cap)",
+                     "frac_of_burst_peak": round(route_tf / pk["bf16"], 4),
+                     "flop_per_byte": round(route_flops / (C * BYTES_PER_CHUNK), 1),
+                     "hbm": {"achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
+                             "frac": round(achieved / pk["hbm"], 4)},
+                     "traffic": ROUTE_DRAM_TRAFFIC(C),
                      "traffic_unit": "GB per launch",
-                     "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of this "
-                                     "kernel on a 192,961-chunk bank (2072 B per chunk), scaled "
-                                     "by chunks to this bank",
                      "peak_source": pk["src"]},
         "stages_ms": {"route": round(seg[0], 4), "topk": round(seg[1], 4),
                       "gather": round(seg[2], 4), "attn": round(seg[3], 4),

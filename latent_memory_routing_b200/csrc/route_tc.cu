@@ -39,6 +39,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "msa_common.cuh"
 #include "route_tc.cuh"
@@ -55,18 +56,23 @@ constexpr int kWindow = 256;  // documents cached per tile for chunk -> doc
 constexpr int kEpiBar = 1;    // named barrier of the epilogue warps
 constexpr int kMaxStages = 8;
 
-template <int N, int D, bool kPrep>
+// kPair: a CTA pair (cluster of 2, cta_group::2) shares each MMA -- M = 256
+// chunks (128 per CTA), each CTA holding half of the N query columns -- so a
+// CTA's stage carries half the query bytes (prepared bank, N = 256 only).
+template <int N, int D, bool kPrep, bool kPair = false>
 struct Cfg {
+  static_assert(!kPair || (kPrep && N == 256), "pairs take the prepared bank, 256 columns");
   static constexpr int KB = D / 64;                   // 64-element K blocks per head
   static constexpr int SKB = kPrep ? 1 : KB;          // K blocks per stage
   static constexpr int SPH = KB / SKB;                // stages per head
+  static constexpr int NB = kPair ? N / 2 : N;        // query columns in this CTA's stage
   static constexpr int A_BYTES = SKB * kTile * 128;
-  static constexpr int B_BYTES = SKB * N * 128;
+  static constexpr int B_BYTES = SKB * NB * 128;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES_FIT = (200 * 1024) / STAGE;
   static constexpr int STAGES = STAGES_FIT > kMaxStages ? kMaxStages : STAGES_FIT;
   static constexpr int TMEM_COLS = 2 * N;
-  static constexpr uint32_t IDESC = tc::idesc_bf16_f32(kTile, N);
+  static constexpr uint32_t IDESC = tc::idesc_bf16_f32(kPair ? 2 * kTile : kTile, N);
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE;
   static_assert(STAGES >= 2, "need a double-buffered ring");
   static_assert(N % 64 == 0 && N >= 64 && N <= 256, "N");
@@ -180,22 +186,28 @@ __device__ __forceinline__ void reduce32(const uint32_t (&r)[32], int cs, int NT
   }
 }
 
-template <int N, int D, bool kPrep>
+template <int N, int D, bool kPrep, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 int H, int NT, int T, int n_pass, int64_t C, int64_t n_tiles,
                 const int64_t* __restrict__ coff, int n_docs, uint32_t* __restrict__ doc_u,
                 uint32_t* __restrict__ chunk_u, int* __restrict__ status) {
-  using K = Cfg<N, D, kPrep>;
+  using K = Cfg<N, D, kPrep, kPair>;
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ Aux aux;
   unsigned char* ring = tc::smem_align<1024>(smem_dyn);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // contiguous tile range of this CTA
-  const int64_t tb = (int64_t)blockIdx.x * n_tiles / gridDim.x;
-  const int64_t te = (int64_t)(blockIdx.x + 1) * n_tiles / gridDim.x;
+  // A unit is one 128-chunk tile, or for a CTA pair two adjacent tiles (the
+  // even CTA takes the first); each CTA (pair) owns a contiguous unit range.
+  const uint32_t crank = kPair ? tc::cluster_ctarank() : 0u;
+  constexpr int kStep = kPair ? 2 : 1;  // tiles per unit
+  const int64_t n_units = (n_tiles + kStep - 1) / kStep;
+  const int64_t grp = blockIdx.x / kStep, n_grp = gridDim.x / kStep;
+  const int64_t tb = grp * n_units / n_grp;
+  const int64_t te = (grp + 1) * n_units / n_grp;
+  auto unit_tile = [&](int64_t u) { return u * kStep + crank; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < K::STAGES; ++i) {
@@ -205,17 +217,26 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&aux.accf[i], 1);
-      tc::mbar_init(&aux.acce[i], kEpiWarps);
+      // a pair's leader waits for both CTAs' epilogue warps
+      tc::mbar_init(&aux.acce[i], kEpiWarps * kStep);
     }
     aux.abort_flag = 0;
     tc::fence_mbar_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(&aux.tmem_base, K::TMEM_COLS);
-    tc::tmem_relinquish();
+    if constexpr (kPair) {
+      tc::tmem_alloc_pair(&aux.tmem_base, K::TMEM_COLS);
+      tc::tmem_relinquish_pair();
+    } else {
+      tc::tmem_alloc(&aux.tmem_base, K::TMEM_COLS);
+      tc::tmem_relinquish();
+    }
   }
   tc::tc_fence_before();
   __syncthreads();
+  // the peer's loads and arrivals target the leader's barriers: both CTAs'
+  // barriers are initialised before either CTA goes on
+  if constexpr (kPair) tc::cluster_sync();
   tc::tc_fence_after();
   const uint32_t tmem = aux.tmem_base;
   volatile int* abort_flag = &aux.abort_flag;
@@ -228,7 +249,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
       uint32_t u = 0;
       bool stop = false;
       for (int p = 0; p < n_pass && !stop; ++p)
-        for (int64_t tile = tb; tile < te && !stop; ++tile)
+        for (int64_t un = tb; un < te && !stop; ++un)
           for (int h = 0; h < H && !stop; ++h)
             for (int s = 0; s < K::SPH; ++s, ++u) {
               const int st = u % K::STAGES;
@@ -239,29 +260,46 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 stop = true;
                 break;
               }
+              const int64_t tile = unit_tile(un);
               unsigned char* a = ring + st * K::STAGE;
               unsigned char* b = a + K::A_BYTES;
-              tc::mbar_arrive_expect_tx(&aux.full[st], K::STAGE);
+              if constexpr (kPair) {
+                // both CTAs' bytes count on the leader's barrier, which the
+                // leader alone arms
+                const uint32_t fb = tc::mapa_shared(&aux.full[st], 0);
+                if (crank == 0) tc::mbar_arrive_expect_tx(&aux.full[st], 2 * K::STAGE);
+                const int x = s * 64;
+                tc::tma_load_3d_pair(a, &tm_k, fb, x, h, (int32_t)(tile * kTile));
+                tc::tma_load_3d_pair(b, &tm_q, fb, x, p * N + (int)crank * K::NB, h);
+              } else {
+                tc::mbar_arrive_expect_tx(&aux.full[st], K::STAGE);
 #pragma unroll
-              for (int kb = 0; kb < K::SKB; ++kb) {
-                const int x = (s * K::SKB + kb) * 64;
-                tc::tma_load_3d(a + kb * kTile * 128, &tm_k, &aux.full[st], x, h,
-                                (int32_t)(tile * kTile));
-                tc::tma_load_3d(b + kb * N * 128, &tm_q, &aux.full[st], x, p * N, h);
+                for (int kb = 0; kb < K::SKB; ++kb) {
+                  const int x = (s * K::SKB + kb) * 64;
+                  tc::tma_load_3d(a + kb * kTile * 128, &tm_k, &aux.full[st], x, h,
+                                  (int32_t)(tile * kTile));
+                  tc::tma_load_3d(b + kb * N * 128, &tm_q, &aux.full[st], x, p * N, h);
+                }
               }
             }
-      // Drain: every load issued must have landed before the CTA exits.
+      // Drain: every load issued must have landed before the CTA exits (a
+      // pair's loads, both CTAs', complete on the leader's barriers, and the
+      // peer leaves only after the leader, at the closing cluster barrier).
       const uint32_t issued = u;
-      for (uint32_t v = issued > (uint32_t)K::STAGES ? issued - K::STAGES : 0; v < issued; ++v)
-        tc::mbar_wait(&aux.full[v % K::STAGES], (v / K::STAGES) & 1u);
+      if (crank == 0)
+        for (uint32_t v = issued > (uint32_t)K::STAGES ? issued - K::STAGES : 0; v < issued; ++v)
+          tc::mbar_wait(&aux.full[v % K::STAGES], (v / K::STAGES) & 1u);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
+    if (lane == 0 && crank == 0) {  // a pair's MMAs are issued by its leader
       uint32_t u = 0, it = 0;
       bool stop = false;
+      // a pair's commits go to the barrier in each CTA
+      const uint32_t peer_empty0 = kPair ? tc::mapa_shared(&aux.empty[0], 1) : 0u;
+      const uint32_t peer_accf0 = kPair ? tc::mapa_shared(&aux.accf[0], 1) : 0u;
       for (int p = 0; p < n_pass && !stop; ++p)
-        for (int64_t tile = tb; tile < te && !stop; ++tile, ++it) {
+        for (int64_t un = tb; un < te && !stop; ++un, ++it) {
           const int ab = it & 1;
           const uint32_t aph = (it >> 1) & 1u;
           const uint32_t d_tmem = tmem + ab * N;
@@ -288,12 +326,27 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
               for (int kk = 0; kk < K::SKB * 4; ++kk) {
                 const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside the swizzle atom
                 const uint64_t ad = tc::sdesc_kmajor_sw128(a0 + (kk >> 2) * (kTile * 128) + koff);
-                const uint64_t bd = tc::sdesc_kmajor_sw128(b0 + (kk >> 2) * (N * 128) + koff);
-                tc::mma_bf16_ss(d_tmem, ad, bd, K::IDESC, (h > 0 || s > 0 || kk > 0) ? 1u : 0u);
+                const uint64_t bd =
+                    tc::sdesc_kmajor_sw128(b0 + (kk >> 2) * (K::NB * 128) + koff);
+                const uint32_t acc = (h > 0 || s > 0 || kk > 0) ? 1u : 0u;
+                if constexpr (kPair) tc::mma_bf16_ss_pair(d_tmem, ad, bd, K::IDESC, acc);
+                else tc::mma_bf16_ss(d_tmem, ad, bd, K::IDESC, acc);
               }
-              tc::mma_commit(&aux.empty[st]);
+              if constexpr (kPair) {
+                tc::mma_commit_pair(tc::smem_u32(&aux.empty[st]));
+                tc::mma_commit_pair(peer_empty0 + st * (uint32_t)sizeof(uint64_t));
+              } else {
+                tc::mma_commit(&aux.empty[st]);
+              }
             }
-          if (!stop) tc::mma_commit(&aux.accf[ab]);
+          if (!stop) {
+            if constexpr (kPair) {
+              tc::mma_commit_pair(tc::smem_u32(&aux.accf[ab]));
+              tc::mma_commit_pair(peer_accf0 + ab * (uint32_t)sizeof(uint64_t));
+            } else {
+              tc::mma_commit(&aux.accf[ab]);
+            }
+          }
         }
     }
   } else if (warp < 2 + kXWarps) {
@@ -354,7 +407,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
       // first tile of the pass: look its document window up synchronously
       if (tb < te) {
         if (ew == 0) {
-          const int64_t d0 = warp_find_segment(coff, n_docs, tb * kTile);
+          const int64_t d0 = warp_find_segment(coff, n_docs, unit_tile(tb) * kTile);
           if (lane == 0) aux.d0 = (int)d0;
         }
         epi_bar();
@@ -365,10 +418,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         epi_bar();
       }
-      for (int64_t tile = tb; tile < te; ++tile, ++it) {
+      for (int64_t un = tb; un < te; ++un, ++it) {
         const int ab = it & 1;
         const uint32_t aph = (it >> 1) & 1u;
-        const int64_t c0 = tile * kTile;
+        const int64_t c0 = unit_tile(un) * kTile;
         const int64_t c = c0 + row;
         const int d0 = aux.d0;
         const int64_t wend = aux.win[kWindow];
@@ -387,11 +440,11 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
           }
         }
         // next tile's window: base document and prefetch into registers
-        const bool has_next = tile + 1 < te;
+        const bool has_next = un + 1 < te;
         int d0n = d0;
         int64_t w0 = INT64_MAX, w1 = INT64_MAX, w2 = INT64_MAX;
         if (has_next) {
-          const int64_t cn = c0 + kTile;
+          const int64_t cn = c0 + kStep * kTile;  // this CTA's next tile
           if (cn < wend) {
             int lo = 0, hi = kWindow;
             while (hi - lo > 1) {
@@ -443,7 +496,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&aux.acce[ab]);
+        if (lane == 0) {
+          if constexpr (kPair) tc::mbar_arrive_cluster(tc::mapa_shared(&aux.acce[ab], 0));
+          else tc::mbar_arrive(&aux.acce[ab]);
+        }
         epi_bar();  // everyone is done with this tile's window
         if (has_next) {
           aux.win[et] = w0;
@@ -460,9 +516,13 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
   tc::tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair frees TMEM or leaves while the other may still
+  // signal its barriers
+  if constexpr (kPair) tc::cluster_sync();
   if (warp == 1) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, K::TMEM_COLS);
+    if constexpr (kPair) tc::tmem_dealloc_pair(tmem, K::TMEM_COLS);
+    else tc::tmem_dealloc(tmem, K::TMEM_COLS);
   }
 }
 
@@ -524,26 +584,47 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N, int D, bool kPrep>
+template <int N, int D, bool kPrep, bool kPair = false>
 int launch(int B, int T, int H, const __nv_bfloat16* qhat, int n_pad, const __nv_bfloat16* kr,
            int64_t C, const int64_t* coff, int n_docs, uint32_t* doc_u, uint32_t* chunk_u,
            int* status, cudaStream_t s) {
-  using K = Cfg<N, D, kPrep>;
+  using K = Cfg<N, D, kPrep, kPair>;
   CUtensorMap tm_k, tm_q;
   if (!make_map(&tm_k, kr, D, H, C, (uint64_t)D * 2, (uint64_t)H * D * 2, 1, kTile))
     return note_cuda(cudaErrorInvalidValue);
-  if (!make_map(&tm_q, qhat, D, n_pad, H, (uint64_t)D * 2, (uint64_t)n_pad * D * 2, N, 1))
+  if (!make_map(&tm_q, qhat, D, n_pad, H, (uint64_t)D * 2, (uint64_t)n_pad * D * 2, K::NB, 1))
     return note_cuda(cudaErrorInvalidValue);
-  auto kern = route_tc_kernel<N, D, kPrep>;
+  auto kern = route_tc_kernel<N, D, kPrep, kPair>;
   int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
   const int64_t n_tiles = (C + kTile - 1) / kTile;
-  const int grid = (int)std::min<int64_t>(n_tiles, num_sms());
   const int NT = B * T;
   const int n_pass = n_pad / N;
-  kern<<<grid, kThreads, K::SMEM, s>>>(tm_k, tm_q, H, NT, T, n_pass, C, n_tiles, coff, n_docs,
-                                       doc_u, chunk_u, status);
-  return check_launch();
+  if constexpr (kPair) {
+    // one CTA pair per TPC (two SMs), each pair a contiguous range of
+    // 256-chunk units
+    const int64_t n_units = (n_tiles + 1) / 2;
+    const int pairs = (int)std::min<int64_t>(n_units, std::max(1, num_sms() / 2));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = K::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return note_cuda(cudaLaunchKernelEx(&cfg, kern, tm_k, tm_q, H, NT, T, n_pass, C, n_tiles,
+                                        coff, n_docs, doc_u, chunk_u, status));
+  } else {
+    const int grid = (int)std::min<int64_t>(n_tiles, num_sms());
+    kern<<<grid, kThreads, K::SMEM, s>>>(tm_k, tm_q, H, NT, T, n_pass, C, n_tiles, coff, n_docs,
+                                         doc_u, chunk_u, status);
+    return check_launch();
+  }
 }
 
 }  // namespace
@@ -560,6 +641,20 @@ int route_tc_launch(int B, int T, int H, int D, const __nv_bfloat16* qhat, int n
                     cudaStream_t s) {
   const int N = n_pad <= 128 ? n_pad : 256;
   if (!aligned16(qhat) || !aligned16(kr)) return MSA_ERR_INVALID_ARG;
+  // a prepared bank at 256 columns runs on CTA pairs unless MSA_ROUTE_PAIRS=0
+  // asks for the single-CTA kernel (both compute the same scores)
+  static const bool pairs = [] {
+    const char* e = getenv("MSA_ROUTE_PAIRS");
+    return !(e && e[0] == '0');
+  }();
+  if (prepared && N == 256 && pairs) {
+    if (D == 128)
+      return launch<256, 128, true, true>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u,
+                                          chunk_u, status, s);
+    if (D == 64)
+      return launch<256, 64, true, true>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u,
+                                         chunk_u, status, s);
+  }
 #define MSA_ROUTE_CASE(NN, DD, PP)                                                        \
   if (N == NN && D == DD && prepared == PP)                                                \
     return launch<NN, DD, PP>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u, chunk_u, \
