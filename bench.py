@@ -44,8 +44,9 @@ def ROUTE_DRAM_TRAFFIC(C):
     """DRAM bytes (GB) of one route_tc_kernel launch over C chunks, from the
     ncu dram__bytes_read.sum + dram__bytes_write.sum of the current kernel on
     a smaller bank, scaled by chunks (the kernel's traffic grows with the
-    chunks it scans); None until the current kernel has been captured."""
-    return None
+    chunks it scans).  Pair kernel on a 192,961-chunk bank: 396.06 MB read +
+    3.85 MB written = 2072.5 B per chunk, against 2048 algorithmic."""
+    return round((396.060416e6 + 3.851008e6) / 192961 * C / 1e9, 3)
 
 
 def peaks():
@@ -589,7 +590,30 @@ CASES = {
     "prefill_b1_t4096": dict(B=1, T=4096, T_loc=4096, M=384),
     "prefill_b2_t8192": dict(B=2, T=8192, T_loc=8192, M=384),
     "decode_b64_t2048": dict(B=64, T=1, T_loc=2048, M=250),
+    "route_bank_10m_b64": None,  # routing, not attention: see run_route_case
 }
+
+
+def run_route_case():
+    """The bank_10m decode step's routing: 64 single-token queries over the
+    prepared 10M-token bank (160K chunks), three calls."""
+    import torch
+
+    from latent_memory_routing_b200 import build as _b
+    from latent_memory_routing_b200 import pipeline, synth
+    _b.build()
+    lengths = synth.bank_10m_lengths()
+    coff = pipeline.chunk_offsets(synth.tok_offsets(lengths).cuda())
+    w = synth.bank_10m(coff.cpu(), "cuda")
+    hat = pipeline.prepare_bank(w["kr_bar"])
+    B, H, D = w["B"], hat.shape[1], hat.shape[2]
+    router = pipeline.Router(torch.bfloat16, B, 1, H, D, "cuda", prepared=True)
+    ds = torch.empty((B, len(lengths)), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        router(w["q_r"], hat, coff, len(lengths), ds)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": "route_bank_10m_b64", "n_chunks": int(coff[-1]),
+                      "score_max": float(ds.max())}))
 
 
 def run_case(name: str):
@@ -597,6 +621,8 @@ def run_case(name: str):
 
     from latent_memory_routing_b200 import build as _b
     from latent_memory_routing_b200 import pipeline, synth
+    if name == "route_bank_10m_b64":
+        return run_route_case()
     _b.build()
     c = CASES[name]
     B, T, T_loc, M, Hq, H, D = c["B"], c["T"], c["T_loc"], c["M"], 32, 8, 128
@@ -628,7 +654,7 @@ def main():
     ap.add_argument("--n-docs", type=int, default=100000,
                     help="documents in the bank (fewer only to profile a small case)")
     ap.add_argument("--case", choices=sorted(CASES),
-                    help="run one attention kernel shape three times (for profiling) and exit")
+                    help="run one kernel shape three times (for profiling) and exit")
     args = ap.parse_args()
     if args.case:
         run_case(args.case)

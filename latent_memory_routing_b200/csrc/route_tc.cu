@@ -69,11 +69,18 @@ struct Cfg {
   static constexpr int A_BYTES = SKB * kTile * 128;
   static constexpr int B_BYTES = SKB * NB * 128;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES_FIT = (200 * 1024) / STAGE;
+  static constexpr int STAGES_FIT =
+      (200 * 1024 - (N <= 128 ? kEpiWarps * (N * 33 + 32) * 4 : 0)) / STAGE;
   static constexpr int STAGES = STAGES_FIT > kMaxStages ? kMaxStages : STAGES_FIT;
   static constexpr int TMEM_COLS = 2 * N;
   static constexpr uint32_t IDESC = tc::idesc_bf16_f32(kPair ? 2 * kTile : kTile, N);
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE;
+  // column-owner epilogue (queries of fewer than 32 tokens, N <= 128): per
+  // epilogue warp, the warp's 32 rows x N per-query maxima, [slot][33]
+  // (padded: row-wise writes and slot-wise reads both conflict-free), and
+  // the 32 rows' document ids
+  static constexpr int SCR_WORDS = N <= 128 ? N * 33 + 32 : 0;
+  static constexpr size_t SCR = (size_t)kEpiWarps * SCR_WORDS * 4;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + SCR;
   static_assert(STAGES >= 2, "need a double-buffered ring");
   static_assert(N % 64 == 0 && N >= 64 && N <= 256, "N");
 };
@@ -477,28 +484,102 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         tc::tc_fence_after();
         const uint32_t tbase = tmem + lane_addr + ab * N;
-        int b = col0 / T;
-        int t = col0 - b * T;
-        float m = -INFINITY;
         uint32_t r0[32], r1[32];
-        tc::tmem_ld32(tbase, r0);
-        tc::tmem_ld_wait();
+        if (K::SCR_WORDS > 0 && T < 32) {
+          // Column-owner epilogue.  (1) each row folds its columns into one
+          // maximum per query (slot) and parks it in shared memory, which
+          // frees the accumulator at once; (2) lane s owns slot s (s + 32,
+          // ...) and walks the warp's 32 rows in chunk order -- a
+          // document's rows are one run -- with one atomicMax per run.
+          uint32_t* scr = reinterpret_cast<uint32_t*>(ring + K::STAGES * K::STAGE) +
+                          ew * K::SCR_WORDS;
+          int* dw = reinterpret_cast<int*>(scr + N * 33);
+          dw[lane] = dd;
+          const int col_end = min(col0 + N, NT);
+          const int b_first = col0 / T;
+          int tq = col0 - b_first * T;  // token of the current query
+          int slot = 0;
+          float m = -INFINITY;
+          auto fold32 = [&](const uint32_t (&r)[32], int cs) {
 #pragma unroll
-        for (int j = 0; j < N / 32; j += 2) {
-          if (j + 1 < N / 32) tc::tmem_ld32(tbase + (j + 1) * 32, r1);
-          reduce32(r0, col0 + j * 32, NT, T, j + 1 == N / 32, m, b, t, emit);
+            for (int i = 0; i < 32; ++i) {
+              const int col = cs + i;
+              if (col >= col_end) break;  // warp-uniform
+              m = fmaxf(m, __uint_as_float(r[i]));
+              if (++tq == T || col + 1 == col_end) {
+                const uint32_t o = valid ? f2o(m) : 0u;
+                scr[slot * 33 + lane] = o;
+                if (chunk_u && valid) atomicMax(chunk_u + (int64_t)(b_first + slot) * C + c, o);
+                m = -INFINITY;
+                if (tq == T) {
+                  tq = 0;
+                  ++slot;
+                }
+              }
+            }
+          };
+          tc::tmem_ld32(tbase, r0);
           tc::tmem_ld_wait();
-          if (j + 1 < N / 32) {
-            if (j + 2 < N / 32) tc::tmem_ld32(tbase + (j + 2) * 32, r0);
-            reduce32(r1, col0 + (j + 1) * 32, NT, T, j + 2 == N / 32, m, b, t, emit);
+#pragma unroll
+          for (int j = 0; j < N / 32; j += 2) {
+            if (j + 1 < N / 32) tc::tmem_ld32(tbase + (j + 1) * 32, r1);
+            fold32(r0, col0 + j * 32);
             tc::tmem_ld_wait();
+            if (j + 1 < N / 32) {
+              if (j + 2 < N / 32) tc::tmem_ld32(tbase + (j + 2) * 32, r0);
+              fold32(r1, col0 + (j + 1) * 32);
+              tc::tmem_ld_wait();
+            }
           }
-        }
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (kPair) tc::mbar_arrive_cluster(tc::mapa_shared(&aux.acce[ab], 0));
-          else tc::mbar_arrive(&aux.acce[ab]);
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (kPair) tc::mbar_arrive_cluster(tc::mapa_shared(&aux.acce[ab], 0));
+            else tc::mbar_arrive(&aux.acce[ab]);
+          }
+          const int n_slots = (col_end - 1) / T - b_first + 1;
+          for (int sl = lane; sl < n_slots; sl += 32) {
+            uint32_t* doc_row = doc_u + (int64_t)(b_first + sl) * n_docs;
+            const uint32_t* v = scr + sl * 33;
+            int cd = dw[0];
+            uint32_t cur = v[0];
+            for (int rr = 1; rr < 32; ++rr) {
+              const int d = dw[rr];
+              const uint32_t k = v[rr];
+              if (d != cd) {
+                if (cd >= 0) atomicMax(doc_row + cd, cur);
+                cd = d;
+                cur = k;
+              } else {
+                cur = max(cur, k);
+              }
+            }
+            if (cd >= 0) atomicMax(doc_row + cd, cur);
+          }
+          __syncwarp();  // the next tile rewrites scr and dw
+        } else {
+          int b = col0 / T;
+          int t = col0 - b * T;
+          float m = -INFINITY;
+          tc::tmem_ld32(tbase, r0);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < N / 32; j += 2) {
+            if (j + 1 < N / 32) tc::tmem_ld32(tbase + (j + 1) * 32, r1);
+            reduce32(r0, col0 + j * 32, NT, T, j + 1 == N / 32, m, b, t, emit);
+            tc::tmem_ld_wait();
+            if (j + 1 < N / 32) {
+              if (j + 2 < N / 32) tc::tmem_ld32(tbase + (j + 2) * 32, r0);
+              reduce32(r1, col0 + (j + 1) * 32, NT, T, j + 2 == N / 32, m, b, t, emit);
+              tc::tmem_ld_wait();
+            }
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (kPair) tc::mbar_arrive_cluster(tc::mapa_shared(&aux.acce[ab], 0));
+            else tc::mbar_arrive(&aux.acce[ab]);
+          }
         }
         epi_bar();  // everyone is done with this tile's window
         if (has_next) {

@@ -180,6 +180,8 @@ def _route(q_r, kr, coff, n_docs, with_chunks=True, prepared=False):
     (2, 150, 8, 128, 40),     # 300 columns: two passes over the bank
     (1, 64, 2, 64, 70),       # D = 64, H = 2
     (5, 3, 1, 128, 33),       # H = 1
+    (100, 1, 8, 128, 50),     # N = 128, one column per query
+    (12, 10, 8, 128, 45),     # N = 128, ten-token queries
 ])
 def test_route_bf16_vs_oracle(B, T, H, D, n_docs, prepared):
     g = torch.Generator(device="cuda").manual_seed(100 + B * T)
