@@ -20,6 +20,7 @@
 // splits.  The RoPE cos/sin of every local position is computed once per
 // call (exact angle reduction in double) into the workspace.
 #include <algorithm>
+#include <cstdlib>
 
 #include "attn_tc.cuh"
 #include "msa_common.cuh"
@@ -258,12 +259,28 @@ int launch_simt(int B, int Tq, int T_loc, int Hq, int H, const void* q, const vo
 }  // namespace
 }  // namespace msa
 
+namespace msa {
+namespace {
+// bf16 decode runs on the tensor-core kernel unless MSA_DECODE_TC=0 selects
+// the CUDA-core kernel (both compute the same attention)
+bool decode_tc_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("MSA_DECODE_TC");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+}  // namespace
+}  // namespace msa
+
 extern "C" size_t msa_sparse_attn_workspace_size(msa_dtype dt, int B, int T, int T_loc, int Hq,
                                                  int H, int D, int m_cap) {
   using namespace msa;
   if (B <= 0 || T <= 0 || T_loc < T || H <= 0 || Hq % H || D <= 0 || m_cap < 0) return 0;
   if (dt == MSA_BF16 && attn_decode_supported(T, Hq, H, D))
-    return std::max<size_t>(attn_decode_workspace_size(B, T_loc, Hq, H, D, m_cap), 256);
+    return std::max<size_t>({attn_decode_workspace_size(B, T_loc, Hq, H, D, m_cap),
+                             attn_decode_tc_workspace_size(B, T_loc, Hq, H, D, m_cap),
+                             (size_t)256});
   if (dt == MSA_BF16 && attn_tc_supported(B, T, T_loc, Hq, H, D, m_cap))
     return attn_tc_workspace_size(B, T, T_loc, Hq, H, D, m_cap);
   return plan(B, T, T_loc, Hq, H, D, m_cap, num_sms()).total;
@@ -286,6 +303,12 @@ extern "C" int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
   const float qscale = sc * kLog2e;
+  if (dt == MSA_BF16 && attn_decode_tc_supported(T, Hq, H, D) && decode_tc_enabled()) {
+    const size_t need = attn_decode_tc_workspace_size(B, T_loc, Hq, H, D, m_cap);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+    return attn_decode_tc_launch(B, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len, m_cap, k_loc,
+                                 v_loc, pos0, rope_base, qscale, out, ws, s);
+  }
   if (dt == MSA_BF16 && attn_decode_supported(T, Hq, H, D)) {
     const size_t need = attn_decode_workspace_size(B, T_loc, Hq, H, D, m_cap);
     if (need && (!ws || ws_bytes < need || !aligned16(ws))) return MSA_ERR_WORKSPACE;

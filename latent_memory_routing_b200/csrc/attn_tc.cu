@@ -95,14 +95,7 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// UMMA descriptor of an MN-major, 128B-swizzled operand whose MN extent is
-// split in 64-element (128 B) column blocks `lbo` bytes apart and whose K
-// rows are 128 B apart (8-row swizzle atoms 1024 B apart): the layout of a
-// TMA box {64 MN, rows K} stored block after block.
-__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo) {
-  return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
+using tc::sdesc_mnmajor_sw128;
 
 // 2^x by the SFU (ex2.approx, ~2 ulp); its result feeds a bf16 P tile.
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -560,6 +553,11 @@ bool map3(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int b
 }
 
 }  // namespace
+
+bool tma_map_sw128_bf16(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int bh,
+                        int br) {
+  return map3(m, ptr, D, heads, rows, bh, br);
+}
 
 bool tma_map_rows_bf16(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int br) {
   auto fn = encode_fn();

@@ -25,6 +25,20 @@ int attn_decode_launch(int B, int T_loc, int Hq, int H, int D, const void* q, co
                        void* ws, cudaStream_t s);
 
 // Tensor map of a bf16 [rows][heads][D] array viewed as dims {D, heads,
+// rows}, 128-byte swizzle, box {64, bh, br}: 64-element K blocks of br rows,
+// the layout of a K-major (or, read the other way, MN-major) UMMA operand.
+bool tma_map_sw128_bf16(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int bh,
+                        int br);
+
+// bf16 decode on the tcgen05 tensor cores (attn_decode_tc.cu).
+bool attn_decode_tc_supported(int T, int Hq, int H, int D);
+size_t attn_decode_tc_workspace_size(int B, int T_loc, int Hq, int H, int D, int m_cap);
+int attn_decode_tc_launch(int B, int T_loc, int Hq, int H, int D, const void* q,
+                          const void* k_mem, const void* v_mem, const int32_t* mem_len,
+                          int m_cap, const void* k_loc, const void* v_loc, int pos0,
+                          float rope_base, float qscale, void* out, void* ws, cudaStream_t s);
+
+// Tensor map of a bf16 [rows][heads][D] array viewed as dims {D, heads,
 // rows}, no swizzle, box {D, 1, br}: one head's D-vector of br consecutive
 // rows, stored densely (D * 2 bytes per row).  False if the driver's encoder
 // is unavailable or rejects the shape.

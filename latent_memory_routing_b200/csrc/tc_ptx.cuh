@@ -256,6 +256,15 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// UMMA descriptor of an MN-major, 128B-swizzled operand whose MN extent is
+// split in 64-element (128 B) column blocks `lbo` bytes apart and whose K
+// rows are 128 B apart (8-row swizzle atoms 1024 B apart): the layout of a
+// TMA box {64 MN, rows K} stored block after block.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo) {
+  return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1),
 // A and B bf16 (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 =
 // 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
