@@ -10,12 +10,14 @@
 //
 // Design.  Decode is HBM-bound (every K/V byte is read once); the tensor
 // cores take the two contractions off the CUDA cores so that the few
-// instructions left per key hide under the stream.  One CTA of 14 warps per
-// (key split, batch element, KV head) serves the G query heads of the KV
-// head, padded to N = 16 MMA columns:
+// instructions left per key hide under the stream.  A persistent grid of at
+// most one CTA of 14 warps per SM walks work items -- a key split of one
+// (batch element, KV head), serving the G query heads of the KV head padded
+// to N = 16 MMA columns -- with one continuous pipeline across items, so
+// the stream never drains between them:
 //   * warp 0 TMA-loads 128-key K and V tiles (128B-swizzled, 64-dim blocks)
-//     into a 3-stage ring -- memory tiles first, then local tiles, so no
-//     tile mixes the two;
+//     into a 3-stage ring -- per item, memory tiles first, then local tiles,
+//     so no tile mixes the two;
 //   * warps 2, 3, 8..13 (rotators) apply RoPE to local K tiles in shared
 //     memory in the relative form <R(p_q) q, R(p_k) k> = <R(Delta) q,
 //     R(delta) k>: a key's rotation by its offset delta in the tile uses a
@@ -34,8 +36,9 @@
 //     into Q) against a per-head reference maximum that moves only when a
 //     score exceeds it by more than 2^8 -- then O^T is rescaled in TMEM --,
 //     keep per-thread partial row sums (reduced once at the end), and write
-//     P^T (bf16) as the B operand of P V.
-// Splits write (max, sum, O) partials that the split-KV combine kernel
+//     P^T (bf16) as the B operand of P V; at an item's last tile they reduce
+//     the row sums and write the item's output.
+// The query buffers are double-buffered by item and by tile.  Splits write (max, sum, O) partials that the split-KV combine kernel
 // merges; a single split writes the normalised output directly.  Every wait
 // is bounded; after a timeout every role walks its loop without waiting.
 #include <cudaTypedefs.h>
@@ -69,11 +72,11 @@ constexpr uint32_t kTmemCols = 64;         // S buffers: 0..31, O^T: 32..47
 
 struct DTS {  // dynamic shared memory, offsets from a 1024-byte aligned base
   static constexpr size_t RING = 0;
-  static constexpr size_t QMEM = RING + (size_t)kTStages * kStageBytes;
-  static constexpr size_t QT = QMEM + kQBytes;       // [2]
-  static constexpr size_t P = QT + 2 * kQBytes;      // [2]
-  static constexpr size_t QRAW = P + 2 * kPBytes;    // [16][128] f32, scaled raw query
-  static constexpr size_t RED = QRAW + (size_t)kNH * kDim * 4;  // [4][16] f32
+  static constexpr size_t QMEM = RING + (size_t)kTStages * kStageBytes;  // [2] by item
+  static constexpr size_t QT = QMEM + 2 * kQBytes;   // [2] by tile
+  static constexpr size_t P = QT + 2 * kQBytes;      // [2] by tile
+  static constexpr size_t QRAW = P + 2 * kPBytes;    // [2][16][128] bf16 raw query, by item
+  static constexpr size_t RED = QRAW + 2 * (size_t)kNH * kDim * 2;  // [4][16] f32
   static constexpr size_t FLAGS = RED + 4 * kNH * 4;            // [2][4] int
   static constexpr size_t ALLOC = FLAGS + 2 * 4 * 4 + 1024;
   static_assert(QMEM % 1024 == 0 && QT % 1024 == 0 && P % 1024 == 0, "swizzle atoms");
@@ -113,52 +116,92 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int k, int rows) {
                     (kk & 7) * 2);
 }
 
+// One work item: a key split of one (batch element, KV head).  Every role
+// walks the same sequence -- the CTA's items blockIdx.x, blockIdx.x + grid,
+// ..., empty ones skipped, and their tiles -- through its own cursor.
+struct Cur {
+  int it, k, j, nt;      // item, its ordinal among this CTA's non-empty items, tile, tiles
+  int b, g, sp, M, n_mt, j_lo;
+};
+
 template <int G>
 __global__ void __launch_bounds__(kTThreads, 1)
 attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
                       const __grid_constant__ CUtensorMap tm_vm,
                       const __grid_constant__ CUtensorMap tm_kl,
                       const __grid_constant__ CUtensorMap tm_vl, int T_loc, int Hq, int H,
-                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ mem_len,
-                      int m_cap, int64_t pos0, double base, float qscale, int n_split,
-                      const float2* __restrict__ cs_tab, __nv_bfloat16* __restrict__ out,
-                      float* __restrict__ part_o, float2* __restrict__ part_ml,
-                      int* __restrict__ status) {
+                      int n_items, const __nv_bfloat16* __restrict__ q,
+                      const int32_t* __restrict__ mem_len, int m_cap, int64_t pos0, double base,
+                      float qscale, int n_split, const float2* __restrict__ cs_tab,
+                      __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
+                      float2* __restrict__ part_ml, int* __restrict__ status) {
   static_assert(G >= 1 && G <= kNH, "heads per KV head");
   constexpr int HALF = kDim / 2;
   extern __shared__ __align__(1024) unsigned char dsm[];
   __shared__ DTAux aux;
   unsigned char* sm = tc::smem_align<1024>(dsm);
   unsigned char* ring = sm + DTS::RING;
-  unsigned char* qmem = sm + DTS::QMEM;
-  unsigned char* qt = sm + DTS::QT;
-  unsigned char* pbuf = sm + DTS::P;
-  float* qraw = reinterpret_cast<float*>(sm + DTS::QRAW);
+  unsigned char* qmem = sm + DTS::QMEM;  // [2] by item
+  unsigned char* qt = sm + DTS::QT;      // [2] by tile
+  unsigned char* pbuf = sm + DTS::P;     // [2] by tile
+  __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(sm + DTS::QRAW);  // [2][16][128]
   float* red = reinterpret_cast<float*>(sm + DTS::RED);
   int* flags = reinterpret_cast<int*>(sm + DTS::FLAGS);
-
-  const int split = blockIdx.x;
-  const int b = blockIdx.y / H, g = blockIdx.y % H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int M = min(max(mem_len[b], 0), m_cap);
-  const int n_mt = (M + kTK - 1) / kTK;
-  const int n_all = n_mt + (T_loc + kTK - 1) / kTK;
-  const int j_lo = (int)((int64_t)split * n_all / n_split);
-  const int j_hi = (int)((int64_t)(split + 1) * n_all / n_split);
-  const int nt = j_hi - j_lo;
-  if (nt <= 0) {  // an empty split: neutral partial
-    for (int e = tid; e < G * kDim; e += kTThreads) {
-      const int64_t row_id = (int64_t)b * Hq + g * G + e / kDim;
-      part_o[(row_id * n_split + split) * kDim + e % kDim] = 0.f;
-      if (e % kDim == 0) part_ml[row_id * n_split + split] = make_float2(-INFINITY, 0.f);
-    }
-    return;
-  }
-  auto tile_mem = [&](int jj) { return jj < n_mt; };
-  auto tile_key0 = [&](int jj) { return jj < n_mt ? jj * kTK : (jj - n_mt) * kTK; };
-  auto tile_valid = [&](int jj) {
-    return jj < n_mt ? min(kTK, M - jj * kTK) : min(kTK, T_loc - (jj - n_mt) * kTK);
+
+  auto load_item = [&](Cur& c) {
+    c.sp = c.it % n_split;
+    const int bg = c.it / n_split;
+    c.b = bg / H;
+    c.g = bg % H;
+    c.M = min(max(mem_len[c.b], 0), m_cap);
+    c.n_mt = (c.M + kTK - 1) / kTK;
+    const int n_all = c.n_mt + (T_loc + kTK - 1) / kTK;
+    c.j_lo = (int)((int64_t)c.sp * n_all / n_split);
+    c.nt = (int)((int64_t)(c.sp + 1) * n_all / n_split) - c.j_lo;
   };
+  auto first = [&](Cur& c) -> bool {
+    c.k = 0;
+    c.j = 0;
+    for (c.it = blockIdx.x; c.it < n_items; c.it += gridDim.x) {
+      load_item(c);
+      if (c.nt > 0) return true;
+    }
+    return false;
+  };
+  auto next = [&](Cur& c) -> bool {
+    if (++c.j < c.nt) return true;
+    c.j = 0;
+    ++c.k;
+    for (c.it += gridDim.x; c.it < n_items; c.it += gridDim.x) {
+      load_item(c);
+      if (c.nt > 0) return true;
+    }
+    return false;
+  };
+  auto tile_mem = [&](const Cur& c) { return c.j_lo + c.j < c.n_mt; };
+  auto tile_key0 = [&](const Cur& c) {
+    const int jj = c.j_lo + c.j;
+    return jj < c.n_mt ? jj * kTK : (jj - c.n_mt) * kTK;
+  };
+  auto tile_valid = [&](const Cur& c) {
+    const int jj = c.j_lo + c.j;
+    return jj < c.n_mt ? min(kTK, c.M - jj * kTK) : min(kTK, T_loc - (jj - c.n_mt) * kTK);
+  };
+
+  // an empty split (more splits than tiles): neutral partials
+  if (n_split > 1) {
+    Cur c;
+    for (c.it = blockIdx.x; c.it < n_items; c.it += gridDim.x) {
+      load_item(c);
+      if (c.nt > 0) continue;
+      for (int e = tid; e < G * kDim; e += kTThreads) {
+        const int64_t row_id = (int64_t)c.b * Hq + c.g * G + e / kDim;
+        part_o[(row_id * n_split + c.sp) * kDim + e % kDim] = 0.f;
+        if (e % kDim == 0) part_ml[row_id * n_split + c.sp] = make_float2(-INFINITY, 0.f);
+      }
+    }
+  }
 
   if (tid == 0) {
     for (int i = 0; i < kTStages; ++i) {
@@ -179,29 +222,9 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     tc::tmem_alloc(&aux.tmem_base, kTmemCols);
     tc::tmem_relinquish();
   }
-  // zero the per-tile query buffers and P^T (rows >= G stay zero), keep the
-  // scaled raw query, and build R(p_q) q for the memory tiles (all 16 rows)
-  for (int e = tid; e < (2 * kQBytes + 2 * kPBytes) / 16; e += kTThreads)
-    reinterpret_cast<uint4*>(qt)[e] = make_uint4(0, 0, 0, 0);
-  for (int e = tid; e < G * kDim; e += kTThreads)
-    qraw[e] = __bfloat162float(q[((int64_t)b * Hq + g * G) * kDim + e]) * qscale;
-  if (n_mt > j_lo) {
-    for (int e = tid; e < kNH * HALF; e += kTThreads) {
-      const int h = e / HALF, i = e % HALF;
-      float y1 = 0.f, y2 = 0.f;
-      if (h < G) {
-        const __nv_bfloat16* qp = q + ((int64_t)b * Hq + g * G + h) * kDim;
-        const float x1 = __bfloat162float(qp[i]) * qscale;
-        const float x2 = __bfloat162float(qp[i + HALF]) * qscale;
-        const float2 c = rope_cs(pos0 + T_loc - 1, rope_inv_freq(base, i, kDim));
-        y1 = x1 * c.x - x2 * c.y;
-        y2 = x2 * c.x + x1 * c.y;
-      }
-      *reinterpret_cast<__nv_bfloat16*>(qmem + sw128_off(h, i, kNH)) = __float2bfloat16(y1);
-      *reinterpret_cast<__nv_bfloat16*>(qmem + sw128_off(h, i + HALF, kNH)) =
-          __float2bfloat16(y2);
-    }
-  }
+  // all query and P^T buffers start at zero (rows >= G stay zero)
+  for (int e = tid; e < (4 * kQBytes + 2 * kPBytes) / 16; e += kTThreads)
+    reinterpret_cast<uint4*>(qmem)[e] = make_uint4(0, 0, 0, 0);
   tc::fence_proxy_async_smem();
   tc::tc_fence_before();
   __syncthreads();
@@ -219,66 +242,74 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued = 0;
-      for (int j = 0; j < nt; ++j) {
-        const int st = j % kTStages;
-        wait_or_abort(&aux.sfree[st], ((j / kTStages) & 1) ^ 1);
+      Cur c;
+      int u = 0;
+      for (bool ok = first(c); ok; ok = next(c), ++u) {
+        const int st = u % kTStages;
+        wait_or_abort(&aux.sfree[st], ((u / kTStages) & 1) ^ 1);
         if (*abort_flag) break;
-        const int jj = j_lo + j;
         unsigned char* kd = ring + (size_t)st * kStageBytes;
-        const bool mem = tile_mem(jj);
-        const int row0 = mem ? b * m_cap + tile_key0(jj) : b * T_loc + tile_key0(jj);
+        const bool mem = tile_mem(c);
+        const int row0 = (mem ? c.b * m_cap : c.b * T_loc) + tile_key0(c);
         const CUtensorMap* mk = mem ? &tm_km : &tm_kl;
         const CUtensorMap* mv = mem ? &tm_vm : &tm_vl;
         tc::mbar_arrive_expect_tx(&aux.full[st], kStageBytes);
-        tc::tma_load_3d(kd, mk, &aux.full[st], 0, g, row0);
-        tc::tma_load_3d(kd + kBlk, mk, &aux.full[st], 64, g, row0);
-        tc::tma_load_3d(kd + kTileBytes, mv, &aux.full[st], 0, g, row0);
-        tc::tma_load_3d(kd + kTileBytes + kBlk, mv, &aux.full[st], 64, g, row0);
-        ++issued;
+        tc::tma_load_3d(kd, mk, &aux.full[st], 0, c.g, row0);
+        tc::tma_load_3d(kd + kBlk, mk, &aux.full[st], 64, c.g, row0);
+        tc::tma_load_3d(kd + kTileBytes, mv, &aux.full[st], 0, c.g, row0);
+        tc::tma_load_3d(kd + kTileBytes + kBlk, mv, &aux.full[st], 64, c.g, row0);
       }
-      for (int v = issued > kTStages ? issued - kTStages : 0; v < issued; ++v)
+      for (int v = u > kTStages ? u - kTStages : 0; v < u; ++v)
         tc::mbar_wait(&aux.full[v % kTStages], (v / kTStages) & 1);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
-      auto issue_s = [&](int j) {
-        const int st = j % kTStages;
-        wait_or_abort(&aux.kready[st], (j / kTStages) & 1);
+      Cur cs, cp;  // the S cursor runs two tiles ahead of the P V cursor
+      int us = 0, up = 0;
+      bool hs = first(cs), hp = first(cp);
+      auto issue_s = [&]() {
+        const int st = us % kTStages;
+        wait_or_abort(&aux.kready[st], (us / kTStages) & 1);
         tc::tc_fence_after();
         const uint32_t a0 = tc::smem_u32(ring + (size_t)st * kStageBytes);
-        const uint32_t b0 = tc::smem_u32(tile_mem(j_lo + j) ? qmem : qt + (j & 1) * kQBytes);
+        const uint32_t b0 =
+            tc::smem_u32(tile_mem(cs) ? qmem + (cs.k & 1) * kQBytes : qt + (us & 1) * kQBytes);
 #pragma unroll
         for (int kk = 0; kk < kDim / 16; ++kk) {
           const uint32_t koff = (kk & 3) * 32;
-          tc::mma_bf16_ss(tmem + (j & 1) * kNH,
+          tc::mma_bf16_ss(tmem + (us & 1) * kNH,
                           tc::sdesc_kmajor_sw128(a0 + (kk >> 2) * kBlk + koff),
                           tc::sdesc_kmajor_sw128(b0 + (kk >> 2) * (kNH * 128) + koff), kIdescS,
                           kk > 0 ? 1u : 0u);
         }
-        tc::mma_commit(&aux.sfull[j & 1]);
+        tc::mma_commit(&aux.sfull[us & 1]);
+        ++us;
+        hs = next(cs);
       };
-      auto issue_pv = [&](int j) {
-        const int st = j % kTStages;
-        wait_or_abort(&aux.pfull[j & 1], (j >> 1) & 1);
+      auto issue_pv = [&]() {
+        const int st = up % kTStages;
+        wait_or_abort(&aux.pfull[up & 1], (up >> 1) & 1);
         tc::tc_fence_after();
         const uint32_t v0 = tc::smem_u32(ring + (size_t)st * kStageBytes + kTileBytes);
-        const uint32_t p0 = tc::smem_u32(pbuf + (j & 1) * kPBytes);
+        const uint32_t p0 = tc::smem_u32(pbuf + (up & 1) * kPBytes);
+        const bool first_tile = cp.j == 0, last_tile = cp.j == cp.nt - 1;
 #pragma unroll
         for (int kk = 0; kk < kTK / 16; ++kk)
           tc::mma_bf16_ss(tmem + 2 * kNH, tc::sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kBlk),
                           tc::sdesc_kmajor_sw128(p0 + (kk >> 2) * (kNH * 128) + (kk & 3) * 32),
-                          kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                          kIdescO, (!first_tile || kk > 0) ? 1u : 0u);
         tc::mma_commit(&aux.sfree[st]);
         tc::mma_commit(&aux.pvdone);
-        if (j == nt - 1) tc::mma_commit(&aux.odone);
+        if (last_tile) tc::mma_commit(&aux.odone);  // this item's O^T is final
+        ++up;
+        hp = next(cp);
       };
-      issue_s(0);
-      if (nt > 1) issue_s(1);
-      for (int j = 0; j < nt; ++j) {
-        issue_pv(j);
-        if (j + 2 < nt) issue_s(j + 2);
+      if (hs) issue_s();
+      if (hs) issue_s();
+      while (hp) {
+        issue_pv();
+        if (hs) issue_s();
       }
     }
   } else if (warp >= 4 && warp < 4 + kSoftWarps) {
@@ -287,18 +318,21 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     const int r = w4 * 32 + lane;       // key row of S^T, dim row of O^T
     const uint32_t lane_addr = (uint32_t)(w4 * 32) << 16;
     float m_ref[G], l_part[G];
+    Cur c;
+    int u = 0;
+    for (bool ok = first(c); ok; ok = next(c), ++u) {
+      if (c.j == 0) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m_ref[h] = -INFINITY;
-      l_part[h] = 0.f;
-    }
-    for (int j = 0; j < nt; ++j) {
-      wait_or_abort(&aux.sfull[j & 1], (j >> 1) & 1);
+        for (int h = 0; h < G; ++h) {
+          m_ref[h] = -INFINITY;
+          l_part[h] = 0.f;
+        }
+      }
+      wait_or_abort(&aux.sfull[u & 1], (u >> 1) & 1);
       tc::tc_fence_after();
-      const int jj = j_lo + j;
-      const bool valid = r < tile_valid(jj);
+      const bool valid = r < tile_valid(c);
       uint32_t sv[16];
-      tc::tmem_ld16(tmem + lane_addr + (j & 1) * kNH, sv);
+      tc::tmem_ld16(tmem + lane_addr + (u & 1) * kNH, sv);
       tc::tmem_ld_wait();
       float s[G];
       bool need = false;
@@ -308,11 +342,10 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         need |= s[h] > m_ref[h] + kRescaleLog2;
       }
       const int any_w = __any_sync(0xffffffffu, need);
-      if (lane == 0) flags[(j & 1) * 4 + w4] = any_w;
+      int* fl = flags + (u & 1) * 4;
+      if (lane == 0) fl[w4] = any_w;
       soft_bar();
-      const bool any = flags[(j & 1) * 4] | flags[(j & 1) * 4 + 1] | flags[(j & 1) * 4 + 2] |
-                       flags[(j & 1) * 4 + 3];
-      if (any) {  // uniform: new reference maxima from the tile's maxima
+      if (fl[0] | fl[1] | fl[2] | fl[3]) {  // uniform: new reference maxima
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float mx = s[h];
@@ -325,7 +358,8 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         bool rescale = false;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float mt = fmaxf(fmaxf(red[h], red[kNH + h]), fmaxf(red[2 * kNH + h], red[3 * kNH + h]));
+          const float mt =
+              fmaxf(fmaxf(red[h], red[kNH + h]), fmaxf(red[2 * kNH + h], red[3 * kNH + h]));
           alpha[h] = 1.f;
           if (mt > m_ref[h] + kRescaleLog2) {
             alpha[h] = m_ref[h] == -INFINITY ? 0.f : ex2a(m_ref[h] - mt);
@@ -334,10 +368,10 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           }
           l_part[h] *= alpha[h];
         }
-        if (rescale && j > 0) {
-          // O^T holds P V of tiles < j: wait for the last of them, then
-          // scale each head's column (the TMEM columns of this thread's dim)
-          wait_or_abort(&aux.pvdone, (j - 1) & 1);
+        if (rescale && c.j > 0) {
+          // O^T holds P V of this item's earlier tiles: wait for the last
+          // one (tile u-1), then scale each head's column in TMEM
+          wait_or_abort(&aux.pvdone, (u - 1) & 1);
           tc::tc_fence_after();
           uint32_t ov[16];
           tc::tmem_ld16(tmem + lane_addr + 2 * kNH, ov);
@@ -348,9 +382,9 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           tmem_st_wait();
         }
       }
-      // P^T column of this key (buffer j&1: its previous reader, P V of tile
-      // j-2, completed before S(j) was issued)
-      unsigned char* pb = pbuf + (j & 1) * kPBytes;
+      // P^T column of this key (buffer u&1: its previous reader, P V of tile
+      // u-2, completed before S(u) was issued)
+      unsigned char* pb = pbuf + (u & 1) * kPBytes;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float p = (valid && m_ref[h] != -INFINITY) ? ex2a(s[h] - m_ref[h]) : 0.f;
@@ -360,59 +394,92 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&aux.pfull[j & 1]);
-    }
-    wait_or_abort(&aux.odone, 0);
-    tc::tc_fence_after();
-    // row sums: per-thread partials reduced over the 128 key lanes
-    soft_bar();  // every thread is past its last read of red
+      if (lane == 0) tc::mbar_arrive(&aux.pfull[u & 1]);
+      if (c.j == c.nt - 1) {
+        // the item's last tile: once its P V is done, reduce the row sums
+        // over the 128 key lanes and write this split's O (dim r per thread)
+        wait_or_abort(&aux.odone, c.k & 1);
+        tc::tc_fence_after();
+        soft_bar();  // every thread is past its reads of red
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float v = l_part[h];
+        for (int h = 0; h < G; ++h) {
+          float v = l_part[h];
 #pragma unroll
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) red[w4 * kNH + h] = v;
-    }
-    soft_bar();
-    uint32_t ov[16];
-    tc::tmem_ld16(tmem + lane_addr + 2 * kNH, ov);
-    tc::tmem_ld_wait();
+          for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) red[w4 * kNH + h] = v;
+        }
+        soft_bar();
+        uint32_t ov[16];
+        tc::tmem_ld16(tmem + lane_addr + 2 * kNH, ov);
+        tc::tmem_ld_wait();
+        tc::tc_fence_before();  // the next item's first P V overwrites O^T
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float l = red[h] + red[kNH + h] + red[2 * kNH + h] + red[3 * kNH + h];
-      const int64_t row_id = (int64_t)b * Hq + g * G + h;  // T == 1
-      const float o = __uint_as_float(ov[h]);
-      if (n_split == 1) {
-        out[row_id * kDim + r] = __float2bfloat16(l > 0.f ? o / l : 0.f);
-      } else {
-        part_o[(row_id * n_split + split) * kDim + r] = o;
-        if (r == 0) part_ml[row_id * n_split + split] = make_float2(m_ref[h], l);
+        for (int h = 0; h < G; ++h) {
+          const float l = red[h] + red[kNH + h] + red[2 * kNH + h] + red[3 * kNH + h];
+          const int64_t row_id = (int64_t)c.b * Hq + c.g * G + h;  // T == 1
+          const float o = __uint_as_float(ov[h]);
+          if (n_split == 1) {
+            out[row_id * kDim + r] = __float2bfloat16(l > 0.f ? o / l : 0.f);
+          } else {
+            part_o[(row_id * n_split + c.sp) * kDim + r] = o;
+            if (r == 0) part_ml[row_id * n_split + c.sp] = make_float2(m_ref[h], l);
+          }
+        }
       }
     }
   } else {
     // ------------------------------------------------------------ rotators
     const int rt = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // 0 .. 255
-    const int c = rt & 7, r0 = rt >> 3;  // 16-byte chunk, first of four rows
-    float2 cs[4][8];                     // (cos, sin) of delta = r0 + 32 q, pair 8c + e
+    const int ch = rt & 7, r0 = rt >> 3;  // 16-byte chunk, first of four rows
+    float2 cs[4][8];                      // (cos, sin) of delta = r0 + 32 q, pair 8 ch + e
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) cs[qq][e] = cs_tab[(r0 + 32 * qq) * HALF + 8 * c + e];
-    const int i_q = rt % HALF;  // query pair this thread rotates
+      for (int e = 0; e < 8; e += 2) {
+        const float4 t =
+            *reinterpret_cast<const float4*>(cs_tab + (r0 + 32 * qq) * HALF + 8 * ch + e);
+        cs[qq][e] = make_float2(t.x, t.y);
+        cs[qq][e + 1] = make_float2(t.z, t.w);
+      }
+    const int i_q = rt % HALF;  // query pair this thread rotates (every item)
     const double wq = rope_inv_freq(base, i_q, kDim);
     const float2 qstep = rope_cs(kTK, wq);
+    const float2 qpos = rope_cs(pos0 + T_loc - 1, wq);  // R(p_q) for memory tiles
     float2 qcs = make_float2(1.f, 0.f);
     bool anchored = false;
-    for (int j = 0; j < nt; ++j) {
-      const int st = j % kTStages, jj = j_lo + j;
-      wait_or_abort(&aux.full[st], (j / kTStages) & 1);
+    Cur c;
+    int u = 0;
+    for (bool ok = first(c); ok; ok = next(c), ++u) {
+      const int st = u % kTStages;
+      wait_or_abort(&aux.full[st], (u / kTStages) & 1);
       unsigned char* kt = ring + (size_t)st * kStageBytes;
-      const int n_valid = tile_valid(jj);
-      if (!tile_mem(jj)) {
-        // the query for this tile: R(Delta) q into buffer j&1, whose last
-        // reader S(j-2) must be done
-        if (j >= 2) wait_or_abort(&aux.sfull[j & 1], ((j - 2) >> 1) & 1);
-        const int Delta = T_loc - 1 - tile_key0(jj);
+      __nv_bfloat16* qr = qraw + (c.k & 1) * kNH * kDim;
+      if (c.j == 0) {
+        // a new item: its raw query and R(p_q) q go to buffers k&1, whose
+        // last readers (S of item k-2, at or before tile u-1) must be done
+        if (u >= 1) wait_or_abort(&aux.sfull[(u - 1) & 1], ((u - 1) >> 1) & 1);
+        for (int e = rt; e < G * kDim; e += 32 * kRotWarps)
+          qr[e] = q[((int64_t)c.b * Hq + c.g * G) * kDim + e];
+        asm volatile("bar.sync %0, %1;" ::"n"(kSmBar + 1), "n"(32 * kRotWarps) : "memory");
+        if (c.n_mt > c.j_lo) {
+          unsigned char* qm = qmem + (c.k & 1) * kQBytes;
+          for (int e = rt; e < G * HALF; e += 32 * kRotWarps) {
+            const int h = e / HALF;
+            const float x1 = __bfloat162float(qr[h * kDim + i_q]) * qscale;
+            const float x2 = __bfloat162float(qr[h * kDim + i_q + HALF]) * qscale;
+            *reinterpret_cast<__nv_bfloat16*>(qm + sw128_off(h, i_q, kNH)) =
+                __float2bfloat16(x1 * qpos.x - x2 * qpos.y);
+            *reinterpret_cast<__nv_bfloat16*>(qm + sw128_off(h, i_q + HALF, kNH)) =
+                __float2bfloat16(x2 * qpos.x + x1 * qpos.y);
+          }
+        }
+        anchored = false;
+      }
+      const int n_valid = tile_valid(c);
+      if (!tile_mem(c)) {
+        // R(Delta) q into buffer u&1, whose last reader S(u-2) must be done
+        if (u >= 2) wait_or_abort(&aux.sfull[u & 1], ((u - 2) >> 1) & 1);
+        const int Delta = T_loc - 1 - tile_key0(c);
         if (!anchored) {
           qcs = rope_cs(Delta, wq);
           anchored = true;
@@ -421,22 +488,23 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           qcs.y = qcs.y * qstep.x - qcs.x * qstep.y;
           qcs.x = cc;
         }
-        unsigned char* qb = qt + (j & 1) * kQBytes;
+        unsigned char* qb = qt + (u & 1) * kQBytes;
         for (int e = rt; e < G * HALF; e += 32 * kRotWarps) {
           const int h = e / HALF;
-          const float x1 = qraw[h * kDim + i_q], x2 = qraw[h * kDim + i_q + HALF];
+          const float x1 = __bfloat162float(qr[h * kDim + i_q]) * qscale;
+          const float x2 = __bfloat162float(qr[h * kDim + i_q + HALF]) * qscale;
           *reinterpret_cast<__nv_bfloat16*>(qb + sw128_off(h, i_q, kNH)) =
               __float2bfloat16(x1 * qcs.x - x2 * qcs.y);
           *reinterpret_cast<__nv_bfloat16*>(qb + sw128_off(h, i_q + HALF, kNH)) =
               __float2bfloat16(x2 * qcs.x + x1 * qcs.y);
         }
         // R(delta) k for this thread's four rows, 8 pairs each: dims
-        // 8c..8c+7 (first block) and their partners 64 + 8c.. (second block,
-        // same swizzled offset)
+        // 8ch..8ch+7 (first block) and their partners 64 + 8ch.. (second
+        // block, same swizzled offset)
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
           const int rr = r0 + 32 * qq;
-          const uint32_t off = rr * 128 + ((c ^ (rr & 7)) << 4);
+          const uint32_t off = rr * 128 + ((ch ^ (rr & 7)) << 4);
           uint4* p1 = reinterpret_cast<uint4*>(kt + off);
           uint4* p2 = reinterpret_cast<uint4*>(kt + kBlk + off);
           float x1[8], x2[8], y1[8], y2[8];
@@ -486,9 +554,10 @@ struct DTPlan {
   size_t tab_bytes, po_bytes, ml_bytes, total;
 };
 
-// Key splits: the grid runs in waves of one CTA per SM and a CTA pays a
-// pipeline start; take the split count with the fewest tile-slots per SM
-// (waves x tiles per CTA), plus half a tile per CTA for the start.
+// Key splits: each of min(items, SMs) CTAs walks items round-robin, so the
+// busiest CTA runs ceil(items / CTAs) items of ceil(tiles / splits) tiles;
+// take the split count that makes that smallest, charging a quarter tile per
+// item for its query set-up and output.
 DTPlan dt_plan(int B, int Hq, int H, int T_loc, int m_cap) {
   DTPlan p{};
   const int64_t base = (int64_t)B * H;
@@ -497,8 +566,8 @@ DTPlan dt_plan(int B, int Hq, int H, int T_loc, int m_cap) {
   double best = 1e30;
   int pick = 1;
   for (int ns = 1; ns <= std::min<int64_t>(tiles, 32); ++ns) {
-    const int64_t waves = (base * ns + sms - 1) / sms;
-    const double cost = (double)waves * ((tiles + ns - 1) / ns + 0.5);
+    const int64_t items = base * ns, grid = std::min(items, sms);
+    const double cost = (double)((items + grid - 1) / grid) * ((tiles + ns - 1) / ns + 0.25);
     if (cost < best - 1e-9) {
       best = cost;
       pick = ns;
@@ -537,8 +606,10 @@ int launch_dtc(int B, int T_loc, int Hq, int H, const void* q, const void* k_mem
   auto kern = attn_decode_tc_kernel<G>;
   rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)DTS::ALLOC);
   if (rc) return rc;
-  const dim3 grid((unsigned)p.n_split, (unsigned)(B * H));
-  kern<<<grid, kTThreads, DTS::ALLOC, s>>>(tkm, tvm, tkl, tvl, T_loc, Hq, H,
+  const int64_t n_items = (int64_t)p.n_split * B * H;
+  if (n_items > INT32_MAX) return MSA_ERR_UNSUPPORTED;
+  const int grid = (int)std::min<int64_t>(n_items, num_sms());
+  kern<<<grid, kTThreads, DTS::ALLOC, s>>>(tkm, tvm, tkl, tvl, T_loc, Hq, H, (int)n_items,
                                            static_cast<const __nv_bfloat16*>(q), mem_len, m_cap,
                                            pos0, (double)rope_base, qscale, p.n_split, tab,
                                            static_cast<__nv_bfloat16*>(out), part_o, part_ml,

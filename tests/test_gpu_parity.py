@@ -553,6 +553,7 @@ def test_attention_prefill_tensor_core_shapes(B, T, T_loc, Hq, H, D, m_cap, mem_
     (1, 100, 16, 1, 500, [500]),            # G = 16, one KV head
     (2, 90, 32, 8, 64, [0, 0]),             # no memory rows at all
     (4, 4096, 32, 8, 1024, [1000, 0, 1024, 513]),  # long context, several splits
+    (48, 130, 16, 8, 300, [0, 1, 127, 128, 129, 255, 256, 300] * 6),  # many items per CTA
 ])
 def test_attention_decode_shapes(B, T_loc, Hq, H, m_cap, mem_lens):
     """bf16 decode over 64-key tiles: rows past mem_len hold NaN and must not
