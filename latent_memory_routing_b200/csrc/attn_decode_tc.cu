@@ -16,8 +16,10 @@
 // to N = 16 MMA columns -- with one continuous pipeline across items, so
 // the stream never drains between them:
 //   * warp 0 TMA-loads 128-key K and V tiles (128B-swizzled, 64-dim blocks)
-//     into a 3-stage ring -- per item, memory tiles first, then local tiles,
-//     so no tile mixes the two;
+//     into 3-slot K and V rings, one lane each -- per item, memory tiles
+//     first, then local tiles, so no tile mixes the two; a K slot is
+//     released when S has read it, a V slot when P V has, so the K stream
+//     runs ahead;
 //   * warps 2, 3, 8..13 (rotators) apply RoPE to local K tiles in shared
 //     memory in the relative form <R(p_q) q, R(p_k) k> = <R(Delta) q,
 //     R(delta) k>: a key's rotation by its offset delta in the tile uses a
@@ -83,7 +85,10 @@ struct DTS {  // dynamic shared memory, offsets from a 1024-byte aligned base
 };
 
 struct DTAux {
-  uint64_t full[kTStages], kready[kTStages], sfree[kTStages], sfull[2], pfull[2], pvdone, odone;
+  // K and V tiles of a stage arrive and leave separately: a K slot is free
+  // once S has read it, a V slot once P V has
+  uint64_t kfull[kTStages], vfull[kTStages], kready[kTStages], kfree[kTStages], vfree[kTStages];
+  uint64_t sfull[2], pfull[2], pvdone, odone;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -205,9 +210,11 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
 
   if (tid == 0) {
     for (int i = 0; i < kTStages; ++i) {
-      tc::mbar_init(&aux.full[i], 1);
+      tc::mbar_init(&aux.kfull[i], 1);
+      tc::mbar_init(&aux.vfull[i], 1);
       tc::mbar_init(&aux.kready[i], kRotWarps);
-      tc::mbar_init(&aux.sfree[i], 1);
+      tc::mbar_init(&aux.kfree[i], 1);
+      tc::mbar_init(&aux.vfree[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&aux.sfull[i], 1);
@@ -240,27 +247,29 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // ----------------------------------------------------------- producers
+    // lane 0 streams the K tiles, lane 1 the V tiles, each gated by its own
+    // slot releases, so K loads run ahead of the V slots P V still holds
+    if (lane < 2) {
+      const bool isv = lane == 1;
+      uint64_t* fullb = isv ? aux.vfull : aux.kfull;
+      uint64_t* freeb = isv ? aux.vfree : aux.kfree;
       Cur c;
       int u = 0;
       for (bool ok = first(c); ok; ok = next(c), ++u) {
         const int st = u % kTStages;
-        wait_or_abort(&aux.sfree[st], ((u / kTStages) & 1) ^ 1);
+        wait_or_abort(&freeb[st], ((u / kTStages) & 1) ^ 1);
         if (*abort_flag) break;
-        unsigned char* kd = ring + (size_t)st * kStageBytes;
+        unsigned char* d = ring + (size_t)st * kStageBytes + (isv ? kTileBytes : 0);
         const bool mem = tile_mem(c);
         const int row0 = (mem ? c.b * m_cap : c.b * T_loc) + tile_key0(c);
-        const CUtensorMap* mk = mem ? &tm_km : &tm_kl;
-        const CUtensorMap* mv = mem ? &tm_vm : &tm_vl;
-        tc::mbar_arrive_expect_tx(&aux.full[st], kStageBytes);
-        tc::tma_load_3d(kd, mk, &aux.full[st], 0, c.g, row0);
-        tc::tma_load_3d(kd + kBlk, mk, &aux.full[st], 64, c.g, row0);
-        tc::tma_load_3d(kd + kTileBytes, mv, &aux.full[st], 0, c.g, row0);
-        tc::tma_load_3d(kd + kTileBytes + kBlk, mv, &aux.full[st], 64, c.g, row0);
+        const CUtensorMap* m = mem ? (isv ? &tm_vm : &tm_km) : (isv ? &tm_vl : &tm_kl);
+        tc::mbar_arrive_expect_tx(&fullb[st], kTileBytes);
+        tc::tma_load_3d(d, m, &fullb[st], 0, c.g, row0);
+        tc::tma_load_3d(d + kBlk, m, &fullb[st], 64, c.g, row0);
       }
       for (int v = u > kTStages ? u - kTStages : 0; v < u; ++v)
-        tc::mbar_wait(&aux.full[v % kTStages], (v / kTStages) & 1);
+        tc::mbar_wait(&fullb[v % kTStages], (v / kTStages) & 1);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
@@ -284,12 +293,14 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
                           kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&aux.sfull[us & 1]);
+        tc::mma_commit(&aux.kfree[st]);  // S has read the K slot
         ++us;
         hs = next(cs);
       };
       auto issue_pv = [&]() {
         const int st = up % kTStages;
         wait_or_abort(&aux.pfull[up & 1], (up >> 1) & 1);
+        wait_or_abort(&aux.vfull[st], (up / kTStages) & 1);
         tc::tc_fence_after();
         const uint32_t v0 = tc::smem_u32(ring + (size_t)st * kStageBytes + kTileBytes);
         const uint32_t p0 = tc::smem_u32(pbuf + (up & 1) * kPBytes);
@@ -299,7 +310,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           tc::mma_bf16_ss(tmem + 2 * kNH, tc::sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kBlk),
                           tc::sdesc_kmajor_sw128(p0 + (kk >> 2) * (kNH * 128) + (kk & 3) * 32),
                           kIdescO, (!first_tile || kk > 0) ? 1u : 0u);
-        tc::mma_commit(&aux.sfree[st]);
+        tc::mma_commit(&aux.vfree[st]);  // P V has read the V slot
         tc::mma_commit(&aux.pvdone);
         if (last_tile) tc::mma_commit(&aux.odone);  // this item's O^T is final
         ++up;
@@ -451,7 +462,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     int u = 0;
     for (bool ok = first(c); ok; ok = next(c), ++u) {
       const int st = u % kTStages;
-      wait_or_abort(&aux.full[st], (u / kTStages) & 1);
+      wait_or_abort(&aux.kfull[st], (u / kTStages) & 1);
       unsigned char* kt = ring + (size_t)st * kStageBytes;
       __nv_bfloat16* qr = qraw + (c.k & 1) * kNH * kDim;
       if (c.j == 0) {
@@ -520,7 +531,13 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         }
       } else if (n_valid < kTK) {
         // memory rows past mem_len hold whatever the caller's buffer holds:
-        // zero their V so that 0 * V stays 0 in P V
+        // zero their V (once it has landed) so that 0 * V stays 0 in P V,
+        // which is issued after S(u) and so after this tile's kready.  The V
+        // stream may trail the K stream by a whole ring, so first wait for
+        // the slot's previous tile (u - 3) to leave it: then the vfull
+        // parity below can only mean tile u.
+        if (u >= kTStages) wait_or_abort(&aux.vfree[st], ((u / kTStages) - 1) & 1);
+        wait_or_abort(&aux.vfull[st], (u / kTStages) & 1);
         unsigned char* vt = kt + kTileBytes;
         for (int e = rt; e < (kTK - n_valid) * 16; e += 32 * kRotWarps) {
           const int rr = n_valid + e / 16, cc = e % 16;
