@@ -264,6 +264,35 @@ int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, int H,
                     float rope_base, float scale, void* out, void* ws,
                     size_t ws_bytes, msa_stream_t stream);
 
+/* Fused context assembly + sparse attention -- [HYSEN] §"Memory must be
+ * encoded offline ..." (only the selected documents' K/V are loaded and
+ * joined with the local context) and §"Routing happens inside attention
+ * ...": the same attention as msa_gather_kv followed by msa_sparse_attn,
+ * reading the selected documents' pooled rows straight from the bank (no
+ * gathered copy).
+ *   idx          [B][k] int32 (device): document ids in rank order.
+ *   chunk_offsets[n_docs+1] int64 (device); k_bar, v_bar [n_chunks][H][D]
+ *                (dt): one layer of the bank (device or pinned, mapped host
+ *                memory).
+ *   m_cap        upper bound of a query's memory rows (sizes the workspace;
+ *                rows past it are dropped and MSA_ERR_CAPACITY is recorded).
+ *   mem_len      [B] int32, written when not NULL: memory rows used.
+ *   q, k_loc, v_loc, pos0, rope_base, scale, out: as msa_sparse_attn.
+ * Each document's rows are read in 8-row groups; the rows of its last group
+ * past its end are bank rows masked out (the bank must hold finite values).
+ * Supported (else MSA_ERR_UNSUPPORTED): bf16, D = 128, T = 1 (decode),
+ * Hq/H in {1,2,4,8,16}, 1 <= k <= min(n_docs, 1024), n_chunks < 2^31.
+ * The workspace size is 0 for unsupported shapes. */
+size_t msa_sparse_attn_fused_workspace_size(msa_dtype dt, int B, int T, int T_loc, int Hq,
+                                            int H, int D, int k, int m_cap);
+int msa_sparse_attn_fused(msa_dtype dt, int B, int T, int T_loc, int Hq, int H, int D,
+                          const void* q, const int32_t* idx, int k,
+                          const int64_t* chunk_offsets, int n_docs, const void* k_bar,
+                          const void* v_bar, int64_t n_chunks, int m_cap, const void* k_loc,
+                          const void* v_loc, int pos0, float rope_base, float scale,
+                          void* out, int32_t* mem_len, void* ws, size_t ws_bytes,
+                          msa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,9 +25,12 @@ from .msa import (  # noqa: F401
     msa_route_scores_prepared,
     msa_route_workspace_size,
     msa_sparse_attn,
+    msa_sparse_attn_fused,
+    msa_sparse_attn_fused_workspace_size,
     msa_sparse_attn_workspace_size,
     msa_status_string,
     msa_topk_docs,
+    msa_topk_merge_shards,
     msa_topk_workspace_size,
     msa_version,
 )

@@ -129,14 +129,21 @@ struct Cur {
   int b, g, sp, M, n_mt, j_lo;
 };
 
-template <int G>
+// kFused: the memory rows come straight from the pooled bank -- per query
+// a list of 8-row groups (first bank row, rows that belong to the document)
+// in rank order -- instead of a gathered [B][m_cap] buffer; tm_km / tm_vm
+// then map the bank with 8-row boxes (one 128B-swizzle atom each), and a
+// memory tile is 16 groups.  Rows past a document's end within its last
+// group are real bank rows, masked out.
+template <int G, bool kFused>
 __global__ void __launch_bounds__(kTThreads, 1)
 attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
                       const __grid_constant__ CUtensorMap tm_vm,
                       const __grid_constant__ CUtensorMap tm_kl,
                       const __grid_constant__ CUtensorMap tm_vl, int T_loc, int Hq, int H,
                       int n_items, const __nv_bfloat16* __restrict__ q,
-                      const int32_t* __restrict__ mem_len, int m_cap, int64_t pos0, double base,
+                      const int32_t* __restrict__ mem_len, int m_cap,
+                      const int2* __restrict__ groups, int max_groups, int64_t pos0, double base,
                       float qscale, int n_split, const float2* __restrict__ cs_tab,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
                       float2* __restrict__ part_ml, int* __restrict__ status) {
@@ -159,7 +166,8 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     const int bg = c.it / n_split;
     c.b = bg / H;
     c.g = bg % H;
-    c.M = min(max(mem_len[c.b], 0), m_cap);
+    // fused: mem_len holds the query's group count; its memory is 8 rows a group
+    c.M = kFused ? 8 * min(max(mem_len[c.b], 0), max_groups) : min(max(mem_len[c.b], 0), m_cap);
     c.n_mt = (c.M + kTK - 1) / kTK;
     const int n_all = c.n_mt + (T_loc + kTK - 1) / kTK;
     c.j_lo = (int)((int64_t)c.sp * n_all / n_split);
@@ -262,11 +270,24 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         if (*abort_flag) break;
         unsigned char* d = ring + (size_t)st * kStageBytes + (isv ? kTileBytes : 0);
         const bool mem = tile_mem(c);
-        const int row0 = (mem ? c.b * m_cap : c.b * T_loc) + tile_key0(c);
         const CUtensorMap* m = mem ? (isv ? &tm_vm : &tm_km) : (isv ? &tm_vl : &tm_kl);
         tc::mbar_arrive_expect_tx(&fullb[st], kTileBytes);
-        tc::tma_load_3d(d, m, &fullb[st], 0, c.g, row0);
-        tc::tma_load_3d(d + kBlk, m, &fullb[st], 64, c.g, row0);
+        if (kFused && mem) {
+          // 16 groups of 8 bank rows; past the query's last group, repeat it
+          // (finite rows, masked) so every row of the tile is written
+          const int ng = c.M / 8, g0 = tile_key0(c) / 8;
+          const int2* gq = groups + (int64_t)c.b * max_groups;
+#pragma unroll 4
+          for (int gi = 0; gi < kTK / 8; ++gi) {
+            const int src = gq[min(g0 + gi, ng - 1)].x;
+            tc::tma_load_3d(d + gi * 1024, m, &fullb[st], 0, c.g, src);
+            tc::tma_load_3d(d + kBlk + gi * 1024, m, &fullb[st], 64, c.g, src);
+          }
+        } else {
+          const int row0 = (mem ? c.b * m_cap : c.b * T_loc) + tile_key0(c);
+          tc::tma_load_3d(d, m, &fullb[st], 0, c.g, row0);
+          tc::tma_load_3d(d + kBlk, m, &fullb[st], 64, c.g, row0);
+        }
       }
       for (int v = u > kTStages ? u - kTStages : 0; v < u; ++v)
         tc::mbar_wait(&fullb[v % kTStages], (v / kTStages) & 1);
@@ -341,7 +362,11 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       }
       wait_or_abort(&aux.sfull[u & 1], (u >> 1) & 1);
       tc::tc_fence_after();
-      const bool valid = r < tile_valid(c);
+      bool valid = r < tile_valid(c);
+      if (kFused && tile_mem(c)) {  // its group holds the row, and the row its document's
+        const int grp = (tile_key0(c) + r) / 8;
+        valid = grp < c.M / 8 && (r & 7) < groups[(int64_t)c.b * max_groups + grp].y;
+      }
       uint32_t sv[16];
       tc::tmem_ld16(tmem + lane_addr + (u & 1) * kNH, sv);
       tc::tmem_ld_wait();
@@ -529,7 +554,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           *p1 = Vec16<__nv_bfloat16>::pack(y1);
           *p2 = Vec16<__nv_bfloat16>::pack(y2);
         }
-      } else if (n_valid < kTK) {
+      } else if (!kFused && n_valid < kTK) {
         // memory rows past mem_len hold whatever the caller's buffer holds:
         // zero their V (once it has landed) so that 0 * V stays 0 in P V,
         // which is issued after S(u) and so after this tile's kready.  The V
@@ -603,8 +628,10 @@ template <int G>
 int launch_dtc(int B, int T_loc, int Hq, int H, const void* q, const void* k_mem,
                const void* v_mem, const int32_t* mem_len, int m_cap, const void* k_loc,
                const void* v_loc, int pos0, float rope_base, float qscale, void* out, void* ws,
-               cudaStream_t s) {
-  const DTPlan p = dt_plan(B, Hq, H, T_loc, m_cap);
+               cudaStream_t s, const FusedMemory* fm) {
+  // fused: the memory is at most 8 * max_groups rows a query (for the plan)
+  const int mem_rows_cap = fm ? 8 * fm->max_groups : m_cap;
+  const DTPlan p = dt_plan(B, Hq, H, T_loc, mem_rows_cap);
   unsigned char* w = static_cast<unsigned char*>(ws);
   float2* tab = reinterpret_cast<float2*>(w);
   float* part_o = reinterpret_cast<float*>(w + p.tab_bytes);
@@ -613,27 +640,52 @@ int launch_dtc(int B, int T_loc, int Hq, int H, const void* q, const void* k_mem
   int rc = check_launch();
   if (rc) return rc;
   CUtensorMap tkm, tvm, tkl, tvl;
-  const bool has_mem = m_cap > 0;
-  const int64_t mem_rows = has_mem ? (int64_t)B * m_cap : (int64_t)B * T_loc;
-  if (!tma_map_sw128_bf16(&tkm, has_mem ? k_mem : k_loc, kDim, H, mem_rows, 1, kTK) ||
-      !tma_map_sw128_bf16(&tvm, has_mem ? v_mem : v_loc, kDim, H, mem_rows, 1, kTK) ||
-      !tma_map_sw128_bf16(&tkl, k_loc, kDim, H, (int64_t)B * T_loc, 1, kTK) ||
-      !tma_map_sw128_bf16(&tvl, v_loc, kDim, H, (int64_t)B * T_loc, 1, kTK))
-    return note_cuda(cudaErrorInvalidValue);
-  auto kern = attn_decode_tc_kernel<G>;
+  bool ok;
+  if (fm) {  // the bank itself, 8-row boxes (one swizzle atom)
+    ok = tma_map_sw128_bf16(&tkm, fm->k_bar, kDim, H, fm->n_chunks, 1, 8) &&
+         tma_map_sw128_bf16(&tvm, fm->v_bar, kDim, H, fm->n_chunks, 1, 8);
+  } else {
+    const bool has_mem = m_cap > 0;
+    const int64_t mem_rows = has_mem ? (int64_t)B * m_cap : (int64_t)B * T_loc;
+    ok = tma_map_sw128_bf16(&tkm, has_mem ? k_mem : k_loc, kDim, H, mem_rows, 1, kTK) &&
+         tma_map_sw128_bf16(&tvm, has_mem ? v_mem : v_loc, kDim, H, mem_rows, 1, kTK);
+  }
+  ok = ok && tma_map_sw128_bf16(&tkl, k_loc, kDim, H, (int64_t)B * T_loc, 1, kTK) &&
+       tma_map_sw128_bf16(&tvl, v_loc, kDim, H, (int64_t)B * T_loc, 1, kTK);
+  if (!ok) return note_cuda(cudaErrorInvalidValue);
+  auto kern = fm ? attn_decode_tc_kernel<G, true> : attn_decode_tc_kernel<G, false>;
   rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)DTS::ALLOC);
   if (rc) return rc;
   const int64_t n_items = (int64_t)p.n_split * B * H;
   if (n_items > INT32_MAX) return MSA_ERR_UNSUPPORTED;
   const int grid = (int)std::min<int64_t>(n_items, num_sms());
-  kern<<<grid, kTThreads, DTS::ALLOC, s>>>(tkm, tvm, tkl, tvl, T_loc, Hq, H, (int)n_items,
-                                           static_cast<const __nv_bfloat16*>(q), mem_len, m_cap,
-                                           pos0, (double)rope_base, qscale, p.n_split, tab,
-                                           static_cast<__nv_bfloat16*>(out), part_o, part_ml,
-                                           device_status_ptr());
+  kern<<<grid, kTThreads, DTS::ALLOC, s>>>(
+      tkm, tvm, tkl, tvl, T_loc, Hq, H, (int)n_items, static_cast<const __nv_bfloat16*>(q),
+      fm ? fm->n_groups : mem_len, m_cap, fm ? fm->groups : nullptr, fm ? fm->max_groups : 0,
+      pos0, (double)rope_base, qscale, p.n_split, tab, static_cast<__nv_bfloat16*>(out), part_o,
+      part_ml, device_status_ptr());
   rc = check_launch();
   if (rc || p.n_split == 1) return rc;
   return attn_combine_bf16(B, 1, Hq, kDim, p.n_split, part_o, part_ml, out, s);
+}
+
+int dispatch_dtc(int B, int T_loc, int Hq, int H, int D, const void* q, const void* k_mem,
+                 const void* v_mem, const int32_t* mem_len, int m_cap, const void* k_loc,
+                 const void* v_loc, int pos0, float rope_base, float qscale, void* out, void* ws,
+                 cudaStream_t s, const FusedMemory* fm) {
+  if (!aligned16(k_loc) || !aligned16(v_loc)) return MSA_ERR_INVALID_ARG;
+  if (!fm && m_cap > 0 && (!aligned16(k_mem) || !aligned16(v_mem))) return MSA_ERR_INVALID_ARG;
+  if (fm && (!aligned16(fm->k_bar) || !aligned16(fm->v_bar))) return MSA_ERR_INVALID_ARG;
+  if ((int64_t)B * H > 65535 || (int64_t)B * std::max(m_cap, T_loc) > INT32_MAX)
+    return MSA_ERR_UNSUPPORTED;
+  const int G = Hq / H;
+#define MSA_DTC_CASE(GG)                                                                    \
+  if (D == kDim && G == GG)                                                                 \
+    return launch_dtc<GG>(B, T_loc, Hq, H, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc, \
+                          pos0, rope_base, qscale, out, ws, s, fm);
+  MSA_DTC_CASE(1) MSA_DTC_CASE(2) MSA_DTC_CASE(4) MSA_DTC_CASE(8) MSA_DTC_CASE(16)
+#undef MSA_DTC_CASE
+  return MSA_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -653,19 +705,20 @@ int attn_decode_tc_launch(int B, int T_loc, int Hq, int H, int D, const void* q,
                           const void* k_mem, const void* v_mem, const int32_t* mem_len,
                           int m_cap, const void* k_loc, const void* v_loc, int pos0,
                           float rope_base, float qscale, void* out, void* ws, cudaStream_t s) {
-  if (!aligned16(k_loc) || !aligned16(v_loc) ||
-      (m_cap > 0 && (!aligned16(k_mem) || !aligned16(v_mem))))
-    return MSA_ERR_INVALID_ARG;
-  if ((int64_t)B * H > 65535 || (int64_t)B * std::max(m_cap, T_loc) > INT32_MAX)
-    return MSA_ERR_UNSUPPORTED;
-  const int G = Hq / H;
-#define MSA_DTC_CASE(GG)                                                                    \
-  if (D == kDim && G == GG)                                                                 \
-    return launch_dtc<GG>(B, T_loc, Hq, H, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc, \
-                          pos0, rope_base, qscale, out, ws, s);
-  MSA_DTC_CASE(1) MSA_DTC_CASE(2) MSA_DTC_CASE(4) MSA_DTC_CASE(8) MSA_DTC_CASE(16)
-#undef MSA_DTC_CASE
-  return MSA_ERR_UNSUPPORTED;
+  return dispatch_dtc(B, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc, pos0,
+                      rope_base, qscale, out, ws, s, nullptr);
+}
+
+size_t attn_decode_tc_fused_workspace_size(int B, int T_loc, int Hq, int H, int max_groups) {
+  return dt_plan(B, Hq, H, T_loc, 8 * max_groups).total;
+}
+
+int attn_decode_tc_launch_fused(int B, int T_loc, int Hq, int H, int D, const void* q,
+                                const FusedMemory& fm, const void* k_loc, const void* v_loc,
+                                int pos0, float rope_base, float qscale, void* out, void* ws,
+                                cudaStream_t s) {
+  return dispatch_dtc(B, T_loc, Hq, H, D, q, nullptr, nullptr, nullptr, 8 * fm.max_groups,
+                      k_loc, v_loc, pos0, rope_base, qscale, out, ws, s, &fm);
 }
 
 }  // namespace msa

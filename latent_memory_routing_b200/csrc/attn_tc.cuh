@@ -30,6 +30,18 @@ int attn_decode_launch(int B, int T_loc, int Hq, int H, int D, const void* q, co
 bool tma_map_sw128_bf16(CUtensorMap* m, const void* ptr, int D, int heads, int64_t rows, int bh,
                         int br);
 
+// Memory read straight from the pooled bank (fused assemble + attend): per
+// query b, groups[b * max_groups + i] = (first bank row, rows of the group
+// that belong to its document, 1..8) for i < n_groups[b], in rank order.
+struct FusedMemory {
+  const int2* groups;
+  const int32_t* n_groups;
+  int max_groups;
+  const void* k_bar;
+  const void* v_bar;
+  int64_t n_chunks;
+};
+
 // bf16 decode on the tcgen05 tensor cores (attn_decode_tc.cu).
 bool attn_decode_tc_supported(int T, int Hq, int H, int D);
 size_t attn_decode_tc_workspace_size(int B, int T_loc, int Hq, int H, int D, int m_cap);
@@ -37,6 +49,11 @@ int attn_decode_tc_launch(int B, int T_loc, int Hq, int H, int D, const void* q,
                           const void* k_mem, const void* v_mem, const int32_t* mem_len,
                           int m_cap, const void* k_loc, const void* v_loc, int pos0,
                           float rope_base, float qscale, void* out, void* ws, cudaStream_t s);
+size_t attn_decode_tc_fused_workspace_size(int B, int T_loc, int Hq, int H, int max_groups);
+int attn_decode_tc_launch_fused(int B, int T_loc, int Hq, int H, int D, const void* q,
+                                const FusedMemory& fm, const void* k_loc, const void* v_loc,
+                                int pos0, float rope_base, float qscale, void* out, void* ws,
+                                cudaStream_t s);
 
 // Tensor map of a bf16 [rows][heads][D] array viewed as dims {D, heads,
 // rows}, no swizzle, box {D, 1, br}: one head's D-vector of br consecutive

@@ -65,6 +65,10 @@ _SIGS = {
     "msa_gather_kv": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i, c_p, c_p, c_i, c_p, c_p,
                             c_p, c_p]),
     "msa_sparse_attn_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_i]),
+    "msa_sparse_attn_fused_workspace_size": (c_sz, [c_i] * 9),
+    "msa_sparse_attn_fused": (c_i, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i, c_p, c_i,
+                                    c_p, c_p, c_i64, c_i, c_p, c_p, c_i, c_f, c_f, c_p, c_p,
+                                    c_p, c_sz, c_p]),
     "msa_sparse_attn": (c_i, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_i, c_p,
                               c_p, c_i, c_f, c_f, c_p, c_p, c_sz, c_p]),
 }
@@ -273,3 +277,23 @@ def msa_sparse_attn(dt, B, T, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len, m_cap, 
         dt, B, T, T_loc, Hq, H, D, _ptr(q), _ptr(k_mem), _ptr(v_mem), _ptr(mem_len), m_cap,
         _ptr(k_loc), _ptr(v_loc), pos0, rope_base, scale, _ptr(out), _ptr(ws), ws_bytes,
         _stream(stream)))
+
+
+def msa_sparse_attn_fused_workspace_size(dt, B, T, T_loc, Hq, H, D, k, m_cap) -> int:
+    return lib().msa_sparse_attn_fused_workspace_size(dt, B, T, T_loc, Hq, H, D, k, m_cap)
+
+
+def msa_sparse_attn_fused(dt, B, T, T_loc, Hq, H, D, q, idx, k, chunk_offsets, n_docs, k_bar,
+                          v_bar, n_chunks, m_cap, k_loc, v_loc, pos0, rope_base, scale, out,
+                          mem_len, ws, ws_bytes, stream=None):
+    _numel_ok(q, B * T * Hq * D, "q")
+    _numel_ok(idx, B * k, "idx")
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets")
+    _numel_ok(k_loc, B * T_loc * H * D, "k_loc")
+    _numel_ok(v_loc, B * T_loc * H * D, "v_loc")
+    _numel_ok(out, B * T * Hq * D, "out")
+    _numel_ok(mem_len, B, "mem_len")
+    _check("msa_sparse_attn_fused", lib().msa_sparse_attn_fused(
+        dt, B, T, T_loc, Hq, H, D, _ptr(q), _ptr(idx), k, _ptr(chunk_offsets), n_docs,
+        _ptr(k_bar), _ptr(v_bar), n_chunks, m_cap, _ptr(k_loc), _ptr(v_loc), pos0, rope_base,
+        scale, _ptr(out), _ptr(mem_len), _ptr(ws), ws_bytes, _stream(stream)))

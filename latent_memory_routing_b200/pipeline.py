@@ -131,13 +131,38 @@ class Attention:
         return out
 
 
+class FusedAttention:
+    """msa_sparse_attn_fused for fixed shapes: attention over the selected
+    documents read straight from the bank (no gathered copy)."""
+
+    def __init__(self, dtype, B, T, T_loc, Hq, H, D, k, m_cap, device):
+        self.dt = _m.dtype_code(dtype)
+        self.shape = (B, T, T_loc, Hq, H, D, k, m_cap)
+        n = _m.msa_sparse_attn_fused_workspace_size(self.dt, B, T, T_loc, Hq, H, D, k, m_cap)
+        if n == 0:
+            raise _m.MsaError("msa_sparse_attn_fused", -2, "unsupported shape")
+        self.ws = torch.empty(n, dtype=torch.uint8, device=device)
+        self.mem_len = torch.empty(B, dtype=torch.int32, device=device)
+
+    def __call__(self, q, idx, chunk_offs, k_bar, v_bar, k_loc, v_loc, pos0: int,
+                 rope_base: float = 10000.0, scale: float = 0.0, out=None, stream=None):
+        B, T, T_loc, Hq, H, D, k, m_cap = self.shape
+        if out is None:
+            out = torch.empty((B, T, Hq, D), dtype=q.dtype, device=q.device)
+        _m.msa_sparse_attn_fused(self.dt, B, T, T_loc, Hq, H, D, q, idx, k, chunk_offs,
+                                 chunk_offs.numel() - 1, k_bar, v_bar, k_bar.shape[0], m_cap,
+                                 k_loc, v_loc, pos0, rope_base, scale, out, self.mem_len,
+                                 self.ws, self.ws.numel(), stream)
+        return out
+
+
 class Pipeline:
     """route -> top-k -> gather -> attend over a resident pooled bank (one
     layer), with every buffer allocated once.  With ``prepared=True``,
     ``kr_bar`` is a bank made by ``prepare_bank``."""
 
     def __init__(self, kr_bar, k_bar, v_bar, chunk_offs, *, B, T, T_loc, Hq, k, m_cap,
-                 pos0=None, rope_base=10000.0, prepared=False):
+                 pos0=None, rope_base=10000.0, prepared=False, fused=False):
         C, H, D = kr_bar.shape
         dev = kr_bar.device
         self.kr_bar, self.k_bar, self.v_bar, self.coff = kr_bar, k_bar, v_bar, chunk_offs
@@ -147,7 +172,9 @@ class Pipeline:
         self.pos0 = k if pos0 is None else pos0
         self.rope_base = rope_base
         self.router = Router(kr_bar.dtype, B, T, H, D, dev, prepared=prepared)
-        self.attn = Attention(kr_bar.dtype, B, T, T_loc, Hq, H, D, m_cap, dev)
+        self.fused = fused
+        self.attn = (FusedAttention(kr_bar.dtype, B, T, T_loc, Hq, H, D, k, m_cap, dev) if fused
+                     else Attention(kr_bar.dtype, B, T, T_loc, Hq, H, D, m_cap, dev))
         self.doc_scores = torch.empty((B, self.n_docs), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, k), dtype=torch.int32, device=dev)
         self.top = torch.empty((B, k), dtype=torch.float32, device=dev)
@@ -175,6 +202,11 @@ class Pipeline:
     def __call__(self, q_r, q, k_loc, v_loc, stream=None):
         self.router(q_r, self.kr_bar, self.coff, self.n_docs, self.doc_scores, None, stream)
         topk_docs(self.doc_scores, self.k, self.idx, self.top, self.topk_ws, stream)
+        if self.fused:  # attention reads the selected rows from the bank itself
+            self.attn(q, self.idx, self.coff, self.k_bar, self.v_bar, k_loc, v_loc, self.pos0,
+                      self.rope_base, 0.0, self.out, stream)
+            self.mem_len = self.attn.mem_len
+            return self.out
         gather_kv(self.idx, self.coff, self.k_bar, self.v_bar, self.m_cap, self.k_mem,
                   self.v_mem, self.mem_len, stream)
         self.attn(q, self.k_mem, self.v_mem, self.mem_len, k_loc, v_loc, self.pos0,

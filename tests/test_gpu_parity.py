@@ -583,6 +583,66 @@ def test_attention_decode_shapes(B, T_loc, Hq, H, m_cap, mem_lens):
     status_ok()
 
 
+@pytest.mark.parametrize("B,T_loc,Hq,H,k,n_docs", [
+    (5, 300, 32, 8, 6, 40),      # GQA 4:1, ragged documents
+    (3, 65, 16, 1, 9, 30),       # G = 16, one KV head
+    (4, 200, 8, 8, 3, 12),       # G = 1
+])
+def test_attention_fused_decode_vs_oracle(B, T_loc, Hq, H, k, n_docs):
+    """Fused assembly + decode attention: rows read from the bank in 8-row
+    groups (documents of 1..40 rows, most not a multiple of 8, one document
+    shared by two queries) against the oracle's gather + attention."""
+    D = 128
+    g = torch.Generator(device="cuda").manual_seed(T_loc + n_docs)
+    gc = torch.Generator().manual_seed(T_loc)
+    counts = torch.randint(1, 41, (n_docs,), generator=gc).numpy()
+    counts[0] = 1
+    coff_h = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    C = int(coff_h[-1])
+    kb = synth.randn((C, H, D), torch.bfloat16, "cuda", g)
+    vb = synth.randn((C, H, D), torch.bfloat16, "cuda", g)
+    idx_h = np.stack([np.random.default_rng(b).choice(n_docs, k, replace=False) for b in range(B)])
+    idx_h[1, 0] = idx_h[0, 0]
+    idx_h[0, -1] = 0  # the one-row document
+    idx = torch.from_numpy(idx_h).int().cuda()
+    q = synth.randn((B, 1, Hq, D), torch.bfloat16, "cuda", g)
+    kl = synth.randn((B, T_loc, H, D), torch.bfloat16, "cuda", g)
+    vl = synth.randn((B, T_loc, H, D), torch.bfloat16, "cuda", g)
+    m_cap = int(max(counts[r].sum() for r in idx_h))
+    att = pipeline.FusedAttention(torch.bfloat16, B, 1, T_loc, Hq, H, D, k, m_cap, "cuda")
+    out = att(q, idx, torch.from_numpy(coff_h).cuda(), kb, vb, kl, vl, k)
+    torch.cuda.synchronize()
+    okm, ovm, oml = oracle.gather_kv(idx_h, coff_h, f64(kb), f64(vb))
+    assert att.mem_len.cpu().tolist() == list(oml)
+    want = oracle.sparse_attn(f64(q), okm, ovm, f64(kl), f64(vl), k, 10000.0)
+    got = f64(out)
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got - want)) <= ATTN_BF16
+    status_ok()
+
+
+def test_attention_fused_capacity_and_bad_index():
+    """Fewer groups than the documents need: rows past the capacity are
+    dropped (mem_len says how many were used) and MSA_ERR_CAPACITY is
+    recorded."""
+    D, H, Hq, T_loc, k = 128, 8, 32, 64, 4
+    counts = np.array([30, 30, 30, 30, 30])
+    coff_h = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    g = torch.Generator(device="cuda").manual_seed(3)
+    kb = synth.randn((int(coff_h[-1]), H, D), torch.bfloat16, "cuda", g)
+    vb = synth.randn((int(coff_h[-1]), H, D), torch.bfloat16, "cuda", g)
+    idx = torch.tensor([[0, 1, 2, 3]], dtype=torch.int32, device="cuda")
+    q = synth.randn((1, 1, Hq, D), torch.bfloat16, "cuda", g)
+    kl = synth.randn((1, T_loc, H, D), torch.bfloat16, "cuda", g)
+    att = pipeline.FusedAttention(torch.bfloat16, 1, 1, T_loc, Hq, H, D, k, 40, "cuda")
+    out = att(q, idx, torch.from_numpy(coff_h).cuda(), kb, vb, kl, kl, k)
+    torch.cuda.synchronize()
+    # max_groups = ceil(40/8) + 4 = 9 groups; each document takes 4
+    assert int(att.mem_len[0]) == 30 + 30 + 8
+    assert np.all(np.isfinite(f64(out)))
+    assert msa.msa_device_status(clear=True) == -3
+
+
 def test_attention_decode_10m_workload_full():
     lengths = synth.bank_10m_lengths()
     coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
@@ -597,10 +657,15 @@ def test_attention_decode_10m_workload_full():
                                     torch.from_numpy(coff_h).cuda(), w["k_bar"], w["v_bar"], m_cap)
     att = pipeline.Attention(torch.bfloat16, B, 1, 2048, 32, 8, 128, m_cap, "cuda")
     out = att(w["q"], km, vm, ml, w["k_loc"], w["v_loc"], 16)
+    fatt = pipeline.FusedAttention(torch.bfloat16, B, 1, 2048, 32, 8, 128, 16, m_cap, "cuda")
+    fout = fatt(w["q"], torch.from_numpy(idx).int().cuda(), torch.from_numpy(coff_h).cuda(),
+                w["k_bar"], w["v_bar"], w["k_loc"], w["v_loc"], 16)
     torch.cuda.synchronize()
-    okm, ovm, _ = oracle.gather_kv(idx, coff_h, f64(w["k_bar"]), f64(w["v_bar"]))
+    okm, ovm, oml = oracle.gather_kv(idx, coff_h, f64(w["k_bar"]), f64(w["v_bar"]))
     want = oracle.sparse_attn(f64(w["q"]), okm, ovm, f64(w["k_loc"]), f64(w["v_loc"]), 16)
     assert np.max(np.abs(f64(out) - want)) <= ATTN_BF16
+    assert np.max(np.abs(f64(fout) - want)) <= ATTN_BF16  # the same, read from the bank
+    assert fatt.mem_len.cpu().tolist() == list(oml)
     status_ok()
 
 
