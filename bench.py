@@ -291,6 +291,16 @@ def run_libmsa(args, world, rank, local):
     torch.cuda.synchronize()
     prep_ms = q0.elapsed_time(q1)
 
+    # the same step with fused assembly + attention (no gathered copy)
+    pf = pipeline.Pipeline(w["kr_hat"], w["k_bar"], w["v_bar"], p.coff, B=1, T=w["T"],
+                           T_loc=w["T_loc"], Hq=w["Hq"], k=w["k"], m_cap=p.m_cap,
+                           pos0=w["pos0"], prepared=True, fused=True)
+    pf(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    graph_f = pf.capture(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    fused_ms = time_device(graph_f.replay, args.steps)
+    fused_same_idx = bool(torch.equal(pf.idx, p.idx))
+    del graph_f, pf
+
     launches = count_launches(p, w)
     status = msa.msa_device_status(clear=True)
 
@@ -337,6 +347,11 @@ def run_libmsa(args, world, rank, local):
                       "note": "eager launches with events between stages; the step "
                               "(ms_per_step) replays the same ten launches as one CUDA graph"},
         "route_gchunks_s": round(C / (route_ms * 1e-3) / 1e9, 4),
+        "fused_step": {"ms_per_step": round(fused_ms, 4),
+                       "gchunks_s": round(C * world / (fused_ms * 1e-3) / 1e9, 4),
+                       "note": "route -> top-k -> msa_sparse_attn_fused (memory read from the "
+                               "bank, no gather), one CUDA graph",
+                       "same_topk_as_step": fused_same_idx},
         "route_raw_bank": {"ms": round(raw_ms, 4),
                            "gchunks_s": round(C / (raw_ms * 1e-3) / 1e9, 4),
                            "hbm_frac": round(C * BYTES_PER_CHUNK / (raw_ms * 1e-3) / 1e9 / pk["hbm"], 4),
@@ -465,6 +480,16 @@ def bench_decode(steps: int, peak_hbm: float) -> dict:
                                             p.doc_scores, None), steps)
     ms_attn = time_device(lambda: p.attn(w["q"], p.k_mem, p.v_mem, p.mem_len, w["k_loc"],
                                          w["v_loc"], p.pos0, p.rope_base, 0.0, p.out), steps)
+    pf = pipeline.Pipeline(hat, w["k_bar"], w["v_bar"], coff, B=w["B"], T=1, T_loc=w["T_loc"],
+                           Hq=w["Hq"], k=w["k"], m_cap=m_cap, pos0=w["pos0"], prepared=True,
+                           fused=True)
+    pf(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    graph_f = pf.capture(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    ms_f = time_device(graph_f.replay, steps)
+    ms_attn_f = time_device(lambda: pf.attn(w["q"], pf.idx, pf.coff, pf.k_bar, pf.v_bar,
+                                            w["k_loc"], w["v_loc"], pf.pos0, pf.rope_base, 0.0,
+                                            pf.out), steps)
+    del graph_f
     H, D = p.H, p.D
     rows = int(p.mem_len.sum()) + w["B"] * w["T_loc"]
     attn_bytes = rows * H * D * 2 * 2 + 2 * w["q"].numel() * 2
@@ -478,8 +503,14 @@ def bench_decode(steps: int, peak_hbm: float) -> dict:
            "attn_ms": round(ms_attn, 4),
            "attn_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_hbm,
                              "unit": "GB/s", "frac": round(gbs / peak_hbm, 4)},
+           "fused": {"ms_per_step": round(ms_f, 4),
+                     "decode_tok_s": round(w["B"] / (ms_f * 1e-3), 1),
+                     "attn_ms": round(ms_attn_f, 4),
+                     "attn_gbs": round(attn_bytes / (ms_attn_f * 1e-3) / 1e9, 1),
+                     "note": "route -> top-k -> msa_sparse_attn_fused: memory rows read from "
+                             "the bank in 8-row groups, no gather"},
            "n_chunks": C}
-    del w, p, graph, hat
+    del w, p, pf, graph, hat
     torch.cuda.empty_cache()
     return res
 

@@ -87,13 +87,17 @@ FusedPlan fused_plan(int B, int T, int T_loc, int Hq, int H, int k, int m_cap) {
   p.max_groups = max_groups_for(k, m_cap);
   p.g_bytes = round_up((size_t)B * p.max_groups * sizeof(int2), 256);
   p.n_bytes = round_up((size_t)B * sizeof(int32_t), 256);
-  p.attn_bytes = T == 1 ? attn_decode_tc_fused_workspace_size(B, T_loc, Hq, H, p.max_groups) : 0;
+  p.attn_bytes = T == 1 ? attn_decode_tc_fused_workspace_size(B, T_loc, Hq, H, p.max_groups)
+                        : attn_tc_fused_workspace_size(B, T, T_loc, Hq, H, 128, p.max_groups);
   p.total = p.g_bytes + p.n_bytes + p.attn_bytes;
   return p;
 }
 
-bool fused_supported(msa_dtype dt, int T, int Hq, int H, int D) {
-  return dt == MSA_BF16 && attn_decode_tc_supported(T, Hq, H, D);
+bool fused_supported(msa_dtype dt, int B, int T, int T_loc, int Hq, int H, int D, int k,
+                     int m_cap) {
+  if (dt != MSA_BF16 || D != 128) return false;
+  if (T == 1) return attn_decode_tc_supported(T, Hq, H, D);
+  return attn_tc_supported(B, T, T_loc, Hq, H, D, 8 * max_groups_for(k, m_cap));
 }
 
 }  // namespace
@@ -103,7 +107,7 @@ extern "C" size_t msa_sparse_attn_fused_workspace_size(msa_dtype dt, int B, int 
                                                        int Hq, int H, int D, int k, int m_cap) {
   using namespace msa;
   if (B <= 0 || T <= 0 || T_loc < T || H <= 0 || Hq % H || k <= 0 || m_cap < 0) return 0;
-  if (!fused_supported(dt, T, Hq, H, D)) return 0;
+  if (!fused_supported(dt, B, T, T_loc, Hq, H, D, k, m_cap)) return 0;
   return fused_plan(B, T, T_loc, Hq, H, k, m_cap).total;
 }
 
@@ -123,7 +127,7 @@ extern "C" int msa_sparse_attn_fused(msa_dtype dt, int B, int T, int T_loc, int 
     return MSA_ERR_INVALID_ARG;
   if (!(rope_base > 0.f)) return MSA_ERR_INVALID_ARG;
   if (Hq % H) return MSA_ERR_UNSUPPORTED;
-  if (!fused_supported(dt, T, Hq, H, D)) return MSA_ERR_UNSUPPORTED;
+  if (!fused_supported(dt, B, T, T_loc, Hq, H, D, k, m_cap)) return MSA_ERR_UNSUPPORTED;
   if (n_chunks > INT32_MAX - 8 || B > 0x7fffffff) return MSA_ERR_UNSUPPORTED;
   const FusedPlan p = fused_plan(B, T, T_loc, Hq, H, k, m_cap);
   if ((int64_t)B * p.max_groups * 8 > INT32_MAX) return MSA_ERR_UNSUPPORTED;
@@ -141,6 +145,9 @@ extern "C" int msa_sparse_attn_fused(msa_dtype dt, int B, int T, int T_loc, int 
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
   const float qscale = sc * 1.4426950408889634f;  // log2(e): softmax in base 2
   const FusedMemory fm{groups, n_groups, p.max_groups, k_bar, v_bar, n_chunks};
-  return attn_decode_tc_launch_fused(B, T_loc, Hq, H, D, q, fm, k_loc, v_loc, pos0, rope_base,
-                                     qscale, out, attn_ws, s);
+  if (T == 1)
+    return attn_decode_tc_launch_fused(B, T_loc, Hq, H, D, q, fm, k_loc, v_loc, pos0, rope_base,
+                                       qscale, out, attn_ws, s);
+  return attn_tc_launch_fused(B, T, T_loc, Hq, H, D, q, fm, k_loc, v_loc, pos0, rope_base, qscale,
+                              out, attn_ws, s);
 }

@@ -134,12 +134,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int D>
+// kFused: memory rows read straight from the pooled bank, per query a list
+// of 8-row groups (first bank row, rows of the group inside its document)
+// in rank order; tm_km / tm_vm map the bank with 8-row boxes (one
+// 128B-swizzle atom), a memory tile is 16 groups, and `mem_len` holds the
+// group count.  Rows past a document's end are finite bank rows, masked.
+template <int D, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_km,
                const __grid_constant__ CUtensorMap tm_vm, const __grid_constant__ CUtensorMap tm_kl,
                const __grid_constant__ CUtensorMap tm_vl, int T, int T_loc, int Hq, int H, int G,
-               const int32_t* __restrict__ mem_len, int m_cap, float qscale, int n_split,
+               const int32_t* __restrict__ mem_len, int m_cap, const int2* __restrict__ groups,
+               int max_groups, float qscale, int n_split,
                __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
                float2* __restrict__ part_ml, int* __restrict__ status) {
   using K = ACfg<D>;
@@ -159,7 +165,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int TQ = kRows / G;          // tokens per Q tile
   const int tok0 = mt * kQT * TQ;    // first token of the CTA
   const int n_tok = min(kQT * TQ, T - tok0);
-  const int M = min(max(mem_len[b], 0), m_cap);
+  const int M =
+      kFused ? 8 * min(max(mem_len[b], 0), max_groups) : min(max(mem_len[b], 0), m_cap);
+  const int2* gq = kFused ? groups + (int64_t)b * max_groups : nullptr;
   const int lim_max = T_loc - T + tok0 + n_tok - 1;  // last local key any row sees
   const int n_mt = (M + kKeys - 1) / kKeys;
   const int n_lt = (lim_max + 1 + kKeys - 1) / kKeys;
@@ -231,11 +239,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const bool mem = jj < n_mt;
         const CUtensorMap* mk = mem ? &tm_km : &tm_kl;
         const CUtensorMap* mv = mem ? &tm_vm : &tm_vl;
-        const int row = mem ? b * m_cap + jj * kKeys : b * T_loc + (jj - n_mt) * kKeys;
+        if (kFused && mem) {
+          // 16 groups of 8 bank rows; past the last group, repeat it (finite
+          // rows, masked) so every row of the tile is written
+          const int ng = M / 8, g0 = jj * (kKeys / 8);
+          for (int gi = 0; gi < kKeys / 8; ++gi) {
+            const int src = gq[min(g0 + gi, ng - 1)].x;
 #pragma unroll
-        for (int kb = 0; kb < K::KB; ++kb) {
-          tc::tma_load_3d(k_dst + kb * kKeys * 128, mk, &aux.kv_full[st], kb * 64, g, row);
-          tc::tma_load_3d(v_dst + kb * kKeys * 128, mv, &aux.kv_full[st], kb * 64, g, row);
+            for (int kb = 0; kb < K::KB; ++kb) {
+              tc::tma_load_3d(k_dst + kb * kKeys * 128 + gi * 1024, mk, &aux.kv_full[st],
+                              kb * 64, g, src);
+              tc::tma_load_3d(v_dst + kb * kKeys * 128 + gi * 1024, mv, &aux.kv_full[st],
+                              kb * 64, g, src);
+            }
+          }
+        } else {
+          const int row = mem ? b * m_cap + jj * kKeys : b * T_loc + (jj - n_mt) * kKeys;
+#pragma unroll
+          for (int kb = 0; kb < K::KB; ++kb) {
+            tc::tma_load_3d(k_dst + kb * kKeys * 128, mk, &aux.kv_full[st], kb * 64, g, row);
+            tc::tma_load_3d(v_dst + kb * kKeys * 128, mv, &aux.kv_full[st], kb * 64, g, row);
+          }
         }
         ++issued;
       }
@@ -337,7 +361,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::tmem_ld_wait();
       // keys a row may not see read as -inf (also hides whatever S holds
       // there: rows past mem_len, keys past the causal limit)
-      if (!__all_sync(0xffffffffu, n_vis == kKeys)) {
+      if (kFused && mem) {
+        // valid rows of each of the tile's 16 groups (0 past the last
+        // group), read as the columns reach each group
+        bool all8 = true;
+        for (int gi = 0; gi < kKeys / 8; ++gi) {
+          const int grp = key0 / 8 + gi;
+          all8 &= grp < M / 8 && gq[grp].y == 8;
+        }
+        if (!all8) {
+          int nvg = 0;
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c) {
+            if ((c & 7) == 0) {
+              const int grp = key0 / 8 + (c >> 3);
+              nvg = grp < M / 8 ? gq[grp].y : 0;
+            }
+            if ((c & 7) >= nvg) sv[c] = 0xff800000u;
+          }
+        }
+      } else if (!__all_sync(0xffffffffu, n_vis == kKeys)) {
 #pragma unroll
         for (int c = 0; c < kKeys; ++c)
           if (c >= n_vis) sv[c] = 0xff800000u;
@@ -396,7 +439,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       asm("add.rn.f32x2 %0, %0, %1;" : "+l"(ls2[0]) : "l"(ls2[1]));
       const float ls = __uint_as_float((uint32_t)ls2[0]) + __uint_as_float((uint32_t)(ls2[0] >> 32));
       l_run += ls;
-      if (mem && M - key0 < kKeys) {
+      if (!kFused && mem && M - key0 < kKeys) {
         // rows past mem_len in the last memory tile hold whatever the
         // caller's buffer holds there; zero their V so that 0 * V stays 0
         const int vrow = quad * 32 + lane;  // one V row per thread of group 0
@@ -604,9 +647,10 @@ template <int D>
 int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void* k_mem,
               const void* v_mem, const int32_t* mem_len, int m_cap, const void* k_loc,
               const void* v_loc, int pos0, float rope_base, float qscale, void* out, void* ws,
-              cudaStream_t s) {
+              cudaStream_t s, const FusedMemory* fm) {
   using K = ACfg<D>;
   const int G = Hq / H;
+  if (fm) m_cap = 8 * fm->max_groups;  // memory rows a query can have, for the plan
   const TcPlan p = tc_plan(B, T, T_loc, Hq, H, D, m_cap);
   unsigned char* w = static_cast<unsigned char*>(ws);
   __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(w);
@@ -624,20 +668,25 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   const int64_t mem_rows = std::max<int64_t>((int64_t)B * m_cap, 1);
   const void* km = m_cap > 0 ? k_mem : k_rot;  // any valid address when there is no memory
   const void* vm = m_cap > 0 ? v_mem : v_loc;
-  if (!map3(&tq, q_rot, D, Hq, (int64_t)B * T, G, TQ) ||
-      !map3(&tkm, km, D, H, m_cap > 0 ? mem_rows : (int64_t)B * T_loc, 1, kKeys) ||
-      !map3(&tvm, vm, D, H, m_cap > 0 ? mem_rows : (int64_t)B * T_loc, 1, kKeys) ||
+  const bool mem_ok =
+      fm ? map3(&tkm, fm->k_bar, D, H, fm->n_chunks, 1, 8) &&
+               map3(&tvm, fm->v_bar, D, H, fm->n_chunks, 1, 8)
+         : map3(&tkm, km, D, H, m_cap > 0 ? mem_rows : (int64_t)B * T_loc, 1, kKeys) &&
+               map3(&tvm, vm, D, H, m_cap > 0 ? mem_rows : (int64_t)B * T_loc, 1, kKeys);
+  if (!mem_ok || !map3(&tq, q_rot, D, Hq, (int64_t)B * T, G, TQ) ||
       !map3(&tkl, k_rot, D, H, (int64_t)B * T_loc, 1, kKeys) ||
       !map3(&tvl, v_loc, D, H, (int64_t)B * T_loc, 1, kKeys))
     return note_cuda(cudaErrorInvalidValue);
-  auto kern = attn_tc_kernel<D>;
+  auto kern = fm ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>;
   rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
   const int n_qb = (T + kQT * TQ - 1) / (kQT * TQ);
   if (n_qb > 65535 || B > 65535) return MSA_ERR_UNSUPPORTED;
   const dim3 grid((unsigned)(p.n_split * H), (unsigned)B, (unsigned)n_qb);
-  kern<<<grid, kThreads, K::SMEM, s>>>(tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G, mem_len,
-                                       m_cap, qscale, p.n_split, static_cast<__nv_bfloat16*>(out),
+  kern<<<grid, kThreads, K::SMEM, s>>>(tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G,
+                                       fm ? fm->n_groups : mem_len, m_cap,
+                                       fm ? fm->groups : nullptr, fm ? fm->max_groups : 0,
+                                       qscale, p.n_split, static_cast<__nv_bfloat16*>(out),
                                        part_o, part_ml, device_status_ptr());
   rc = check_launch();
   if (rc || p.n_split == 1) return rc;
@@ -672,9 +721,27 @@ int attn_tc_launch(int B, int T, int T_loc, int Hq, int H, int D, const void* q,
     return MSA_ERR_INVALID_ARG;
   if (D == 64)
     return launch_tc<64>(B, T, T_loc, Hq, H, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc, pos0,
-                         rope_base, qscale, out, ws, s);
+                         rope_base, qscale, out, ws, s, nullptr);
   return launch_tc<128>(B, T, T_loc, Hq, H, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc, pos0,
-                        rope_base, qscale, out, ws, s);
+                        rope_base, qscale, out, ws, s, nullptr);
+}
+
+size_t attn_tc_fused_workspace_size(int B, int T, int T_loc, int Hq, int H, int D,
+                                    int max_groups) {
+  return tc_plan(B, T, T_loc, Hq, H, D, 8 * max_groups).total;
+}
+
+int attn_tc_launch_fused(int B, int T, int T_loc, int Hq, int H, int D, const void* q,
+                         const FusedMemory& fm, const void* k_loc, const void* v_loc, int pos0,
+                         float rope_base, float qscale, void* out, void* ws, cudaStream_t s) {
+  if (!aligned16(q) || !aligned16(k_loc) || !aligned16(v_loc) || !aligned16(out) ||
+      !aligned16(fm.k_bar) || !aligned16(fm.v_bar))
+    return MSA_ERR_INVALID_ARG;
+  if (D == 64)
+    return launch_tc<64>(B, T, T_loc, Hq, H, q, nullptr, nullptr, nullptr, 0, k_loc, v_loc,
+                         pos0, rope_base, qscale, out, ws, s, &fm);
+  return launch_tc<128>(B, T, T_loc, Hq, H, q, nullptr, nullptr, nullptr, 0, k_loc, v_loc, pos0,
+                        rope_base, qscale, out, ws, s, &fm);
 }
 
 }  // namespace msa

@@ -50,6 +50,11 @@ int attn_decode_tc_launch(int B, int T_loc, int Hq, int H, int D, const void* q,
                           int m_cap, const void* k_loc, const void* v_loc, int pos0,
                           float rope_base, float qscale, void* out, void* ws, cudaStream_t s);
 size_t attn_decode_tc_fused_workspace_size(int B, int T_loc, int Hq, int H, int max_groups);
+size_t attn_tc_fused_workspace_size(int B, int T, int T_loc, int Hq, int H, int D,
+                                    int max_groups);
+int attn_tc_launch_fused(int B, int T, int T_loc, int Hq, int H, int D, const void* q,
+                         const FusedMemory& fm, const void* k_loc, const void* v_loc, int pos0,
+                         float rope_base, float qscale, void* out, void* ws, cudaStream_t s);
 int attn_decode_tc_launch_fused(int B, int T_loc, int Hq, int H, int D, const void* q,
                                 const FusedMemory& fm, const void* k_loc, const void* v_loc,
                                 int pos0, float rope_base, float qscale, void* out, void* ws,

@@ -583,15 +583,18 @@ def test_attention_decode_shapes(B, T_loc, Hq, H, m_cap, mem_lens):
     status_ok()
 
 
-@pytest.mark.parametrize("B,T_loc,Hq,H,k,n_docs", [
-    (5, 300, 32, 8, 6, 40),      # GQA 4:1, ragged documents
-    (3, 65, 16, 1, 9, 30),       # G = 16, one KV head
-    (4, 200, 8, 8, 3, 12),       # G = 1
+@pytest.mark.parametrize("B,T,T_loc,Hq,H,k,n_docs", [
+    (5, 1, 300, 32, 8, 6, 40),      # decode, GQA 4:1, ragged documents
+    (3, 1, 65, 16, 1, 9, 30),       # decode, G = 16, one KV head
+    (4, 1, 200, 8, 8, 3, 12),       # decode, G = 1
+    (2, 64, 64, 32, 8, 6, 40),      # prefill
+    (1, 256, 256, 32, 8, 16, 60),   # prefill at the 100M-bank step's shape
+    (2, 300, 700, 16, 8, 7, 25),    # chunked prefill, several key tiles, G = 2
 ])
-def test_attention_fused_decode_vs_oracle(B, T_loc, Hq, H, k, n_docs):
-    """Fused assembly + decode attention: rows read from the bank in 8-row
-    groups (documents of 1..40 rows, most not a multiple of 8, one document
-    shared by two queries) against the oracle's gather + attention."""
+def test_attention_fused_vs_oracle(B, T, T_loc, Hq, H, k, n_docs):
+    """Fused assembly + attention: rows read from the bank in 8-row groups
+    (documents of 1..40 rows, most not a multiple of 8, one document shared
+    by two queries) against the oracle's gather + attention."""
     D = 128
     g = torch.Generator(device="cuda").manual_seed(T_loc + n_docs)
     gc = torch.Generator().manual_seed(T_loc)
@@ -602,14 +605,16 @@ def test_attention_fused_decode_vs_oracle(B, T_loc, Hq, H, k, n_docs):
     kb = synth.randn((C, H, D), torch.bfloat16, "cuda", g)
     vb = synth.randn((C, H, D), torch.bfloat16, "cuda", g)
     idx_h = np.stack([np.random.default_rng(b).choice(n_docs, k, replace=False) for b in range(B)])
-    idx_h[1, 0] = idx_h[0, 0]
-    idx_h[0, -1] = 0  # the one-row document
+    if B > 1:
+        idx_h[1, 0] = idx_h[0, 0]
+    if 0 not in idx_h[0]:
+        idx_h[0, -1] = 0  # the one-row document
     idx = torch.from_numpy(idx_h).int().cuda()
-    q = synth.randn((B, 1, Hq, D), torch.bfloat16, "cuda", g)
+    q = synth.randn((B, T, Hq, D), torch.bfloat16, "cuda", g)
     kl = synth.randn((B, T_loc, H, D), torch.bfloat16, "cuda", g)
     vl = synth.randn((B, T_loc, H, D), torch.bfloat16, "cuda", g)
     m_cap = int(max(counts[r].sum() for r in idx_h))
-    att = pipeline.FusedAttention(torch.bfloat16, B, 1, T_loc, Hq, H, D, k, m_cap, "cuda")
+    att = pipeline.FusedAttention(torch.bfloat16, B, T, T_loc, Hq, H, D, k, m_cap, "cuda")
     out = att(q, idx, torch.from_numpy(coff_h).cuda(), kb, vb, kl, vl, k)
     torch.cuda.synchronize()
     okm, ovm, oml = oracle.gather_kv(idx_h, coff_h, f64(kb), f64(vb))
