@@ -14,6 +14,10 @@ msa_oracle
 msa_loops
     A second, deliberately loop-only implementation for tiny shapes, used to
     pin ``msa_oracle`` against a structurally different restatement.
+msa_backward
+    The backward pass of chunk pooling and routing (gradients of the token
+    tensors and of the routing query / bank from the gradients of the pooled
+    bank and of the document scores), for training with a routing loss.
 """
 
 from .msa_oracle import (  # noqa: F401
@@ -34,4 +38,10 @@ from .msa_oracle import (  # noqa: F401
     gather_kv,
     sparse_attn,
     msa_forward,
+)
+from .msa_backward import (  # noqa: F401,E402
+    cosine_grad,
+    encode_pool_backward,
+    route_argmax,
+    route_scores_backward,
 )
