@@ -264,6 +264,39 @@ int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, int H,
                     float rope_base, float scale, void* out, void* ws,
                     size_t ws_bytes, msa_stream_t stream);
 
+/* Backward of the routing score -- "深度分析MSA" §"四、训练阶段：学习 memory
+ * 与路由": the routing auxiliary loss (BCE or InfoNCE on the document
+ * scores) trains Q_r and K_r.  Given dL/d(doc_scores) it ADDS to the
+ * caller's (zeroed) gradient buffers:
+ *   d_doc    [B][n_docs] float (device): dL/d(doc score); zero entries cost
+ *            nothing.
+ *   dq_r     [B][T][H][D] float, accumulated.
+ *   dkr_bar  [n_chunks][H][D] float, accumulated (gradient of the raw,
+ *            unnormalised pooled routing keys).
+ *   q_r, kr_bar, chunk_offsets: as msa_route_scores (dt f32 or bf16).
+ * A document's score is that of its best (chunk, query token) pair; the
+ * gradient goes to the first maximiser (lowest chunk, then lowest token),
+ * recomputed here in fp32.  Cost: one pass over the document's chunks and
+ * the query's tokens per (query, document) pair with a non-zero gradient.
+ * Supported: D in {64,128}, H <= 16, H*D <= 1024. */
+int msa_route_backward(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
+                       const void* kr_bar, int64_t n_chunks, const int64_t* chunk_offsets,
+                       int n_docs, const float* d_doc, float* dq_r, float* dkr_bar,
+                       msa_stream_t stream);
+
+/* Backward of the memory encoding (chunk pooling with document-wise RoPE on
+ * K) -- the same training step: the gradient of the pooled bank reaches the
+ * token tensors.  All float:
+ *   dk_bar, dv_bar, dkr_bar  [L][n_chunks][H][D] (device).
+ *   dk_tok, dv_tok, dkr_tok  [L][n_tok][H][D], written.
+ * Each token gets its chunk's gradient / (tokens in the chunk); K's is
+ * rotated back by the token's document-wise position.  D in {64,128}. */
+int msa_encode_pool_backward(int L, int64_t n_tok, int n_docs, int H, int D,
+                             const float* dk_bar, const float* dv_bar, const float* dkr_bar,
+                             const int64_t* tok_offsets, const int64_t* chunk_offsets,
+                             int64_t n_chunks, float rope_base, float* dk_tok, float* dv_tok,
+                             float* dkr_tok, msa_stream_t stream);
+
 /* Fused context assembly + sparse attention -- [HYSEN] §"Memory must be
  * encoded offline ..." (only the selected documents' K/V are loaded and
  * joined with the local context) and §"Routing happens inside attention

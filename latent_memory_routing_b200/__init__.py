@@ -18,8 +18,10 @@ from .msa import (  # noqa: F401
     msa_chunk_offsets,
     msa_device_status,
     msa_encode_pool,
+    msa_encode_pool_backward,
     msa_gather_kv,
     msa_last_cuda_error,
+    msa_route_backward,
     msa_route_prepare_bank,
     msa_route_scores,
     msa_route_scores_prepared,

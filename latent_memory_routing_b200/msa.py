@@ -66,6 +66,10 @@ _SIGS = {
                             c_p, c_p]),
     "msa_sparse_attn_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_i]),
     "msa_sparse_attn_fused_workspace_size": (c_sz, [c_i] * 9),
+    "msa_route_backward": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i64, c_p, c_i, c_p, c_p,
+                                 c_p, c_p]),
+    "msa_encode_pool_backward": (c_i, [c_i, c_i64, c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_p,
+                                       c_i64, c_f, c_p, c_p, c_p, c_p]),
     "msa_sparse_attn_fused": (c_i, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i, c_p, c_i,
                                     c_p, c_p, c_i64, c_i, c_p, c_p, c_i, c_f, c_f, c_p, c_p,
                                     c_p, c_sz, c_p]),
@@ -297,3 +301,28 @@ def msa_sparse_attn_fused(dt, B, T, T_loc, Hq, H, D, q, idx, k, chunk_offsets, n
         dt, B, T, T_loc, Hq, H, D, _ptr(q), _ptr(idx), k, _ptr(chunk_offsets), n_docs,
         _ptr(k_bar), _ptr(v_bar), n_chunks, m_cap, _ptr(k_loc), _ptr(v_loc), pos0, rope_base,
         scale, _ptr(out), _ptr(mem_len), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def msa_route_backward(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_docs, d_doc,
+                       dq_r, dkr_bar, stream=None):
+    _numel_ok(q_r, B * T * H * D, "q_r")
+    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
+    _numel_ok(d_doc, B * n_docs, "d_doc")
+    _numel_ok(dq_r, B * T * H * D, "dq_r")
+    _numel_ok(dkr_bar, n_chunks * H * D, "dkr_bar")
+    _check("msa_route_backward", lib().msa_route_backward(
+        dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
+        _ptr(d_doc), _ptr(dq_r), _ptr(dkr_bar), _stream(stream)))
+
+
+def msa_encode_pool_backward(L, n_tok, n_docs, H, D, dk_bar, dv_bar, dkr_bar, tok_offsets,
+                             chunk_offsets, n_chunks, rope_base, dk_tok, dv_tok, dkr_tok,
+                             stream=None):
+    for t, nm in ((dk_bar, "dk_bar"), (dv_bar, "dv_bar"), (dkr_bar, "dkr_bar")):
+        _numel_ok(t, L * n_chunks * H * D, nm)
+    for t, nm in ((dk_tok, "dk_tok"), (dv_tok, "dv_tok"), (dkr_tok, "dkr_tok")):
+        _numel_ok(t, L * n_tok * H * D, nm)
+    _check("msa_encode_pool_backward", lib().msa_encode_pool_backward(
+        L, n_tok, n_docs, H, D, _ptr(dk_bar), _ptr(dv_bar), _ptr(dkr_bar), _ptr(tok_offsets),
+        _ptr(chunk_offsets), n_chunks, rope_base, _ptr(dk_tok), _ptr(dv_tok), _ptr(dkr_tok),
+        _stream(stream)))

@@ -100,6 +100,32 @@ def gather_kv(idx, chunk_offs, k_bar, v_bar, m_cap: int, k_mem=None, v_mem=None,
     return k_mem, v_mem, mem_len
 
 
+def route_backward(q_r, kr_bar, chunk_offs, d_doc, dq_r=None, dkr_bar=None, stream=None):
+    """Gradients of the routing inputs from dL/d(doc_scores): ADDS into dq_r
+    [B][T][H][D] and dkr_bar [C][H][D] (fp32; zero buffers made if None)."""
+    B, T, H, D = q_r.shape
+    C = kr_bar.shape[0]
+    if dq_r is None:
+        dq_r = torch.zeros((B, T, H, D), dtype=torch.float32, device=q_r.device)
+    if dkr_bar is None:
+        dkr_bar = torch.zeros((C, H, D), dtype=torch.float32, device=q_r.device)
+    _m.msa_route_backward(dt_code(q_r), B, T, H, D, q_r, kr_bar, C, chunk_offs,
+                          chunk_offs.numel() - 1, d_doc, dq_r, dkr_bar, stream)
+    return dq_r, dkr_bar
+
+
+def encode_pool_backward(dk_bar, dv_bar, dkr_bar, tok_offs, chunk_offs, n_tok: int,
+                         rope_base: float = 10000.0, stream=None):
+    """Gradients of the token tensors [L][N][H][D] (fp32) from the pooled
+    bank's gradients [L][C][H][D] (fp32)."""
+    L, C, H, D = dk_bar.shape
+    outs = tuple(torch.empty((L, n_tok, H, D), dtype=torch.float32, device=dk_bar.device)
+                 for _ in range(3))
+    _m.msa_encode_pool_backward(L, n_tok, tok_offs.numel() - 1, H, D, dk_bar, dv_bar, dkr_bar,
+                                tok_offs, chunk_offs, C, rope_base, *outs, stream)
+    return outs
+
+
 def to_host_tier(t):
     """A copy of a bank tensor in pinned host memory.  Pinned allocations are
     mapped into every device's address space, so msa_gather_kv reads the

@@ -747,3 +747,62 @@ def test_1m_bank_chain_sampled():
         # the GPU routes its own bf16-rounded bank: allow the bank rounding
         assert abs(float(ds[0, d]) - od) <= ROUTE_ATOL + 2e-3, d
     status_ok()
+
+
+# ------------------------------------------------------------------ backward
+
+def _rel(got, want):
+    return np.max(np.abs(got - want)) / max(np.max(np.abs(want)), 1e-30)
+
+
+def test_encode_pool_backward_vs_oracle():
+    """Token gradients from pooled gradients: /count per chunk, K rotated
+    back by -p; two layers, documents with partial tails and a 1-token one."""
+    L, H, D = 2, 8, 128
+    lengths = np.array([180, 64, 1, 300, 77])
+    toff_h = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    coff_h = oracle.chunk_offsets_from_lengths(lengths)
+    N, C = int(toff_h[-1]), int(coff_h[-1])
+    g = torch.Generator(device="cuda").manual_seed(77)
+    dk, dv, dr = (torch.randn((L, C, H, D), generator=g, device="cuda") for _ in range(3))
+    gk, gv, gr = pipeline.encode_pool_backward(dk, dv, dr, torch.from_numpy(toff_h).cuda(),
+                                               torch.from_numpy(coff_h).cuda(), N)
+    torch.cuda.synchronize()
+    ok, ov, orr = oracle.encode_pool_backward(f64(dk), f64(dv), f64(dr), toff_h)
+    for got, want in ((gk, ok), (gv, ov), (gr, orr)):
+        assert _rel(f64(got), want) <= 1e-5
+    status_ok()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_route_backward_vs_oracle(dtype):
+    """dQ_r and dK̄_r from dL/d(doc_scores), against the oracle, on the
+    (query, document) pairs whose best and second best (chunk, token) pair
+    differ by more than 1e-4 (the argmax is then the same at fp32)."""
+    B, T, H, D, n_docs = 2, 40, 8, 128, 30
+    g = torch.Generator(device="cuda").manual_seed(5)
+    gc = torch.Generator().manual_seed(5)
+    lengths = torch.randint(1, 900, (n_docs,), generator=gc).numpy()
+    coff_h = oracle.chunk_offsets_from_lengths(lengths)
+    C = int(coff_h[-1])
+    q_r = synth.randn((B, T, H, D), dtype, "cuda", g)
+    kr = synth.randn((C, H, D), dtype, "cuda", g)
+    q64, k64 = f64(q_r), f64(kr)
+    qn = q64 / np.linalg.norm(q64, axis=-1, keepdims=True)
+    kn = k64 / np.linalg.norm(k64, axis=-1, keepdims=True)
+    rng = np.random.default_rng(5)
+    d_doc = np.zeros((B, n_docs))
+    for b in range(B):
+        for d in range(n_docs):
+            s = np.einsum("thd,chd->ct", qn[b], kn[coff_h[d]:coff_h[d + 1]]).ravel() / H
+            top2 = np.sort(s)[-2:] if s.size > 1 else np.array([-np.inf, s[0]])
+            if top2[1] - top2[0] > 1e-4 and rng.random() < 0.6:
+                d_doc[b, d] = rng.standard_normal()
+    assert np.count_nonzero(d_doc) >= 10
+    dq, dk = pipeline.route_backward(q_r, kr, torch.from_numpy(coff_h).cuda(),
+                                     torch.from_numpy(d_doc).float().cuda())
+    torch.cuda.synchronize()
+    oq, ok = oracle.route_scores_backward(q64, k64, coff_h, d_doc.astype(np.float32))
+    assert _rel(f64(dq), oq) <= 1e-4
+    assert _rel(f64(dk), ok) <= 1e-4
+    status_ok()
