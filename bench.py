@@ -376,7 +376,8 @@ def run_libmsa(args, world, rank, local):
         torch.cuda.empty_cache()
         line["workloads"] = {"encode_4l": bench_encode(max(args.steps // 4, 3), pk["hbm"]),
                              "bank_10m_decode": bench_decode(args.steps, pk["hbm"]),
-                             "bank_100m_tiered": tiered}
+                             "bank_100m_tiered": tiered,
+                             "backward_1m": bench_backward(max(args.steps // 4, 3), pk["hbm"])}
     return line
 
 
@@ -511,6 +512,59 @@ def bench_decode(steps: int, peak_hbm: float) -> dict:
                              "the bank in 8-row groups, no gather"},
            "n_chunks": C}
     del w, p, pf, graph, hat
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_backward(steps: int, peak_hbm: float) -> dict:
+    """Backward of routing and chunk pooling over the bank_1m document set
+    (1,000 docs, ~1M tokens, ~16.5K chunks): a dense dL/d(doc score) for one
+    128-token query -> dQ_r, dK̄_r; and the pooled banks' fp32 gradients ->
+    the 1M token rows' gradients."""
+    import torch
+
+    from latent_memory_routing_b200 import pipeline, synth
+    lengths = synth.bank_1m_lengths()
+    toff = synth.tok_offsets(lengths).cuda()
+    coff = pipeline.chunk_offsets(toff)
+    C, N = int(coff[-1]), int(toff[-1])
+    w = synth.backward_1m(coff.cpu(), N, "cuda")
+    H, D, T = w["H"], w["D"], w["T"]
+    dq = torch.zeros((1, T, H, D), dtype=torch.float32, device="cuda")
+    dk = torch.zeros((C, H, D), dtype=torch.float32, device="cuda")
+    ws = pipeline.route_backward_workspace(w["q_r"], w["kr_bar"], len(lengths))
+    ms_r = time_device(lambda: pipeline.route_backward(w["q_r"], w["kr_bar"], coff, w["d_doc"],
+                                                       dq, dk, ws=ws), steps)
+    # the argmax scan reads the routing bank once (2*H*D bytes per chunk) and
+    # does 2*H*D FLOP per (chunk, query token): 128 FLOP/B at T=128, below
+    # the ridge, so HBM bounds it; the gradient kernel touches only the
+    # pairs' rows
+    scan_bytes = C * H * D * 2
+    gbs = scan_bytes / (ms_r * 1e-3) / 1e9
+    tf = 2.0 * H * D * C * T / (ms_r * 1e-3) / 1e12
+    del dq, dk
+    outs = tuple(torch.empty((1, N, H, D), dtype=torch.float32, device="cuda") for _ in range(3))
+    ms_p = time_device(lambda: pipeline.encode_pool_backward(
+        w["dk_bar"], w["dv_bar"], w["dkr_bar"], toff, coff, N, out=outs), steps)
+    del outs
+    algo = 3 * C * H * D * 4 + 3 * N * H * D * 4
+    gbs_p = algo / (ms_p * 1e-3) / 1e9
+    res = {"workload": "backward_1m: bank_1m's 1,000 docs (U[256,1792] tokens, %d chunks); "
+                       "dense dL/d(doc score) for one 128-token query; fp32 pooled-bank "
+                       "gradients [1][C][8][128] x 3 -> token gradients [1][%d][8][128] x 3" % (C, N),
+           "route_backward_ms": round(ms_r, 4),
+           "route_backward_roofline": {
+               "bound": "hbm", "achieved": round(gbs, 1), "peak": peak_hbm, "unit": "GB/s",
+               "frac": round(gbs / peak_hbm, 4), "tflops": round(tf, 2),
+               "note": "whole call (query prep, key reset, tcgen05 argmax scan, gradient "
+                       "kernel) against the scan's bank bytes; a 34 MB bank is under one "
+                       "wave of tiles, so launch and pipeline fill dominate"},
+           "pool_backward_ms": round(ms_p, 4),
+           "pool_backward_roofline": {"bound": "hbm", "achieved": round(gbs_p, 1),
+                                      "peak": peak_hbm, "unit": "GB/s",
+                                      "frac": round(gbs_p / peak_hbm, 4)},
+           "n_chunks": C, "n_tok": N}
+    del w
     torch.cuda.empty_cache()
     return res
 

@@ -275,14 +275,25 @@ int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, int H,
  *            unnormalised pooled routing keys).
  *   q_r, kr_bar, chunk_offsets: as msa_route_scores (dt f32 or bf16).
  * A document's score is that of its best (chunk, query token) pair; the
- * gradient goes to the first maximiser (lowest chunk, then lowest token),
- * recomputed here in fp32.  Cost: one pass over the document's chunks and
- * the query's tokens per (query, document) pair with a non-zero gradient.
+ * gradient goes to the first maximiser (lowest chunk, then lowest token) and
+ * is computed in fp32 from q_r and kr_bar.
+ * bf16 with D in {64,128}, H <= 8 and n_chunks * T < 2^32: the maximisers are
+ * found by one tensor-core scan of the bank (as msa_route_scores, the
+ * cosines of bf16 unit rows summed in fp32; pairs whose best two cosines lie
+ * within that rounding may take either) and the gradient kernel visits only
+ * pairs with a non-zero gradient; ws must hold
+ * msa_route_backward_workspace_size() bytes (16-byte aligned) or the call
+ * returns MSA_ERR_WORKSPACE.  Otherwise (fp32, or MSA_ROUTE_BWD_TC=0 in the
+ * environment) the maximisers are recomputed in fp32 on the CUDA cores, one
+ * pass over the document's chunks and the query's tokens per pair with a
+ * non-zero gradient, and ws is unused (workspace size 0).
  * Supported: D in {64,128}, H <= 16, H*D <= 1024. */
+size_t msa_route_backward_workspace_size(msa_dtype dt, int B, int T, int H, int D,
+                                         int64_t n_chunks, int n_docs);
 int msa_route_backward(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
                        const void* kr_bar, int64_t n_chunks, const int64_t* chunk_offsets,
                        int n_docs, const float* d_doc, float* dq_r, float* dkr_bar,
-                       msa_stream_t stream);
+                       void* ws, size_t ws_bytes, msa_stream_t stream);
 
 /* Backward of the memory encoding (chunk pooling with document-wise RoPE on
  * K) -- the same training step: the gradient of the pooled bank reaches the

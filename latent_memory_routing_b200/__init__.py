@@ -22,6 +22,7 @@ from .msa import (  # noqa: F401
     msa_gather_kv,
     msa_last_cuda_error,
     msa_route_backward,
+    msa_route_backward_workspace_size,
     msa_route_prepare_bank,
     msa_route_scores,
     msa_route_scores_prepared,

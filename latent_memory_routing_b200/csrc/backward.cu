@@ -22,18 +22,27 @@
 //    (cos, sin) table built once (angles reduced in double); every token row
 //    of every layer is written once with 16-byte stores: V and K_r get the
 //    pooled gradient / count, K its rotation by -p.  HBM-bound on the writes.
-//  * route_backward_kernel: persistent CTAs over the (query, document) pairs
-//    whose gradient is non-zero.  A CTA recomputes the document's head-mean
-//    cosines for every (chunk, token) pair in fp32 from unit rows staged in
+//  * routing, bf16 (the tensor-core path): finding each document's first
+//    maximiser is the forward scan itself -- every (chunk, token) head-mean
+//    cosine -- so it runs as the tcgen05 routing kernel in its argmax mode
+//    (one 64-bit key per (query, document): score, then ~(chunk, token));
+//    route_grad_kernel then takes one warp per pair with a non-zero gradient
+//    and adds g/H * dcos/dq and g/H * dcos/dk for each head into dq_r and
+//    dkr_bar (fp32, atomically: pairs may share a token or a chunk).  The
+//    maximiser is decided on the scan's bf16 unit rows (fp32 sums); the
+//    gradient is taken from the inputs in fp32.
+//  * routing, fp32 (or MSA_ROUTE_BWD_TC=0): route_backward_kernel,
+//    persistent CTAs over the pairs with a non-zero gradient, recomputes the
+//    document's cosines in fp32 on the CUDA cores from unit rows staged in
 //    shared memory (8 chunks x 16 tokens at a time, two threads per pair),
-//    takes the first maximiser, then adds g/H * dcos/dq and g/H * dcos/dk for
-//    each head into dq_r and dkr_bar (fp32, atomically: pairs may share a
-//    token or a chunk).  Its cost grows with the pairs that carry gradient
-//    -- a loss over the selected documents and some negatives -- not with the
-//    bank.
+//    takes the first maximiser and adds the same gradients.  Its cost grows
+//    with the pairs that carry gradient, not with the bank.
 #include <algorithm>
 
+#include <cstdlib>
+
 #include "msa_common.cuh"
+#include "route_tc.cuh"
 
 namespace msa {
 namespace {
@@ -291,8 +300,101 @@ route_backward_kernel(int B, int T, int H, int D, const E* __restrict__ q_r,
   }
 }
 
+// Gradients at known first maximisers (the tensor-core argmax scan's keys):
+// one warp per (query, document) pair with a non-zero gradient; per head the
+// warp reduces |q|, |k| and q.k over D and adds g/H * dcos/dq and
+// g/H * dcos/dk into dq_r and dkr_bar.
+template <typename E>
+__global__ void __launch_bounds__(256)
+route_grad_kernel(int B, int T, int H, int D, const E* __restrict__ q_r,
+                  const E* __restrict__ kr, const int64_t* __restrict__ coff, int n_docs,
+                  const float* __restrict__ d_doc, const unsigned long long* __restrict__ keys,
+                  float* __restrict__ dq, float* __restrict__ dkr, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t HD = (int64_t)H * D;
+  const int64_t n_pairs = (int64_t)B * n_docs;
+  const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t pr = w0; pr < n_pairs; pr += nw) {
+    const float g = d_doc[pr];
+    if (g == 0.f) continue;
+    const unsigned long long key = keys[pr];
+    if (key == 0ull) {  // no chunk reached this pair (an empty document)
+      if (lane == 0) record_error(status, MSA_ERR_INVALID_ARG);
+      continue;
+    }
+    const int b = (int)(pr / n_docs), d = (int)(pr % n_docs);
+    const uint32_t local = 0xffffffffu - (uint32_t)key;
+    const int64_t cs = coff[d] + local / (uint32_t)T;
+    const int ts = (int)(local % (uint32_t)T);
+    const E* qv = q_r + ((int64_t)b * T + ts) * HD;
+    const E* kv = kr + cs * HD;
+    float* gq_out = dq + ((int64_t)b * T + ts) * HD;
+    float* gk_out = dkr + cs * HD;
+    const float gh = g / (float)H;
+    for (int h = 0; h < H; ++h) {
+      float nq = 0.f, nk = 0.f, dt = 0.f;
+      for (int i = lane; i < D; i += 32) {
+        const float x = to_f(qv[h * D + i]), y = to_f(kv[h * D + i]);
+        nq = fmaf(x, x, nq);
+        nk = fmaf(y, y, nk);
+        dt = fmaf(x, y, dt);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        nq += __shfl_xor_sync(0xffffffffu, nq, o);
+        nk += __shfl_xor_sync(0xffffffffu, nk, o);
+        dt += __shfl_xor_sync(0xffffffffu, dt, o);
+      }
+      const float lq = sqrtf(nq), lk = sqrtf(nk);
+      const float mq = fmaxf(lq, kEps), mk = fmaxf(lk, kEps);
+      const float cosv = dt / (mq * mk);
+      for (int i = lane; i < D; i += 32) {
+        const float x = to_f(qv[h * D + i]), y = to_f(kv[h * D + i]);
+        const float gq = y / (mq * mk) - (lq >= kEps ? cosv * x / (mq * mq) : 0.f);
+        const float gk = x / (mq * mk) - (lk >= kEps ? cosv * y / (mk * mk) : 0.f);
+        atomicAdd(gq_out + h * D + i, gh * gq);
+        atomicAdd(gk_out + h * D + i, gh * gk);
+      }
+    }
+  }
+}
+
+// The tensor-core path: bf16, D in {64, 128}, H <= 8, and every document's
+// (chunk, token) index fits the key's 32 bits (bounded by n_chunks * T).
+bool route_backward_tc(msa_dtype dt, int B, int T, int H, int D, int64_t n_chunks) {
+  static const bool enabled = [] {
+    const char* e = getenv("MSA_ROUTE_BWD_TC");
+    return !(e && e[0] == '0');
+  }();
+  return enabled && dt == MSA_BF16 && (D == 64 || D == 128) && H <= 8 &&
+         (int64_t)B * T <= (1LL << 24) && n_chunks * (int64_t)T < 0xffffffffLL;
+}
+
+struct BwdPlan {
+  int n_pad;
+  size_t q_bytes, key_bytes, total;
+};
+
+BwdPlan bwd_plan(int B, int T, int H, int D, int n_docs) {
+  BwdPlan p{};
+  p.n_pad = (int)route_tc_columns((int64_t)B * T);
+  p.q_bytes = round_up((size_t)p.n_pad * H * D * sizeof(__nv_bfloat16), 256);
+  p.key_bytes = round_up((size_t)B * n_docs * sizeof(unsigned long long), 256);
+  p.total = p.q_bytes + p.key_bytes;
+  return p;
+}
+
 }  // namespace
 }  // namespace msa
+
+extern "C" size_t msa_route_backward_workspace_size(msa_dtype dt, int B, int T, int H, int D,
+                                                    int64_t n_chunks, int n_docs) {
+  using namespace msa;
+  if (B <= 0 || T <= 0 || H <= 0 || n_docs <= 0 || n_chunks <= 0) return 0;
+  if (!route_backward_tc(dt, B, T, H, D, n_chunks)) return 0;
+  return bwd_plan(B, T, H, D, n_docs).total;
+}
 
 extern "C" int msa_encode_pool_backward(int L, int64_t n_tok, int n_docs, int H, int D,
                                         const float* dk_bar, const float* dv_bar,
@@ -326,7 +428,8 @@ extern "C" int msa_encode_pool_backward(int L, int64_t n_tok, int n_docs, int H,
 extern "C" int msa_route_backward(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
                                   const void* kr_bar, int64_t n_chunks,
                                   const int64_t* chunk_offsets, int n_docs, const float* d_doc,
-                                  float* dq_r, float* dkr_bar, msa_stream_t stream) {
+                                  float* dq_r, float* dkr_bar, void* ws, size_t ws_bytes,
+                                  msa_stream_t stream) {
   using namespace msa;
   if (B <= 0 || T <= 0 || H <= 0 || D <= 0 || n_chunks <= 0 || n_docs <= 0)
     return MSA_ERR_INVALID_ARG;
@@ -335,6 +438,30 @@ extern "C" int msa_route_backward(msa_dtype dt, int B, int T, int H, int D, cons
   if (dt != MSA_F32 && dt != MSA_BF16) return MSA_ERR_INVALID_ARG;
   if (n_chunks > 0x7fffffffLL || (int64_t)B * T > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (route_backward_tc(dt, B, T, H, D, n_chunks)) {
+    // (1) the first maximiser of every (query, document) on the tensor
+    // cores; (2) the cosine gradients at those pairs on the CUDA cores
+    const BwdPlan p = bwd_plan(B, T, H, D, n_docs);
+    if (!ws || ws_bytes < p.total || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+    if (!aligned16(q_r) || !aligned16(kr_bar)) return MSA_ERR_INVALID_ARG;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    auto* qhat = reinterpret_cast<__nv_bfloat16*>(w);
+    auto* keys = reinterpret_cast<unsigned long long*>(w + p.q_bytes);
+    const auto* q = static_cast<const __nv_bfloat16*>(q_r);
+    const auto* k = static_cast<const __nv_bfloat16*>(kr_bar);
+    int rc = route_prep_bf16_launch(B * T, H, D, p.n_pad, q, qhat, s);
+    if (rc) return rc;
+    if ((rc = note_cuda(cudaMemsetAsync(keys, 0, (size_t)B * n_docs * 8, s)))) return rc;
+    rc = route_tc_argmax_launch(B, T, H, D, qhat, p.n_pad, k, n_chunks, chunk_offsets, n_docs,
+                                keys, device_status_ptr(), s);
+    if (rc) return rc;
+    const int64_t pairs = (int64_t)B * n_docs;
+    const int grid = (int)std::min<int64_t>((pairs + 7) / 8, 16LL * num_sms());
+    route_grad_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(B, T, H, D, q, k, chunk_offsets, n_docs,
+                                                          d_doc, keys, dq_r, dkr_bar,
+                                                          device_status_ptr());
+    return check_launch();
+  }
   const size_t smem = (size_t)(kRbChunks + kRbTokens) * H * D * sizeof(float);
   const int64_t pairs = (int64_t)B * n_docs;
   const int grid = (int)std::min<int64_t>(pairs, 8LL * num_sms());

@@ -212,6 +212,19 @@ int route_scores_impl(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
 }  // namespace
 }  // namespace msa
 
+namespace msa {
+
+int route_prep_bf16_launch(int NT, int H, int D, int n_pad, const __nv_bfloat16* q_r,
+                           __nv_bfloat16* qhat, cudaStream_t s) {
+  const int64_t rows = (int64_t)n_pad * H;
+  const unsigned blocks = (unsigned)std::min<int64_t>((rows * 32 + 255) / 256 + 1, 1 << 20);
+  route_prep_kernel<__nv_bfloat16, __nv_bfloat16, true><<<blocks, 256, 0, s>>>(
+      NT, H, D, n_pad, q_r, qhat, nullptr, 0, nullptr, 0);
+  return check_launch();
+}
+
+}  // namespace msa
+
 extern "C" int msa_route_scores(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
                                 const void* kr_bar, int64_t n_chunks,
                                 const int64_t* chunk_offsets, int n_docs, float* doc_scores,

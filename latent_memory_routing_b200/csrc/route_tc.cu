@@ -193,12 +193,18 @@ __device__ __forceinline__ void reduce32(const uint32_t (&r)[32], int cs, int NT
   }
 }
 
-template <int N, int D, bool kPrep, bool kPair>
+// kArg: instead of the document maximum, each (query, document) gets the
+// 64-bit key of its first maximiser -- high word the order-preserving score,
+// low word ~((chunk - document's first chunk) * T + token) -- so one
+// atomicMax keeps the highest score, then the lowest chunk, then the lowest
+// token (the host guarantees (chunks of a document) * T < 2^32).
+template <int N, int D, bool kPrep, bool kPair, bool kArg>
 __global__ void __launch_bounds__(kThreads, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 int H, int NT, int T, int n_pass, int64_t C, int64_t n_tiles,
                 const int64_t* __restrict__ coff, int n_docs, uint32_t* __restrict__ doc_u,
-                uint32_t* __restrict__ chunk_u, int* __restrict__ status) {
+                uint32_t* __restrict__ chunk_u, unsigned long long* __restrict__ doc_key,
+                int* __restrict__ status) {
   using K = Cfg<N, D, kPrep, kPair>;
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ Aux aux;
@@ -432,8 +438,9 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int64_t c = c0 + row;
         const int d0 = aux.d0;
         const int64_t wend = aux.win[kWindow];
-        // this row's document
+        // this row's document (and, for kArg, the document's first chunk)
         int dd = -1;
+        int64_t cdoc = 0;
         if (c < C) {
           if (c < wend) {
             int lo = 0, hi = kWindow;  // win[lo] <= c < win[hi]
@@ -442,8 +449,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
               if (aux.win[mid] <= c) lo = mid; else hi = mid;
             }
             dd = d0 + lo;
+            if constexpr (kArg) cdoc = aux.win[lo];
           } else {  // more than kWindow documents in one tile (empty documents)
             dd = bisect_global(coff, d0, n_docs, c);
+            if constexpr (kArg) cdoc = __ldg(coff + dd);
           }
         }
         // next tile's window: base document and prefetch into registers
@@ -485,7 +494,68 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tc::tc_fence_after();
         const uint32_t tbase = tmem + lane_addr + ab * N;
         uint32_t r0[32], r1[32];
-        if (K::SCR_WORDS > 0 && T < 32) {
+        if constexpr (kArg) {
+          // First maximiser: per row and query, the best token (strictly
+          // greater keeps the first); per document, the best row (the key
+          // orders equal scores by chunk, then token).
+          const uint32_t row_base = (uint32_t)((c - cdoc) * T);
+          const bool head = emit.head;
+          auto emit_arg = [&](float mm, int tt, int bb) {
+            unsigned long long x =
+                valid ? ((unsigned long long)f2o(mm) << 32) |
+                            (unsigned long long)(0xffffffffu - (row_base + (uint32_t)tt))
+                      : 0ull;
+#pragma unroll
+            for (int k = 0; k < 5; ++k) {
+              const unsigned long long y = __shfl_down_sync(0xffffffffu, x, 1 << k);
+              if (same & (1u << k)) x = x > y ? x : y;
+            }
+            if (head) atomicMax(doc_key + (int64_t)bb * n_docs + dd, x);
+          };
+          int b = col0 / T;
+          int t = col0 - b * T;
+          float m = -INFINITY;
+          int mt = t;
+          auto fold_arg = [&](const uint32_t (&r)[32], int cs, bool last_chunk) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int col = cs + i;
+              if (col >= NT) break;  // warp-uniform
+              const float v = __uint_as_float(r[i]);
+              if (v > m) {
+                m = v;
+                mt = t;
+              }
+              if ((last_chunk && i == 31) || col + 1 >= NT || t + 1 == T) {
+                emit_arg(m, mt, b);
+                m = -INFINITY;
+              }
+              if (++t == T) {
+                t = 0;
+                ++b;
+              }
+            }
+          };
+          tc::tmem_ld32(tbase, r0);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < N / 32; j += 2) {
+            if (j + 1 < N / 32) tc::tmem_ld32(tbase + (j + 1) * 32, r1);
+            fold_arg(r0, col0 + j * 32, j + 1 == N / 32);
+            tc::tmem_ld_wait();
+            if (j + 1 < N / 32) {
+              if (j + 2 < N / 32) tc::tmem_ld32(tbase + (j + 2) * 32, r0);
+              fold_arg(r1, col0 + (j + 1) * 32, j + 2 == N / 32);
+              tc::tmem_ld_wait();
+            }
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (kPair) tc::mbar_arrive_cluster(tc::mapa_shared(&aux.acce[ab], 0));
+            else tc::mbar_arrive(&aux.acce[ab]);
+          }
+        } else if (K::SCR_WORDS > 0 && T < 32) {
           // Column-owner epilogue.  (1) each row folds its columns into one
           // maximum per query (slot) and parks it in shared memory, which
           // frees the accumulator at once; (2) lane s owns slot s (s + 32,
@@ -665,17 +735,17 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N, int D, bool kPrep, bool kPair = false>
+template <int N, int D, bool kPrep, bool kPair = false, bool kArg = false>
 int launch(int B, int T, int H, const __nv_bfloat16* qhat, int n_pad, const __nv_bfloat16* kr,
            int64_t C, const int64_t* coff, int n_docs, uint32_t* doc_u, uint32_t* chunk_u,
-           int* status, cudaStream_t s) {
+           unsigned long long* doc_key, int* status, cudaStream_t s) {
   using K = Cfg<N, D, kPrep, kPair>;
   CUtensorMap tm_k, tm_q;
   if (!make_map(&tm_k, kr, D, H, C, (uint64_t)D * 2, (uint64_t)H * D * 2, 1, kTile))
     return note_cuda(cudaErrorInvalidValue);
   if (!make_map(&tm_q, qhat, D, n_pad, H, (uint64_t)D * 2, (uint64_t)n_pad * D * 2, K::NB, 1))
     return note_cuda(cudaErrorInvalidValue);
-  auto kern = route_tc_kernel<N, D, kPrep, kPair>;
+  auto kern = route_tc_kernel<N, D, kPrep, kPair, kArg>;
   int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
   const int64_t n_tiles = (C + kTile - 1) / kTile;
@@ -699,11 +769,11 @@ int launch(int B, int T, int H, const __nv_bfloat16* qhat, int n_pad, const __nv
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return note_cuda(cudaLaunchKernelEx(&cfg, kern, tm_k, tm_q, H, NT, T, n_pass, C, n_tiles,
-                                        coff, n_docs, doc_u, chunk_u, status));
+                                        coff, n_docs, doc_u, chunk_u, doc_key, status));
   } else {
     const int grid = (int)std::min<int64_t>(n_tiles, num_sms());
     kern<<<grid, kThreads, K::SMEM, s>>>(tm_k, tm_q, H, NT, T, n_pass, C, n_tiles, coff, n_docs,
-                                         doc_u, chunk_u, status);
+                                         doc_u, chunk_u, doc_key, status);
     return check_launch();
   }
 }
@@ -731,15 +801,15 @@ int route_tc_launch(int B, int T, int H, int D, const __nv_bfloat16* qhat, int n
   if (prepared && N == 256 && pairs) {
     if (D == 128)
       return launch<256, 128, true, true>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u,
-                                          chunk_u, status, s);
+                                          chunk_u, nullptr, status, s);
     if (D == 64)
       return launch<256, 64, true, true>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u,
-                                         chunk_u, status, s);
+                                         chunk_u, nullptr, status, s);
   }
 #define MSA_ROUTE_CASE(NN, DD, PP)                                                        \
   if (N == NN && D == DD && prepared == PP)                                                \
     return launch<NN, DD, PP>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, doc_u, chunk_u, \
-                              status, s);
+                              nullptr, status, s);
   MSA_ROUTE_CASE(64, 64, false)
   MSA_ROUTE_CASE(64, 128, false)
   MSA_ROUTE_CASE(128, 64, false)
@@ -753,6 +823,25 @@ int route_tc_launch(int B, int T, int H, int D, const __nv_bfloat16* qhat, int n
   MSA_ROUTE_CASE(256, 64, true)
   MSA_ROUTE_CASE(256, 128, true)
 #undef MSA_ROUTE_CASE
+  return MSA_ERR_UNSUPPORTED;
+}
+
+int route_tc_argmax_launch(int B, int T, int H, int D, const __nv_bfloat16* qhat, int n_pad,
+                           const __nv_bfloat16* kr, int64_t C, const int64_t* coff, int n_docs,
+                           unsigned long long* doc_key, int* status, cudaStream_t s) {
+  const int N = n_pad <= 128 ? n_pad : 256;
+  if (!aligned16(qhat) || !aligned16(kr)) return MSA_ERR_INVALID_ARG;
+#define MSA_ARG_CASE(NN, DD)                                                             \
+  if (N == NN && D == DD)                                                                 \
+    return launch<NN, DD, false, false, true>(B, T, H, qhat, n_pad, kr, C, coff, n_docs, \
+                                              nullptr, nullptr, doc_key, status, s);
+  MSA_ARG_CASE(64, 64)
+  MSA_ARG_CASE(64, 128)
+  MSA_ARG_CASE(128, 64)
+  MSA_ARG_CASE(128, 128)
+  MSA_ARG_CASE(256, 64)
+  MSA_ARG_CASE(256, 128)
+#undef MSA_ARG_CASE
   return MSA_ERR_UNSUPPORTED;
 }
 

@@ -66,8 +66,9 @@ _SIGS = {
                             c_p, c_p]),
     "msa_sparse_attn_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_i]),
     "msa_sparse_attn_fused_workspace_size": (c_sz, [c_i] * 9),
+    "msa_route_backward_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i, c_i64, c_i]),
     "msa_route_backward": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i64, c_p, c_i, c_p, c_p,
-                                 c_p, c_p]),
+                                 c_p, c_p, c_sz, c_p]),
     "msa_encode_pool_backward": (c_i, [c_i, c_i64, c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_p,
                                        c_i64, c_f, c_p, c_p, c_p, c_p]),
     "msa_sparse_attn_fused": (c_i, [c_i, c_i, c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i, c_p, c_i,
@@ -303,8 +304,12 @@ def msa_sparse_attn_fused(dt, B, T, T_loc, Hq, H, D, q, idx, k, chunk_offsets, n
         scale, _ptr(out), _ptr(mem_len), _ptr(ws), ws_bytes, _stream(stream)))
 
 
+def msa_route_backward_workspace_size(dt, B, T, H, D, n_chunks, n_docs) -> int:
+    return lib().msa_route_backward_workspace_size(dt, B, T, H, D, n_chunks, n_docs)
+
+
 def msa_route_backward(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_docs, d_doc,
-                       dq_r, dkr_bar, stream=None):
+                       dq_r, dkr_bar, ws=None, ws_bytes=0, stream=None):
     _numel_ok(q_r, B * T * H * D, "q_r")
     _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
     _numel_ok(d_doc, B * n_docs, "d_doc")
@@ -312,7 +317,7 @@ def msa_route_backward(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_d
     _numel_ok(dkr_bar, n_chunks * H * D, "dkr_bar")
     _check("msa_route_backward", lib().msa_route_backward(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
-        _ptr(d_doc), _ptr(dq_r), _ptr(dkr_bar), _stream(stream)))
+        _ptr(d_doc), _ptr(dq_r), _ptr(dkr_bar), _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def msa_encode_pool_backward(L, n_tok, n_docs, H, D, dk_bar, dv_bar, dkr_bar, tok_offsets,

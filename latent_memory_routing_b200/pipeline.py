@@ -100,27 +100,40 @@ def gather_kv(idx, chunk_offs, k_bar, v_bar, m_cap: int, k_mem=None, v_mem=None,
     return k_mem, v_mem, mem_len
 
 
-def route_backward(q_r, kr_bar, chunk_offs, d_doc, dq_r=None, dkr_bar=None, stream=None):
+def route_backward_workspace(q_r, kr_bar, n_docs: int):
+    """The workspace msa_route_backward needs for these shapes (None if none)."""
+    B, T, H, D = q_r.shape
+    n = _m.msa_route_backward_workspace_size(dt_code(q_r), B, T, H, D, kr_bar.shape[0], n_docs)
+    return torch.empty(n, dtype=torch.uint8, device=q_r.device) if n else None
+
+
+def route_backward(q_r, kr_bar, chunk_offs, d_doc, dq_r=None, dkr_bar=None, ws=None,
+                   stream=None):
     """Gradients of the routing inputs from dL/d(doc_scores): ADDS into dq_r
-    [B][T][H][D] and dkr_bar [C][H][D] (fp32; zero buffers made if None)."""
+    [B][T][H][D] and dkr_bar [C][H][D] (fp32; zero buffers made if None).
+    ``ws``: from route_backward_workspace (made here if None)."""
     B, T, H, D = q_r.shape
     C = kr_bar.shape[0]
+    if ws is None:
+        ws = route_backward_workspace(q_r, kr_bar, chunk_offs.numel() - 1)
     if dq_r is None:
         dq_r = torch.zeros((B, T, H, D), dtype=torch.float32, device=q_r.device)
     if dkr_bar is None:
         dkr_bar = torch.zeros((C, H, D), dtype=torch.float32, device=q_r.device)
     _m.msa_route_backward(dt_code(q_r), B, T, H, D, q_r, kr_bar, C, chunk_offs,
-                          chunk_offs.numel() - 1, d_doc, dq_r, dkr_bar, stream)
+                          chunk_offs.numel() - 1, d_doc, dq_r, dkr_bar, ws,
+                          0 if ws is None else ws.numel(), stream)
     return dq_r, dkr_bar
 
 
 def encode_pool_backward(dk_bar, dv_bar, dkr_bar, tok_offs, chunk_offs, n_tok: int,
-                         rope_base: float = 10000.0, stream=None):
+                         rope_base: float = 10000.0, out=None, stream=None):
     """Gradients of the token tensors [L][N][H][D] (fp32) from the pooled
-    bank's gradients [L][C][H][D] (fp32)."""
+    bank's gradients [L][C][H][D] (fp32); ``out`` = (dk, dv, dkr) to reuse."""
     L, C, H, D = dk_bar.shape
-    outs = tuple(torch.empty((L, n_tok, H, D), dtype=torch.float32, device=dk_bar.device)
-                 for _ in range(3))
+    outs = out if out is not None else tuple(
+        torch.empty((L, n_tok, H, D), dtype=torch.float32, device=dk_bar.device)
+        for _ in range(3))
     _m.msa_encode_pool_backward(L, n_tok, tok_offs.numel() - 1, H, D, dk_bar, dv_bar, dkr_bar,
                                 tok_offs, chunk_offs, C, rope_base, *outs, stream)
     return outs

@@ -36,7 +36,7 @@ import math
 import torch
 
 SEEDS = {"tiny": 1001, "bank_1m": 1002, "bank_10m": 1003,
-         "bank_100m": 1004, "encode_4l": 1005}
+         "bank_100m": 1004, "encode_4l": 1005, "backward_1m": 1006}
 
 NEEDLE_SIGMA_TOKEN = 0.1
 NEEDLE_SIGMA_POOLED = 0.1 / 8.0
@@ -166,6 +166,31 @@ def bank_1m(device="cpu", n_docs: int = 1000, T: int = 128) -> dict:
     w["v_loc"] = randn((1, T, H, D), dt, device, g)
     plant_token_needles(w["kr_tok"], toff, needles, w["q_r"][0], g)
     return w
+
+
+def backward_1m(chunk_offsets, n_tok: int, device="cpu", T: int = 128) -> dict:
+    """Inputs of the backward of routing and pooling over the bank_1m
+    document set (lengths as ``bank_1m`` draws them; ``chunk_offsets`` and
+    ``n_tok`` from the caller): a pooled routing bank and one T-token query
+    (bf16 N(0,1)), a dense dL/d(doc score) over every document (the shape of
+    an InfoNCE gradient: softmax(scores) - one-hot, drawn here as N(0,1)/n_docs)
+    and fp32 N(0,1) gradients of the pooled K, V and K_r banks."""
+    g = _gen(device, SEEDS["backward_1m"])
+    H, D = 8, 128
+    C = int(chunk_offsets[-1])
+    n_docs = len(chunk_offsets) - 1
+    w = dict(name="backward_1m", H=H, D=D, T=T, B=1, n_docs=n_docs, n_tok=n_tok)
+    w["q_r"] = randn((1, T, H, D), torch.bfloat16, device, g)
+    w["kr_bar"] = randn((C, H, D), torch.bfloat16, device, g)
+    w["d_doc"] = torch.randn((1, n_docs), generator=g, device=device) / n_docs
+    for name in ("dk_bar", "dv_bar", "dkr_bar"):
+        w[name] = torch.randn((1, C, H, D), generator=g, device=device)
+    return w
+
+
+def bank_1m_lengths(n_docs: int = 1000) -> torch.Tensor:
+    """The document lengths ``bank_1m`` draws (its generator's first draw)."""
+    return lengths_uniform(n_docs, 256, 1792, _gen("cpu", SEEDS["bank_1m"]))
 
 
 def bank_10m_lengths(n_docs: int = 10000) -> torch.Tensor:

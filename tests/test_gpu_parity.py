@@ -774,13 +774,37 @@ def test_encode_pool_backward_vs_oracle():
     status_ok()
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_route_backward_vs_oracle(dtype):
+def _clear_gap_grad(q64, k64, coff_h, gap, rng, frac=0.6):
+    """dL/d(doc score): N(0,1) on a random subset of the (query, document)
+    pairs whose best and second-best (chunk, token) head-mean cosines differ
+    by more than `gap` (their first maximiser is then the same in any
+    precision within that gap), 0 elsewhere."""
+    B, T, H, _ = q64.shape
+    n_docs = len(coff_h) - 1
+    qn = q64 / np.linalg.norm(q64, axis=-1, keepdims=True)
+    kn = k64 / np.linalg.norm(k64, axis=-1, keepdims=True)
+    d_doc = np.zeros((B, n_docs))
+    for b in range(B):
+        for d in range(n_docs):
+            s = np.einsum("thd,chd->ct", qn[b], kn[coff_h[d]:coff_h[d + 1]]).ravel() / H
+            top2 = np.sort(s)[-2:] if s.size > 1 else np.array([-np.inf, s[0]])
+            if top2[1] - top2[0] > gap and rng.random() < frac:
+                d_doc[b, d] = rng.standard_normal()
+    return d_doc
+
+
+# (B, T): one 128-column pass; one 64-column pass; 300 query columns in two
+# 256-column passes, the second query's tokens split across them
+@pytest.mark.parametrize("dtype,B,T", [(torch.float32, 2, 40), (torch.bfloat16, 2, 40),
+                                       (torch.bfloat16, 1, 40), (torch.bfloat16, 2, 150)])
+def test_route_backward_vs_oracle(dtype, B, T):
     """dQ_r and dK̄_r from dL/d(doc_scores), against the oracle, on the
-    (query, document) pairs whose best and second best (chunk, token) pair
-    differ by more than 1e-4 (the argmax is then the same at fp32)."""
-    B, T, H, D, n_docs = 2, 40, 8, 128, 30
-    g = torch.Generator(device="cuda").manual_seed(5)
+    (query, document) pairs whose first maximiser is decided beyond rounding:
+    a gap above 1e-4 for the fp32 CUDA-core path, above 4e-3 (the routing
+    score tolerance) for the bf16 path, whose maximisers come from the
+    tensor-core scan of bf16 unit rows."""
+    H, D, n_docs = 8, 128, 30
+    g = torch.Generator(device="cuda").manual_seed(5 + B * T)
     gc = torch.Generator().manual_seed(5)
     lengths = torch.randint(1, 900, (n_docs,), generator=gc).numpy()
     coff_h = oracle.chunk_offsets_from_lengths(lengths)
@@ -788,16 +812,8 @@ def test_route_backward_vs_oracle(dtype):
     q_r = synth.randn((B, T, H, D), dtype, "cuda", g)
     kr = synth.randn((C, H, D), dtype, "cuda", g)
     q64, k64 = f64(q_r), f64(kr)
-    qn = q64 / np.linalg.norm(q64, axis=-1, keepdims=True)
-    kn = k64 / np.linalg.norm(k64, axis=-1, keepdims=True)
-    rng = np.random.default_rng(5)
-    d_doc = np.zeros((B, n_docs))
-    for b in range(B):
-        for d in range(n_docs):
-            s = np.einsum("thd,chd->ct", qn[b], kn[coff_h[d]:coff_h[d + 1]]).ravel() / H
-            top2 = np.sort(s)[-2:] if s.size > 1 else np.array([-np.inf, s[0]])
-            if top2[1] - top2[0] > 1e-4 and rng.random() < 0.6:
-                d_doc[b, d] = rng.standard_normal()
+    gap = 1e-4 if dtype == torch.float32 else 4e-3
+    d_doc = _clear_gap_grad(q64, k64, coff_h, gap, np.random.default_rng(5))
     assert np.count_nonzero(d_doc) >= 10
     dq, dk = pipeline.route_backward(q_r, kr, torch.from_numpy(coff_h).cuda(),
                                      torch.from_numpy(d_doc).float().cuda())
@@ -805,4 +821,53 @@ def test_route_backward_vs_oracle(dtype):
     oq, ok = oracle.route_scores_backward(q64, k64, coff_h, d_doc.astype(np.float32))
     assert _rel(f64(dq), oq) <= 1e-4
     assert _rel(f64(dk), ok) <= 1e-4
+    status_ok()
+
+
+def test_route_backward_first_maximiser_ties():
+    """Exact ties go to the first maximiser: two identical chunk rows and two
+    identical query tokens make four equal best pairs in document 1; the
+    gradient must reach only (its lower chunk, the lower token)."""
+    B, T, H, D = 1, 24, 8, 128
+    lengths = np.array([300, 640, 200])
+    coff_h = oracle.chunk_offsets_from_lengths(lengths)
+    C = int(coff_h[-1])
+    g = torch.Generator(device="cuda").manual_seed(11)
+    q_r = synth.randn((B, T, H, D), torch.bfloat16, "cuda", g)
+    kr = synth.randn((C, H, D), torch.bfloat16, "cuda", g)
+    q_r[0, 17] = q_r[0, 6]
+    c_a, c_b = int(coff_h[1]) + 2, int(coff_h[1]) + 7
+    row = (q_r[0, 6].float() + 0.8 * synth.randn((H, D), torch.float32, "cuda", g))
+    kr[c_a] = row.to(torch.bfloat16)
+    kr[c_b] = kr[c_a]
+    d_doc = torch.zeros((B, 3), dtype=torch.float32, device="cuda")
+    d_doc[0, 1] = 1.0
+    dq, dk = pipeline.route_backward(q_r, kr, torch.from_numpy(coff_h).cuda(), d_doc)
+    torch.cuda.synchronize()
+    oq, ok = oracle.route_scores_backward(f64(q_r), f64(kr), coff_h, f64(d_doc))
+    _, c_star, t_star = oracle.route_argmax(f64(q_r), f64(kr), coff_h)
+    assert (int(c_star[0, 1]), int(t_star[0, 1])) == (c_a, 6)
+    dq_h, dk_h = f64(dq), f64(dk)
+    assert np.count_nonzero(dq_h[0, 17]) == 0 and np.count_nonzero(dk_h[c_b]) == 0
+    assert np.count_nonzero(dq_h[0, 6]) > 0 and np.count_nonzero(dk_h[c_a]) > 0
+    assert _rel(dq_h, oq) <= 1e-4
+    assert _rel(dk_h, ok) <= 1e-4
+    status_ok()
+
+
+def test_route_backward_workspace_contract():
+    """bf16 takes the tensor-core path and needs its workspace; fp32 needs
+    none; a short workspace is refused before any launch."""
+    B, T, H, D, C, n_docs = 1, 16, 8, 128, 40, 4
+    assert msa.msa_route_backward_workspace_size(msa.MSA_BF16, B, T, H, D, C, n_docs) > 0
+    assert msa.msa_route_backward_workspace_size(msa.MSA_F32, B, T, H, D, C, n_docs) == 0
+    q = torch.zeros((B, T, H, D), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((C, H, D), dtype=torch.bfloat16, device="cuda")
+    coff = torch.tensor([0, 10, 20, 30, 40], dtype=torch.int64, device="cuda")
+    dd = torch.zeros((B, n_docs), dtype=torch.float32, device="cuda")
+    dq = torch.zeros((B, T, H, D), dtype=torch.float32, device="cuda")
+    dk = torch.zeros((C, H, D), dtype=torch.float32, device="cuda")
+    with pytest.raises(msa.MsaError):
+        msa.msa_route_backward(msa.MSA_BF16, B, T, H, D, q, k, C, coff, n_docs, dd, dq, dk,
+                               None, 0)
     status_ok()
