@@ -675,8 +675,28 @@ CASES = {
     "prefill_b1_t4096": dict(B=1, T=4096, T_loc=4096, M=384),
     "prefill_b2_t8192": dict(B=2, T=8192, T_loc=8192, M=384),
     "decode_b64_t2048": dict(B=64, T=1, T_loc=2048, M=250),
+    "prefill_b1_t256": dict(B=1, T=256, T_loc=256, M=273),  # the bank_100m step's attention
     "route_bank_10m_b64": None,  # routing, not attention: see run_route_case
+    "topk_b1_100k": None,        # the bank_100m step's top-16: see run_topk_case
 }
+
+
+def run_topk_case():
+    """The bank_100m step's selection: top-16 of 100,000 document scores,
+    three calls."""
+    import torch
+
+    from latent_memory_routing_b200 import build as _b
+    from latent_memory_routing_b200 import pipeline
+    _b.build()
+    g = torch.Generator(device="cuda").manual_seed(3)
+    s = torch.randn((1, 100000), device="cuda", generator=g) * 0.02 + 0.1
+    ws = pipeline.topk_workspace(1, 100000, 16, "cuda")
+    idx = torch.empty((1, 16), dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        pipeline.topk_docs(s, 16, idx, None, ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": "topk_b1_100k", "first": int(idx[0, 0])}))
 
 
 def run_route_case():
@@ -708,6 +728,8 @@ def run_case(name: str):
     from latent_memory_routing_b200 import pipeline, synth
     if name == "route_bank_10m_b64":
         return run_route_case()
+    if name == "topk_b1_100k":
+        return run_topk_case()
     _b.build()
     c = CASES[name]
     B, T, T_loc, M, Hq, H, D = c["B"], c["T"], c["T_loc"], c["M"], 32, 8, 128

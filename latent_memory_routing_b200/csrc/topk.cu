@@ -21,6 +21,14 @@
 //     (a bitonic sort above 2048 candidates) and writes the first k.
 // Very large score vectors whose segments would not fit in shared memory
 // keep their keys in global memory (L2) with the same select.
+// Small k (<= 32, the routing's top-16): a warp keeps a sorted list of its
+// 32 best keys, one per lane, and folds in 32 new keys at a time -- a
+// register bitonic sort of the batch (skipped when no key beats the
+// list's last), then the top 32 of the two sorted lists by one elementwise
+// maximum against the reversed batch and a 5-step bitonic merge.  A
+// 512-thread CTA takes a 1024-key segment (its 16 warps' lists merged the
+// same way, as a tree); a second kernel merges the segments' lists per
+// query.
 #include <algorithm>
 
 #include "msa_common.cuh"
@@ -257,14 +265,153 @@ topk_merge_kernel(int n, int k, int n_cand, const unsigned long long* __restrict
                top_out ? top_out + (int64_t)b * k : nullptr);
 }
 
+// ---------------------------------------------------------------- small k
+constexpr int kSmallK = 32;
+constexpr int kSmallThreads = 512;
+constexpr int kSmallWarps = kSmallThreads / 32;
+constexpr int kSmallBatches = 2;                           // 32-key batches per warp
+constexpr int kSmallSeg = kSmallThreads * kSmallBatches;   // keys per select CTA
+constexpr int kMergeSmemLists = 160;                       // lists a merge CTA stages (40 KB)
+
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
+  return a > b ? a : b;
+}
+__device__ __forceinline__ unsigned long long umin64(unsigned long long a, unsigned long long b) {
+  return a < b ? a : b;
+}
+
+// Sorts one key per lane, descending across lanes 0..31 (bitonic network).
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+      const bool desc = (lane & k) == 0 || k == 32;  // this block's direction
+      const bool lower = (lane & j) == 0;
+      x = (lower == desc) ? umax64(x, y) : umin64(x, y);
+    }
+  return x;
+}
+
+// Top 32 of two descending lists (one key per lane each), descending.
+__device__ __forceinline__ unsigned long long warp_merge_desc(unsigned long long a,
+                                                              unsigned long long b, int lane) {
+  // a descending, b reversed ascending: their elementwise maximum is the top
+  // 32 of the union, as a bitonic sequence
+  unsigned long long z = umax64(a, __shfl_sync(0xffffffffu, b, 31 - lane));
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(0xffffffffu, z, j);
+    z = (lane & j) == 0 ? umax64(z, y) : umin64(z, y);
+  }
+  return z;
+}
+
+// The block's per-warp sorted lists lists[0..kSmallWarps) -> lists[0], by a
+// tree of pairwise merges (log2(warps) levels).
+__device__ __forceinline__ unsigned long long block_merge_lists(
+    unsigned long long (*lists)[32], int warp, int lane) {
+#pragma unroll
+  for (int half = kSmallWarps / 2; half >= 1; half >>= 1) {
+    __syncthreads();
+    if (warp < half) lists[warp][lane] = warp_merge_desc(lists[warp][lane],
+                                                         lists[warp + half][lane], lane);
+  }
+  __syncthreads();
+  return lists[0][lane];
+}
+
+__device__ __forceinline__ void write_small(unsigned long long key, int lane, int k, int64_t row,
+                                            const float* __restrict__ s,
+                                            int32_t* __restrict__ idx_out,
+                                            float* __restrict__ top_out) {
+  if (lane < k) {
+    const uint32_t i = 0xffffffffu - (uint32_t)(key & 0xffffffffull);
+    idx_out[row * k + lane] = (int32_t)i;
+    if (top_out) top_out[row * k + lane] = s[i];
+  }
+}
+
+// grid (n_seg, B).  Each warp folds its 64 keys into a sorted top 32 (a
+// batch's sort is skipped when none of it beats the list's last); the
+// block merges the 16 lists.  n_seg == 1 writes the result, otherwise the
+// segment's sorted list goes to seg_out [B][n_seg][32].
+__global__ void __launch_bounds__(kSmallThreads)
+topk_small_select_kernel(int n, int k, const float* __restrict__ scores,
+                         int32_t* __restrict__ idx_out, float* __restrict__ top_out,
+                         unsigned long long* __restrict__ seg_out) {
+  __shared__ unsigned long long lists[kSmallWarps][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int b = blockIdx.y;
+  const float* s = scores + (int64_t)b * n;
+  const int64_t base = (int64_t)blockIdx.x * kSmallSeg + warp * 32 * kSmallBatches;
+  unsigned long long key[kSmallBatches];
+#pragma unroll
+  for (int i = 0; i < kSmallBatches; ++i) {  // all loads in flight first
+    const int64_t e = base + i * 32 + lane;
+    key[i] = e < n ? cand_key(score_key(__ldg(s + e)), (uint32_t)e) : 0ull;
+  }
+  unsigned long long list = warp_sort_desc(key[0], lane);
+#pragma unroll
+  for (int i = 1; i < kSmallBatches; ++i) {
+    const unsigned long long thr = __shfl_sync(0xffffffffu, list, 31);
+    if (__any_sync(0xffffffffu, key[i] > thr))
+      list = warp_merge_desc(list, warp_sort_desc(key[i], lane), lane);
+  }
+  lists[warp][lane] = list;
+  const unsigned long long acc = block_merge_lists(lists, warp, lane);
+  if (warp == 0) {
+    if (gridDim.x == 1) write_small(acc, lane, k, b, s, idx_out, top_out);
+    else seg_out[((int64_t)b * gridDim.x + blockIdx.x) * 32 + lane] = acc;
+  }
+}
+
+// grid (B): the n_seg sorted lists of one query -> its top-k in rank order.
+// Up to kMergeSmemLists lists are staged in shared memory by the whole block
+// first (one round of loads), then each warp folds its share and the block
+// merges the warps' lists.
+__global__ void __launch_bounds__(kSmallThreads)
+topk_small_merge_kernel(int n, int k, int n_seg, const unsigned long long* __restrict__ seg_in,
+                        const float* __restrict__ scores, int32_t* __restrict__ idx_out,
+                        float* __restrict__ top_out) {
+  __shared__ unsigned long long staged[kMergeSmemLists * 32];
+  __shared__ unsigned long long lists[kSmallWarps][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int b = blockIdx.x;
+  const unsigned long long* src = seg_in + (int64_t)b * n_seg * 32;
+  unsigned long long acc = 0ull;
+  for (int s0 = 0; s0 < n_seg; s0 += kMergeSmemLists) {
+    const int ns = min(kMergeSmemLists, n_seg - s0);
+    __syncthreads();  // the previous round's lists have been read
+    for (int e = threadIdx.x; e < ns * 32; e += kSmallThreads) staged[e] = src[(int64_t)s0 * 32 + e];
+    __syncthreads();
+    for (int sg = warp; sg < ns; sg += kSmallWarps) {
+      const unsigned long long x = staged[sg * 32 + lane];
+      const unsigned long long thr = __shfl_sync(0xffffffffu, acc, 31);
+      if (__any_sync(0xffffffffu, x > thr)) acc = warp_merge_desc(acc, x, lane);
+    }
+  }
+  lists[warp][lane] = acc;
+  acc = block_merge_lists(lists, warp, lane);
+  if (warp == 0) write_small(acc, lane, k, b, scores + (int64_t)b * n, idx_out, top_out);
+}
+
 struct TopkPlan {
   int seg_len, n_seg;
-  bool smem_keys;
+  bool smem_keys, small;
   size_t ws_bytes;
 };
 
 TopkPlan plan(int B, int n, int k) {
   TopkPlan p{};
+  if (k <= kSmallK && (int64_t)(n + kSmallSeg - 1) / kSmallSeg <= 65535) {
+    p.small = true;
+    p.seg_len = kSmallSeg;
+    p.n_seg = (n + kSmallSeg - 1) / kSmallSeg;
+    p.ws_bytes = p.n_seg > 1 ? (size_t)B * p.n_seg * kSmallK * sizeof(unsigned long long) : 0;
+    return p;
+  }
   if (n <= kSegSmem) {
     p.seg_len = n;
     p.n_seg = 1;
@@ -305,6 +452,14 @@ extern "C" int msa_topk_docs(int B, int n_docs, int k, const float* scores, int3
   unsigned long long* cand = p.n_seg > 1 ? static_cast<unsigned long long*>(ws) : nullptr;
   const dim3 grid((unsigned)p.n_seg, (unsigned)B);
   int rc;
+  if (p.small) {
+    topk_small_select_kernel<<<grid, kSmallThreads, 0, s>>>(n_docs, k, scores, idx, top_scores,
+                                                            cand);
+    if ((rc = check_launch()) || p.n_seg == 1) return rc;
+    topk_small_merge_kernel<<<B, kSmallThreads, 0, s>>>(n_docs, k, p.n_seg, cand, scores, idx,
+                                                        top_scores);
+    return check_launch();
+  }
   if (p.smem_keys) {
     const size_t smem = (size_t)p.seg_len * sizeof(uint32_t);
     rc = ensure_smem_attr(reinterpret_cast<const void*>(topk_select_kernel<true>), (int)smem);

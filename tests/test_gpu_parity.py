@@ -312,6 +312,8 @@ def test_route_100m_prefill_sampled(prepared):
     (2, 16384, 16, None), (2, 16385, 16, 64.0),          # one segment / two segments
     (1, 200000, 1024, None),                              # 8 segments of 25K keys (L2 keys)
     (3, 70000, 100, 16.0), (1, 1000000, 16, None),        # many ties; 1M documents
+    (2, 2048, 32, None), (2, 2049, 32, 4.0),              # small-k path: one / two segments
+    (1, 50000, 1, None), (1, 70000, 33, None),            # k = 1; just above the small path
 ])
 def test_topk_identical_to_oracle(B, n, k, quant):
     g = torch.Generator(device="cuda").manual_seed(n + k)
@@ -324,6 +326,22 @@ def test_topk_identical_to_oracle(B, n, k, quant):
     oi, ot = oracle.topk_docs(f64(s), k)
     np.testing.assert_array_equal(idx.cpu().numpy(), oi)
     np.testing.assert_array_equal(f64(top), ot)
+    status_ok()
+
+
+@pytest.mark.parametrize("k", [16, 32, 200])
+def test_topk_sorted_inputs(k):
+    """Ascending scores (every batch of the small-k path improves its list)
+    and descending ones, with runs of exact ties."""
+    n = 40000
+    base = torch.arange(n, device="cuda", dtype=torch.float32) // 3
+    for s in (base[None, :], base.flip(0)[None, :], -base[None, :]):
+        s = s.contiguous()
+        top = torch.empty((1, k), device="cuda")
+        idx, _ = pipeline.topk_docs(s, k, top=top)
+        oi, ot = oracle.topk_docs(f64(s), k)
+        np.testing.assert_array_equal(idx.cpu().numpy(), oi)
+        np.testing.assert_array_equal(f64(top), ot)
     status_ok()
 
 
@@ -518,6 +536,7 @@ def test_attention_vs_oracle(dtype, B, T, T_loc, Hq, H, D, m_cap, mem_lens, pos0
     (2, 300, 700, 32, 8, 128, 500, [500, 129]),   # several key tiles each side
     (3, 64, 64, 8, 8, 64, 130, [128, 0, 1]),       # G = 1, empty and 1-row memory
     (1, 17, 1000, 16, 1, 128, 256, [256]),         # G = 16, chunked prefill
+    (1, 64, 4096, 32, 8, 128, 384, [300]),         # long local context: key-tile splits
 ])
 def test_attention_prefill_tensor_core_shapes(B, T, T_loc, Hq, H, D, m_cap, mem_lens):
     """Rows past mem_len are filled with NaN: they must not reach the
