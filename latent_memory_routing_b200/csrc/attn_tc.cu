@@ -130,39 +130,6 @@ __device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
   return (unsigned long long)__float_as_uint(lo) | ((unsigned long long)__float_as_uint(hi) << 32);
 }
 
-// 2^x for a pair of floats on the FMA pipe, to take part of the softmax's
-// exponentials off the MUFU unit (which alone would bound a tile: one ex2
-// per score).  Range reduction x = r + f with r = round(x) (adding 1.5 * 2^23
-// leaves r in the low mantissa bits) and f in [-0.5, 0.5]; 2^f by a cubic,
-// 2^r by adding r to the exponent field.  The cubic's coefficients are a
-// relative-error fit of 2^f on [-0.5, 0.5] (iteratively reweighted least
-// squares on a dense grid): max relative error 7.5e-5, under the bf16
-// rounding P gets next (2^-9).  x is clamped at -126 so that the exponent
-// field stays non-negative: a masked score (-inf) gives about 1e-38, not 0.
-constexpr float kExp2C0 = 0.9999281168f, kExp2C1 = 0.6932609677f, kExp2C2 = 0.2426105440f,
-                kExp2C3 = 0.0551713221f;
-__device__ __forceinline__ unsigned long long ex2_poly2(unsigned long long x2) {
-  const unsigned long long xc = f2_pack(fmaxf(__uint_as_float((uint32_t)x2), -126.f),
-                                        fmaxf(__uint_as_float((uint32_t)(x2 >> 32)), -126.f));
-  const unsigned long long magic = f2_pack(12582912.f, 12582912.f);
-  const unsigned long long nmagic = f2_pack(-12582912.f, -12582912.f);
-  const unsigned long long neg1 = f2_pack(-1.f, -1.f);
-  unsigned long long t2, r2, f2, p2;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(xc), "l"(magic));
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r2) : "l"(t2), "l"(nmagic));    // round(x)
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(f2) : "l"(r2), "l"(neg1), "l"(xc));  // x - r
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(p2)
-      : "l"(f2_pack(kExp2C3, kExp2C3)), "l"(f2), "l"(f2_pack(kExp2C2, kExp2C2)));
-  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(p2) : "l"(f2), "l"(f2_pack(kExp2C1, kExp2C1)));
-  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(p2) : "l"(f2), "l"(f2_pack(kExp2C0, kExp2C0)));
-  // the low word of t holds r (two's complement) above bit 22's offset;
-  // shifted to the exponent field, the offset bits leave the word
-  const uint32_t lo = (uint32_t)p2 + ((uint32_t)t2 << 23);
-  const uint32_t hi = (uint32_t)(p2 >> 32) + ((uint32_t)(t2 >> 32) << 23);
-  return (unsigned long long)lo | ((unsigned long long)hi << 32);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -462,19 +429,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const int k0 = c * 64 + 2 * e;
           unsigned long long x2 = (unsigned long long)sv[k0] | ((unsigned long long)sv[k0 + 1] << 32);
           asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(x2) : "l"(sc2), "l"(nm2));
-          // 3 pairs in 8 on the FMA pipe, the rest on MUFU: the split that
-          // balances the two per tile
-          unsigned long long p2;
-          float p0, p1;
-          if ((e & 7) < 3) {
-            p2 = ex2_poly2(x2);
-            p0 = __uint_as_float((uint32_t)p2);
-            p1 = __uint_as_float((uint32_t)(p2 >> 32));
-          } else {
-            p0 = ex2_approx(__uint_as_float((uint32_t)x2));
-            p1 = ex2_approx(__uint_as_float((uint32_t)(x2 >> 32)));
-            p2 = f2_pack(p0, p1);
-          }
+          const float p0 = ex2_approx(__uint_as_float((uint32_t)x2));
+          const float p1 = ex2_approx(__uint_as_float((uint32_t)(x2 >> 32)));
+          const unsigned long long p2 = f2_pack(p0, p1);
           asm("add.rn.f32x2 %0, %0, %1;" : "+l"(ls2[e & 1]) : "l"(p2));
           w[e] = pack_bf16(p0, p1);
         }
