@@ -11,7 +11,7 @@
 // Design.  Decode is HBM-bound (every K/V byte is read once); the tensor
 // cores take the two contractions off the CUDA cores so that the few
 // instructions left per key hide under the stream.  A persistent grid of at
-// most one CTA of 14 warps per SM walks work items -- a key split of one
+// most one CTA of 15 warps per SM walks work items -- a key split of one
 // (batch element, KV head), serving the G query heads of the KV head padded
 // to N = 16 MMA columns -- with one continuous pipeline across items, so
 // the stream never drains between them:
@@ -29,10 +29,12 @@
 //     rotated and meet R(p_q) q.  In a memory tile that ends early they zero
 //     the V rows past mem_len;
 //   * warp 1 issues S^T = K Q^T (M = 128 keys, N = 16, K = 128) into one of
-//     two TMEM buffers and O^T += V^T P^T (M = 128 dims, N = 16, K = 128
-//     keys; V read MN-major) into the O^T TMEM columns, in the order
-//     S(0) S(1) | PV(0) S(2) | PV(1) S(3) ..., so the softmax of a tile runs
-//     under the next tile's S;
+//     two TMEM buffers as soon as a K tile is rotated, and the last warp
+//     issues O^T += V^T P^T (M = 128 dims, N = 16, K = 128 keys; V read
+//     MN-major) into the O^T TMEM columns as soon as P and the V tile are
+//     there -- two issuers, so that S never queues behind a P V that waits
+//     for its V tile (the V stream, whose slots are held longest, sets the
+//     pace);
 //   * warps 4..7 (softmax, one thread per TMEM lane: a key row of S^T, a dim
 //     row of O^T) turn S into P (base-2 exponent domain, the scale folded
 //     into Q) against a per-head reference maximum that moves only when a
@@ -60,7 +62,8 @@ constexpr int kDim = 128;                  // head dim
 constexpr int kTStages = 3;
 constexpr int kRotWarps = 8;
 constexpr int kSoftWarps = 4;
-constexpr int kTThreads = 32 * (2 + kRotWarps + kSoftWarps);
+constexpr int kPvWarp = 2 + kRotWarps + kSoftWarps;  // the P V issuer, last warp
+constexpr int kTThreads = 32 * (kPvWarp + 1);
 constexpr int kBlk = kTK * 128;            // one 64-dim block of a K or V tile: 16 KB
 constexpr int kTileBytes = 2 * kBlk;       // K or V tile: 32 KB
 constexpr int kStageBytes = 2 * kTileBytes;
@@ -88,7 +91,7 @@ struct DTAux {
   // K and V tiles of a stage arrive and leave separately: a K slot is free
   // once S has read it, a V slot once P V has
   uint64_t kfull[kTStages], vfull[kTStages], kready[kTStages], kfree[kTStages], vfree[kTStages];
-  uint64_t sfull[2], pfull[2], pvdone, odone;
+  uint64_t sfull[2], pfull[2], pvdone[2], odone;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -228,7 +231,8 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       tc::mbar_init(&aux.sfull[i], 1);
       tc::mbar_init(&aux.pfull[i], kSoftWarps);
     }
-    tc::mbar_init(&aux.pvdone, 1);
+    tc::mbar_init(&aux.pvdone[0], 1);
+    tc::mbar_init(&aux.pvdone[1], 1);
     tc::mbar_init(&aux.odone, 1);
     aux.abort_flag = 0;
     tc::fence_mbar_init();
@@ -293,14 +297,17 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         tc::mbar_wait(&fullb[v % kTStages], (v / kTStages) & 1);
     }
   } else if (warp == 1) {
-    // ----------------------------------------------------------------- MMA
+    // ------------------------------------------------------------- S MMA
+    // S(u) as soon as its K tile is rotated (kready) and its TMEM buffer
+    // u&1 has been read by the softmax of tile u-2 (pfull of u-2): the P V
+    // stream, issued by its own warp, does not hold it back
     if (lane == 0) {
-      Cur cs, cp;  // the S cursor runs two tiles ahead of the P V cursor
-      int us = 0, up = 0;
-      bool hs = first(cs), hp = first(cp);
-      auto issue_s = [&]() {
+      Cur cs;
+      int us = 0;
+      for (bool hs = first(cs); hs; hs = next(cs), ++us) {
         const int st = us % kTStages;
         wait_or_abort(&aux.kready[st], (us / kTStages) & 1);
+        if (us >= 2) wait_or_abort(&aux.pfull[us & 1], ((us - 2) >> 1) & 1);
         tc::tc_fence_after();
         const uint32_t a0 = tc::smem_u32(ring + (size_t)st * kStageBytes);
         const uint32_t b0 =
@@ -315,10 +322,15 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         }
         tc::mma_commit(&aux.sfull[us & 1]);
         tc::mma_commit(&aux.kfree[st]);  // S has read the K slot
-        ++us;
-        hs = next(cs);
-      };
-      auto issue_pv = [&]() {
+      }
+    }
+  } else if (warp == kPvWarp) {
+    // ----------------------------------------------------------- P V MMA
+    // P V(u) as soon as P(u) is written and V(u) has landed
+    if (lane == 0) {
+      Cur cp;
+      int up = 0;
+      for (bool hp = first(cp); hp; hp = next(cp), ++up) {
         const int st = up % kTStages;
         wait_or_abort(&aux.pfull[up & 1], (up >> 1) & 1);
         wait_or_abort(&aux.vfull[st], (up / kTStages) & 1);
@@ -331,17 +343,9 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           tc::mma_bf16_ss(tmem + 2 * kNH, tc::sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kBlk),
                           tc::sdesc_kmajor_sw128(p0 + (kk >> 2) * (kNH * 128) + (kk & 3) * 32),
                           kIdescO, (!first_tile || kk > 0) ? 1u : 0u);
-        tc::mma_commit(&aux.vfree[st]);  // P V has read the V slot
-        tc::mma_commit(&aux.pvdone);
+        tc::mma_commit(&aux.vfree[st]);        // P V has read the V slot
+        tc::mma_commit(&aux.pvdone[up & 1]);   // ... and the P buffer up&1
         if (last_tile) tc::mma_commit(&aux.odone);  // this item's O^T is final
-        ++up;
-        hp = next(cp);
-      };
-      if (hs) issue_s();
-      if (hs) issue_s();
-      while (hp) {
-        issue_pv();
-        if (hs) issue_s();
       }
     }
   } else if (warp >= 4 && warp < 4 + kSoftWarps) {
@@ -407,7 +411,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         if (rescale && c.j > 0) {
           // O^T holds P V of this item's earlier tiles: wait for the last
           // one (tile u-1), then scale each head's column in TMEM
-          wait_or_abort(&aux.pvdone, (u - 1) & 1);
+          wait_or_abort(&aux.pvdone[(u - 1) & 1], ((u - 1) >> 1) & 1);
           tc::tc_fence_after();
           uint32_t ov[16];
           tc::tmem_ld16(tmem + lane_addr + 2 * kNH, ov);
@@ -418,8 +422,9 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           tmem_st_wait();
         }
       }
-      // P^T column of this key (buffer u&1: its previous reader, P V of tile
-      // u-2, completed before S(u) was issued)
+      // P^T column of this key into buffer u&1, once its previous reader,
+      // P V of tile u-2, is done
+      if (u >= 2) wait_or_abort(&aux.pvdone[u & 1], ((u - 2) >> 1) & 1);
       unsigned char* pb = pbuf + (u & 1) * kPBytes;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
