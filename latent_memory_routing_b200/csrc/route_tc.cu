@@ -571,6 +571,20 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
           int slot = 0;
           float m = -INFINITY;
           auto fold32 = [&](const uint32_t (&r)[32], int cs) {
+            if (T == 1) {
+              // one query per column: every column is parked as it is, with
+              // no loop-carried state (independent stores)
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int col = cs + i;
+                if (col < col_end) {  // warp-uniform
+                  const uint32_t o = valid ? f2o(__uint_as_float(r[i])) : 0u;
+                  scr[(col - col0) * 33 + lane] = o;
+                  if (chunk_u && valid) atomicMax(chunk_u + (int64_t)col * C + c, o);
+                }
+              }
+              return;
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int col = cs + i;
@@ -608,20 +622,25 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             else tc::mbar_arrive(&aux.acce[ab]);
           }
           const int n_slots = (col_end - 1) / T - b_first + 1;
+          // the warp's document runs are the same for every slot: bit rr of
+          // `heads` marks a row that starts one (warp-uniform branches below)
+          const unsigned heads = __ballot_sync(0xffffffffu, lane == 0 || up != dd);
           for (int sl = lane; sl < n_slots; sl += 32) {
             uint32_t* doc_row = doc_u + (int64_t)(b_first + sl) * n_docs;
             const uint32_t* v = scr + sl * 33;
+            uint32_t vals[32];
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) vals[rr] = v[rr];  // all loads first
             int cd = dw[0];
-            uint32_t cur = v[0];
+            uint32_t cur = vals[0];
+#pragma unroll
             for (int rr = 1; rr < 32; ++rr) {
-              const int d = dw[rr];
-              const uint32_t k = v[rr];
-              if (d != cd) {
+              if ((heads >> rr) & 1u) {
                 if (cd >= 0) atomicMax(doc_row + cd, cur);
-                cd = d;
-                cur = k;
+                cd = dw[rr];
+                cur = vals[rr];
               } else {
-                cur = max(cur, k);
+                cur = max(cur, vals[rr]);
               }
             }
             if (cd >= 0) atomicMax(doc_row + cd, cur);
