@@ -84,18 +84,7 @@ struct AAux {
   int abort_flag;
 };
 
-// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16; A is M x K bf16 in TMEM,
-// row m in lane m, elements 2c and 2c+1 of K packed in column c.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
+using tc::mma_bf16_ts;
 using tc::sdesc_mnmajor_sw128;
 
 // 2^x by the SFU (ex2.approx, ~2 ulp); its result feeds a bf16 P tile.
