@@ -44,9 +44,9 @@ def ROUTE_DRAM_TRAFFIC(C):
     """DRAM bytes (GB) of one route_tc_kernel launch over C chunks, from the
     ncu dram__bytes_read.sum + dram__bytes_write.sum of the current kernel on
     a smaller bank, scaled by chunks (the kernel's traffic grows with the
-    chunks it scans).  Pair kernel on a 192,961-chunk bank: 396.06 MB read +
-    3.85 MB written = 2072.5 B per chunk, against 2048 algorithmic."""
-    return round((396.060416e6 + 3.851008e6) / 192961 * C / 1e9, 3)
+    chunks it scans).  Pair kernel on a 192,961-chunk bank: 396.11 MB read +
+    4.08 MB written = 2073.9 B per chunk, against 2048 algorithmic."""
+    return round((396.111872e6 + 4.078592e6) / 192961 * C / 1e9, 3)
 
 
 def peaks():
