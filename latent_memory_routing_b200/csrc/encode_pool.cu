@@ -8,14 +8,30 @@
 // §"三、文档如何变成 memory" / "2. chunk 压缩" (64 tokens per chunk,
 // K -> K̄, V -> V̄, K_r -> K̄_r by mean pooling, 180 tokens -> 3 chunks).
 //
-// Design (HBM-bound stream): one CTA per chunk, looping over the L layers so
-// the chunk's RoPE table is built once.  Each thread owns two 16-byte vectors
+// Design (HBM-bound stream).  encode_tma_kernel (the default): persistent
+// CTAs, one per SM, each owning a contiguous range of chunks.  One producer
+// thread streams, per (chunk, layer), the chunk's contiguous token rows of K,
+// V and K_r with 1-D bulk copies (cp.async.bulk, 32 KB stages, a two-stage
+// ring per tensor, so that each ring has one consumer group and a group
+// never waits on a slot another group's stage may still hold) -- the copy
+// engine keeps up to 192 KB in flight per SM without a load instruction per
+// 16 bytes; three consumer groups (one per tensor) each own
+// one 16-byte vector of a head and its rotate-half partner, add every row of
+// their tensor from shared memory into fp32 registers (K rotated by the
+// token's document-wise position from the chunk's (cos, sin) table) and write
+// the chunk's mean row once, so no partial sums cross threads.
+// encode_pool_kernel (MSA_ENCODE_TMA=0): one CTA per chunk, looping over the
+// L layers so the chunk's RoPE table is built once.  Each thread owns two 16-byte vectors
 // of one head -- elements [v*VEC, v*VEC+VEC) and the rotate-half partners at
 // +D/2 -- so the rotation needs no data exchange; R token rows are in flight
 // per CTA.  Loads are 16-byte, coalesced and L1-bypassing; sums are fp32;
 // the R partial sums are combined through shared memory and each output row
 // is written once with 16-byte stores.
+#include <algorithm>
+#include <cstdlib>
+
 #include "msa_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace msa {
 namespace {
@@ -140,6 +156,211 @@ encode_pool_kernel(int L, int64_t n_tok, int n_docs, int H, int R,
   }
 }
 
+constexpr int kEncStage = 16384;  // bytes per ring stage
+constexpr int kEncStages = 4;     // stages per tensor: one ring per consumer group
+
+// Threads: one producer warp + three consumer groups of Ug (U rounded up to
+// a warp) threads, U = H * (D/2) / VEC.
+template <typename T, int D>
+constexpr int enc_tma_max_threads() {
+  return 32 + 3 * (16 * (D / 2) / Vec16<T>::N);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(enc_tma_max_threads<T, D>(), 1)
+encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS,
+                  const T* __restrict__ k_tok, const T* __restrict__ v_tok,
+                  const T* __restrict__ kr_tok, const int64_t* __restrict__ tok_off,
+                  const int64_t* __restrict__ chunk_off, int64_t n_chunks, double base,
+                  int chunk, T* __restrict__ k_bar, T* __restrict__ v_bar,
+                  T* __restrict__ kr_bar, int* status) {
+  constexpr int VEC = Vec16<T>::N;
+  constexpr int HALF = D / 2;
+  constexpr int UPH = HALF / VEC;
+  extern __shared__ __align__(1024) unsigned char enc_dsm[];
+  unsigned char* ring = tc::smem_align<1024>(enc_dsm);
+  // ring of tensor t: stages [t * kEncStages, (t + 1) * kEncStages)
+  float2* cs_tab = reinterpret_cast<float2*>(ring + 3 * kEncStages * kEncStage);  // [64][HALF]
+  __shared__ uint64_t full[3 * kEncStages], empty[3 * kEncStages];
+  __shared__ double w_tab[HALF];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row_elems = (int64_t)H * D;
+  const uint32_t row_bytes = (uint32_t)(row_elems * sizeof(T));
+  const int64_t cb = (int64_t)blockIdx.x * n_chunks / gridDim.x;
+  const int64_t ce = (int64_t)(blockIdx.x + 1) * n_chunks / gridDim.x;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3 * kEncStages; ++i) {
+      tc::mbar_init(&full[i], 1);
+      tc::mbar_init(&empty[i], Ug / 32);
+    }
+    abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < HALF; i += blockDim.x) w_tab[i] = rope_inv_freq(base, i, D);
+  __syncthreads();
+  volatile int* abort_v = &abort_flag;
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    if (*abort_v) return;
+    if (!tc::mbar_wait(bar, parity)) {
+      record_error(status, MSA_ERR_TIMEOUT);
+      *abort_v = 1;
+    }
+  };
+  // the chunk's document: a bisection for the first chunk, then a forward
+  // walk (a CTA's chunks are consecutive), with the document's offsets kept
+  // in registers so that most chunks need no global load
+  int64_t d = 0;
+  {
+    int64_t lo = 0, hi = n_docs;
+    while (hi - lo > 1) {
+      const int64_t mid = (lo + hi) >> 1;
+      if (__ldg(chunk_off + mid) <= cb) lo = mid; else hi = mid;
+    }
+    d = lo;
+  }
+  int64_t c_lo = __ldg(chunk_off + d), c_hi = __ldg(chunk_off + d + 1);
+  int64_t t_lo = __ldg(tok_off + d), t_hi = __ldg(tok_off + d + 1);
+  auto locate = [&](int64_t c, int64_t& tok0, int& rows, int64_t& p0) {
+    while (c >= c_hi && d + 1 < n_docs) {
+      ++d;
+      c_lo = c_hi;
+      c_hi = __ldg(chunk_off + d + 1);
+      t_lo = t_hi;
+      t_hi = __ldg(tok_off + d + 1);
+    }
+    const int64_t j = c - c_lo;
+    tok0 = t_lo + j * chunk;
+    const int64_t left = t_hi - tok0;
+    rows = (int)(left < 0 ? 0 : (left < chunk ? left : chunk));
+    p0 = j * chunk;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const T* src[3] = {k_tok, v_tok, kr_tok};
+      uint32_t ut[3] = {0, 0, 0};  // stages issued to each tensor's ring
+      for (int64_t c = cb; c < ce; ++c) {
+        int64_t tok0, p0;
+        int rows;
+        locate(c, tok0, rows, p0);
+        const int nstg = (rows + RS - 1) / RS;
+        for (int l = 0; l < L; ++l)
+          for (int g = 0; g < nstg; ++g)
+            for (int t = 0; t < 3; ++t) {
+              const uint32_t u = ut[t]++;
+              const int st = t * kEncStages + (int)(u % kEncStages);
+              wait(&empty[st], ((u / kEncStages) & 1) ^ 1);
+              if (*abort_v) continue;
+              const int nr = min(RS, rows - g * RS);
+              tc::mbar_arrive_expect_tx(&full[st], (uint32_t)nr * row_bytes);
+              tc::bulk_load(ring + (size_t)st * kEncStage,
+                            src[t] + ((int64_t)l * n_tok + tok0 + (int64_t)g * RS) * row_elems,
+                            (uint32_t)nr * row_bytes, &full[st]);
+            }
+      }
+      // every copy issued must land before the CTA exits
+      for (int t = 0; t < 3; ++t)
+        for (uint32_t v = ut[t] > (uint32_t)kEncStages ? ut[t] - kEncStages : 0; v < ut[t]; ++v)
+          tc::mbar_wait(&full[t * kEncStages + v % kEncStages], (v / kEncStages) & 1);
+    }
+  } else {
+    // ----------------------------------------------------------- consumers
+    const int t = (warp - 1) / (Ug / 32);         // 0: K, 1: V, 2: K_r
+    const int jt = (int)threadIdx.x - 32 - t * Ug;  // index in the group
+    const bool active = jt < U;
+    const int h = jt / UPH, v = jt % UPH;
+    const int64_t col_lo = (int64_t)h * D + v * VEC;
+    T* dst = t == 0 ? k_bar : (t == 1 ? v_bar : kr_bar);
+    uint32_t u = 0;
+    for (int64_t c = cb; c < ce; ++c) {
+      int64_t tok0, p0;
+      int rows;
+      locate(c, tok0, rows, p0);
+      const int nstg = (rows + RS - 1) / RS;
+      if (t == 0) {  // the K group rebuilds the chunk's (cos, sin) table
+        asm volatile("bar.sync 1, %0;" ::"r"(Ug) : "memory");  // old table no longer read
+        // frequency i: an exact anchor at p0 (angle reduced in double), then
+        // one rotation by w_i per row, in double
+        for (int i = jt; i < HALF; i += Ug) {
+          const double w = w_tab[i];
+          double sa, ca, sw, cw;
+          const double two_pi = 6.283185307179586;
+          const double th = (double)p0 * w;
+          sincos(fma(-rint(th * (1.0 / two_pi)), two_pi, th), &sa, &ca);
+          sincos(w, &sw, &cw);
+          for (int r = 0; r < rows; ++r) {
+            cs_tab[r * HALF + i] = make_float2((float)ca, (float)sa);
+            const double cn = ca * cw - sa * sw;
+            sa = sa * cw + ca * sw;
+            ca = cn;
+          }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(Ug) : "memory");
+      }
+      const float inv_n = rows > 0 ? 1.0f / (float)rows : 0.f;
+      for (int l = 0; l < L; ++l) {
+        float a1[VEC], a2[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) a1[e] = a2[e] = 0.f;
+        for (int g = 0; g < nstg; ++g, ++u) {
+          const int st = t * kEncStages + (int)(u % kEncStages);
+          wait(&full[st], (u / kEncStages) & 1);
+          const int nr = min(RS, rows - g * RS);
+          if (active && !*abort_v) {
+            const unsigned char* base_row = ring + (size_t)st * kEncStage;
+            for (int rr = 0; rr < nr; ++rr) {
+              const unsigned char* row = base_row + (size_t)rr * row_bytes;
+              const uint4 q1 = *reinterpret_cast<const uint4*>(row + col_lo * sizeof(T));
+              const uint4 q2 =
+                  *reinterpret_cast<const uint4*>(row + (col_lo + HALF) * sizeof(T));
+              float x1[VEC], x2[VEC];
+              Vec16<T>::unpack(q1, x1);
+              Vec16<T>::unpack(q2, x2);
+              if (t == 0) {
+                const float2* cs = cs_tab + (g * RS + rr) * HALF + v * VEC;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                  const float2 q = cs[e];
+                  a1[e] += x1[e] * q.x - x2[e] * q.y;
+                  a2[e] += x2[e] * q.x + x1[e] * q.y;
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                  a1[e] += x1[e];
+                  a2[e] += x2[e];
+                }
+              }
+            }
+          }
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&empty[st]);
+        }
+        if (active) {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            a1[e] *= inv_n;
+            a2[e] *= inv_n;
+          }
+          T* o = dst + ((int64_t)l * n_chunks + c) * row_elems + col_lo;
+          st16(o, Vec16<T>::pack(a1));
+          st16(o + HALF, Vec16<T>::pack(a2));
+        }
+      }
+    }
+  }
+}
+
+bool encode_tma_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("MSA_ENCODE_TMA");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 __global__ void chunk_offsets_kernel(int n_docs, const int64_t* __restrict__ tok_off,
                                      int chunk, int64_t* __restrict__ chunk_off,
                                      int* status) {
@@ -177,6 +398,24 @@ int launch_encode(int L, int64_t n_tok, int n_docs, int H, const void* k,
                   const int64_t* coff, int64_t n_chunks, float base, int chunk,
                   void* kb, void* vb, void* rb, cudaStream_t s) {
   constexpr int VEC = Vec16<T>::N;
+  const int64_t row_bytes = (int64_t)H * D * (int64_t)sizeof(T);
+  if (encode_tma_enabled() && row_bytes % 16 == 0 && row_bytes <= kEncStage) {
+    const int U = H * (D / 2 / VEC);
+    const int Ug = (U + 31) / 32 * 32;
+    const int RS = (int)std::min<int64_t>(chunk, kEncStage / row_bytes);
+    const size_t smem =
+        1024 + (size_t)3 * kEncStages * kEncStage + sizeof(float2) * kMaxChunk * (D / 2);
+    auto kern = encode_tma_kernel<T, D>;
+    int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem);
+    if (rc) return rc;
+    if (n_chunks == 0) return MSA_OK;
+    const int grid = (int)std::min<int64_t>(n_chunks, num_sms());
+    kern<<<grid, 32 + 3 * Ug, smem, s>>>(
+        L, n_tok, n_docs, H, U, Ug, RS, static_cast<const T*>(k), static_cast<const T*>(v),
+        static_cast<const T*>(kr), toff, coff, n_chunks, (double)base, chunk,
+        static_cast<T*>(kb), static_cast<T*>(vb), static_cast<T*>(rb), device_status_ptr());
+    return check_launch();
+  }
   const int U = H * (D / 2 / VEC);
   const int R = U >= kEncThreads ? 1 : kEncThreads / U;
   const int threads = U * R;
