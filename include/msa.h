@@ -42,6 +42,19 @@
  *     per-device status word read with msa_device_status().
  *   - Tensors read with 16-byte vector loads must be 16-byte aligned; this
  *     is checked and reported as MSA_ERR_INVALID_ARG.
+ *   - Environment switches, read once per process, choose between kernels
+ *     that compute the same results (for comparison and profiling):
+ *       MSA_ROUTE_PAIRS=0   prepared-bank routing on single CTAs instead of
+ *                           CTA pairs;
+ *       MSA_DECODE_TC=0     decode attention on the CUDA cores instead of
+ *                           the tensor cores;
+ *       MSA_ENCODE_TMA=0    chunk pooling by per-chunk CTAs with plain loads
+ *                           instead of bulk copies;
+ *       MSA_ROUTE_BWD_TC=0  the routing backward's maximisers recomputed on
+ *                           the CUDA cores (fp32) instead of the tensor-core
+ *                           scan;
+ *       MSA_ATTN_SPLITS=n   at most n (1..16) key-tile splits in prefill
+ *                           attention (default 3).
  */
 #ifndef MSA_H
 #define MSA_H
