@@ -380,10 +380,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
       for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(sv[c]);
 #pragma unroll
-      for (int c = 8; c < kKeys; c += 16)
+      for (int c = 8; c + 16 <= kKeys; c += 16)
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           mx[u] = fmax3(mx[u], __uint_as_float(sv[c + u]), __uint_as_float(sv[c + 8 + u]));
+      if ((kKeys - 8) % 16)  // the last 8 keys
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], __uint_as_float(sv[kKeys - 8 + u]));
       const float mraw = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
                                fmaxf(mx[6], mx[7]));
       const float mt = mraw * qscale;  // qscale > 0 keeps the order
