@@ -661,7 +661,11 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(step * 1e3, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n_chunks": C},
+        "config": {"workload": WORKLOAD, "n_chunks": C, "n_docs": len(lengths),
+                   "global_batch": world, "seq_len": int(w["T"]), "top_k": int(w["k"]),
+                   "m_cap": int(w["k"]) * int((coff_h[1:] - coff_h[:-1]).max()),
+                   "parallelism": "rank 0 only (host cores)",
+                   "l2": "the 3.2 GB routing bank streams through the 126 MB L2 every step"},
         "cpu_baseline": {**cb, "value": round(value, 8)},
         "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
