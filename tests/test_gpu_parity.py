@@ -814,15 +814,18 @@ def _clear_gap_grad(q64, k64, coff_h, gap, rng, frac=0.6):
 
 # (B, T): one 128-column pass; one 64-column pass; 300 query columns in two
 # 256-column passes, the second query's tokens split across them
-@pytest.mark.parametrize("dtype,B,T", [(torch.float32, 2, 40), (torch.bfloat16, 2, 40),
-                                       (torch.bfloat16, 1, 40), (torch.bfloat16, 2, 150)])
-def test_route_backward_vs_oracle(dtype, B, T):
+@pytest.mark.parametrize("dtype,B,T,H,D", [
+    (torch.float32, 2, 40, 8, 128), (torch.bfloat16, 2, 40, 8, 128),
+    (torch.bfloat16, 1, 40, 8, 128), (torch.bfloat16, 2, 150, 8, 128),
+    (torch.bfloat16, 3, 20, 4, 64),                      # D = 64 scan, 64 columns
+])
+def test_route_backward_vs_oracle(dtype, B, T, H, D):
     """dQ_r and dK̄_r from dL/d(doc_scores), against the oracle, on the
     (query, document) pairs whose first maximiser is decided beyond rounding:
     a gap above 1e-4 for the fp32 CUDA-core path, above 4e-3 (the routing
     score tolerance) for the bf16 path, whose maximisers come from the
     tensor-core scan of bf16 unit rows."""
-    H, D, n_docs = 8, 128, 30
+    n_docs = 30
     g = torch.Generator(device="cuda").manual_seed(5 + B * T)
     gc = torch.Generator().manual_seed(5)
     lengths = torch.randint(1, 900, (n_docs,), generator=gc).numpy()
