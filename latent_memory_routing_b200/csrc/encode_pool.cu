@@ -9,8 +9,8 @@
 // K -> K̄, V -> V̄, K_r -> K̄_r by mean pooling, 180 tokens -> 3 chunks).
 //
 // Design (HBM-bound stream).  encode_tma_kernel (the default): persistent
-// CTAs, one per SM, each owning a contiguous range of chunks.  One producer
-// thread streams, per (chunk, layer), the chunk's contiguous token rows of K,
+// CTAs, one per SM, each owning a contiguous range of chunks.  Three producer
+// threads stream, per (chunk, layer), the chunk's contiguous token rows of K,
 // V and K_r with 1-D bulk copies (cp.async.bulk, 32 KB stages, a two-stage
 // ring per tensor, so that each ring has one consumer group and a group
 // never waits on a slot another group's stage may still hold) -- the copy
@@ -238,32 +238,32 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const T* src[3] = {k_tok, v_tok, kr_tok};
-      uint32_t ut[3] = {0, 0, 0};  // stages issued to each tensor's ring
+    // lane t streams tensor t into its own ring, so that no ring waits
+    // behind another's slot
+    if (lane < 3) {
+      const int t = lane;
+      const T* src = t == 0 ? k_tok : (t == 1 ? v_tok : kr_tok);
+      uint32_t u = 0;  // stages issued to this tensor's ring
       for (int64_t c = cb; c < ce; ++c) {
         int64_t tok0, p0;
         int rows;
         locate(c, tok0, rows, p0);
         const int nstg = (rows + RS - 1) / RS;
         for (int l = 0; l < L; ++l)
-          for (int g = 0; g < nstg; ++g)
-            for (int t = 0; t < 3; ++t) {
-              const uint32_t u = ut[t]++;
-              const int st = t * kEncStages + (int)(u % kEncStages);
-              wait(&empty[st], ((u / kEncStages) & 1) ^ 1);
-              if (*abort_v) continue;
-              const int nr = min(RS, rows - g * RS);
-              tc::mbar_arrive_expect_tx(&full[st], (uint32_t)nr * row_bytes);
-              tc::bulk_load(ring + (size_t)st * kEncStage,
-                            src[t] + ((int64_t)l * n_tok + tok0 + (int64_t)g * RS) * row_elems,
-                            (uint32_t)nr * row_bytes, &full[st]);
-            }
+          for (int g = 0; g < nstg; ++g, ++u) {
+            const int st = t * kEncStages + (int)(u % kEncStages);
+            wait(&empty[st], ((u / kEncStages) & 1) ^ 1);
+            if (*abort_v) continue;
+            const int nr = min(RS, rows - g * RS);
+            tc::mbar_arrive_expect_tx(&full[st], (uint32_t)nr * row_bytes);
+            tc::bulk_load(ring + (size_t)st * kEncStage,
+                          src + ((int64_t)l * n_tok + tok0 + (int64_t)g * RS) * row_elems,
+                          (uint32_t)nr * row_bytes, &full[st]);
+          }
       }
       // every copy issued must land before the CTA exits
-      for (int t = 0; t < 3; ++t)
-        for (uint32_t v = ut[t] > (uint32_t)kEncStages ? ut[t] - kEncStages : 0; v < ut[t]; ++v)
-          tc::mbar_wait(&full[t * kEncStages + v % kEncStages], (v / kEncStages) & 1);
+      for (uint32_t v = u > (uint32_t)kEncStages ? u - kEncStages : 0; v < u; ++v)
+        tc::mbar_wait(&full[t * kEncStages + v % kEncStages], (v / kEncStages) & 1);
     }
   } else {
     // ----------------------------------------------------------- consumers
