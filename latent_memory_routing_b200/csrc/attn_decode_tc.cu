@@ -552,9 +552,11 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       __nv_bfloat16* qr = qraw + (c.k & 1) * kNH * kDim;
       if (c.j == 0) {
         // a new item (before its first K tile lands): its raw query and
-        // R(p_q) q go to buffers k&1, whose last readers (S of item k-2, at
-        // or before tile u-1) must be done
-        if (u >= 1) wait_or_abort(&aux.sfull[(u - 1) & 1], ((u - 1) >> 1) & 1);
+        // R(p_q) q go to buffers k&1, whose last readers -- S of item k-2,
+        // at or before tile u-2, as item k-1 has at least one tile -- must
+        // be done (S completes in order); S(u-1), the previous item's last,
+        // may still be running
+        if (u >= 2) wait_or_abort(&aux.sfull[u & 1], ((u - 2) >> 1) & 1);
         if (qpre_it != c.it) prefetch_q(c.it);
 #pragma unroll
         for (int i = 0; i < kQPer; ++i) {
