@@ -238,6 +238,53 @@ class Pipeline:
             self(q_r, q, k_loc, v_loc)
         return graph
 
+    def capture_from_host(self, q_r_h, q_h, k_loc_h, v_loc_h, out_h, idx_h):
+        """Records one step that starts from pinned host inputs and ends with
+        the output and the selected documents back in pinned host memory, as
+        one CUDA graph: Q_r is uploaded first and routing starts at once,
+        while Q and the local K/V are uploaded on a second stream; attention
+        waits for both.  ``graph.replay()`` runs the whole step, copies
+        included.  Returns the graph (the device-side copies of the inputs
+        live in this object)."""
+        dev = {name: torch.empty(t.shape, dtype=t.dtype, device=self.kr_bar.device)
+               for name, t in (("q_r", q_r_h), ("q", q_h), ("k_loc", k_loc_h),
+                               ("v_loc", v_loc_h))}
+        self._host_step_inputs = dev
+        side = torch.cuda.Stream()
+
+        def step():
+            main = torch.cuda.current_stream()
+            side.wait_stream(main)
+            with torch.cuda.stream(side):  # attention inputs, under the routing
+                dev["q"].copy_(q_h, non_blocking=True)
+                dev["k_loc"].copy_(k_loc_h, non_blocking=True)
+                dev["v_loc"].copy_(v_loc_h, non_blocking=True)
+            dev["q_r"].copy_(q_r_h, non_blocking=True)
+            self.router(dev["q_r"], self.kr_bar, self.coff, self.n_docs, self.doc_scores, None)
+            topk_docs(self.doc_scores, self.k, self.idx, self.top, self.topk_ws)
+            if not self.fused:
+                gather_kv(self.idx, self.coff, self.k_bar, self.v_bar, self.m_cap, self.k_mem,
+                          self.v_mem, self.mem_len)
+            main.wait_stream(side)
+            if self.fused:
+                self.attn(dev["q"], self.idx, self.coff, self.k_bar, self.v_bar, dev["k_loc"],
+                          dev["v_loc"], self.pos0, self.rope_base, 0.0, self.out)
+            else:
+                self.attn(dev["q"], self.k_mem, self.v_mem, self.mem_len, dev["k_loc"],
+                          dev["v_loc"], self.pos0, self.rope_base, 0.0, self.out)
+            out_h.copy_(self.out, non_blocking=True)
+            idx_h.copy_(self.idx, non_blocking=True)
+
+        warm = torch.cuda.Stream()
+        warm.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(warm):
+            step()
+        torch.cuda.current_stream().wait_stream(warm)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        return graph
+
     def __call__(self, q_r, q, k_loc, v_loc, stream=None):
         self.router(q_r, self.kr_bar, self.coff, self.n_docs, self.doc_scores, None, stream)
         topk_docs(self.doc_scores, self.k, self.idx, self.top, self.topk_ws, stream)
