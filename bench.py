@@ -375,7 +375,9 @@ def run_libmsa(args, world, rank, local):
         line["workloads"] = {"encode_4l": bench_encode(max(args.steps // 4, 3), pk["hbm"]),
                              "bank_10m_decode": bench_decode(args.steps, pk["hbm"]),
                              "bank_100m_tiered": tiered,
-                             "backward_1m": bench_backward(max(args.steps // 4, 3), pk["hbm"])}
+                             "backward_1m": bench_backward(max(args.steps // 4, 3), pk["hbm"]),
+                             "prefill_sweep": bench_prefill_sweep(max(args.steps // 2, 3),
+                                                                  pk["bf16"])}
     return line
 
 
@@ -563,6 +565,37 @@ def bench_backward(steps: int, peak_hbm: float) -> dict:
                                       "frac": round(gbs_p / peak_hbm, 4)},
            "n_chunks": C, "n_tok": N}
     del w
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_prefill_sweep(steps: int, peak_bf16: float) -> dict:
+    """Causal prefill attention alone at longer contexts than the bank_100m
+    step's 256 tokens (whose attention is latency-bound): 32 query heads,
+    8 KV heads, D=128, 384 memory rows, T = T_loc."""
+    import torch
+
+    from latent_memory_routing_b200 import pipeline, synth
+    res = {"note": "tensor-core prefill, FLOPs = 4*D per visible (query row, key) pair, "
+                   "fraction of the measured burst bf16 peak", "shapes": []}
+    for (B, T, M) in ((1, 4096, 384), (2, 8192, 384), (1, 16384, 384)):
+        Hq, H, D = 32, 8, 128
+        g = torch.Generator(device="cuda").manual_seed(B * T)
+        dt = torch.bfloat16
+        q = synth.randn((B, T, Hq, D), dt, "cuda", g)
+        km = synth.randn((B, M, H, D), dt, "cuda", g)
+        vm = synth.randn((B, M, H, D), dt, "cuda", g)
+        kl = synth.randn((B, T, H, D), dt, "cuda", g)
+        vl = synth.randn((B, T, H, D), dt, "cuda", g)
+        ml = torch.full((B,), M, dtype=torch.int32, device="cuda")
+        att = pipeline.Attention(dt, B, T, T, Hq, H, D, M, "cuda")
+        out = torch.empty((B, T, Hq, D), dtype=dt, device="cuda")
+        ms = time_device(lambda: att(q, km, vm, ml, kl, vl, 16, out=out), steps)
+        pairs = B * sum(M + i + 1 for i in range(T))
+        tf = 4.0 * D * Hq * pairs / (ms * 1e-3) / 1e12
+        res["shapes"].append({"B": B, "T": T, "T_loc": T, "M": M, "ms": round(ms, 4),
+                              "tflops": round(tf, 1), "frac_burst": round(tf / peak_bf16, 4)})
+        del q, km, vm, kl, vl, att, out
     torch.cuda.empty_cache()
     return res
 
