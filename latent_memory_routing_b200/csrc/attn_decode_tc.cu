@@ -73,7 +73,7 @@ constexpr int kSmBar = 1;                  // named barrier of the softmax warps
 constexpr float kRescaleLog2 = 8.f;
 constexpr uint32_t kIdescS = tc::idesc_bf16_f32(kTK, kNH);
 constexpr uint32_t kIdescO = tc::idesc_bf16_f32(kDim, kNH) | (1u << 15);  // A MN-major
-constexpr uint32_t kTmemCols = 64;         // S buffers: 0..31, O^T by item parity: 32..63
+constexpr uint32_t kTmemCols = 64;         // S buffers: 0..31, O^T: 32..47
 
 struct DTS {  // dynamic shared memory, offsets from a 1024-byte aligned base
   static constexpr size_t RING = 0;
@@ -83,9 +83,7 @@ struct DTS {  // dynamic shared memory, offsets from a 1024-byte aligned base
   static constexpr size_t QRAW = P + 2 * kPBytes;    // [2][16][128] bf16 raw query, by item
   static constexpr size_t RED = QRAW + 2 * (size_t)kNH * kDim * 2;  // [4][16] f32
   static constexpr size_t FLAGS = RED + 4 * kNH * 4;            // [2][4] int
-  static constexpr size_t REDL = FLAGS + 2 * 4 * 4;             // [2][4][16] f32, by item
-  static constexpr size_t REDM = REDL + 2 * 4 * kNH * 4;        // [2][16] f32, by item
-  static constexpr size_t ALLOC = REDM + 2 * kNH * 4 + 1024;
+  static constexpr size_t ALLOC = FLAGS + 2 * 4 * 4 + 1024;
   static_assert(QMEM % 1024 == 0 && QT % 1024 == 0 && P % 1024 == 0, "swizzle atoms");
 };
 
@@ -93,7 +91,7 @@ struct DTAux {
   // K and V tiles of a stage arrive and leave separately: a K slot is free
   // once S has read it, a V slot once P V has
   uint64_t kfull[kTStages], vfull[kTStages], kready[kTStages], kfree[kTStages], vfree[kTStages];
-  uint64_t sfull[2], pfull[2], pvdone[2], odone[2];
+  uint64_t sfull[2], pfull[2], pvdone[2], odone;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -132,7 +130,6 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int k, int rows) {
 struct Cur {
   int it, k, j, nt;      // item, its ordinal among this CTA's non-empty items, tile, tiles
   int b, g, sp, M, n_mt, j_lo;
-  int pf_it, pf_ml;      // the next item and its mem_len, loaded one item ahead
 };
 
 // kFused: the memory rows come straight from the pooled bank -- per query
@@ -167,22 +164,13 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   int* flags = reinterpret_cast<int*>(sm + DTS::FLAGS);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // mem_len of item `it` (0 past the last item); each role's cursor loads
-  // the next item's one item ahead, so that no role waits on that global
-  // load at an item boundary
-  auto ml_of = [&](int it) -> int {
-    return it < n_items ? mem_len[(it / n_split) / H] : 0;
-  };
   auto load_item = [&](Cur& c) {
     c.sp = c.it % n_split;
     const int bg = c.it / n_split;
     c.b = bg / H;
     c.g = bg % H;
-    const int ml = c.pf_it == c.it ? c.pf_ml : ml_of(c.it);
-    c.pf_it = c.it + gridDim.x;
-    c.pf_ml = ml_of(c.pf_it);
     // fused: mem_len holds the query's group count; its memory is 8 rows a group
-    c.M = kFused ? 8 * min(max(ml, 0), max_groups) : min(max(ml, 0), m_cap);
+    c.M = kFused ? 8 * min(max(mem_len[c.b], 0), max_groups) : min(max(mem_len[c.b], 0), m_cap);
     c.n_mt = (c.M + kTK - 1) / kTK;
     const int n_all = c.n_mt + (T_loc + kTK - 1) / kTK;
     c.j_lo = (int)((int64_t)c.sp * n_all / n_split);
@@ -191,7 +179,6 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   auto first = [&](Cur& c) -> bool {
     c.k = 0;
     c.j = 0;
-    c.pf_it = -1;
     for (c.it = blockIdx.x; c.it < n_items; c.it += gridDim.x) {
       load_item(c);
       if (c.nt > 0) return true;
@@ -221,7 +208,6 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   // an empty split (more splits than tiles): neutral partials
   if (n_split > 1) {
     Cur c;
-    c.pf_it = -1;
     for (c.it = blockIdx.x; c.it < n_items; c.it += gridDim.x) {
       load_item(c);
       if (c.nt > 0) continue;
@@ -247,8 +233,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     }
     tc::mbar_init(&aux.pvdone[0], 1);
     tc::mbar_init(&aux.pvdone[1], 1);
-    tc::mbar_init(&aux.odone[0], 1);
-    tc::mbar_init(&aux.odone[1], 1);
+    tc::mbar_init(&aux.odone, 1);
     aux.abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -355,13 +340,12 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         const bool first_tile = cp.j == 0, last_tile = cp.j == cp.nt - 1;
 #pragma unroll
         for (int kk = 0; kk < kTK / 16; ++kk)
-          tc::mma_bf16_ss(tmem + (2 + (cp.k & 1)) * kNH,
-                          tc::sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kBlk),
+          tc::mma_bf16_ss(tmem + 2 * kNH, tc::sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kBlk),
                           tc::sdesc_kmajor_sw128(p0 + (kk >> 2) * (kNH * 128) + (kk & 3) * 32),
                           kIdescO, (!first_tile || kk > 0) ? 1u : 0u);
         tc::mma_commit(&aux.vfree[st]);        // P V has read the V slot
         tc::mma_commit(&aux.pvdone[up & 1]);   // ... and the P buffer up&1
-        if (last_tile) tc::mma_commit(&aux.odone[cp.k & 1]);  // this item's O^T is final
+        if (last_tile) tc::mma_commit(&aux.odone);  // this item's O^T is final
       }
     }
   } else if (warp >= 4 && warp < 4 + kSoftWarps) {
@@ -370,34 +354,6 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     const int r = w4 * 32 + lane;       // key row of S^T, dim row of O^T
     const uint32_t lane_addr = (uint32_t)(w4 * 32) << 16;
     float m_ref[G], l_part[G];
-    float* redl = reinterpret_cast<float*>(sm + DTS::REDL);  // [2][4][16] by item
-    float* redm = reinterpret_cast<float*>(sm + DTS::REDM);  // [2][16] by item
-    int pend_k = -1, pend_b = 0, pend_g = 0, pend_sp = 0;      // an item awaiting its output
-    // Writes item pend_k's output once its last P V is done: the row sums
-    // from the four warps' partials, O^T from the item's TMEM buffer (dim r
-    // per thread).  Its buffers are next written two items later.
-    auto finalize = [&]() {
-      wait_or_abort(&aux.odone[pend_k & 1], (pend_k >> 1) & 1);
-      tc::tc_fence_after();
-      soft_bar();  // the four warps' partial sums are in redl
-      const float* rl = redl + (pend_k & 1) * 4 * kNH;
-      uint32_t ov[16];
-      tc::tmem_ld16(tmem + lane_addr + (2 + (pend_k & 1)) * kNH, ov);
-      tc::tmem_ld_wait();
-      tc::tc_fence_before();  // item pend_k + 2's first P V overwrites this O^T
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float l = rl[h] + rl[kNH + h] + rl[2 * kNH + h] + rl[3 * kNH + h];
-        const int64_t row_id = (int64_t)pend_b * Hq + pend_g * G + h;  // T == 1
-        const float o = __uint_as_float(ov[h]);
-        if (n_split == 1) {
-          out[row_id * kDim + r] = __float2bfloat16(l > 0.f ? o / l : 0.f);
-        } else {
-          part_o[(row_id * n_split + pend_sp) * kDim + r] = o;
-          if (r == 0) part_ml[row_id * n_split + pend_sp] = make_float2(redm[(pend_k & 1) * kNH + h], l);
-        }
-      }
-    };
     Cur c;
     int u = 0;
     for (bool ok = first(c); ok; ok = next(c), ++u) {
@@ -458,12 +414,11 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           wait_or_abort(&aux.pvdone[(u - 1) & 1], ((u - 1) >> 1) & 1);
           tc::tc_fence_after();
           uint32_t ov[16];
-          const uint32_t t_o = tmem + lane_addr + (2 + (c.k & 1)) * kNH;
-          tc::tmem_ld16(t_o, ov);
+          tc::tmem_ld16(tmem + lane_addr + 2 * kNH, ov);
           tc::tmem_ld_wait();
 #pragma unroll
           for (int h = 0; h < G; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
-          tmem_st16(t_o, ov);
+          tmem_st16(tmem + lane_addr + 2 * kNH, ov);
           tmem_st_wait();
         }
       }
@@ -481,32 +436,38 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&aux.pfull[u & 1]);
-      // the previous item's output, deferred to here (after this tile's P
-      // is out) so that the softmax moves on to the next item while that
-      // item's last P V completes
-      if (pend_k >= 0) {
-        finalize();
-        pend_k = -1;
-      }
       if (c.j == c.nt - 1) {
-        // the item's last tile: reduce the row sums over this warp's 32 key
-        // lanes now (into the item's slot) and leave the rest for later
-        float* rl = redl + (c.k & 1) * 4 * kNH;
+        // the item's last tile: once its P V is done, reduce the row sums
+        // over the 128 key lanes and write this split's O (dim r per thread)
+        wait_or_abort(&aux.odone, c.k & 1);
+        tc::tc_fence_after();
+        soft_bar();  // every thread is past its reads of red
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float v = l_part[h];
 #pragma unroll
           for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane == 0) rl[w4 * kNH + h] = v;
-          if (w4 == 0 && lane == 0) redm[(c.k & 1) * kNH + h] = m_ref[h];
+          if (lane == 0) red[w4 * kNH + h] = v;
         }
-        pend_k = c.k;
-        pend_b = c.b;
-        pend_g = c.g;
-        pend_sp = c.sp;
+        soft_bar();
+        uint32_t ov[16];
+        tc::tmem_ld16(tmem + lane_addr + 2 * kNH, ov);
+        tc::tmem_ld_wait();
+        tc::tc_fence_before();  // the next item's first P V overwrites O^T
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float l = red[h] + red[kNH + h] + red[2 * kNH + h] + red[3 * kNH + h];
+          const int64_t row_id = (int64_t)c.b * Hq + c.g * G + h;  // T == 1
+          const float o = __uint_as_float(ov[h]);
+          if (n_split == 1) {
+            out[row_id * kDim + r] = __float2bfloat16(l > 0.f ? o / l : 0.f);
+          } else {
+            part_o[(row_id * n_split + c.sp) * kDim + r] = o;
+            if (r == 0) part_ml[row_id * n_split + c.sp] = make_float2(m_ref[h], l);
+          }
+        }
       }
     }
-    if (pend_k >= 0) finalize();
   } else {
     // ------------------------------------------------------------ rotators
     const int rt = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // 0 .. 255
@@ -527,43 +488,19 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     const float2 qpos = rope_cs(pos0 + T_loc - 1, wq);  // R(p_q) for memory tiles
     float2 qcs = make_float2(1.f, 0.f);
     bool anchored = false;
-    // this thread's share of an item's raw query (G x 128 bf16 over 256
-    // threads), loaded one item ahead into registers
-    constexpr int kQPer = kNH * kDim / (32 * kRotWarps);
-    __nv_bfloat16 qpre[kQPer];
-    int qpre_it = -1;
-    auto prefetch_q = [&](int it) {
-      qpre_it = -1;
-      if (it >= n_items) return;
-      const int bg = it / n_split;
-      const __nv_bfloat16* src = q + ((int64_t)(bg / H) * Hq + (bg % H) * G) * kDim;
-#pragma unroll
-      for (int i = 0; i < kQPer; ++i) {
-        const int e = rt + i * 32 * kRotWarps;
-        if (e < G * kDim) qpre[i] = src[e];
-      }
-      qpre_it = it;
-    };
     Cur c;
     int u = 0;
     for (bool ok = first(c); ok; ok = next(c), ++u) {
       const int st = u % kTStages;
+      wait_or_abort(&aux.kfull[st], (u / kTStages) & 1);
       unsigned char* kt = ring + (size_t)st * kStageBytes;
       __nv_bfloat16* qr = qraw + (c.k & 1) * kNH * kDim;
       if (c.j == 0) {
-        // a new item (before its first K tile lands): its raw query and
-        // R(p_q) q go to buffers k&1, whose last readers -- S of item k-2,
-        // at or before tile u-2, as item k-1 has at least one tile -- must
-        // be done (S completes in order); S(u-1), the previous item's last,
-        // may still be running
-        if (u >= 2) wait_or_abort(&aux.sfull[u & 1], ((u - 2) >> 1) & 1);
-        if (qpre_it != c.it) prefetch_q(c.it);
-#pragma unroll
-        for (int i = 0; i < kQPer; ++i) {
-          const int e = rt + i * 32 * kRotWarps;
-          if (e < G * kDim) qr[e] = qpre[i];
-        }
-        prefetch_q(c.pf_it);  // the next item's, in flight during this one
+        // a new item: its raw query and R(p_q) q go to buffers k&1, whose
+        // last readers (S of item k-2, at or before tile u-1) must be done
+        if (u >= 1) wait_or_abort(&aux.sfull[(u - 1) & 1], ((u - 1) >> 1) & 1);
+        for (int e = rt; e < G * kDim; e += 32 * kRotWarps)
+          qr[e] = q[((int64_t)c.b * Hq + c.g * G) * kDim + e];
         asm volatile("bar.sync %0, %1;" ::"n"(kSmBar + 1), "n"(32 * kRotWarps) : "memory");
         if (c.n_mt > c.j_lo) {
           unsigned char* qm = qmem + (c.k & 1) * kQBytes;
@@ -579,7 +516,6 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         }
         anchored = false;
       }
-      wait_or_abort(&aux.kfull[st], (u / kTStages) & 1);
       const int n_valid = tile_valid(c);
       if (!tile_mem(c)) {
         // R(Delta) q into buffer u&1, whose last reader S(u-2) must be done
