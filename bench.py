@@ -326,11 +326,11 @@ def run_libmsa(args, world, rank, local):
         "roofline": {"bound": "tensor",
                      "kernel": "route_tc_kernel on CTA pairs, prepared bank "
                                "(msa_route_scores_prepared call)",
-                     "achieved": round(route_tf, 1), "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                     "frac": round(route_tf / pk["bf16_sus"], 4),
-                     "peak_kind": "sustained bf16 (the kernel runs back to back for seconds "
-                                  "under the power cap)",
-                     "frac_of_burst_peak": round(route_tf / pk["bf16"], 4),
+                     "achieved": round(route_tf, 1), "peak": pk["bf16"], "unit": "TFLOP/s",
+                     "frac": round(route_tf / pk["bf16"], 4),
+                     "peak_kind": "burst bf16 (the timed region is tens of milliseconds, "
+                                  "short of the seconds-long power-cap regime)",
+                     "frac_of_sustained_peak": round(route_tf / pk["bf16_sus"], 4),
                      "flop_per_byte": round(route_flops / (C * BYTES_PER_CHUNK), 1),
                      "hbm": {"achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
                              "frac": round(achieved / pk["hbm"], 4)},
@@ -340,7 +340,7 @@ def run_libmsa(args, world, rank, local):
         "stages_ms": {"route": round(seg[0], 4), "topk": round(seg[1], 4),
                       "gather": round(seg[2], 4), "attn": round(seg[3], 4),
                       "note": "eager launches with events between stages; the step "
-                              "(ms_per_step) replays the same ten launches as one CUDA graph"},
+                              "(ms_per_step) replays the same launches as one CUDA graph"},
         "route_gchunks_s": round(C / (route_ms * 1e-3) / 1e9, 4),
         "fused_step": {"ms_per_step": round(fused_ms, 4),
                        "gchunks_s": round(C * world / (fused_ms * 1e-3) / 1e9, 4),
