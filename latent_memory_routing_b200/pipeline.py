@@ -254,12 +254,14 @@ class Pipeline:
 
         def step():
             main = torch.cuda.current_stream()
+            # Q_r first: the uploads share one copy engine, so the others
+            # are made to follow it and run under the routing
+            dev["q_r"].copy_(q_r_h, non_blocking=True)
             side.wait_stream(main)
             with torch.cuda.stream(side):  # attention inputs, under the routing
                 dev["q"].copy_(q_h, non_blocking=True)
                 dev["k_loc"].copy_(k_loc_h, non_blocking=True)
                 dev["v_loc"].copy_(v_loc_h, non_blocking=True)
-            dev["q_r"].copy_(q_r_h, non_blocking=True)
             self.router(dev["q_r"], self.kr_bar, self.coff, self.n_docs, self.doc_scores, None)
             topk_docs(self.doc_scores, self.k, self.idx, self.top, self.topk_ws)
             if not self.fused:
