@@ -825,12 +825,17 @@ def main():
         run_case(args.case)
         return
     args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        # the oracle on rank 0's host cores: no device and no process group;
+        # under torchrun the other ranks exit at once
+        line = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
+                             int(os.environ.get("RANK", "0")))
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     world, rank, local = dist_setup(args.gpus)
     try:
-        if args.impl == "reference":
-            line = run_reference(args, world, rank)
-        else:
-            line = run_libmsa(args, world, rank, local)
+        line = run_libmsa(args, world, rank, local)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:
