@@ -609,10 +609,11 @@ def attn_flops_per_step(p) -> float:
     return 4.0 * D * Hq * pairs
 
 
-def cpu_baseline(w, p, C, sample_chunks: int = 16384) -> dict:
+def cpu_baseline(w, p, C, route_seconds: float = 10.0, slice_chunks: int = 16384) -> dict:
     """The float64 oracle, as it stands, on a bounded sample of the step:
-    routing over ``sample_chunks`` chunks (scaled to the full bank), then
-    top-k, gather and attention at full size."""
+    routing over 16,384-chunk slices spread evenly over the bank until about
+    ``route_seconds`` of routing time is spent (scaled to the full bank),
+    then top-k, gather and attention at full size."""
     import numpy as np
     import torch
 
@@ -625,10 +626,20 @@ def cpu_baseline(w, p, C, sample_chunks: int = 16384) -> dict:
     cores = len(os.sched_getaffinity(0))
     coff_h = p.coff.cpu().numpy()
     q_r = w["q_r"].double().cpu().numpy()
-    kr_s = w["kr_bar"][:sample_chunks].double().cpu().numpy()
-    t0 = time.perf_counter()
-    oracle.route_chunk_scores(q_r, kr_s)
-    t_route = (time.perf_counter() - t0) * C / sample_chunks
+    n_slices = max(C // slice_chunks, 1)
+    stride = C // n_slices
+    t_spent, done = 0.0, 0
+    while done < n_slices and (done == 0 or t_spent < route_seconds):
+        # slice i of the visiting order 0, n/2, n/4, 3n/4, ... (bit-reversed)
+        i = int(f"{done:032b}"[::-1], 2) * n_slices >> 32
+        s0 = i * stride
+        kr_s = w["kr_bar"][s0:s0 + slice_chunks].double().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.route_chunk_scores(q_r, kr_s)
+        t_spent += time.perf_counter() - t0
+        done += 1
+    sampled = min(done * slice_chunks, C)
+    t_route = t_spent * C / sampled
     # full-size top-k / gather / attention (on seeded scores, independent of
     # the GPU): the gather reads a compact host copy of the selected rows
     rng = np.random.default_rng(0)
@@ -644,8 +655,9 @@ def cpu_baseline(w, p, C, sample_chunks: int = 16384) -> dict:
     step = t_route + t_rest
     return {"value": round(C / step / 1e9, 8), "unit": UNIT, "cores": cores, "blas_threads": blas,
             "kind": "oracle", "seconds_per_step_est": round(step, 3),
-            "sample": f"routing timed on {sample_chunks} of {C} chunks and scaled by "
-                      f"{C / sample_chunks:.1f}; top-k, gather and attention timed at full size"}
+            "sample": f"routing timed on {done} slices of {slice_chunks} chunks spread over the "
+                      f"bank ({sampled} of {C} chunks, {t_spent:.1f} s) and scaled by "
+                      f"{C / sampled:.1f}; top-k, gather and attention timed at full size"}
 
 
 def _compact(k_bank, v_bank, coff_h, docs):
@@ -682,7 +694,7 @@ def run_reference(args, world, rank):
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        cb = cpu_baseline(w, p, C, sample_chunks=4096)
+        cb = cpu_baseline(w, p, C, route_seconds=1.0)
         if i >= args.warmup:
             times.append(cb["seconds_per_step_est"])
     step = statistics.median(times)
