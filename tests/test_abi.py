@@ -2,7 +2,6 @@
 include/msa.h declares, and rejects bad arguments on the host before any
 CUDA work (no GPU needed for these paths)."""
 
-import ctypes
 
 import pytest
 

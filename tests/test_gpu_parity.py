@@ -18,7 +18,6 @@ Full-size workloads are checked on sampled outputs that the oracle computes
 one by one.
 """
 
-import math
 
 import numpy as np
 import pytest

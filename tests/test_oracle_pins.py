@@ -9,7 +9,6 @@ or a transposed operand in the oracle fails at least one of them; the
 that a pin fires.
 """
 
-import math
 import os
 
 import numpy as np
