@@ -97,6 +97,23 @@ const char* msa_version(void);
  * queued on `stream`; blocks the host until that work is done. */
 int msa_device_status(int32_t* host_out, int clear, msa_stream_t stream);
 
+/* Failure-detection check of the bounded device waits.  Every pipelined
+ * kernel (routing scan, chunk pooling, prefill and decode attention) waits on
+ * mbarriers for at most a fixed time; a wait that runs out records
+ * MSA_ERR_TIMEOUT in the device status word and the kernel winds down, so a
+ * lost arrival becomes an error status instead of a hung GPU.  This call runs
+ * that path alone: one thread initialises an mbarrier expecting one arrival
+ * and waits for its first phase for at most limit_ns nanoseconds.
+ *   arrive != 0  the thread arrives first: the wait succeeds at once and
+ *                nothing is recorded;
+ *   arrive == 0  nothing arrives: the wait expires after limit_ns and
+ *                MSA_ERR_TIMEOUT is recorded in the device status word.
+ * The kernel holds no asynchronous copy and no tensor memory, so the context
+ * stays usable either way.  1000 <= limit_ns <= 10^10 (10 s), else
+ * MSA_ERR_INVALID_ARG (checked before any CUDA call).  Asynchronous on
+ * `stream`; read the outcome with msa_device_status. */
+int msa_check_bounded_wait(int64_t limit_ns, int arrive, msa_stream_t stream);
+
 /* Chunk offsets of the bank -- [DEEP] §"三、文档如何变成 memory",
  * "2. chunk 压缩": every `chunk` (64) tokens of a document form one chunk and
  * a trailing partial chunk is kept (180 tokens -> 3 chunks).

@@ -15,6 +15,7 @@ from .msa import (  # noqa: F401
     MSA_BF16,
     MSA_F32,
     MsaError,
+    msa_check_bounded_wait,
     msa_chunk_offsets,
     msa_device_status,
     msa_encode_pool,

@@ -47,6 +47,7 @@ _SIGS = {
     "msa_last_cuda_error": (c_i, []),
     "msa_version": (ctypes.c_char_p, []),
     "msa_device_status": (c_i, [c_p, c_i, c_p]),
+    "msa_check_bounded_wait": (c_i, [c_i64, c_i, c_p]),
     "msa_chunk_offsets": (c_i, [c_i, c_p, c_i, c_p, c_p]),
     "msa_encode_pool": (c_i, [c_i, c_i, c_i64, c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_p,
                               c_i64, c_f, c_i, c_p, c_p, c_p, c_p]),
@@ -163,6 +164,11 @@ def msa_device_status(clear: bool = True, stream=None) -> int:
     _check("msa_device_status",
            lib().msa_device_status(ctypes.addressof(out), int(clear), _stream(stream)))
     return out.value
+
+
+def msa_check_bounded_wait(limit_ns: int, arrive: bool, stream=None):
+    _check("msa_check_bounded_wait",
+           lib().msa_check_bounded_wait(int(limit_ns), int(arrive), _stream(stream)))
 
 
 def msa_chunk_offsets(n_docs, tok_offsets, chunk, chunk_offsets, stream=None):

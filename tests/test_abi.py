@@ -46,6 +46,13 @@ def test_host_validation_topk(lib):
     assert f(1, 10, 2, NULL, 16, NULL, NULL, 0, NULL) == -1     # NULL scores
 
 
+def test_host_validation_bounded_wait(lib):
+    f = lib.msa_check_bounded_wait
+    assert f(999, 0, NULL) == -1                  # limit below 1 us
+    assert f(10_000_000_001, 0, NULL) == -1       # limit above 10 s
+    assert f(-5, 1, NULL) == -1
+
+
 def test_host_validation_route(lib):
     f = lib.msa_route_scores
     p = 256
