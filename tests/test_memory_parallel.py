@@ -1,5 +1,5 @@
 """Memory Parallel host logic on the CPU: the shard plan, and the candidate
-exchange between two gloo ranks, checked against the oracle's unsharded
+exchange between 2, 3 and 4 gloo ranks, checked against the oracle's unsharded
 routing + top-k.  (The merge kernel itself is checked on the GPU in
 test_gpu_parity.py, with the shards emulated in one process.)"""
 
@@ -95,7 +95,8 @@ def _rank_main(rank, world, port, seed, k, fail_q):
         gid = ci.numpy().astype(np.int64) + base[:, None, None]
         full, _ = oracle.route_scores(q_r, kr, off)
         want, _ = oracle.topk_docs(full, k)
-        assert plan[0][0] <= 7 < plan[0][1] <= 50 < plan[1][1]
+        shard = [next(r for r, pr in enumerate(plan) if pr[0] <= d < pr[1]) for d in (7, 50)]
+        assert shard[0] < shard[1]  # the tie crosses a shard boundary
         for b in range(2):
             s = cs.numpy()[:, b].reshape(-1).astype(np.float64)
             g = gid[:, b].reshape(-1)
@@ -115,10 +116,52 @@ def _free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("world", [2])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_exchange_and_merge_gloo(world):
     ctx = mp.get_context("spawn")
     fail_q = ctx.SimpleQueue()
     mp.start_processes(_rank_main, args=(world, _free_port(), 3, 4, fail_q), nprocs=world,
                        join=True, start_method="spawn")
     assert fail_q.empty()
+
+
+def _rank_dies_main(rank, world, port, fail_q, done_q):
+    """Rank 1 raises after joining the group and before the exchange; rank 0
+    must see its exchange end with an error (the peer's connection closes, or
+    the group's short timeout expires) instead of waiting for good."""
+    import datetime
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        raise RuntimeError("rank 1 fails before the exchange (injected on the host)")
+    s = torch.zeros((2, 4), dtype=torch.float32)
+    i = torch.zeros((2, 4), dtype=torch.int32)
+    try:
+        mpar.exchange_candidates(s, i)
+    except Exception as e:  # detected: report and leave
+        done_q.put(f"rank 0 detected: {type(e).__name__}")
+        return
+    fail_q.put("rank 0: the exchange completed without its peer")
+
+
+def test_rank_failure_before_exchange_is_detected():
+    ctx = mp.get_context("spawn")
+    fail_q, done_q = ctx.SimpleQueue(), ctx.SimpleQueue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_dies_main, args=(r, 2, port, fail_q, done_q))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    alive = [p.pid for p in procs if p.is_alive()]
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert not alive, "a rank did not finish"
+    assert fail_q.empty(), fail_q.get()
+    assert not done_q.empty(), "rank 0 did not report the failure"
+    assert done_q.get().startswith("rank 0 detected")
+    assert procs[0].exitcode == 0 and procs[1].exitcode != 0
