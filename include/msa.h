@@ -55,6 +55,21 @@
  *                           scan;
  *       MSA_ATTN_SPLITS=n   at most n (1..16) key-tile splits in prefill
  *                           attention (default 3).
+ *   - Debug build (libmsa_debug.so: the same sources compiled with
+ *     -DMSA_DEBUG).  Its kernels are the release kernels.  What changes is
+ *     that every compute entry point, after its host checks, validates on
+ *     the device the index arrays it is given:
+ *       - CSR offsets must be non-negative, non-decreasing and within the
+ *         tensor they index;
+ *       - memory lengths must lie in [0, m_cap].
+ *     The call waits for that check and returns MSA_ERR_INVALID_ARG before
+ *     any of its kernels reads through a bad array.  At its end it waits for
+ *     its own work and returns a CUDA error or the status word's first
+ *     error, such as MSA_ERR_CAPACITY.  The word is read, not cleared, so an
+ *     earlier unread error is returned too.  While the stream is being
+ *     captured into a CUDA graph nothing waits: the checks are captured with
+ *     the call and record into the status word.  msa_check_bounded_wait is
+ *     not wrapped.
  */
 #ifndef MSA_H
 #define MSA_H

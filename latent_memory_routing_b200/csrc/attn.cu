@@ -286,11 +286,11 @@ extern "C" size_t msa_sparse_attn_workspace_size(msa_dtype dt, int B, int T, int
   return plan(B, T, T_loc, Hq, H, D, m_cap, num_sms()).total;
 }
 
-extern "C" int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, int H, int D,
-                               const void* q, const void* k_mem, const void* v_mem,
-                               const int32_t* mem_len, int m_cap, const void* k_loc,
-                               const void* v_loc, int pos0, float rope_base, float scale,
-                               void* out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+static int sparse_attn_body(msa_dtype dt, int B, int T, int T_loc, int Hq, int H, int D,
+                            const void* q, const void* k_mem, const void* v_mem,
+                            const int32_t* mem_len, int m_cap, const void* k_loc,
+                            const void* v_loc, int pos0, float rope_base, float scale,
+                            void* out, void* ws, size_t ws_bytes, msa_stream_t stream) {
   using namespace msa;
   if (B <= 0 || T <= 0 || T_loc < T || H <= 0 || Hq <= 0 || m_cap < 0 || pos0 < 0)
     return MSA_ERR_INVALID_ARG;
@@ -301,6 +301,7 @@ extern "C" int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, in
   if (dt != MSA_F32 && dt != MSA_BF16) return MSA_ERR_INVALID_ARG;
   if ((int64_t)B * H > 65535 || (int64_t)m_cap + T_loc > (1LL << 30)) return MSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = debug_check_mem_len(mem_len, B, m_cap, s)) return rc;
   const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)D);
   const float qscale = sc * kLog2e;
   if (dt == MSA_BF16 && attn_decode_tc_supported(T, Hq, H, D) && decode_tc_enabled()) {
@@ -343,4 +344,15 @@ extern "C" int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, in
              : launch_simt<__nv_bfloat16, 128>(B, T, T_loc, Hq, H, q, k_mem, v_mem, mem_len,
                                                m_cap, k_loc, v_loc, p, cs, qscale, part_o,
                                                part_ml, out, s);
+}
+
+extern "C" int msa_sparse_attn(msa_dtype dt, int B, int T, int T_loc, int Hq, int H, int D,
+                               const void* q, const void* k_mem, const void* v_mem,
+                               const int32_t* mem_len, int m_cap, const void* k_loc,
+                               const void* v_loc, int pos0, float rope_base, float scale,
+                               void* out, void* ws, size_t ws_bytes, msa_stream_t stream) {
+  return msa::debug_finish(sparse_attn_body(dt, B, T, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len,
+                                            m_cap, k_loc, v_loc, pos0, rope_base, scale, out,
+                                            ws, ws_bytes, stream),
+                           reinterpret_cast<cudaStream_t>(stream));
 }

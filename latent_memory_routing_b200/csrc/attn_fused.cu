@@ -133,6 +133,7 @@ extern "C" int msa_sparse_attn_fused(msa_dtype dt, int B, int T, int T_loc, int 
   if ((int64_t)B * p.max_groups * 8 > INT32_MAX) return MSA_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < p.total || !aligned16(ws)) return MSA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = debug_check_offsets(chunk_offsets, n_docs, n_chunks, s)) return rc;
   unsigned char* w = static_cast<unsigned char*>(ws);
   int2* groups = reinterpret_cast<int2*>(w);
   int32_t* n_groups = reinterpret_cast<int32_t*>(w + p.g_bytes);
@@ -146,8 +147,10 @@ extern "C" int msa_sparse_attn_fused(msa_dtype dt, int B, int T, int T_loc, int 
   const float qscale = sc * 1.4426950408889634f;  // log2(e): softmax in base 2
   const FusedMemory fm{groups, n_groups, p.max_groups, k_bar, v_bar, n_chunks};
   if (T == 1)
-    return attn_decode_tc_launch_fused(B, T_loc, Hq, H, D, q, fm, k_loc, v_loc, pos0, rope_base,
-                                       qscale, out, attn_ws, s);
-  return attn_tc_launch_fused(B, T, T_loc, Hq, H, D, q, fm, k_loc, v_loc, pos0, rope_base, qscale,
+    rc = attn_decode_tc_launch_fused(B, T_loc, Hq, H, D, q, fm, k_loc, v_loc, pos0, rope_base,
+                                     qscale, out, attn_ws, s);
+  else
+    rc = attn_tc_launch_fused(B, T, T_loc, Hq, H, D, q, fm, k_loc, v_loc, pos0, rope_base, qscale,
                               out, attn_ws, s);
+  return debug_finish(rc, s);
 }

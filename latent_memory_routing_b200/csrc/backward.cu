@@ -414,6 +414,8 @@ extern "C" int msa_encode_pool_backward(int L, int64_t n_tok, int n_docs, int H,
     return MSA_ERR_INVALID_ARG;
   if (n_chunks > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = debug_check_offsets(tok_offsets, n_docs, n_tok, s)) return rc;
+  if (int rc = debug_check_offsets(chunk_offsets, n_docs, n_chunks, s)) return rc;
   if (D == 64)
     pool_backward_kernel<64><<<(unsigned)n_chunks, kPbThreads, 0, s>>>(
         L, n_tok, n_docs, H, dk_bar, dv_bar, dkr_bar, tok_offsets, chunk_offsets, n_chunks,
@@ -422,7 +424,7 @@ extern "C" int msa_encode_pool_backward(int L, int64_t n_tok, int n_docs, int H,
     pool_backward_kernel<128><<<(unsigned)n_chunks, kPbThreads, 0, s>>>(
         L, n_tok, n_docs, H, dk_bar, dv_bar, dkr_bar, tok_offsets, chunk_offsets, n_chunks,
         (double)rope_base, dk_tok, dv_tok, dkr_tok);
-  return check_launch();
+  return debug_finish(check_launch(), s);
 }
 
 extern "C" int msa_route_backward(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
@@ -438,6 +440,7 @@ extern "C" int msa_route_backward(msa_dtype dt, int B, int T, int H, int D, cons
   if (dt != MSA_F32 && dt != MSA_BF16) return MSA_ERR_INVALID_ARG;
   if (n_chunks > 0x7fffffffLL || (int64_t)B * T > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = debug_check_offsets(chunk_offsets, n_docs, n_chunks, s)) return rc;
   if (route_backward_tc(dt, B, T, H, D, n_chunks)) {
     // (1) the first maximiser of every (query, document) on the tensor
     // cores; (2) the cosine gradients at those pairs on the CUDA cores
@@ -460,7 +463,7 @@ extern "C" int msa_route_backward(msa_dtype dt, int B, int T, int H, int D, cons
     route_grad_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(B, T, H, D, q, k, chunk_offsets, n_docs,
                                                           d_doc, keys, dq_r, dkr_bar,
                                                           device_status_ptr());
-    return check_launch();
+    return debug_finish(check_launch(), s);
   }
   const size_t smem = (size_t)(kRbChunks + kRbTokens) * H * D * sizeof(float);
   const int64_t pairs = (int64_t)B * n_docs;
@@ -480,5 +483,5 @@ extern "C" int msa_route_backward(msa_dtype dt, int B, int T, int H, int D, cons
                                      static_cast<const __nv_bfloat16*>(kr_bar), chunk_offsets,
                                      n_docs, d_doc, dq_r, dkr_bar, device_status_ptr());
   }
-  return check_launch();
+  return debug_finish(check_launch(), s);
 }

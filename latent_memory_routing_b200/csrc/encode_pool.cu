@@ -442,10 +442,11 @@ extern "C" int msa_chunk_offsets(int n_docs, const int64_t* tok_offsets,
   if (n_docs <= 0 || !tok_offsets || !chunk_offsets) return MSA_ERR_INVALID_ARG;
   if (chunk < 1 || chunk > msa::kMaxChunk) return MSA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (int rc = msa::debug_check_offsets(tok_offsets, n_docs, INT64_MAX, s)) return rc;
   msa::chunk_offsets_kernel<<<1, 1024, 0, s>>>(n_docs, tok_offsets, chunk,
                                                chunk_offsets,
                                                msa::device_status_ptr());
-  return msa::check_launch();
+  return msa::debug_finish(msa::check_launch(), s);
 }
 
 extern "C" int msa_encode_pool(msa_dtype dt, int L, int64_t n_tok, int n_docs,
@@ -467,22 +468,23 @@ extern "C" int msa_encode_pool(msa_dtype dt, int L, int64_t n_tok, int n_docs,
   if (H < 1 || H > 16 || (D != 64 && D != 128)) return MSA_ERR_UNSUPPORTED;
   if (n_chunks > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dt == MSA_F32) {
-    return D == 64 ? launch_encode<float, 64>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
-                                              tok_offsets, chunk_offsets, n_chunks,
-                                              rope_base, chunk, k_bar, v_bar, kr_bar, s)
-                   : launch_encode<float, 128>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
-                                               tok_offsets, chunk_offsets, n_chunks,
-                                               rope_base, chunk, k_bar, v_bar, kr_bar, s);
-  }
-  if (dt == MSA_BF16) {
-    return D == 64
-               ? launch_encode<__nv_bfloat16, 64>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
-                                                  tok_offsets, chunk_offsets, n_chunks,
-                                                  rope_base, chunk, k_bar, v_bar, kr_bar, s)
-               : launch_encode<__nv_bfloat16, 128>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
-                                                   tok_offsets, chunk_offsets, n_chunks,
-                                                   rope_base, chunk, k_bar, v_bar, kr_bar, s);
-  }
-  return MSA_ERR_INVALID_ARG;
+  if (dt != MSA_F32 && dt != MSA_BF16) return MSA_ERR_INVALID_ARG;
+  if (int rc = debug_check_offsets(tok_offsets, n_docs, n_tok, s)) return rc;
+  if (int rc = debug_check_offsets(chunk_offsets, n_docs, n_chunks, s)) return rc;
+  int rc;
+  if (dt == MSA_F32)
+    rc = D == 64 ? launch_encode<float, 64>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
+                                            tok_offsets, chunk_offsets, n_chunks, rope_base,
+                                            chunk, k_bar, v_bar, kr_bar, s)
+                 : launch_encode<float, 128>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
+                                             tok_offsets, chunk_offsets, n_chunks, rope_base,
+                                             chunk, k_bar, v_bar, kr_bar, s);
+  else
+    rc = D == 64 ? launch_encode<__nv_bfloat16, 64>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
+                                                    tok_offsets, chunk_offsets, n_chunks,
+                                                    rope_base, chunk, k_bar, v_bar, kr_bar, s)
+                 : launch_encode<__nv_bfloat16, 128>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
+                                                     tok_offsets, chunk_offsets, n_chunks,
+                                                     rope_base, chunk, k_bar, v_bar, kr_bar, s);
+  return debug_finish(rc, s);
 }

@@ -98,11 +98,13 @@ extern "C" int msa_gather_kv(msa_dtype dt, int B, int k, int H, int D, const int
   if (row_bytes % 16) return MSA_ERR_UNSUPPORTED;
   if (B > 65535) return MSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the bank's row count is not an argument here: offsets are checked for order only
+  if (int rc = debug_check_offsets(chunk_offsets, n_docs, INT64_MAX, s)) return rc;
   const dim3 grid((unsigned)(k * kSplit), (unsigned)B);
   gather_kernel<<<grid, 256, 0, s>>>(k, n_docs, (int)(row_bytes / 16), idx, chunk_offsets,
                                      static_cast<const uint4*>(k_bar),
                                      static_cast<const uint4*>(v_bar), m_cap,
                                      static_cast<uint4*>(k_mem), static_cast<uint4*>(v_mem),
                                      mem_len, device_status_ptr());
-  return check_launch();
+  return debug_finish(check_launch(), s);
 }

@@ -60,7 +60,8 @@ extern "C" int msa_topk_merge_shards(int B, int world, int k, const float* cand_
   if (B <= 0 || world <= 0 || k <= 0 || !cand_scores || !cand_idx || !doc_base || !idx)
     return MSA_ERR_INVALID_ARG;
   if ((int64_t)world * k > kMaxCands || B > 0x7fffffff) return MSA_ERR_UNSUPPORTED;
-  merge_shards_kernel<<<(unsigned)B, kMergeThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  merge_shards_kernel<<<(unsigned)B, kMergeThreads, 0, s>>>(
       B, world, k, cand_scores, cand_idx, doc_base, idx, top_scores, device_status_ptr());
-  return check_launch();
+  return debug_finish(check_launch(), s);
 }

@@ -43,6 +43,31 @@ __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// ------------------------------------------------------------- debug build
+//
+// Built with -DMSA_DEBUG (libmsa_debug.so), every entry point checks the
+// device-side index arrays it is given before any kernel reads through them,
+// and waits for its own work.  A check launches a small validation kernel,
+// waits for it and returns the device status word's error, if one is set
+// (the word is not cleared), so a bad input comes back as an error status
+// from the call that received it and the hot kernels never run on it.
+// While the stream is being captured into a CUDA graph nothing waits: the
+// validation kernels are captured too and record into the status word.  In
+// the release build these functions are empty and compile away.
+#ifdef MSA_DEBUG
+// CSR offsets [n+1]: 0 <= off[0] <= off[1] <= ... <= off[n] <= total.
+int debug_check_offsets(const int64_t* off, int n, int64_t total, cudaStream_t s);
+// Per-query memory lengths [B]: 0 <= mem_len[b] <= m_cap.
+int debug_check_mem_len(const int32_t* mem_len, int B, int m_cap, cudaStream_t s);
+// End of an entry point: rc if it is an error; otherwise waits for the
+// stream and returns a CUDA error or the status word's error, if any.
+int debug_finish(int rc, cudaStream_t s);
+#else
+inline int debug_check_offsets(const int64_t*, int, int64_t, cudaStream_t) { return MSA_OK; }
+inline int debug_check_mem_len(const int32_t*, int, int, cudaStream_t) { return MSA_OK; }
+inline int debug_finish(int rc, cudaStream_t) { return rc; }
+#endif
+
 // ------------------------------------------------------------ element types
 
 template <typename T> struct Elem;

@@ -174,6 +174,7 @@ int route_scores_impl(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
   const int64_t n_chunk_u = chunk_scores ? (int64_t)B * n_chunks : 0;
   const int sms = num_sms();
   int rc;
+  if ((rc = debug_check_offsets(chunk_offsets, n_docs, n_chunks, s))) return rc;
   if (dt == MSA_F32) {
     const int64_t rows = (int64_t)NT * H;
     const unsigned blocks = (unsigned)std::min<int64_t>((rows * 32 + 255) / 256 + 1, 1 << 20);
@@ -206,7 +207,7 @@ int route_scores_impl(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
     if (rc) return rc;
   }
   route_finalize_kernel<<<(unsigned)sms * 4, 256, 0, s>>>(doc_u, n_doc_u, chunk_u, n_chunk_u);
-  return check_launch();
+  return debug_finish(check_launch(), s);
 }
 
 }  // namespace
@@ -251,7 +252,9 @@ extern "C" int msa_route_prepare_bank(msa_dtype dt, int64_t n_chunks, int H, int
   if (n_chunks <= 0 || H <= 0 || !kr_bar || !kr_hat) return MSA_ERR_INVALID_ARG;
   if (!aligned16(kr_bar) || !aligned16(kr_hat)) return MSA_ERR_INVALID_ARG;
   if (dt != MSA_BF16 || (D != 64 && D != 128)) return MSA_ERR_UNSUPPORTED;
-  return route_prepare_bank_launch(n_chunks * H, D, static_cast<const __nv_bfloat16*>(kr_bar),
-                                   static_cast<__nv_bfloat16*>(kr_hat),
-                                   reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return debug_finish(route_prepare_bank_launch(n_chunks * H, D,
+                                                static_cast<const __nv_bfloat16*>(kr_bar),
+                                                static_cast<__nv_bfloat16*>(kr_hat), s),
+                      s);
 }

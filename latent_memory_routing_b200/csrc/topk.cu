@@ -439,9 +439,8 @@ extern "C" size_t msa_topk_workspace_size(int B, int n_docs, int k) {
   return msa::plan(B, n_docs, k).ws_bytes;
 }
 
-extern "C" int msa_topk_docs(int B, int n_docs, int k, const float* scores, int32_t* idx,
-                             float* top_scores, void* ws, size_t ws_bytes,
-                             msa_stream_t stream) {
+static int topk_docs_body(int B, int n_docs, int k, const float* scores, int32_t* idx,
+                          float* top_scores, void* ws, size_t ws_bytes, msa_stream_t stream) {
   using namespace msa;
   if (B <= 0 || n_docs <= 0 || k <= 0 || k > n_docs || k > kMaxK) return MSA_ERR_INVALID_ARG;
   if (!scores || !idx) return MSA_ERR_INVALID_ARG;
@@ -481,4 +480,12 @@ extern "C" int msa_topk_docs(int B, int n_docs, int k, const float* scores, int3
   if (rc) return rc;
   topk_merge_kernel<<<B, kThreads, smem, s>>>(n_docs, k, n_cand, cand, scores, idx, top_scores);
   return check_launch();
+}
+
+extern "C" int msa_topk_docs(int B, int n_docs, int k, const float* scores, int32_t* idx,
+                             float* top_scores, void* ws, size_t ws_bytes,
+                             msa_stream_t stream) {
+  return msa::debug_finish(
+      topk_docs_body(B, n_docs, k, scores, idx, top_scores, ws, ws_bytes, stream),
+      reinterpret_cast<cudaStream_t>(stream));
 }

@@ -7,6 +7,12 @@ integer device addresses.  ``stream`` defaults to torch's current stream on
 the current device.  A non-zero status raises ``MsaError``; the library must
 have been built (``python -m latent_memory_routing_b200.build``) -- there is
 no fallback.
+
+With ``MSA_DEBUG=1`` in the environment the binding loads
+``libmsa_debug.so`` (``python -m latent_memory_routing_b200.build --debug``)
+instead: the same kernels, with every call first checking the device-side
+index arrays it is given and then waiting for its own work, so that a
+device-detected error is raised by the call that caused it.
 """
 
 from __future__ import annotations
@@ -16,7 +22,8 @@ import os
 import re
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libmsa.so")
+LIB_PATH = os.path.join(PKG, "libmsa_debug.so" if os.environ.get("MSA_DEBUG") == "1"
+                         else "libmsa.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "msa.h")
 
 MSA_F32 = 0

@@ -82,3 +82,50 @@ def test_workspace_sizes_are_monotone(lib):
     b = msa.msa_route_workspace_size(1, 2, 256, 8, 128)
     assert 0 < a < b
     assert msa.msa_route_workspace_size(1, 0, 256, 8, 128) == 0
+
+
+@pytest.fixture(scope="module")
+def debug_lib():
+    """libmsa_debug.so (same sources built with -DMSA_DEBUG), loaded beside
+    the release library under its own handle."""
+    import ctypes
+
+    from latent_memory_routing_b200 import build
+    handle = ctypes.CDLL(build.build(debug=True))
+    for name, (res, args) in msa._SIGS.items():
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    return handle
+
+
+def test_debug_library_exports_every_call(debug_lib):
+    missing = [n for n in msa.header_symbols() if not hasattr(debug_lib, n)]
+    assert not missing, missing
+
+
+def test_debug_library_rejects_the_same_host_arguments(debug_lib):
+    f = debug_lib.msa_topk_docs
+    assert f(1, 10, 11, 16, 16, NULL, NULL, 0, NULL) == -1
+    p = 256
+    g = debug_lib.msa_route_scores
+    assert g(1, 1, 4, 8, 96, p, p, 10, p, 2, p, NULL, p, 1 << 20, NULL) == -2
+    assert g(1, 1, 4, 8, 128, p, p, 10, p, 2, p, NULL, NULL, 0, NULL) == -6
+
+
+def test_input_checks_exist_only_in_the_debug_build(debug_lib):
+    """The release library carries none of the debug build's checks (they
+    compile away), the debug library carries all three."""
+    import subprocess
+
+    from latent_memory_routing_b200 import build
+
+    def checks(path):
+        out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True,
+                             text=True, check=True).stdout
+        return {n for n in ("debug_check_offsets", "debug_check_mem_len", "debug_finish")
+                if n in out}
+
+    assert checks(build.LIB_DEBUG) == {"debug_check_offsets", "debug_check_mem_len",
+                                       "debug_finish"}
+    assert checks(build.LIB) == set()
