@@ -42,9 +42,10 @@
 //     keep per-thread partial row sums (reduced once at the end), and write
 //     P^T (bf16) as the B operand of P V; at an item's last tile they reduce
 //     the row sums and write the item's output.
-// The query buffers are double-buffered by item and by tile.  Splits write (max, sum, O) partials that the split-KV combine kernel
-// merges; a single split writes the normalised output directly.  Every wait
-// is bounded; after a timeout every role walks its loop without waiting.
+// The query buffers are double-buffered by item and by tile.  Splits write
+// (max, sum, O) partials that the split-KV combine kernel merges; a single
+// split writes the normalised output directly.  Every wait is bounded; after
+// a timeout every role walks its loop without waiting.
 #include <cudaTypedefs.h>
 
 #include <algorithm>

@@ -12,26 +12,33 @@
 //   * rope_prep_kernel rotates Q (to pos0 + T_loc - T + i) and the local K
 //     (to pos0 + j) once per call into bf16 workspace copies, one launch,
 //     cos/sin per position built in shared memory (angles reduced in double).
-//   * attn_tc_kernel: one CTA per (128 query rows, KV head, batch, key split;
-//     up to 3 splits of the key tiles, merged by the split-KV combine
-//     kernel, when there are too few row tiles to fill the SMs).  GQA rows
-//     are packed as (token, head of the group): a TMA box of
-//     {64 d, G heads, 128/G tokens} lands as 128 rows of 128 B -- the Q tile
-//     of all G query heads sharing one KV head.  Key tiles of 128 rows come
-//     first from the memory (mem_len rows) then from the local context
-//     (up to the block's last visible key), each as K and V TMA boxes.
-//     - warp 0 (one lane): TMA producer, 2-stage K/V ring;
-//     - warp 1 (one lane): tcgen05.mma S = Q K^T (M=128, N=128 keys, K=D)
-//       into one of two TMEM buffers, and O += P V (M=128, N=D, K=128 keys,
-//       V read MN-major straight from its TMA tile) into the TMEM output
-//       accumulator; the S of tile j+1 is issued before the P V of tile j;
-//     - warps 2..5 (one thread per row): online softmax in fp32 -- the
-//       tile's scores read once from TMEM, masked row maximum, p = 2^(s - m)
-//       (SFU ex2) written as bf16 into a double-buffered shared P tile
-//       (128B-swizzled, the MMA's A operand), row sum.  O accumulates in
-//       TMEM; a row rescales O and its sum only when its maximum grows by
-//       more than 2^8 (then p <= 256 meanwhile), which after the first tiles
-//       is rare.
+//   * attn_tc_kernel: one CTA per (two Q tiles of 128 rows, KV head, batch,
+//     key split), query blocks dispatched heaviest first (causal work grows
+//     with the block index).  Up to 3 splits of the key tiles, at most one
+//     per 8 tiles, are merged by the split-KV combine kernel when there are
+//     too few query blocks to fill the SMs.  GQA rows are packed as (token,
+//     head of the group): a TMA box of {64 d, G heads, 128/G tokens} lands as
+//     128 rows of 128 B -- a Q tile of all G query heads sharing one KV head.
+//     Key tiles of 128 rows come first from the memory (mem_len rows, clamped
+//     to [0, m_cap]) then from the local context (up to the block's last
+//     visible key), each as K and V TMA boxes.
+//     - warpgroup 0: warp 0 (one lane) loads the Q tiles, then runs a 2-stage
+//       K/V ring; warp 1 (one lane) issues tcgen05.mma.  S_i = Q_i K^T
+//       (M = 128, N = 128 keys, K = D) goes to the 128 TMEM columns of Q tile
+//       i; O_i += P_i V (M = 128, N = D, K = 128 keys) reads P_i from those
+//       same TMEM columns (the A operand in tensor memory) and V MN-major
+//       straight from its TMA tile.  The issue order
+//       S_0(0) S_1(0) | P_0V(0) S_0(1) P_1V(0) S_1(1) | ...
+//       keeps one softmax warpgroup busy while the tensor core serves the
+//       other;
+//     - warpgroups 1 and 2 (one per Q tile, one thread per row, registers
+//       moved to them by setmaxnreg): online softmax in fp32 -- the tile's
+//       scores read once from TMEM, masked row maximum, p = 2^(s - m) (SFU
+//       ex2) packed to bf16 and written back over S in TMEM, row sum.  O
+//       accumulates in TMEM; a row rescales O and its sum only when its
+//       maximum grows by more than 2^8 (then p <= 256 meanwhile), which after
+//       the first tiles is rare.  In the last memory tile, warpgroup 1 zeroes
+//       the V rows past mem_len in shared memory before P V reads them.
 //   * Every mbarrier wait is bounded; a timeout records MSA_ERR_TIMEOUT and
 //     all roles finish their loops without waiting.
 #include <cudaTypedefs.h>

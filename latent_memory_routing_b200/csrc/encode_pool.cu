@@ -11,7 +11,7 @@
 // Design (HBM-bound stream).  encode_tma_kernel (the default): persistent
 // CTAs, one per SM, each owning a contiguous range of chunks.  Three producer
 // threads stream, per (chunk, layer), the chunk's contiguous token rows of K,
-// V and K_r with 1-D bulk copies (cp.async.bulk, 32 KB stages, a two-stage
+// V and K_r with 1-D bulk copies (cp.async.bulk, 16 KB stages, a four-stage
 // ring per tensor, so that each ring has one consumer group and a group
 // never waits on a slot another group's stage may still hold) -- the copy
 // engine keeps up to 192 KB in flight per SM without a load instruction per

@@ -34,7 +34,11 @@
 //     query's tokens (a tree maximum when 32 columns belong to one query),
 //     then over the rows of each document inside the warp (segmented
 //     shuffle maximum), and issue one order-preserving atomicMax per
-//     (query, document segment).
+//     (query, document segment).  For queries of fewer than 32 tokens the
+//     epilogue parks per-query maxima in shared memory and walks document
+//     runs from a warp-uniform run mask instead (the column-owner epilogue);
+//   * argmax mode (kArg, for the routing backward): the same scan keeps each
+//     (query, document)'s first maximising (chunk, token) as a 64-bit key.
 // Scores never round-trip through HBM.  No cluster multicast is used.
 #include <cudaTypedefs.h>
 
