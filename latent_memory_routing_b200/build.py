@@ -11,7 +11,8 @@ are rebuilt only when a source or header is newer.
 -DMSA_DEBUG: every entry point validates the device-side index arrays it is
 given (CSR offsets, memory lengths) before its kernels read through them and
 waits for its own work, returning device-detected errors from the call
-itself.  Its kernels are otherwise those of the release library.
+itself.  Its kernels are otherwise those of the release library: sources
+that do not call the debug checks are linked from the release objects.
 """
 
 from __future__ import annotations
@@ -62,14 +63,29 @@ def _compile(src: str, verbose: bool, out_dir: str, extra: list[str]) -> str:
     return obj
 
 
+def _uses_debug_hooks(src: str) -> bool:
+    """True if the source calls the debug build's checks (or tests for it);
+    every other source compiles to the same object in both builds."""
+    with open(src, encoding="utf-8") as f:
+        text = f.read()
+    return "debug_check_" in text or "debug_finish" in text or "MSA_DEBUG" in text
+
+
 def build(verbose: bool = False, debug: bool = False) -> str:
-    out_dir = os.path.join(BUILD, "debug") if debug else BUILD
     lib = LIB_DEBUG if debug else LIB
-    extra = ["-DMSA_DEBUG"] if debug else []
-    os.makedirs(out_dir, exist_ok=True)
+    debug_dir = os.path.join(BUILD, "debug")
+    os.makedirs(BUILD, exist_ok=True)
+    if debug:
+        os.makedirs(debug_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+    def obj(src: str) -> str:
+        if debug and _uses_debug_hooks(src):
+            return _compile(src, verbose, debug_dir, ["-DMSA_DEBUG"])
+        return _compile(src, verbose, BUILD, [])
+
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 4)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose, out_dir, extra), srcs))
+        objs = list(ex.map(obj, srcs))
     if (not os.path.exists(lib)
             or max(os.path.getmtime(o) for o in objs) > os.path.getmtime(lib)):
         tmp = lib + ".tmp"
