@@ -224,14 +224,7 @@ def run_libmsa(args, world, rank, local):
     graph = p.capture(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
     for _ in range(3):
         graph.replay()
-    # nvidia-smi samples every 200 ms, far longer than the timed steps, so
-    # the sampler runs over about 1 s of the same replays just before the
-    # timed region and about 0.5 s just after it (untimed); the timed region
-    # itself is exactly args.steps replays between the two barriers
-    n_pad = int(min(5000, max(20, 1000.0 / max(sum(seg), 1e-3))))
     clocks = Clocks(local)
-    for _ in range(n_pad):
-        graph.replay()
     barrier(world)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -240,12 +233,7 @@ def run_libmsa(args, world, rank, local):
         graph.replay()
     t_end.record()
     barrier(world)
-    for _ in range(n_pad // 2):
-        graph.replay()
-    torch.cuda.synchronize()
     clk = clocks.stop()
-    clk["window"] = (f"{n_pad} untimed replays of the step before the timed region and "
-                     f"{n_pad // 2} after it")
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     ms_step = total_ms / args.steps
     value = C * world / (ms_step * 1e-3) / 1e9
