@@ -144,12 +144,28 @@ def _check(name: str, rc: int):
         raise MsaError(name, rc, detail)
 
 
-def _numel_ok(t, n, what):
+_ESIZE = {MSA_F32: 4, MSA_BF16: 2}
+F32, I32, I64 = 4, 4, 8  # element sizes of the fixed-type arguments
+
+
+def _es(dt) -> int | None:
+    """Element size of a `dt`-typed tensor (None for an unknown dt, which the
+    library itself rejects)."""
+    return _ESIZE.get(dt)
+
+
+def _numel_ok(t, n, what, esize=None):
+    """Checks a tensor argument: contiguous, at least n elements and, given
+    the element size the call uses, at least n * esize bytes (a tensor of a
+    narrower type than the call reads would be overrun)."""
     if t is not None and not isinstance(t, int):
         if not t.is_contiguous():
             raise ValueError(f"{what} must be contiguous")
         if t.numel() < n:
             raise ValueError(f"{what} holds {t.numel()} elements, needs {n}")
+        if esize and t.numel() * t.element_size() < n * esize:
+            raise ValueError(f"{what} holds {t.numel() * t.element_size()} bytes, needs "
+                             f"{n * esize} ({n} elements of {esize} bytes)")
 
 
 # ---------------------------------------------------------------- entry points
@@ -179,8 +195,8 @@ def msa_check_bounded_wait(limit_ns: int, arrive: bool, stream=None):
 
 
 def msa_chunk_offsets(n_docs, tok_offsets, chunk, chunk_offsets, stream=None):
-    _numel_ok(tok_offsets, n_docs + 1, "tok_offsets")
-    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets")
+    _numel_ok(tok_offsets, n_docs + 1, "tok_offsets", I64)
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
     _check("msa_chunk_offsets", lib().msa_chunk_offsets(
         n_docs, _ptr(tok_offsets), chunk, _ptr(chunk_offsets), _stream(stream)))
 
@@ -189,9 +205,11 @@ def msa_encode_pool(dt, L, n_tok, n_docs, H, D, k_tok, v_tok, kr_tok, tok_offset
                     chunk_offsets, n_chunks, rope_base, chunk, k_bar, v_bar, kr_bar,
                     stream=None):
     for t, what in ((k_tok, "k_tok"), (v_tok, "v_tok"), (kr_tok, "kr_tok")):
-        _numel_ok(t, L * n_tok * H * D, what)
+        _numel_ok(t, L * n_tok * H * D, what, _es(dt))
     for t, what in ((k_bar, "k_bar"), (v_bar, "v_bar"), (kr_bar, "kr_bar")):
-        _numel_ok(t, L * n_chunks * H * D, what)
+        _numel_ok(t, L * n_chunks * H * D, what, _es(dt))
+    _numel_ok(tok_offsets, n_docs + 1, "tok_offsets", I64)
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
     _check("msa_encode_pool", lib().msa_encode_pool(
         dt, L, n_tok, n_docs, H, D, _ptr(k_tok), _ptr(v_tok), _ptr(kr_tok),
         _ptr(tok_offsets), _ptr(chunk_offsets), n_chunks, rope_base, chunk,
@@ -204,28 +222,30 @@ def msa_route_workspace_size(dt, B, T, H, D) -> int:
 
 def msa_route_scores(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_docs,
                      doc_scores, chunk_scores, ws, ws_bytes, stream=None):
-    _numel_ok(q_r, B * T * H * D, "q_r")
-    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
-    _numel_ok(doc_scores, B * n_docs, "doc_scores")
-    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores")
+    _numel_ok(q_r, B * T * H * D, "q_r", _es(dt))
+    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar", _es(dt))
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
+    _numel_ok(doc_scores, B * n_docs, "doc_scores", F32)
+    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores", F32)
     _check("msa_route_scores", lib().msa_route_scores(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def msa_route_prepare_bank(dt, n_chunks, H, D, kr_bar, kr_hat, stream=None):
-    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
-    _numel_ok(kr_hat, n_chunks * H * D, "kr_hat")
+    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar", _es(dt))
+    _numel_ok(kr_hat, n_chunks * H * D, "kr_hat", _es(dt))
     _check("msa_route_prepare_bank", lib().msa_route_prepare_bank(
         dt, n_chunks, H, D, _ptr(kr_bar), _ptr(kr_hat), _stream(stream)))
 
 
 def msa_route_scores_prepared(dt, B, T, H, D, q_r, kr_hat, n_chunks, chunk_offsets, n_docs,
                               doc_scores, chunk_scores, ws, ws_bytes, stream=None):
-    _numel_ok(q_r, B * T * H * D, "q_r")
-    _numel_ok(kr_hat, n_chunks * H * D, "kr_hat")
-    _numel_ok(doc_scores, B * n_docs, "doc_scores")
-    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores")
+    _numel_ok(q_r, B * T * H * D, "q_r", _es(dt))
+    _numel_ok(kr_hat, n_chunks * H * D, "kr_hat", _es(dt))
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
+    _numel_ok(doc_scores, B * n_docs, "doc_scores", F32)
+    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores", F32)
     _check("msa_route_scores_prepared", lib().msa_route_scores_prepared(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_hat), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws_bytes, _stream(stream)))
@@ -239,10 +259,11 @@ def msa_route_scores_noalloc(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offset
                              doc_scores, chunk_scores, stream=None):
     """msa_route_scores with the library's fixed scratch array instead of a
     caller workspace (for callers that cannot allocate device memory)."""
-    _numel_ok(q_r, B * T * H * D, "q_r")
-    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
-    _numel_ok(doc_scores, B * n_docs, "doc_scores")
-    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores")
+    _numel_ok(q_r, B * T * H * D, "q_r", _es(dt))
+    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar", _es(dt))
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
+    _numel_ok(doc_scores, B * n_docs, "doc_scores", F32)
+    _numel_ok(chunk_scores, B * n_chunks, "chunk_scores", F32)
     _check("msa_route_scores_noalloc", lib().msa_route_scores_noalloc(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(doc_scores), _ptr(chunk_scores), _stream(stream)))
@@ -254,18 +275,20 @@ def msa_topk_workspace_size(B, n_docs, k) -> int:
 
 def msa_topk_merge_shards(B, world, k, cand_scores, cand_idx, doc_base, idx, top_scores,
                           stream=None):
-    _numel_ok(cand_scores, world * B * k, "cand_scores")
-    _numel_ok(cand_idx, world * B * k, "cand_idx")
-    _numel_ok(doc_base, world, "doc_base")
-    _numel_ok(idx, B * k, "idx")
+    _numel_ok(cand_scores, world * B * k, "cand_scores", F32)
+    _numel_ok(cand_idx, world * B * k, "cand_idx", I32)
+    _numel_ok(doc_base, world, "doc_base", I32)
+    _numel_ok(idx, B * k, "idx", I32)
+    _numel_ok(top_scores, B * k, "top_scores", F32)
     _check("msa_topk_merge_shards", lib().msa_topk_merge_shards(
         B, world, k, _ptr(cand_scores), _ptr(cand_idx), _ptr(doc_base), _ptr(idx),
         _ptr(top_scores), _stream(stream)))
 
 
 def msa_topk_docs(B, n_docs, k, scores, idx, top_scores, ws, ws_bytes, stream=None):
-    _numel_ok(scores, B * n_docs, "scores")
-    _numel_ok(idx, B * k, "idx")
+    _numel_ok(scores, B * n_docs, "scores", F32)
+    _numel_ok(idx, B * k, "idx", I32)
+    _numel_ok(top_scores, B * k, "top_scores", F32)
     _check("msa_topk_docs", lib().msa_topk_docs(
         B, n_docs, k, _ptr(scores), _ptr(idx), _ptr(top_scores), _ptr(ws), ws_bytes,
         _stream(stream)))
@@ -273,9 +296,11 @@ def msa_topk_docs(B, n_docs, k, scores, idx, top_scores, ws, ws_bytes, stream=No
 
 def msa_gather_kv(dt, B, k, H, D, idx, chunk_offsets, n_docs, k_bar, v_bar, m_cap, k_mem,
                   v_mem, mem_len, stream=None):
-    _numel_ok(idx, B * k, "idx")
-    _numel_ok(k_mem, B * m_cap * H * D, "k_mem")
-    _numel_ok(v_mem, B * m_cap * H * D, "v_mem")
+    _numel_ok(idx, B * k, "idx", I32)
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
+    _numel_ok(k_mem, B * m_cap * H * D, "k_mem", _es(dt))
+    _numel_ok(v_mem, B * m_cap * H * D, "v_mem", _es(dt))
+    _numel_ok(mem_len, B, "mem_len", I32)
     _check("msa_gather_kv", lib().msa_gather_kv(
         dt, B, k, H, D, _ptr(idx), _ptr(chunk_offsets), n_docs, _ptr(k_bar), _ptr(v_bar),
         m_cap, _ptr(k_mem), _ptr(v_mem), _ptr(mem_len), _stream(stream)))
@@ -287,10 +312,13 @@ def msa_sparse_attn_workspace_size(dt, B, T, T_loc, Hq, H, D, m_cap) -> int:
 
 def msa_sparse_attn(dt, B, T, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len, m_cap, k_loc, v_loc,
                     pos0, rope_base, scale, out, ws, ws_bytes, stream=None):
-    _numel_ok(q, B * T * Hq * D, "q")
-    _numel_ok(k_loc, B * T_loc * H * D, "k_loc")
-    _numel_ok(v_loc, B * T_loc * H * D, "v_loc")
-    _numel_ok(out, B * T * Hq * D, "out")
+    _numel_ok(q, B * T * Hq * D, "q", _es(dt))
+    _numel_ok(k_mem, B * m_cap * H * D, "k_mem", _es(dt))
+    _numel_ok(v_mem, B * m_cap * H * D, "v_mem", _es(dt))
+    _numel_ok(mem_len, B, "mem_len", I32)
+    _numel_ok(k_loc, B * T_loc * H * D, "k_loc", _es(dt))
+    _numel_ok(v_loc, B * T_loc * H * D, "v_loc", _es(dt))
+    _numel_ok(out, B * T * Hq * D, "out", _es(dt))
     _check("msa_sparse_attn", lib().msa_sparse_attn(
         dt, B, T, T_loc, Hq, H, D, _ptr(q), _ptr(k_mem), _ptr(v_mem), _ptr(mem_len), m_cap,
         _ptr(k_loc), _ptr(v_loc), pos0, rope_base, scale, _ptr(out), _ptr(ws), ws_bytes,
@@ -304,13 +332,15 @@ def msa_sparse_attn_fused_workspace_size(dt, B, T, T_loc, Hq, H, D, k, m_cap) ->
 def msa_sparse_attn_fused(dt, B, T, T_loc, Hq, H, D, q, idx, k, chunk_offsets, n_docs, k_bar,
                           v_bar, n_chunks, m_cap, k_loc, v_loc, pos0, rope_base, scale, out,
                           mem_len, ws, ws_bytes, stream=None):
-    _numel_ok(q, B * T * Hq * D, "q")
-    _numel_ok(idx, B * k, "idx")
-    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets")
-    _numel_ok(k_loc, B * T_loc * H * D, "k_loc")
-    _numel_ok(v_loc, B * T_loc * H * D, "v_loc")
-    _numel_ok(out, B * T * Hq * D, "out")
-    _numel_ok(mem_len, B, "mem_len")
+    _numel_ok(q, B * T * Hq * D, "q", _es(dt))
+    _numel_ok(idx, B * k, "idx", I32)
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
+    _numel_ok(k_bar, n_chunks * H * D, "k_bar", _es(dt))
+    _numel_ok(v_bar, n_chunks * H * D, "v_bar", _es(dt))
+    _numel_ok(k_loc, B * T_loc * H * D, "k_loc", _es(dt))
+    _numel_ok(v_loc, B * T_loc * H * D, "v_loc", _es(dt))
+    _numel_ok(out, B * T * Hq * D, "out", _es(dt))
+    _numel_ok(mem_len, B, "mem_len", I32)
     _check("msa_sparse_attn_fused", lib().msa_sparse_attn_fused(
         dt, B, T, T_loc, Hq, H, D, _ptr(q), _ptr(idx), k, _ptr(chunk_offsets), n_docs,
         _ptr(k_bar), _ptr(v_bar), n_chunks, m_cap, _ptr(k_loc), _ptr(v_loc), pos0, rope_base,
@@ -323,11 +353,12 @@ def msa_route_backward_workspace_size(dt, B, T, H, D, n_chunks, n_docs) -> int:
 
 def msa_route_backward(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_docs, d_doc,
                        dq_r, dkr_bar, ws=None, ws_bytes=0, stream=None):
-    _numel_ok(q_r, B * T * H * D, "q_r")
-    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar")
-    _numel_ok(d_doc, B * n_docs, "d_doc")
-    _numel_ok(dq_r, B * T * H * D, "dq_r")
-    _numel_ok(dkr_bar, n_chunks * H * D, "dkr_bar")
+    _numel_ok(q_r, B * T * H * D, "q_r", _es(dt))
+    _numel_ok(kr_bar, n_chunks * H * D, "kr_bar", _es(dt))
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
+    _numel_ok(d_doc, B * n_docs, "d_doc", F32)
+    _numel_ok(dq_r, B * T * H * D, "dq_r", F32)
+    _numel_ok(dkr_bar, n_chunks * H * D, "dkr_bar", F32)
     _check("msa_route_backward", lib().msa_route_backward(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(d_doc), _ptr(dq_r), _ptr(dkr_bar), _ptr(ws), ws_bytes, _stream(stream)))
@@ -337,9 +368,11 @@ def msa_encode_pool_backward(L, n_tok, n_docs, H, D, dk_bar, dv_bar, dkr_bar, to
                              chunk_offsets, n_chunks, rope_base, dk_tok, dv_tok, dkr_tok,
                              stream=None):
     for t, nm in ((dk_bar, "dk_bar"), (dv_bar, "dv_bar"), (dkr_bar, "dkr_bar")):
-        _numel_ok(t, L * n_chunks * H * D, nm)
+        _numel_ok(t, L * n_chunks * H * D, nm, F32)
     for t, nm in ((dk_tok, "dk_tok"), (dv_tok, "dv_tok"), (dkr_tok, "dkr_tok")):
-        _numel_ok(t, L * n_tok * H * D, nm)
+        _numel_ok(t, L * n_tok * H * D, nm, F32)
+    _numel_ok(tok_offsets, n_docs + 1, "tok_offsets", I64)
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
     _check("msa_encode_pool_backward", lib().msa_encode_pool_backward(
         L, n_tok, n_docs, H, D, _ptr(dk_bar), _ptr(dv_bar), _ptr(dkr_bar), _ptr(tok_offsets),
         _ptr(chunk_offsets), n_chunks, rope_base, _ptr(dk_tok), _ptr(dv_tok), _ptr(dkr_tok),

@@ -129,3 +129,74 @@ def test_input_checks_exist_only_in_the_debug_build(debug_lib):
     assert checks(build.LIB_DEBUG) == {"debug_check_offsets", "debug_check_mem_len",
                                        "debug_finish"}
     assert checks(build.LIB) == set()
+
+
+class _StubLib:
+    """Stands in for libmsa.so: records which entry points were reached."""
+
+    def __init__(self):
+        self.called = []
+
+    def __getattr__(self, name):
+        def fn(*args):
+            self.called.append(name)
+            return 0
+        return fn
+
+
+@pytest.fixture
+def stub(monkeypatch):
+    s = _StubLib()
+    monkeypatch.setattr(msa, "lib", lambda *a, **k: s)
+    return s
+
+
+def test_binding_rejects_narrower_element_types(stub):
+    """A tensor of a narrower type than the call reads (bf16 where fp32 is
+    declared, int32 offsets where int64 are read) would be overrun by the
+    kernel: the binding refuses it before the library is called."""
+    import torch
+    f32, bf16 = torch.float32, torch.bfloat16
+    i32, i64 = torch.int32, torch.int64
+    with pytest.raises(ValueError, match="bytes"):
+        msa.msa_topk_docs(1, 10, 2, torch.zeros(10, dtype=bf16), torch.zeros(2, dtype=i32),
+                          None, None, 0, stream=0)
+    with pytest.raises(ValueError, match="bytes"):
+        msa.msa_chunk_offsets(3, torch.zeros(4, dtype=i32), 64, torch.zeros(4, dtype=i64),
+                              stream=0)
+    B, T, T_loc, Hq, H, D, m_cap = 1, 2, 2, 4, 2, 64, 3
+    ok = dict(q=torch.zeros(B * T * Hq * D, dtype=f32),
+              k_mem=torch.zeros(B * m_cap * H * D, dtype=f32),
+              v_mem=torch.zeros(B * m_cap * H * D, dtype=f32),
+              mem_len=torch.zeros(B, dtype=i32),
+              k_loc=torch.zeros(B * T_loc * H * D, dtype=f32),
+              v_loc=torch.zeros(B * T_loc * H * D, dtype=f32),
+              out=torch.zeros(B * T * Hq * D, dtype=f32))
+
+    def attn(**kw):
+        a = {**ok, **kw}
+        msa.msa_sparse_attn(msa.MSA_F32, B, T, T_loc, Hq, H, D, a["q"], a["k_mem"], a["v_mem"],
+                            a["mem_len"], m_cap, a["k_loc"], a["v_loc"], 2, 10000.0, 0.0,
+                            a["out"], None, 0, stream=0)
+
+    attn()  # matching types reach the library
+    assert stub.called == ["msa_sparse_attn"]
+    for name in ("q", "k_mem", "v_mem", "k_loc", "v_loc", "out"):
+        with pytest.raises(ValueError, match=name):
+            attn(**{name: ok[name].to(bf16)})
+    with pytest.raises(ValueError, match="mem_len"):
+        attn(mem_len=torch.zeros(B, dtype=torch.int16))
+    assert stub.called == ["msa_sparse_attn"]  # no refused call reached it
+
+
+def test_binding_rejects_short_offsets_and_outputs(stub):
+    import torch
+    with pytest.raises(ValueError, match="chunk_offsets"):
+        msa.msa_route_scores(msa.MSA_BF16, 1, 1, 8, 128, torch.zeros(1024, dtype=torch.bfloat16),
+                             torch.zeros(10 * 1024, dtype=torch.bfloat16), 10,
+                             torch.zeros(3, dtype=torch.int64), 3,
+                             torch.zeros(3), None, None, 0, stream=0)
+    with pytest.raises(ValueError, match="top_scores"):
+        msa.msa_topk_docs(2, 10, 4, torch.zeros(20), torch.zeros(8, dtype=torch.int32),
+                          torch.zeros(7), None, 0, stream=0)
+    assert stub.called == []
