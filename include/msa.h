@@ -368,9 +368,14 @@ int msa_encode_pool_backward(int L, int64_t n_tok, int n_docs, int H, int D,
  *   mem_len      [B] int32, written when not NULL: memory rows used.
  *   q, k_loc, v_loc, pos0, rope_base, scale, out: as msa_sparse_attn.
  * Each document's rows are read in 8-row groups; the rows of its last group
- * past its end are bank rows masked out (the bank must hold finite values).
- * Supported (else MSA_ERR_UNSUPPORTED): bf16, D = 128, T = 1 (decode),
- * Hq/H in {1,2,4,8,16}, 1 <= k <= min(n_docs, 1024), n_chunks < 2^31.
+ * past its end are other bank rows, masked out of the softmax and with their
+ * V zeroed, so whatever they hold (NaN included) does not reach the output.
+ * Supported (else MSA_ERR_UNSUPPORTED): bf16, D = 128, Hq/H in
+ * {1,2,4,8,16}, 1 <= k <= min(n_docs, 1024), n_chunks < 2^31, and either
+ *   T = 1 (decode, on the tensor-core decode kernel), or
+ *   2 <= T <= T_loc (prefill, on the tensor-core prefill kernel), with
+ *   B <= 65535 and B*T, B*T_loc and B*8*(ceil(m_cap/8) + k) each <= 2^30
+ *   (a query's memory is padded to whole 8-row groups per document).
  * The workspace size is 0 for unsupported shapes. */
 size_t msa_sparse_attn_fused_workspace_size(msa_dtype dt, int B, int T, int T_loc, int Hq,
                                             int H, int D, int k, int m_cap);

@@ -138,7 +138,8 @@ struct Cur {
 // in rank order -- instead of a gathered [B][m_cap] buffer; tm_km / tm_vm
 // then map the bank with 8-row boxes (one 128B-swizzle atom each), and a
 // memory tile is 16 groups.  Rows past a document's end within its last
-// group are real bank rows, masked out.
+// group are other bank rows: masked out, and their V zeroed in shared memory
+// by the rotators (as the rows past mem_len of a gathered memory tile).
 template <int G, bool kFused>
 __global__ void __launch_bounds__(kTThreads, 1)
 attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
@@ -560,7 +561,28 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           *p1 = Vec16<__nv_bfloat16>::pack(y1);
           *p2 = Vec16<__nv_bfloat16>::pack(y2);
         }
-      } else if (!kFused && n_valid < kTK) {
+      } else if (kFused) {
+        // rows of a group past its document's end (and the repeated groups
+        // past the query's last one) are other bank rows: zero their V as
+        // below, so a non-finite bank value cannot turn 0 * V into NaN
+        const int g0 = tile_key0(c) / 8, ng = c.M / 8;
+        const int2* gq = groups + (int64_t)c.b * max_groups;
+        bool partial = false;
+        for (int gi = 0; gi < kTK / 8; ++gi)
+          partial |= g0 + gi >= ng || gq[g0 + gi].y < 8;
+        if (partial) {
+          if (u >= kTStages) wait_or_abort(&aux.vfree[st], ((u / kTStages) - 1) & 1);
+          wait_or_abort(&aux.vfull[st], (u / kTStages) & 1);
+          unsigned char* vt = kt + kTileBytes;
+          for (int e = rt; e < kTK * 16; e += 32 * kRotWarps) {
+            const int rr = e / 16, cc = e % 16, grp = g0 + rr / 8;
+            const int nv = grp < ng ? gq[grp].y : 0;
+            if ((rr & 7) >= nv)
+              *reinterpret_cast<uint4*>(vt + (cc >> 3) * kBlk + rr * 128 + ((cc & 7) << 4)) =
+                  make_uint4(0, 0, 0, 0);
+          }
+        }
+      } else if (n_valid < kTK) {
         // memory rows past mem_len hold whatever the caller's buffer holds:
         // zero their V (once it has landed) so that 0 * V stays 0 in P V,
         // which is issued after S(u) and so after this tile's kready.  The V

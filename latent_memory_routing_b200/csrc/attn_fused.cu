@@ -13,8 +13,9 @@
 // 128B-swizzle atom of a 64-element K block, which a TMA box of 8 rows
 // writes correctly at any 8-row-aligned place of a tile -- and a query's
 // memory is the concatenation of its documents' groups in rank order.  The
-// rows of a document's last group that lie past its end are real bank rows
-// (finite) that the attention masks out; memory order does not change
+// rows of a document's last group that lie past its end are other bank rows:
+// the attention masks their scores and zeroes their V in shared memory, so
+// they change nothing whatever they hold; memory order does not change
 // attention, so the padding changes nothing but the work.
 // assemble_groups_kernel (one CTA per query) writes the group list; the
 // attention kernels load memory tiles group by group.

@@ -38,7 +38,8 @@
 //       accumulates in TMEM; a row rescales O and its sum only when its
 //       maximum grows by more than 2^8 (then p <= 256 meanwhile), which after
 //       the first tiles is rare.  In the last memory tile, warpgroup 1 zeroes
-//       the V rows past mem_len in shared memory before P V reads them.
+//       the V rows past mem_len in shared memory before P V reads them (in
+//       the fused form, the rows of any group past its document's end).
 //   * Every mbarrier wait is bounded; a timeout records MSA_ERR_TIMEOUT and
 //     all roles finish their loops without waiting.
 #include <cudaTypedefs.h>
@@ -135,7 +136,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // of 8-row groups (first bank row, rows of the group inside its document)
 // in rank order; tm_km / tm_vm map the bank with 8-row boxes (one
 // 128B-swizzle atom), a memory tile is 16 groups, and `mem_len` holds the
-// group count.  Rows past a document's end are finite bank rows, masked.
+// group count.  Rows past a document's end are other bank rows: masked, and
+// their V zeroed in shared memory before P V reads it.
 template <int D, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_km,
@@ -358,10 +360,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::tmem_ld_wait();
       // keys a row may not see read as -inf (also hides whatever S holds
       // there: rows past mem_len, keys past the causal limit)
+      bool all8 = true;  // fused memory tile: every row belongs to its document
       if (kFused && mem) {
         // valid rows of each of the tile's 16 groups (0 past the last
         // group), read as the columns reach each group
-        bool all8 = true;
         for (int gi = 0; gi < kKeys / 8; ++gi) {
           const int grp = key0 / 8 + gi;
           all8 &= grp < M / 8 && gq[grp].y == 8;
@@ -444,6 +446,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // caller's buffer holds there; zero their V so that 0 * V stays 0
         const int vrow = quad * 32 + lane;  // one V row per thread of group 0
         if (qt == 0 && vrow >= M - key0) {
+          unsigned char* vp = sKV + (j % kStages) * K::STAGE + K::K_BYTES + vrow * 128;
+#pragma unroll
+          for (int kb = 0; kb < K::KB; ++kb)
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<uint4*>(vp + kb * (kKeys * 128) + q * 16) = make_uint4(0, 0, 0, 0);
+        }
+        tc::fence_proxy_async_smem();
+      }
+      if (kFused && mem && !all8) {
+        // rows of a group past its document's end (and the repeated groups
+        // past the query's last one) are other bank rows: their p is 0, and
+        // their V is zeroed so that a non-finite bank value cannot turn
+        // 0 * V into NaN
+        const int vrow = quad * 32 + lane;  // one V row per thread of group 0
+        const int grp = key0 / 8 + vrow / 8;
+        const int nv = grp < M / 8 ? gq[grp].y : 0;
+        if (qt == 0 && (vrow & 7) >= nv) {
           unsigned char* vp = sKV + (j % kStages) * K::STAGE + K::K_BYTES + vrow * 128;
 #pragma unroll
           for (int kb = 0; kb < K::KB; ++kb)

@@ -41,7 +41,12 @@ int scratch_ptr(void** out) {
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
     rc = note_cuda(cudaGetSymbolAddress(&p, g_route_scratch));
-    if (rc) return rc;
+    if (rc) {
+      // recorded for msa_last_cuda_error(); cleared from the runtime so that
+      // the next call's launch check does not report it again
+      cudaGetLastError();
+      return rc;
+    }
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];

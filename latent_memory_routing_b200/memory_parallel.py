@@ -61,17 +61,51 @@ def local_offsets(chunk_offsets, plan, rank: int):
     return off[d0:d1 + 1] - c0
 
 
-def exchange_candidates(scores, ids, group=None):
+def _torch_stream(stream):
+    """A torch stream object for a stream argument of the binding (None,
+    a torch.cuda.Stream or a raw cudaStream_t handle)."""
+    import torch
+    if stream is None or isinstance(stream, torch.cuda.Stream):
+        return stream
+    return torch.cuda.ExternalStream(int(stream))
+
+
+def exchange_candidates(scores, ids, group=None, stream=None):
     """All-gathers every rank's ``[B][k]`` local candidates (scores float32,
     local ids int32) into ``[world][B][k]`` tensors on the same device: one
-    collective per tensor, every rank in the same order."""
+    collective per tensor, every rank in the same order.
+
+    Device tensors: with NCCL the all-gathers are ordered after the work
+    queued on ``stream`` (torch's current stream if None) and the results are
+    ready for work queued on it afterwards.  With gloo (a CPU group) device
+    candidates are staged through pinned host memory -- the copy to the host
+    waits for ``stream`` -- and copied back on it."""
+    import contextlib
+
     import torch
     import torch.distributed as dist
     world = dist.get_world_size(group)
-    out_s = torch.empty((world,) + tuple(scores.shape), dtype=scores.dtype, device=scores.device)
-    out_i = torch.empty((world,) + tuple(ids.shape), dtype=ids.dtype, device=ids.device)
-    dist.all_gather(list(out_s.unbind(0)), scores.contiguous(), group=group)
-    dist.all_gather(list(out_i.unbind(0)), ids.contiguous(), group=group)
+    ts = _torch_stream(stream) if scores.is_cuda else None
+    ctx = torch.cuda.stream(ts) if ts is not None else contextlib.nullcontext()
+    with ctx:
+        out_s = torch.empty((world,) + tuple(scores.shape), dtype=scores.dtype,
+                            device=scores.device)
+        out_i = torch.empty((world,) + tuple(ids.shape), dtype=ids.dtype, device=ids.device)
+        staged = scores.is_cuda and dist.get_backend(group) == "gloo"
+        if staged:
+            hs = torch.empty(scores.shape, dtype=scores.dtype, pin_memory=True)
+            hi = torch.empty(ids.shape, dtype=ids.dtype, pin_memory=True)
+            hs.copy_(scores)  # synchronous: waits for the stream's top-k
+            hi.copy_(ids)
+            gs = torch.empty(out_s.shape, dtype=scores.dtype)
+            gi = torch.empty(out_i.shape, dtype=ids.dtype)
+            dist.all_gather(list(gs.unbind(0)), hs, group=group)
+            dist.all_gather(list(gi.unbind(0)), hi, group=group)
+            out_s.copy_(gs)
+            out_i.copy_(gi)
+        else:
+            dist.all_gather(list(out_s.unbind(0)), scores.contiguous(), group=group)
+            dist.all_gather(list(out_i.unbind(0)), ids.contiguous(), group=group)
     return out_s, out_i
 
 
@@ -115,7 +149,7 @@ class MemoryParallelRouter:
     def __call__(self, q_r, stream=None):
         self.router(q_r, self.kr, self.coff, self.n_local, self.doc_scores, None, stream)
         topk_docs(self.doc_scores, self.k, self.loc_idx, self.loc_top, self.topk_ws, stream)
-        cs, ci = exchange_candidates(self.loc_top, self.loc_idx, self.group)
+        cs, ci = exchange_candidates(self.loc_top, self.loc_idx, self.group, stream)
         merge_shards(cs, ci, self.doc_base, self.k, self.idx, self.top, stream)
         return self.idx, self.top
 

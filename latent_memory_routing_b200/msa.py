@@ -144,28 +144,66 @@ def _check(name: str, rc: int):
         raise MsaError(name, rc, detail)
 
 
-_ESIZE = {MSA_F32: 4, MSA_BF16: 2}
-F32, I32, I64 = 4, 4, 8  # element sizes of the fixed-type arguments
+# Element type of each tensor argument: the call's `dt` for floating-point
+# tensors, and these fixed types for the rest.
+F32, I32, I64 = "f32", "i32", "i64"
 
 
-def _es(dt) -> int | None:
-    """Element size of a `dt`-typed tensor (None for an unknown dt, which the
-    library itself rejects)."""
-    return _ESIZE.get(dt)
+def _torch_dtype(kind):
+    import torch
+    return {MSA_F32: torch.float32, MSA_BF16: torch.bfloat16, F32: torch.float32,
+            I32: torch.int32, I64: torch.int64}.get(kind)
 
 
-def _numel_ok(t, n, what, esize=None):
-    """Checks a tensor argument: contiguous, at least n elements and, given
-    the element size the call uses, at least n * esize bytes (a tensor of a
-    narrower type than the call reads would be overrun)."""
-    if t is not None and not isinstance(t, int):
-        if not t.is_contiguous():
-            raise ValueError(f"{what} must be contiguous")
-        if t.numel() < n:
-            raise ValueError(f"{what} holds {t.numel()} elements, needs {n}")
-        if esize and t.numel() * t.element_size() < n * esize:
-            raise ValueError(f"{what} holds {t.numel() * t.element_size()} bytes, needs "
-                             f"{n * esize} ({n} elements of {esize} bytes)")
+def _es(dt):
+    """The element type of a `dt`-typed tensor (None for an unknown dt, which
+    the library itself rejects)."""
+    return dt if dt in (MSA_F32, MSA_BF16) else None
+
+
+def _device_ok(t, host_ok: bool) -> bool:
+    """A tensor the kernels may read: on the current CUDA device, or (where
+    the call reads a tiered bank over the host link) in pinned host memory."""
+    import torch
+    if t.is_cuda:
+        return t.device.index == torch.cuda.current_device()
+    return host_ok and t.is_pinned()
+
+
+def _numel_ok(t, n, what, kind=None, host_ok=False):
+    """Checks a tensor argument before its address goes to the library:
+    contiguous, of exactly the element type the call reads (`kind`: a dt code
+    or F32/I32/I64), holding at least n elements, and on the current device
+    (pinned host memory only where ``host_ok``).  Raw integer addresses are
+    the caller's responsibility and pass unchecked."""
+    if t is None or isinstance(t, int):
+        return
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    want = _torch_dtype(kind)
+    if want is not None and t.dtype != want:
+        raise ValueError(f"{what} is {t.dtype}, the call reads {want}")
+    if t.numel() < n:
+        raise ValueError(f"{what} holds {t.numel()} elements, needs {n}")
+    if not _device_ok(t, host_ok):
+        where = "the current CUDA device or pinned host memory" if host_ok else \
+            "the current CUDA device"
+        raise ValueError(f"{what} is on {t.device}{' (pageable)' if not t.is_cuda else ''}; "
+                         f"the kernels read it from {where}")
+
+
+def _ws_ok(ws, ws_bytes):
+    """A workspace tensor must lie on the current device and hold at least
+    the ws_bytes the library is told it may use."""
+    if ws is None or isinstance(ws, int):
+        return
+    if not ws.is_contiguous():
+        raise ValueError("ws must be contiguous")
+    if ws.numel() * ws.element_size() < ws_bytes:
+        raise ValueError(f"ws holds {ws.numel() * ws.element_size()} bytes, "
+                         f"ws_bytes says {ws_bytes}")
+    if not _device_ok(ws, False):
+        raise ValueError(f"ws is on {ws.device}; it must be on the current CUDA device")
 
 
 # ---------------------------------------------------------------- entry points
@@ -227,6 +265,7 @@ def msa_route_scores(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_doc
     _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
     _numel_ok(doc_scores, B * n_docs, "doc_scores", F32)
     _numel_ok(chunk_scores, B * n_chunks, "chunk_scores", F32)
+    _ws_ok(ws, ws_bytes)
     _check("msa_route_scores", lib().msa_route_scores(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws_bytes, _stream(stream)))
@@ -246,6 +285,7 @@ def msa_route_scores_prepared(dt, B, T, H, D, q_r, kr_hat, n_chunks, chunk_offse
     _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
     _numel_ok(doc_scores, B * n_docs, "doc_scores", F32)
     _numel_ok(chunk_scores, B * n_chunks, "chunk_scores", F32)
+    _ws_ok(ws, ws_bytes)
     _check("msa_route_scores_prepared", lib().msa_route_scores_prepared(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_hat), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(doc_scores), _ptr(chunk_scores), _ptr(ws), ws_bytes, _stream(stream)))
@@ -289,6 +329,7 @@ def msa_topk_docs(B, n_docs, k, scores, idx, top_scores, ws, ws_bytes, stream=No
     _numel_ok(scores, B * n_docs, "scores", F32)
     _numel_ok(idx, B * k, "idx", I32)
     _numel_ok(top_scores, B * k, "top_scores", F32)
+    _ws_ok(ws, ws_bytes)
     _check("msa_topk_docs", lib().msa_topk_docs(
         B, n_docs, k, _ptr(scores), _ptr(idx), _ptr(top_scores), _ptr(ws), ws_bytes,
         _stream(stream)))
@@ -298,6 +339,10 @@ def msa_gather_kv(dt, B, k, H, D, idx, chunk_offsets, n_docs, k_bar, v_bar, m_ca
                   v_mem, mem_len, stream=None):
     _numel_ok(idx, B * k, "idx", I32)
     _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
+    # the bank's row count sits on the device (chunk_offsets[n_docs]); its
+    # type and placement are checked here: device or pinned host tier
+    for t, what in ((k_bar, "k_bar"), (v_bar, "v_bar")):
+        _numel_ok(t, 0, what, _es(dt), host_ok=True)
     _numel_ok(k_mem, B * m_cap * H * D, "k_mem", _es(dt))
     _numel_ok(v_mem, B * m_cap * H * D, "v_mem", _es(dt))
     _numel_ok(mem_len, B, "mem_len", I32)
@@ -319,6 +364,7 @@ def msa_sparse_attn(dt, B, T, T_loc, Hq, H, D, q, k_mem, v_mem, mem_len, m_cap, 
     _numel_ok(k_loc, B * T_loc * H * D, "k_loc", _es(dt))
     _numel_ok(v_loc, B * T_loc * H * D, "v_loc", _es(dt))
     _numel_ok(out, B * T * Hq * D, "out", _es(dt))
+    _ws_ok(ws, ws_bytes)
     _check("msa_sparse_attn", lib().msa_sparse_attn(
         dt, B, T, T_loc, Hq, H, D, _ptr(q), _ptr(k_mem), _ptr(v_mem), _ptr(mem_len), m_cap,
         _ptr(k_loc), _ptr(v_loc), pos0, rope_base, scale, _ptr(out), _ptr(ws), ws_bytes,
@@ -335,12 +381,13 @@ def msa_sparse_attn_fused(dt, B, T, T_loc, Hq, H, D, q, idx, k, chunk_offsets, n
     _numel_ok(q, B * T * Hq * D, "q", _es(dt))
     _numel_ok(idx, B * k, "idx", I32)
     _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
-    _numel_ok(k_bar, n_chunks * H * D, "k_bar", _es(dt))
-    _numel_ok(v_bar, n_chunks * H * D, "v_bar", _es(dt))
+    _numel_ok(k_bar, n_chunks * H * D, "k_bar", _es(dt), host_ok=True)
+    _numel_ok(v_bar, n_chunks * H * D, "v_bar", _es(dt), host_ok=True)
     _numel_ok(k_loc, B * T_loc * H * D, "k_loc", _es(dt))
     _numel_ok(v_loc, B * T_loc * H * D, "v_loc", _es(dt))
     _numel_ok(out, B * T * Hq * D, "out", _es(dt))
     _numel_ok(mem_len, B, "mem_len", I32)
+    _ws_ok(ws, ws_bytes)
     _check("msa_sparse_attn_fused", lib().msa_sparse_attn_fused(
         dt, B, T, T_loc, Hq, H, D, _ptr(q), _ptr(idx), k, _ptr(chunk_offsets), n_docs,
         _ptr(k_bar), _ptr(v_bar), n_chunks, m_cap, _ptr(k_loc), _ptr(v_loc), pos0, rope_base,
@@ -359,6 +406,7 @@ def msa_route_backward(dt, B, T, H, D, q_r, kr_bar, n_chunks, chunk_offsets, n_d
     _numel_ok(d_doc, B * n_docs, "d_doc", F32)
     _numel_ok(dq_r, B * T * H * D, "dq_r", F32)
     _numel_ok(dkr_bar, n_chunks * H * D, "dkr_bar", F32)
+    _ws_ok(ws, ws_bytes)
     _check("msa_route_backward", lib().msa_route_backward(
         dt, B, T, H, D, _ptr(q_r), _ptr(kr_bar), n_chunks, _ptr(chunk_offsets), n_docs,
         _ptr(d_doc), _ptr(dq_r), _ptr(dkr_bar), _ptr(ws), ws_bytes, _stream(stream)))

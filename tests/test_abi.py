@@ -146,24 +146,52 @@ class _StubLib:
 
 @pytest.fixture
 def stub(monkeypatch):
+    """The stubbed library, with CPU tensors standing in for device tensors
+    (the placement check is exercised on its own below)."""
+    s = _StubLib()
+    monkeypatch.setattr(msa, "lib", lambda *a, **k: s)
+    monkeypatch.setattr(msa, "_device_ok", lambda t, host_ok: True)
+    return s
+
+
+@pytest.fixture
+def stub_strict(monkeypatch):
+    """The stubbed library with the binding's real placement check: on a
+    machine without a GPU every tensor is a host tensor."""
     s = _StubLib()
     monkeypatch.setattr(msa, "lib", lambda *a, **k: s)
     return s
 
 
-def test_binding_rejects_narrower_element_types(stub):
-    """A tensor of a narrower type than the call reads (bf16 where fp32 is
-    declared, int32 offsets where int64 are read) would be overrun by the
-    kernel: the binding refuses it before the library is called."""
+def test_binding_rejects_other_element_types(stub):
+    """A tensor of another type than the call reads would be misread by the
+    kernel: a narrower one (bf16 where fp32 is declared, int32 offsets where
+    int64 are read) overrun, a wider one (fp32 q in a bf16 call, int64 ids
+    where int32 are read) reinterpreted.  The binding refuses both before
+    the library is called."""
     import torch
     f32, bf16 = torch.float32, torch.bfloat16
     i32, i64 = torch.int32, torch.int64
-    with pytest.raises(ValueError, match="bytes"):
+    with pytest.raises(ValueError, match="scores is torch.bfloat16"):
         msa.msa_topk_docs(1, 10, 2, torch.zeros(10, dtype=bf16), torch.zeros(2, dtype=i32),
                           None, None, 0, stream=0)
-    with pytest.raises(ValueError, match="bytes"):
+    with pytest.raises(ValueError, match="idx is torch.int64"):
+        msa.msa_topk_docs(1, 10, 2, torch.zeros(10, dtype=f32), torch.zeros(2, dtype=i64),
+                          None, None, 0, stream=0)
+    with pytest.raises(ValueError, match="tok_offsets is torch.int32"):
         msa.msa_chunk_offsets(3, torch.zeros(4, dtype=i32), 64, torch.zeros(4, dtype=i64),
                               stream=0)
+    with pytest.raises(ValueError, match="q_r is torch.float32"):
+        msa.msa_route_scores(msa.MSA_BF16, 1, 1, 8, 128, torch.zeros(1024, dtype=f32),
+                             torch.zeros(10 * 1024, dtype=bf16), 10,
+                             torch.zeros(4, dtype=i64), 3, torch.zeros(3), None, None, 0,
+                             stream=0)
+    with pytest.raises(ValueError, match="mem_len is torch.int64"):
+        msa.msa_gather_kv(msa.MSA_BF16, 1, 2, 8, 128, torch.zeros(2, dtype=i32),
+                          torch.zeros(4, dtype=i64), 3, torch.zeros(1024, dtype=bf16),
+                          torch.zeros(1024, dtype=bf16), 4, torch.zeros(4096, dtype=bf16),
+                          torch.zeros(4096, dtype=bf16), torch.zeros(1, dtype=i64), stream=0)
+    assert stub.called == []
     B, T, T_loc, Hq, H, D, m_cap = 1, 2, 2, 4, 2, 64, 3
     ok = dict(q=torch.zeros(B * T * Hq * D, dtype=f32),
               k_mem=torch.zeros(B * m_cap * H * D, dtype=f32),
@@ -186,7 +214,49 @@ def test_binding_rejects_narrower_element_types(stub):
             attn(**{name: ok[name].to(bf16)})
     with pytest.raises(ValueError, match="mem_len"):
         attn(mem_len=torch.zeros(B, dtype=torch.int16))
+    with pytest.raises(ValueError, match="mem_len"):
+        attn(mem_len=torch.zeros(B, dtype=torch.int64))
     assert stub.called == ["msa_sparse_attn"]  # no refused call reached it
+
+
+def test_binding_refuses_a_workspace_smaller_than_ws_bytes(stub):
+    """The library trusts ws_bytes: a tensor holding fewer bytes would be
+    written past its end, so the binding compares the two first."""
+    import torch
+    q = torch.zeros(1024, dtype=torch.bfloat16)
+    kr = torch.zeros(10 * 1024, dtype=torch.bfloat16)
+    coff = torch.zeros(4, dtype=torch.int64)
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="ws holds 4096 bytes, ws_bytes says 8192"):
+        msa.msa_route_scores(msa.MSA_BF16, 1, 1, 8, 128, q, kr, 10, coff, 3, torch.zeros(3),
+                             None, ws, 8192, stream=0)
+    with pytest.raises(ValueError, match="ws holds"):
+        msa.msa_topk_docs(1, 10, 2, torch.zeros(10), torch.zeros(2, dtype=torch.int32), None,
+                          torch.zeros(16, dtype=torch.uint8), 17, stream=0)
+    assert stub.called == []
+    msa.msa_route_scores(msa.MSA_BF16, 1, 1, 8, 128, q, kr, 10, coff, 3, torch.zeros(3),
+                         None, ws, 4096, stream=0)
+    assert stub.called == ["msa_route_scores"]
+
+
+def test_binding_refuses_host_tensors(stub_strict):
+    """A pageable host tensor's address would reach the kernels as if it were
+    device memory: refused.  Pinned host memory is accepted only for the
+    bank of a tiered gather or fused attention (read over the host link);
+    on this machine no tensor is pinned, so the bank is refused too."""
+    import torch
+    with pytest.raises(ValueError, match="scores is on cpu .pageable.; the kernels read it "
+                                         "from the current CUDA device$"):
+        msa.msa_topk_docs(1, 10, 2, torch.zeros(10), torch.zeros(2, dtype=torch.int32), None,
+                          None, 0, stream=0)
+    with pytest.raises(ValueError, match="k_bar .* or pinned host memory"):
+        msa.msa_gather_kv(msa.MSA_BF16, 1, 2, 8, 128, 1 << 20, 1 << 20, 3,
+                          torch.zeros(1024, dtype=torch.bfloat16), 1 << 20, 4, 1 << 20,
+                          1 << 20, 1 << 20, stream=0)
+    assert stub_strict.called == []
+    # raw integer addresses are the caller's responsibility
+    msa.msa_topk_docs(1, 10, 2, 1 << 20, 1 << 20, None, None, 0, stream=0)
+    assert stub_strict.called == ["msa_topk_docs"]
 
 
 def test_binding_rejects_short_offsets_and_outputs(stub):
