@@ -12,8 +12,14 @@ synthetic bf16 tensors.
 ``value`` = chunks routed per second over the whole step (Gchunks/s), inputs
 resident in HBM.  ``e2e`` repeats the measurement through the same C-ABI
 calls with the per-step inputs copied from pinned host memory and the
-output / top-k read back inside the timed region.  N > 1 runs one
-independent replica per GPU (weak scaling, no data-path collective).
+output / top-k read back inside the timed region.  N > 1 runs Memory
+Parallel: the prepared routing bank is split by document range across the N
+GPUs, each rank routes the query over its own range and keeps its local
+top-16, the ranks all-gather their candidates over NCCL and merge them into
+the global top-16 (msa_topk_merge_shards), and the rank serving the query
+gathers from the content bank (replicated in every GPU's HBM) and attends.
+The total work is fixed (the 100M bank), so scaling is strong; ``value`` is
+the bank's chunks over the step time, max over ranks.
 ``--impl reference`` times the float64 oracle on the host cores on a bounded
 sample of the same workload.
 """
@@ -110,13 +116,18 @@ class Clocks:
                 "reasons": sorted(reasons)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, force_group: bool = False):
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+    if world == 1 and force_group:  # a process group of one, for the sharded step
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29531")
+        os.environ.setdefault("RANK", "0")
+        os.environ.setdefault("WORLD_SIZE", "1")
+    if world > 1 or force_group:
         import datetime
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -144,19 +155,13 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
-def build_workload(rank: int, n_docs: int = 100000):
-    import torch
-
+def build_workload(n_docs: int = 100000):
     from latent_memory_routing_b200 import pipeline, synth
     lengths = synth.bank_100m_lengths(n_docs)
     toff = synth.tok_offsets(lengths).cuda()
     coff = pipeline.chunk_offsets(toff)
     coff_h = coff.cpu()
     w = synth.bank_100m(coff_h, "cuda", n_docs=n_docs)
-    if rank:  # independent replica per rank: different query draws
-        g = torch.Generator(device="cuda").manual_seed(7919 * rank)
-        for key in ("q", "q_r", "k_loc", "v_loc"):
-            w[key] = synth.randn(tuple(w[key].shape), torch.bfloat16, "cuda", g)
     max_chunks = int((coff_h[1:] - coff_h[:-1]).max())
     m_cap = w["k"] * max_chunks
     # the routing bank is prepared once when the memory is built (unit rows)
@@ -165,6 +170,19 @@ def build_workload(rank: int, n_docs: int = 100000):
                           T_loc=w["T_loc"], Hq=w["Hq"], k=w["k"], m_cap=m_cap, pos0=w["pos0"],
                           prepared=True)
     return w, p, int(coff_h[-1])
+
+
+def step_config(world: int, C: int, n_docs: int, n_docs_arg: int, T: int, k: int,
+                m_cap: int) -> dict:
+    """The workload description both arms print for the same N."""
+    return {"workload": WORKLOAD if n_docs_arg == 100000 else
+            f"bank_100m recipe cut to {n_docs_arg} docs (profiling case)",
+            "n_chunks": C, "n_docs": n_docs, "global_batch": 1, "seq_len": T, "top_k": k,
+            "m_cap": m_cap,
+            "parallelism": (f"memory parallel x{world}: routing bank split by document range, "
+                            "candidates all-gathered over NCCL" if world > 1 else
+                            "one GPU holds the whole routing bank"),
+            "l2": "the 3.2 GB routing bank streams through the 126 MB L2 every step"}
 
 
 def timed_step(p, w, ev):
@@ -201,7 +219,7 @@ def run_libmsa(args, world, rank, local):
     from latent_memory_routing_b200 import msa, pipeline
     _b.build()
     msa.lib()
-    w, p, C = build_workload(rank, args.n_docs)
+    w, p, C = build_workload(args.n_docs)
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
     for _ in range(max(args.warmup, 3)):
@@ -236,7 +254,7 @@ def run_libmsa(args, world, rank, local):
     clk = clocks.stop()
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     ms_step = total_ms / args.steps
-    value = C * world / (ms_step * 1e-3) / 1e9
+    value = C / (ms_step * 1e-3) / 1e9
 
     # ---- end to end through host buffers: one graph per step that uploads
     # the step's inputs from pinned host memory (the attention's under the
@@ -312,14 +330,9 @@ def run_libmsa(args, world, rank, local):
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) pooled bank drawn at chunk level + planted needles)",
-        "config": {"workload": WORKLOAD if args.n_docs == 100000 else
-                   f"bank_100m recipe cut to {args.n_docs} docs (profiling case)",
-                   "n_chunks": C, "n_docs": p.n_docs, "global_batch": world,
-                   "seq_len": w["T"], "top_k": w["k"], "m_cap": p.m_cap,
-                   "parallelism": f"replica x{world}",
-                   "l2": "the 3.2 GB routing bank streams through the 126 MB L2 every step"},
+        "config": step_config(world, C, p.n_docs, args.n_docs, w["T"], w["k"], p.m_cap),
         # 256 query columns: 2*H*D*256 = 524,288 FLOP per 2,048-byte chunk row
         # = 256 FLOP/B, above the measured ridge (sustained 210, burst 249):
         # the scan is bound by the tensor pipe, with HBM just below it
@@ -343,7 +356,7 @@ def run_libmsa(args, world, rank, local):
                               "(ms_per_step) replays the same launches as one CUDA graph"},
         "route_gchunks_s": round(C / (route_ms * 1e-3) / 1e9, 4),
         "fused_step": {"ms_per_step": round(fused_ms, 4),
-                       "gchunks_s": round(C * world / (fused_ms * 1e-3) / 1e9, 4),
+                       "gchunks_s": round(C / (fused_ms * 1e-3) / 1e9, 4),
                        "note": "route -> top-k -> msa_sparse_attn_fused (memory read from the "
                                "bank, no gather), one CUDA graph",
                        "same_topk_as_step": fused_same_idx},
@@ -355,7 +368,7 @@ def run_libmsa(args, world, rank, local):
         "sparse_attn_tok_s": round(w["T"] / (seg[3] * 1e-3), 1),
         "sparse_attn_tflops": round(attn_flops / (seg[3] * 1e-3) / 1e12, 3),
         "sparse_attn_tc_frac": round(attn_flops / (seg[3] * 1e-3) / 1e12 / pk["bf16"], 5),
-        "e2e": {"value": round(C * world / (e2e_ms * 1e-3) / 1e9, 4), "unit": UNIT,
+        "e2e": {"value": round(C / (e2e_ms * 1e-3) / 1e9, 4), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "same_output_as_step": e2e_same,
                 "note": "one CUDA graph per step from pinned host inputs to pinned host "
@@ -373,13 +386,192 @@ def run_libmsa(args, world, rank, local):
         tiered = bench_tiered(w, p, args.steps, ms_step)
         del p, w
         torch.cuda.empty_cache()
-        line["workloads"] = {"encode_4l": bench_encode(max(args.steps // 4, 3), pk["hbm"]),
+        line["workloads"] = {"bank_1m": bench_bank_1m(args.steps, pk),
+                             "encode_4l": bench_encode(max(args.steps // 4, 3), pk["hbm"]),
                              "bank_10m_decode": bench_decode(args.steps, pk["hbm"]),
                              "bank_100m_tiered": tiered,
                              "backward_1m": bench_backward(max(args.steps // 4, 3), pk["hbm"]),
                              "prefill_sweep": bench_prefill_sweep(max(args.steps // 2, 3),
                                                                   pk["bf16"])}
     return line
+
+
+def run_memory_parallel(args, world, rank, local):
+    """The step as Memory Parallel over `world` GPUs (one process each).
+
+    Every rank draws the same seeded bank, keeps only the prepared routing
+    keys of its own document range (shard_plan) and the content bank K̄/V̄
+    (replicated: 6.6 GB of a GPU's 180 GB).  A step: route the query over the
+    rank's range, local top-16, one NCCL all-gather of the (score, id)
+    candidates, merge into the global top-16 (every rank gets the same), and
+    on the rank that serves the query (query_block) gather and attend.  No
+    peer memory is read; the only data-path collective is the all-gather.
+    """
+    import torch
+
+    from latent_memory_routing_b200 import build as _b
+    from latent_memory_routing_b200 import memory_parallel as mpar
+    from latent_memory_routing_b200 import msa, pipeline, synth
+    _b.build()
+    msa.lib()
+    lengths = synth.bank_100m_lengths(args.n_docs)
+    toff = synth.tok_offsets(lengths).cuda()
+    coff = pipeline.chunk_offsets(toff)
+    coff_h = coff.cpu()
+    w = synth.bank_100m(coff_h, "cuda", n_docs=args.n_docs)  # the same bytes on every rank
+    C = int(coff_h[-1])
+    n_docs, k, T = len(lengths), w["k"], w["T"]
+    plan = mpar.shard_plan(coff_h.numpy(), world, k)
+    d0, d1, c0, c1 = plan[rank]
+    shard = pipeline.prepare_bank(w["kr_bar"][c0:c1])  # this rank's routing keys only
+    del w["kr_bar"]
+    torch.cuda.empty_cache()
+    local_coff = torch.from_numpy(mpar.local_offsets(coff_h.numpy(), plan, rank)).cuda()
+    m_cap = k * int((coff_h[1:] - coff_h[:-1]).max())
+    mpp = mpar.MemoryParallelPipeline(shard, local_coff, coff, w["k_bar"], w["v_bar"], plan, rank,
+                                      B=1, T=T, T_loc=w["T_loc"], Hq=w["Hq"], k=k, m_cap=m_cap,
+                                      pos0=w["pos0"])
+    rt = mpp.route
+    b0, b1 = mpp.b0, mpp.b1
+    blk = {n: w[n][b0:b1].contiguous() for n in ("q", "k_loc", "v_loc")}
+
+    def step():
+        return mpp(w["q_r"], blk["q"], blk["k_loc"], blk["v_loc"])
+
+    def staged_step(ev):
+        """The same launches as step(), with events between the stages."""
+        ev[0].record()
+        rt.router(w["q_r"], rt.kr, rt.coff, rt.n_local, rt.doc_scores, None)
+        ev[1].record()
+        pipeline.topk_docs(rt.doc_scores, k, rt.loc_idx, rt.loc_top, rt.topk_ws)
+        ev[2].record()
+        cs, ci = mpar.exchange_candidates(rt.loc_top, rt.loc_idx, rt.group)
+        ev[3].record()
+        mpar.merge_shards(cs, ci, rt.doc_base, k, rt.idx, rt.top)
+        ev[4].record()
+        if b1 > b0:
+            pipeline.gather_kv(rt.idx[b0:b1], coff, w["k_bar"], w["v_bar"], m_cap, mpp.k_mem,
+                               mpp.v_mem, mpp.mem_len)
+        ev[5].record()
+        if b1 > b0:
+            mpp.attn(blk["q"], mpp.k_mem, mpp.v_mem, mpp.mem_len, blk["k_loc"], blk["v_loc"],
+                     mpp.pos0, mpp.rope_base, 0.0, mpp.out)
+        ev[6].record()
+
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    names = ["route", "topk_local", "exchange", "merge", "gather", "attn"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        staged_step(evs[i])
+    barrier(world)
+    seg = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(6)]
+
+    clocks = Clocks(local)
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    barrier(world)
+    clk = clocks.stop()
+    ms_step = max_over_ranks(t0.elapsed_time(t1), world) / args.steps
+
+    # end to end: the step's inputs uploaded from pinned host memory and the
+    # output and selection read back, inside the timed region
+    host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory().copy_(t.cpu())
+            for n, t in (("q_r", w["q_r"]), ("q", blk["q"]), ("k_loc", blk["k_loc"]),
+                         ("v_loc", blk["v_loc"]))}
+    dev = {n: torch.empty_like(t, device="cuda") for n, t in host.items()}
+    out_h = torch.empty((max(b1 - b0, 1),) + tuple(mpp.out.shape[1:]),
+                        dtype=mpp.out.dtype).pin_memory()
+    idx_h = torch.empty(rt.idx.shape, dtype=rt.idx.dtype).pin_memory()
+
+    def e2e_step():
+        for n in dev:
+            dev[n].copy_(host[n], non_blocking=True)
+        out = mpp(dev["q_r"], dev["q"], dev["k_loc"], dev["v_loc"])
+        if b1 > b0:
+            out_h[:b1 - b0].copy_(out[:b1 - b0], non_blocking=True)
+        idx_h.copy_(rt.idx, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = (b1 - b0) * out_h[0].numel() * out_h.element_size() + \
+        idx_h.numel() * idx_h.element_size()
+    h2d = int(max_over_ranks(float(h2d), world))
+    d2h = int(max_over_ranks(float(d2h), world))
+
+    import torch.distributed as dist
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        step()
+        torch.cuda.synchronize()
+    launches = sum(1 for e in prof.events()
+                   if e.device_type.name == "CUDA" and "msa" in e.name)
+    launches = int(max_over_ranks(float(launches), world))
+    status = msa.msa_device_status(clear=True)
+    idx_all = [torch.empty_like(rt.idx) for _ in range(world)]
+    if world > 1:
+        dist.all_gather(idx_all, rt.idx)
+    else:
+        idx_all = [rt.idx]
+    same_sel = all(torch.equal(x, idx_all[0]) for x in idx_all)
+    seg_max = [max_over_ranks(x, world) for x in seg]
+    if rank != 0:
+        return None
+    pk = peaks()
+    C_r = c1 - c0
+    route_flops = 2.0 * 8 * 128 * 256 * C_r
+    route_tf = route_flops / (seg[0] * 1e-3) / 1e12
+    return {
+        "metric": METRIC, "value": round(C / (ms_step * 1e-3) / 1e9, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) pooled bank drawn at chunk level + planted needles)",
+        "config": step_config(world, C, n_docs, args.n_docs, T, k, m_cap),
+        "roofline": {"bound": "tensor",
+                     "kernel": "route_tc_kernel on CTA pairs over rank 0's shard "
+                               f"({C_r} of {C} chunks)",
+                     "achieved": round(route_tf, 1), "peak": pk["bf16"], "unit": "TFLOP/s",
+                     "frac": round(route_tf / pk["bf16"], 4),
+                     "hbm": {"achieved": round(C_r * BYTES_PER_CHUNK / (seg[0] * 1e-3) / 1e9, 1),
+                             "peak": pk["hbm"], "unit": "GB/s",
+                             "frac": round(C_r * BYTES_PER_CHUNK / (seg[0] * 1e-3) / 1e9
+                                           / pk["hbm"], 4)},
+                     "traffic": ROUTE_DRAM_TRAFFIC(C_r), "traffic_unit": "GB per launch",
+                     "peak_source": pk["src"]},
+        "stages_ms": {**{n: round(x, 4) for n, x in zip(names, seg_max)},
+                      "note": "eager launches with events between stages, max over ranks per "
+                              "stage; the step's own timing has no events"},
+        "shards": [{"docs": [a, b], "chunks": [c, d]} for a, b, c, d in plan],
+        "same_selection_on_every_rank": same_sel,
+        "e2e": {"value": round(C / (e2e_ms * 1e-3) / 1e9, 4), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "per step: Q_r (every rank) and the served block's Q and local K/V "
+                        "uploaded from pinned host memory, the output and the selection read "
+                        "back"},
+        "gpu_launches": launches * args.steps,
+        "gpu_launches_per_step": launches,
+        "device_status": status,
+        "clocks": clk,
+    }
 
 
 def bench_tiered(w, p, steps: int, resident_ms: float) -> dict:
@@ -433,6 +625,98 @@ def time_device(fn, steps: int) -> float:
     return e0.elapsed_time(e1) / steps
 
 
+def time_device_flushed(fn, steps: int, flush) -> float:
+    """Mean device milliseconds per call with the L2 flushed before every
+    call (``flush`` writes a buffer larger than the L2; its time is not
+    counted): for workloads whose inputs fit in the 126 MB L2."""
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for e0, e1 in evs:
+        flush()
+        e0.record()
+        fn()
+        e1.record()
+    torch.cuda.synchronize()
+    return sum(e0.elapsed_time(e1) for e0, e1 in evs) / steps
+
+
+def bench_bank_1m(steps: int, pk: dict) -> dict:
+    """1M-token bank (1,000 token-level documents encoded by msa_encode_pool,
+    16,312 chunks), one 128-token prefill query: route over the prepared bank
+    -> top-16 -> gather -> attention, per stage and as one CUDA graph.  The
+    bank (33 MB of routing keys) fits in the L2, so the L2 is flushed before
+    every timed call."""
+    import torch
+
+    from latent_memory_routing_b200 import pipeline, synth
+    w = synth.bank_1m("cuda")
+    toff = w["tok_offsets"].cuda()
+    coff = pipeline.chunk_offsets(toff)
+    coff_h = coff.cpu()
+    C = int(coff_h[-1])
+    kb, vb, rb = pipeline.encode_pool(w["k_tok"], w["v_tok"], w["kr_tok"], toff, coff, C)
+    for name in ("k_tok", "v_tok", "kr_tok"):
+        del w[name]
+    hat = pipeline.prepare_bank(rb[0])
+    m_cap = w["k"] * int((coff_h[1:] - coff_h[:-1]).max())
+    p = pipeline.Pipeline(hat, kb[0], vb[0], coff, B=1, T=w["T"], T_loc=w["T_loc"], Hq=w["Hq"],
+                          k=w["k"], m_cap=m_cap, pos0=w["pos0"], prepared=True)
+    p(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    graph = p.capture(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        scratch.fill_(1)
+
+    ms = time_device_flushed(graph.replay, steps, flush)
+    ms_route = time_device_flushed(lambda: p.router(w["q_r"], p.kr_bar, p.coff, p.n_docs,
+                                                    p.doc_scores, None), steps, flush)
+    ms_topk = time_device_flushed(lambda: pipeline.topk_docs(p.doc_scores, p.k, p.idx, p.top,
+                                                             p.topk_ws), steps, flush)
+    ms_gather = time_device_flushed(lambda: pipeline.gather_kv(
+        p.idx, p.coff, p.k_bar, p.v_bar, p.m_cap, p.k_mem, p.v_mem, p.mem_len), steps, flush)
+    ms_attn = time_device_flushed(lambda: p.attn(w["q"], p.k_mem, p.v_mem, p.mem_len,
+                                                 w["k_loc"], w["v_loc"], p.pos0, p.rope_base,
+                                                 0.0, p.out), steps, flush)
+    rows = int(p.mem_len.sum())
+    H, D = p.H, p.D
+    route_bytes = C * BYTES_PER_CHUNK
+    gather_bytes = 2 * 2 * rows * H * D * 2  # K and V rows, read and written
+    attn_flops = attn_flops_per_step(p)
+    hbm = lambda b, t: round(b / (t * 1e-3) / 1e9 / pk["hbm"], 4)  # noqa: E731
+    res = {"workload": "bank_1m: 1,000 token-level docs of U[256,1792] tokens encoded by "
+                       "msa_encode_pool (16,312 chunks), 4 planted needles; one 128-token "
+                       "prefill query, 128 local tokens, top-16",
+           "ms_per_step": round(ms, 4), "gchunks_s": round(C / (ms * 1e-3) / 1e9, 4),
+           "l2": "flushed (256 MB write) before every timed call",
+           "stages_ms": {"route": round(ms_route, 4), "topk": round(ms_topk, 4),
+                         "gather": round(ms_gather, 4), "attn": round(ms_attn, 4)},
+           "route_roofline": {"bound": "hbm", "bytes": route_bytes,
+                              "achieved": round(route_bytes / (ms_route * 1e-3) / 1e9, 1),
+                              "peak": pk["hbm"], "unit": "GB/s",
+                              "frac": hbm(route_bytes, ms_route),
+                              "note": "128 query columns: 128 FLOP per byte, below the ridge; "
+                                      "a 33 MB scan is about one wave of tiles, so the launch "
+                                      "and pipeline fill weigh"},
+           "gather_roofline": {"bound": "hbm", "bytes": gather_bytes,
+                               "achieved": round(gather_bytes / (ms_gather * 1e-3) / 1e9, 1),
+                               "peak": pk["hbm"], "unit": "GB/s",
+                               "frac": hbm(gather_bytes, ms_gather)},
+           "attn_roofline": {"bound": "tensor", "flops": attn_flops,
+                             "achieved": round(attn_flops / (ms_attn * 1e-3) / 1e12, 2),
+                             "peak": pk["bf16"], "unit": "TFLOP/s",
+                             "frac": round(attn_flops / (ms_attn * 1e-3) / 1e12 / pk["bf16"], 5),
+                             "note": "0.4 GFLOP: latency-bound"},
+           "n_chunks": C, "mem_rows": rows}
+    del graph, p, w, kb, vb, rb, hat, scratch
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_encode(steps: int, peak_hbm: float) -> dict:
     """4 routed layers x 1M tokens: doc-wise RoPE + 64-token chunk means."""
     import torch
@@ -482,6 +766,10 @@ def bench_decode(steps: int, peak_hbm: float) -> dict:
                                             p.doc_scores, None), steps)
     ms_attn = time_device(lambda: p.attn(w["q"], p.k_mem, p.v_mem, p.mem_len, w["k_loc"],
                                          w["v_loc"], p.pos0, p.rope_base, 0.0, p.out), steps)
+    ms_topk = time_device(lambda: pipeline.topk_docs(p.doc_scores, p.k, p.idx, p.top,
+                                                     p.topk_ws), steps)
+    ms_gather = time_device(lambda: pipeline.gather_kv(p.idx, p.coff, p.k_bar, p.v_bar, p.m_cap,
+                                                       p.k_mem, p.v_mem, p.mem_len), steps)
     pf = pipeline.Pipeline(hat, w["k_bar"], w["v_bar"], coff, B=w["B"], T=1, T_loc=w["T_loc"],
                            Hq=w["Hq"], k=w["k"], m_cap=m_cap, pos0=w["pos0"], prepared=True,
                            fused=True)
@@ -496,12 +784,20 @@ def bench_decode(steps: int, peak_hbm: float) -> dict:
     rows = int(p.mem_len.sum()) + w["B"] * w["T_loc"]
     attn_bytes = rows * H * D * 2 * 2 + 2 * w["q"].numel() * 2
     gbs = attn_bytes / (ms_attn * 1e-3) / 1e9
+    gather_bytes = 2 * 2 * int(p.mem_len.sum()) * H * D * 2  # K and V rows, read and written
     res = {"workload": "bank_10m: 10,000 docs, lengths LogNormal(ln 800, 0.65) in [64, 8192], "
                        "pooled bf16 bank; 64 single-token decode queries, 2,048 local tokens, top-16",
            "ms_per_step": round(ms, 4), "decode_tok_s": round(w["B"] / (ms * 1e-3), 1),
            "route_ms": round(ms_route, 4),
            "route_gchunks_s": round(C / (ms_route * 1e-3) / 1e9, 4),
            "route_hbm_frac": round(C * BYTES_PER_CHUNK / (ms_route * 1e-3) / 1e9 / peak_hbm, 4),
+           "topk_ms": round(ms_topk, 4),
+           "gather_ms": round(ms_gather, 4),
+           "gather_roofline": {"bound": "hbm", "bytes": gather_bytes,
+                               "achieved": round(gather_bytes / (ms_gather * 1e-3) / 1e9, 1),
+                               "peak": peak_hbm, "unit": "GB/s",
+                               "frac": round(gather_bytes / (ms_gather * 1e-3) / 1e9 / peak_hbm,
+                                             4)},
            "attn_ms": round(ms_attn, 4),
            "attn_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_hbm,
                              "unit": "GB/s", "frac": round(gbs / peak_hbm, 4)},
@@ -570,6 +866,12 @@ def bench_backward(steps: int, peak_hbm: float) -> dict:
     return res
 
 
+# (B, T = T_loc, memory rows) of the prefill sweep; the GPU tests check each
+# point against the oracle on sampled query rows at its own size
+PREFILL_SWEEP = ((1, 4096, 384), (2, 8192, 384), (1, 16384, 384), (1, 32768, 384),
+                 (16, 4096, 384), (16, 2048, 384))
+
+
 def bench_prefill_sweep(steps: int, peak_bf16: float) -> dict:
     """Causal prefill attention alone at longer contexts than the bank_100m
     step's 256 tokens (whose attention is latency-bound): 32 query heads,
@@ -579,7 +881,7 @@ def bench_prefill_sweep(steps: int, peak_bf16: float) -> dict:
     from latent_memory_routing_b200 import pipeline, synth
     res = {"note": "tensor-core prefill, FLOPs = 4*D per visible (query row, key) pair, "
                    "fraction of the measured burst bf16 peak", "shapes": []}
-    for (B, T, M) in ((1, 4096, 384), (2, 8192, 384), (1, 16384, 384)):
+    for (B, T, M) in PREFILL_SWEEP:
         Hq, H, D = 32, 8, 128
         g = torch.Generator(device="cuda").manual_seed(B * T)
         dt = torch.bfloat16
@@ -684,9 +986,10 @@ def run_reference(args, world, rank):
 
     from latent_memory_routing_b200 import synth
     import oracle
-    lengths = synth.bank_100m_lengths()
+    lengths = synth.bank_100m_lengths(args.n_docs)
     coff_h = oracle.chunk_offsets_from_lengths(lengths.numpy())
-    w = synth.bank_100m(coff_h, "cuda" if torch.cuda.is_available() else "cpu")
+    w = synth.bank_100m(coff_h, "cuda" if torch.cuda.is_available() else "cpu",
+                        n_docs=args.n_docs)
     C = int(coff_h[-1])
 
     class P:  # the few pipeline attributes the baseline reads
@@ -715,13 +1018,11 @@ def run_reference(args, world, rank):
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 8), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(step * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": round(step * 1e3, 1), "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n_chunks": C, "n_docs": len(lengths),
-                   "global_batch": world, "seq_len": int(w["T"]), "top_k": int(w["k"]),
-                   "m_cap": int(w["k"]) * int((coff_h[1:] - coff_h[:-1]).max()),
-                   "parallelism": "rank 0 only (host cores)",
-                   "l2": "the 3.2 GB routing bank streams through the 126 MB L2 every step"},
+        "config": step_config(world, C, len(lengths), args.n_docs, int(w["T"]), int(w["k"]),
+                              int(w["k"]) * int((coff_h[1:] - coff_h[:-1]).max())),
+        "where": "rank 0's host cores (the float64 oracle; no device work)",
         "sampled_step": {
             "chunks_routed_per_step": int(round(sum(chunks) / len(chunks))),
             "of_chunks": C, "timed_seconds": round(sum(secs), 2),
@@ -852,6 +1153,8 @@ def main():
                     help="skip the encode and decode workloads reported beside the step")
     ap.add_argument("--n-docs", type=int, default=100000,
                     help="documents in the bank (fewer only to profile a small case)")
+    ap.add_argument("--sharded", action="store_true",
+                    help="run the Memory Parallel step even on one GPU (a group of one)")
     ap.add_argument("--case", choices=sorted(CASES),
                     help="run one kernel shape three times (for profiling) and exit")
     args = ap.parse_args()
@@ -867,13 +1170,16 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = dist_setup(args.gpus, force_group=args.sharded)
     try:
-        line = run_libmsa(args, world, rank, local)
+        if world > 1 or args.sharded:
+            line = run_memory_parallel(args, world, rank, local)
+        else:
+            line = run_libmsa(args, world, rank, local)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:
-        if world > 1:
+        if world > 1 or args.sharded:
             import torch.distributed as dist
             dist.destroy_process_group()
 

@@ -11,23 +11,25 @@
 // Design.  Decode is HBM-bound (every K/V byte is read once); the tensor
 // cores take the two contractions off the CUDA cores so that the few
 // instructions left per key hide under the stream.  A persistent grid of at
-// most one CTA of 15 warps per SM walks work items -- a key split of one
-// (batch element, KV head), serving the G query heads of the KV head padded
-// to N = 16 MMA columns -- with one continuous pipeline across items, so
-// the stream never drains between them:
+// most one CTA of 15 warps per SM takes work items -- a chunk of consecutive
+// key tiles of one (batch element, KV head), serving the G query heads of
+// the KV head padded to N = 16 MMA columns -- from a global counter as it
+// goes (a CTA that runs faster takes more, so the CTAs end together), with
+// one continuous pipeline across items, so the stream never drains between
+// them:
 //   * warp 0 TMA-loads 128-key K and V tiles (128B-swizzled, 64-dim blocks)
-//     into 3-slot K and V rings, one lane each -- per item, memory tiles
+//     into 3-slot K and V rings, one lane each -- the K lane also takes the
+//     next chunk and publishes it to the other roles -- per item, memory tiles
 //     first, then local tiles, so no tile mixes the two; a K slot is
 //     released when S has read it, a V slot when P V has, so the K stream
 //     runs ahead;
 //   * warps 2, 3, 8..13 (rotators) apply RoPE to local K tiles in shared
 //     memory in the relative form <R(p_q) q, R(p_k) k> = <R(Delta) q,
-//     R(delta) k>: a key's rotation by its offset delta in the tile uses a
-//     per-call (delta, frequency) table, and the query, rotated once per
-//     tile by the tile's distance Delta to it (one complex step per tile from
-//     an exact anchor), is written as the MMA's B operand; memory keys are not
-//     rotated and meet R(p_q) q.  In a memory tile that ends early they zero
-//     the V rows past mem_len;
+//     R(delta) k>: a key's rotation by its offset delta in the tile, and
+//     the query, rotated per tile by the tile's distance Delta to it (one
+//     complex step per tile from an anchor the host computed exactly), is
+//     written as the MMA's B operand; memory keys are not rotated and meet
+//     R(p_q) q;
 //   * warp 1 issues S^T = K Q^T (M = 128 keys, N = 16, K = 128) into one of
 //     two TMEM buffers as soon as a K tile is rotated, and the last warp
 //     issues O^T += V^T P^T (M = 128 dims, N = 16, K = 128 keys; V read
@@ -40,15 +42,22 @@
 //     into Q) against a per-head reference maximum that moves only when a
 //     score exceeds it by more than 2^8 -- then O^T is rescaled in TMEM --,
 //     keep per-thread partial row sums (reduced once at the end), and write
-//     P^T (bf16) as the B operand of P V; at an item's last tile they reduce
+//     P^T (bf16) as the B operand of P V (a masked memory row -- past
+//     mem_len, or past its document's end in the fused form -- also has its
+//     V row zeroed in shared memory); at an item's last tile they reduce
 //     the row sums and write the item's output.
-// The query buffers are double-buffered by item and by tile.  Splits write
-// (max, sum, O) partials that the split-KV combine kernel merges; a single
-// split writes the normalised output directly.  Every wait is bounded; after
-// a timeout every role walks its loop without waiting.
+// The query buffers are double-buffered by item and by tile.  The chunks of
+// one (batch element, KV head) write (max, sum, O) partials, and the last of
+// them to finish merges them into the output (an arrival counter), so no
+// second launch combines them; a lone chunk writes the output directly.  The
+// RoPE constants come from the host (no double-precision arithmetic on the
+// device), so nothing precedes the kernel but the reset of its counters.  Every wait is bounded; after a timeout every role walks its
+// loop without waiting.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
+#include <cstdlib>
 
 #include "attn_tc.cuh"
 #include "msa_common.cuh"
@@ -60,14 +69,24 @@ namespace {
 constexpr int kTK = 128;                   // keys per tile (M of S^T)
 constexpr int kNH = 16;                    // MMA columns: G <= 16 heads, padded
 constexpr int kDim = 128;                  // head dim
-constexpr int kTStages = 3;
+// K and V rings of 128-key tiles: a K slot is held from its load to S, a V
+// slot from its load to P V (after S and the softmax), so the V ring is the
+// deeper one
+#ifndef MSA_DTC_KST
+#define MSA_DTC_KST 3
+#endif
+#ifndef MSA_DTC_VST
+#define MSA_DTC_VST 3
+#endif
+constexpr int kKSt = MSA_DTC_KST;
+constexpr int kVSt = MSA_DTC_VST;
+
 constexpr int kRotWarps = 8;
 constexpr int kSoftWarps = 4;
 constexpr int kPvWarp = 2 + kRotWarps + kSoftWarps;  // the P V issuer, last warp
 constexpr int kTThreads = 32 * (kPvWarp + 1);
 constexpr int kBlk = kTK * 128;            // one 64-dim block of a K or V tile: 16 KB
 constexpr int kTileBytes = 2 * kBlk;       // K or V tile: 32 KB
-constexpr int kStageBytes = 2 * kTileBytes;
 constexpr int kQBytes = kNH * kDim * 2;    // Q [16][128] bf16: two 2 KB blocks
 constexpr int kPBytes = kNH * kTK * 2;     // P^T [16][128] bf16: two 2 KB blocks
 constexpr int kSmBar = 1;                  // named barrier of the softmax warps
@@ -78,24 +97,55 @@ constexpr uint32_t kTmemCols = 64;         // S buffers: 0..31, O^T: 32..47
 
 struct DTS {  // dynamic shared memory, offsets from a 1024-byte aligned base
   static constexpr size_t RING = 0;
-  static constexpr size_t QMEM = RING + (size_t)kTStages * kStageBytes;  // [2] by item
+  static constexpr size_t VRING = RING + (size_t)kKSt * kTileBytes;
+  static constexpr size_t QMEM = VRING + (size_t)kVSt * kTileBytes;  // [2] by item
   static constexpr size_t QT = QMEM + 2 * kQBytes;   // [2] by tile
   static constexpr size_t P = QT + 2 * kQBytes;      // [2] by tile
   static constexpr size_t QRAW = P + 2 * kPBytes;    // [2][16][128] bf16 raw query, by item
   static constexpr size_t RED = QRAW + 2 * (size_t)kNH * kDim * 2;  // [4][16] f32
-  static constexpr size_t FLAGS = RED + 4 * kNH * 4;            // [2][4] int
-  static constexpr size_t ALLOC = FLAGS + 2 * 4 * 4 + 1024;
+  static constexpr size_t FLAGS = RED + 4 * kNH * 4;            // [2][4] int + 4 int
+  static constexpr size_t ALLOC = FLAGS + 3 * 4 * 4 + 1024;
   static_assert(QMEM % 1024 == 0 && QT % 1024 == 0 && P % 1024 == 0, "swizzle atoms");
+  static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
 };
+
+// Ring of chunk ids published by the K producer: read by the V producer,
+// the two MMA issuers (one lane each), the softmax warps and the rotator
+// warps (one arrival per warp).
+constexpr int kSched = 4;
+constexpr int kSchedReaders = 3 + kSoftWarps + kRotWarps;
 
 struct DTAux {
   // K and V tiles of a stage arrive and leave separately: a K slot is free
   // once S has read it, a V slot once P V has
-  uint64_t kfull[kTStages], vfull[kTStages], kready[kTStages], kfree[kTStages], vfree[kTStages];
+  uint64_t kfull[kKSt], vfull[kVSt], kready[kKSt], kfree[kKSt], vfree[kVSt];
   uint64_t sfull[2], pfull[2], pvdone[2], odone;
+  uint64_t sched_full[kSched], sched_empty[kSched];
+  int sched_id[kSched];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// RoPE constants of a call, computed on the host in double and rounded
+// once: the kernel does no double-precision arithmetic (FP64 is slow on this
+// part, and a handful of double operations per thread held up the first
+// tiles by microseconds).  For pair i (of kDim / 2):
+//   w[i]      inverse frequency base^(-2i/D);
+//   qpos[i]   R(p_q w_i), the query's own position p_q = pos0 + T_loc - 1;
+//   qdelta[i] R((T_loc - 1) w_i), the distance from local key 0 to the query;
+//   qstep[i]  R(kTK w_i), one key tile.
+struct RopeTab {
+  float w[kDim / 2];
+  float2 qpos[kDim / 2], qdelta[kDim / 2], qstep[kDim / 2];
+};
+
+// Complex product a * conj(b): rotation by angle(a) - angle(b).
+__device__ __forceinline__ float2 cmul_conj(float2 a, float2 b) {
+  return make_float2(a.x * b.x + a.y * b.y, a.y * b.x - a.x * b.y);
+}
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+  return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
+}
 
 __device__ __forceinline__ void soft_bar() {
   asm volatile("bar.sync %0, %1;" ::"n"(kSmBar), "n"(32 * kSoftWarps) : "memory");
@@ -125,12 +175,17 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int k, int rows) {
                     (kk & 7) * 2);
 }
 
-// One work item: a key split of one (batch element, KV head).  Every role
-// walks the same sequence -- the CTA's items blockIdx.x, blockIdx.x + grid,
-// ..., empty ones skipped, and their tiles -- through its own cursor.
+// One work item: a chunk of the key tiles of one (batch element, KV head).
+// Chunks are handed out at run time: the K producer lane takes the next
+// chunk id from a global counter (atomicAdd) when it has issued the last
+// loads of its current chunk and publishes it in a small shared-memory ring;
+// every other role reads the ring in the same order, so all roles walk the
+// same sequence -- chunks with no tiles skipped -- through their own cursor.
+// A CTA that runs ahead takes more chunks, so the CTAs end together.
 struct Cur {
-  int it, k, j, nt;      // item, its ordinal among this CTA's non-empty items, tile, tiles
-  int b, g, sp, M, n_mt, j_lo;
+  int su;                // ring entries read (or, for the K producer, published)
+  int k, j, nt;          // ordinal of the chunk among this CTA's non-empty ones, tile, tiles
+  int item, b, g, sp, n_eff, M, n_mt, j_lo;
 };
 
 // kFused: the memory rows come straight from the pooled bank -- per query
@@ -139,17 +194,29 @@ struct Cur {
 // then map the bank with 8-row boxes (one 128B-swizzle atom each), and a
 // memory tile is 16 groups.  Rows past a document's end within its last
 // group are other bank rows: masked out, and their V zeroed in shared memory
-// by the rotators (as the rows past mem_len of a gathered memory tile).
+// by the softmax (as the rows past mem_len of a gathered memory tile).
+//
+// Chunk ids: the first n_whole ids are whole items (item = id; item =
+// b * H + g).  Whole items fill complete rounds of the grid; the remaining
+// n_tail items, which would leave most CTAs idle in a last partial round,
+// are cut into chunks: id = n_whole + sp * n_tail + t is chunk sp of item
+// n_whole + t, and an item of nt key tiles is cut into n_eff = min(n_ch, nt)
+// chunks of consecutive tiles (chunks sp >= n_eff hold none).  A cut item's
+// chunks write (max, sum, O) partials; the last of them to finish (an
+// arrival counter per cut item) merges them and writes the output, so no
+// second launch combines them.  counters[0] (chunk counter) and
+// counters[1 + t] (arrivals) are zero at launch.
 template <int G, bool kFused>
 __global__ void __launch_bounds__(kTThreads, 1)
 attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
                       const __grid_constant__ CUtensorMap tm_vm,
                       const __grid_constant__ CUtensorMap tm_kl,
                       const __grid_constant__ CUtensorMap tm_vl, int T_loc, int Hq, int H,
-                      int n_items, const __nv_bfloat16* __restrict__ q,
+                      int n_whole, int n_tail, int n_ch, const __nv_bfloat16* __restrict__ q,
                       const int32_t* __restrict__ mem_len, int m_cap,
-                      const int2* __restrict__ groups, int max_groups, int64_t pos0, double base,
-                      float qscale, int n_split, const float2* __restrict__ cs_tab,
+                      const int2* __restrict__ groups, int max_groups,
+                      const __grid_constant__ RopeTab rope, float qscale,
+                      int* __restrict__ counters,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
                       float2* __restrict__ part_ml, int* __restrict__ status) {
   static_assert(G >= 1 && G <= kNH, "heads per KV head");
@@ -157,45 +224,100 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   extern __shared__ __align__(1024) unsigned char dsm[];
   __shared__ DTAux aux;
   unsigned char* sm = tc::smem_align<1024>(dsm);
-  unsigned char* ring = sm + DTS::RING;
-  unsigned char* qmem = sm + DTS::QMEM;  // [2] by item
+  unsigned char* ring = sm + DTS::RING;    // K ring
+  unsigned char* vring = sm + DTS::VRING;  // V ring
+  unsigned char* qmem = sm + DTS::QMEM;  // [2] by chunk
   unsigned char* qt = sm + DTS::QT;      // [2] by tile
   unsigned char* pbuf = sm + DTS::P;     // [2] by tile
   __nv_bfloat16* qraw = reinterpret_cast<__nv_bfloat16*>(sm + DTS::QRAW);  // [2][16][128]
   float* red = reinterpret_cast<float*>(sm + DTS::RED);
   int* flags = reinterpret_cast<int*>(sm + DTS::FLAGS);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n_chunks = n_whole + n_tail * n_ch;
+  const int n_lt = (T_loc + kTK - 1) / kTK;
 
-  auto load_item = [&](Cur& c) {
-    c.sp = c.it % n_split;
-    const int bg = c.it / n_split;
-    c.b = bg / H;
-    c.g = bg % H;
+  auto load_chunk = [&](Cur& c, int id) {
+    if (id < n_whole) {
+      c.sp = 0;
+      c.item = id;
+    } else {
+      c.sp = (id - n_whole) / n_tail;
+      c.item = n_whole + (id - n_whole) % n_tail;
+    }
+    c.b = c.item / H;
+    c.g = c.item % H;
     // fused: mem_len holds the query's group count; its memory is 8 rows a group
     c.M = kFused ? 8 * min(max(mem_len[c.b], 0), max_groups) : min(max(mem_len[c.b], 0), m_cap);
     c.n_mt = (c.M + kTK - 1) / kTK;
-    const int n_all = c.n_mt + (T_loc + kTK - 1) / kTK;
-    c.j_lo = (int)((int64_t)c.sp * n_all / n_split);
-    c.nt = (int)((int64_t)(c.sp + 1) * n_all / n_split) - c.j_lo;
+    const int n_all = c.n_mt + n_lt;
+    c.n_eff = c.item < n_whole ? 1 : min(n_ch, n_all);
+    if (c.sp >= c.n_eff) {
+      c.nt = 0;
+      return;
+    }
+    c.j_lo = (int)((int64_t)c.sp * n_all / c.n_eff);
+    c.nt = (int)((int64_t)(c.sp + 1) * n_all / c.n_eff) - c.j_lo;
   };
-  auto first = [&](Cur& c) -> bool {
+  volatile int* abort_flag = &aux.abort_flag;
+  auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
+    if (*abort_flag) return;
+    if (!tc::mbar_wait(bar, parity)) {
+      record_error(status, MSA_ERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+  };
+  // K producer: take the next chunk from the counter and publish it.  The
+  // counter is read early (`ahead`, taken as the current chunk's last tile
+  // is issued) so that its round trip overlaps that tile's load.
+  int ahead = -1;
+  auto grab = [&](Cur& c) -> bool {
+    for (;;) {
+      const int slot = c.su % kSched;
+      wait_or_abort(&aux.sched_empty[slot], ((c.su / kSched) & 1) ^ 1);
+      int id = -1;
+      if (!*abort_flag) {
+        const int t = ahead >= 0 ? ahead : atomicAdd(counters, 1);
+        ahead = -1;
+        id = t < n_chunks ? t : -1;
+      }
+      aux.sched_id[slot] = id;
+      tc::mbar_arrive(&aux.sched_full[slot]);  // release: the id is visible to the waiters
+      ++c.su;
+      if (id < 0) return false;
+      load_chunk(c, id);
+      if (c.nt > 0) {
+        c.j = 0;
+        return true;
+      }
+    }
+  };
+  // every other role: read the next published chunk (`whole_warp`: all 32
+  // lanes read, lane 0 arrives for the warp)
+  auto fetch = [&](Cur& c, bool whole_warp) -> bool {
+    for (;;) {
+      const int slot = c.su % kSched;
+      wait_or_abort(&aux.sched_full[slot], (c.su / kSched) & 1);
+      const int id = *abort_flag ? -1 : aux.sched_id[slot];
+      if (whole_warp) __syncwarp();
+      if (!whole_warp || lane == 0) tc::mbar_arrive(&aux.sched_empty[slot]);
+      ++c.su;
+      if (id < 0) return false;
+      load_chunk(c, id);
+      if (c.nt > 0) {
+        c.j = 0;
+        return true;
+      }
+    }
+  };
+  auto first = [&](Cur& c, int role) -> bool {
+    c.su = 0;
     c.k = 0;
-    c.j = 0;
-    for (c.it = blockIdx.x; c.it < n_items; c.it += gridDim.x) {
-      load_item(c);
-      if (c.nt > 0) return true;
-    }
-    return false;
+    return role == 0 ? grab(c) : fetch(c, role == 2);
   };
-  auto next = [&](Cur& c) -> bool {
+  auto next = [&](Cur& c, int role) -> bool {
     if (++c.j < c.nt) return true;
-    c.j = 0;
     ++c.k;
-    for (c.it += gridDim.x; c.it < n_items; c.it += gridDim.x) {
-      load_item(c);
-      if (c.nt > 0) return true;
-    }
-    return false;
+    return role == 0 ? grab(c) : fetch(c, role == 2);
   };
   auto tile_mem = [&](const Cur& c) { return c.j_lo + c.j < c.n_mt; };
   auto tile_key0 = [&](const Cur& c) {
@@ -207,26 +329,14 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     return jj < c.n_mt ? min(kTK, c.M - jj * kTK) : min(kTK, T_loc - (jj - c.n_mt) * kTK);
   };
 
-  // an empty split (more splits than tiles): neutral partials
-  if (n_split > 1) {
-    Cur c;
-    for (c.it = blockIdx.x; c.it < n_items; c.it += gridDim.x) {
-      load_item(c);
-      if (c.nt > 0) continue;
-      for (int e = tid; e < G * kDim; e += kTThreads) {
-        const int64_t row_id = (int64_t)c.b * Hq + c.g * G + e / kDim;
-        part_o[(row_id * n_split + c.sp) * kDim + e % kDim] = 0.f;
-        if (e % kDim == 0) part_ml[row_id * n_split + c.sp] = make_float2(-INFINITY, 0.f);
-      }
-    }
-  }
-
   if (tid == 0) {
-    for (int i = 0; i < kTStages; ++i) {
+    for (int i = 0; i < kKSt; ++i) {
       tc::mbar_init(&aux.kfull[i], 1);
-      tc::mbar_init(&aux.vfull[i], 1);
       tc::mbar_init(&aux.kready[i], kRotWarps);
       tc::mbar_init(&aux.kfree[i], 1);
+    }
+    for (int i = 0; i < kVSt; ++i) {
+      tc::mbar_init(&aux.vfull[i], 1);
       tc::mbar_init(&aux.vfree[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -236,6 +346,10 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     tc::mbar_init(&aux.pvdone[0], 1);
     tc::mbar_init(&aux.pvdone[1], 1);
     tc::mbar_init(&aux.odone, 1);
+    for (int i = 0; i < kSched; ++i) {
+      tc::mbar_init(&aux.sched_full[i], 1);
+      tc::mbar_init(&aux.sched_empty[i], kSchedReaders);
+    }
     aux.abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -251,36 +365,32 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = aux.tmem_base;
-  volatile int* abort_flag = &aux.abort_flag;
-  auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
-    if (*abort_flag) return;
-    if (!tc::mbar_wait(bar, parity)) {
-      record_error(status, MSA_ERR_TIMEOUT);
-      *abort_flag = 1;
-    }
-  };
 
   if (warp == 0) {
     // ----------------------------------------------------------- producers
-    // lane 0 streams the K tiles, lane 1 the V tiles, each gated by its own
-    // slot releases, so K loads run ahead of the V slots P V still holds
+    // lane 0 streams the K tiles (and takes the chunks), lane 1 the V tiles,
+    // each gated by its own slot releases, so K loads run ahead of the V
+    // slots P V still holds
     if (lane < 2) {
       const bool isv = lane == 1;
+      const int role = isv ? 1 : 0;
       uint64_t* fullb = isv ? aux.vfull : aux.kfull;
+      const int nst = isv ? kVSt : kKSt;
       uint64_t* freeb = isv ? aux.vfree : aux.kfree;
       Cur c;
       int u = 0;
-      for (bool ok = first(c); ok; ok = next(c), ++u) {
-        const int st = u % kTStages;
-        wait_or_abort(&freeb[st], ((u / kTStages) & 1) ^ 1);
+      for (bool ok = first(c, role); ok; ok = next(c, role), ++u) {
+        const int st = u % nst;
+        if (!isv && c.j == c.nt - 1) ahead = atomicAdd(counters, 1);  // the next chunk
+        wait_or_abort(&freeb[st], ((u / nst) & 1) ^ 1);
         if (*abort_flag) break;
-        unsigned char* d = ring + (size_t)st * kStageBytes + (isv ? kTileBytes : 0);
+        unsigned char* d = (isv ? vring : ring) + (size_t)st * kTileBytes;
         const bool mem = tile_mem(c);
         const CUtensorMap* m = mem ? (isv ? &tm_vm : &tm_km) : (isv ? &tm_vl : &tm_kl);
         tc::mbar_arrive_expect_tx(&fullb[st], kTileBytes);
         if (kFused && mem) {
           // 16 groups of 8 bank rows; past the query's last group, repeat it
-          // (finite rows, masked) so every row of the tile is written
+          // (masked, V zeroed) so every row of the tile is written
           const int ng = c.M / 8, g0 = tile_key0(c) / 8;
           const int2* gq = groups + (int64_t)c.b * max_groups;
 #pragma unroll 4
@@ -294,9 +404,10 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           tc::tma_load_3d(d, m, &fullb[st], 0, c.g, row0);
           tc::tma_load_3d(d + kBlk, m, &fullb[st], 64, c.g, row0);
         }
+
       }
-      for (int v = u > kTStages ? u - kTStages : 0; v < u; ++v)
-        tc::mbar_wait(&fullb[v % kTStages], (v / kTStages) & 1);
+      for (int v = u > nst ? u - nst : 0; v < u; ++v)
+        tc::mbar_wait(&fullb[v % nst], (v / nst) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- S MMA
@@ -306,12 +417,12 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     if (lane == 0) {
       Cur cs;
       int us = 0;
-      for (bool hs = first(cs); hs; hs = next(cs), ++us) {
-        const int st = us % kTStages;
-        wait_or_abort(&aux.kready[st], (us / kTStages) & 1);
+      for (bool hs = first(cs, 1); hs; hs = next(cs, 1), ++us) {
+        const int st = us % kKSt;
+        wait_or_abort(&aux.kready[st], (us / kKSt) & 1);
         if (us >= 2) wait_or_abort(&aux.pfull[us & 1], ((us - 2) >> 1) & 1);
         tc::tc_fence_after();
-        const uint32_t a0 = tc::smem_u32(ring + (size_t)st * kStageBytes);
+        const uint32_t a0 = tc::smem_u32(ring + (size_t)st * kTileBytes);
         const uint32_t b0 =
             tc::smem_u32(tile_mem(cs) ? qmem + (cs.k & 1) * kQBytes : qt + (us & 1) * kQBytes);
 #pragma unroll
@@ -332,12 +443,12 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     if (lane == 0) {
       Cur cp;
       int up = 0;
-      for (bool hp = first(cp); hp; hp = next(cp), ++up) {
-        const int st = up % kTStages;
+      for (bool hp = first(cp, 1); hp; hp = next(cp, 1), ++up) {
+        const int st = up % kVSt;
         wait_or_abort(&aux.pfull[up & 1], (up >> 1) & 1);
-        wait_or_abort(&aux.vfull[st], (up / kTStages) & 1);
+        wait_or_abort(&aux.vfull[st], (up / kVSt) & 1);
         tc::tc_fence_after();
-        const uint32_t v0 = tc::smem_u32(ring + (size_t)st * kStageBytes + kTileBytes);
+        const uint32_t v0 = tc::smem_u32(vring + (size_t)st * kTileBytes);
         const uint32_t p0 = tc::smem_u32(pbuf + (up & 1) * kPBytes);
         const bool first_tile = cp.j == 0, last_tile = cp.j == cp.nt - 1;
 #pragma unroll
@@ -347,7 +458,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
                           kIdescO, (!first_tile || kk > 0) ? 1u : 0u);
         tc::mma_commit(&aux.vfree[st]);        // P V has read the V slot
         tc::mma_commit(&aux.pvdone[up & 1]);   // ... and the P buffer up&1
-        if (last_tile) tc::mma_commit(&aux.odone);  // this item's O^T is final
+        if (last_tile) tc::mma_commit(&aux.odone);  // this chunk's O^T is final
       }
     }
   } else if (warp >= 4 && warp < 4 + kSoftWarps) {
@@ -358,7 +469,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     float m_ref[G], l_part[G];
     Cur c;
     int u = 0;
-    for (bool ok = first(c); ok; ok = next(c), ++u) {
+    for (bool ok = first(c, 2); ok; ok = next(c, 2), ++u) {
       if (c.j == 0) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -372,6 +483,22 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       if (kFused && tile_mem(c)) {  // its group holds the row, and the row its document's
         const int grp = (tile_key0(c) + r) / 8;
         valid = grp < c.M / 8 && (r & 7) < groups[(int64_t)c.b * max_groups + grp].y;
+      }
+      if (!valid && tile_mem(c)) {
+        // this memory row lies past mem_len (whatever the caller's buffer
+        // holds there) or past its document's end (another document's bank
+        // row): zero its V once it has landed, so that 0 * V stays 0 in P V.
+        // P V waits for this thread's pfull arrival below, so V(u + kVSt)
+        // cannot land in the slot before P V(u) has released it; and P V of
+        // tile u-3, awaited for tile u-1, means every earlier V has landed:
+        // the parity of tile u names this tile.
+        const int st = u % kVSt;
+        wait_or_abort(&aux.vfull[st], (u / kVSt) & 1);
+        unsigned char* vt = vring + (size_t)st * kTileBytes;
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc)
+          *reinterpret_cast<uint4*>(vt + (cc >> 3) * kBlk + r * 128 + ((cc & 7) << 4)) =
+              make_uint4(0, 0, 0, 0);
       }
       uint32_t sv[16];
       tc::tmem_ld16(tmem + lane_addr + (u & 1) * kNH, sv);
@@ -411,7 +538,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           l_part[h] *= alpha[h];
         }
         if (rescale && c.j > 0) {
-          // O^T holds P V of this item's earlier tiles: wait for the last
+          // O^T holds P V of this chunk's earlier tiles: wait for the last
           // one (tile u-1), then scale each head's column in TMEM
           wait_or_abort(&aux.pvdone[(u - 1) & 1], ((u - 1) >> 1) & 1);
           tc::tc_fence_after();
@@ -439,8 +566,8 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&aux.pfull[u & 1]);
       if (c.j == c.nt - 1) {
-        // the item's last tile: once its P V is done, reduce the row sums
-        // over the 128 key lanes and write this split's O (dim r per thread)
+        // the chunk's last tile: once its P V is done, reduce the row sums
+        // over the 128 key lanes and write this chunk's O (dim r per thread)
         wait_or_abort(&aux.odone, c.k & 1);
         tc::tc_fence_after();
         soft_bar();  // every thread is past its reads of red
@@ -455,17 +582,78 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         uint32_t ov[16];
         tc::tmem_ld16(tmem + lane_addr + 2 * kNH, ov);
         tc::tmem_ld_wait();
-        tc::tc_fence_before();  // the next item's first P V overwrites O^T
+        tc::tc_fence_before();  // the next chunk's first P V overwrites O^T
+        const int64_t row0 = (int64_t)c.item * G;  // = b * Hq + g * G (T == 1)
+        if (c.n_eff == 1) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float l = red[h] + red[kNH + h] + red[2 * kNH + h] + red[3 * kNH + h];
-          const int64_t row_id = (int64_t)c.b * Hq + c.g * G + h;  // T == 1
-          const float o = __uint_as_float(ov[h]);
-          if (n_split == 1) {
-            out[row_id * kDim + r] = __float2bfloat16(l > 0.f ? o / l : 0.f);
-          } else {
-            part_o[(row_id * n_split + c.sp) * kDim + r] = o;
-            if (r == 0) part_ml[row_id * n_split + c.sp] = make_float2(m_ref[h], l);
+          for (int h = 0; h < G; ++h) {
+            const float l = red[h] + red[kNH + h] + red[2 * kNH + h] + red[3 * kNH + h];
+            const float o = __uint_as_float(ov[h]);
+            out[(row0 + h) * kDim + r] = __float2bfloat16(l > 0.f ? o / l : 0.f);
+          }
+        } else {
+          const int tail = c.item - n_whole;  // cut items only
+          const int64_t pidx = (int64_t)tail * n_ch + c.sp;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            part_o[(pidx * G + h) * kDim + r] = __uint_as_float(ov[h]);
+            if (r == 0) {
+              const float l = red[h] + red[kNH + h] + red[2 * kNH + h] + red[3 * kNH + h];
+              part_ml[pidx * G + h] = make_float2(m_ref[h], l);
+            }
+          }
+          // publish the partial, then count this chunk's arrival; the last
+          // of the item's n_eff chunks merges them.  The group barrier orders
+          // every thread's partial before the counting thread's device-scope
+          // fence and atomic (the fence is cumulative), and the merging
+          // side's fence orders the count before its reads.
+          soft_bar();
+          if (r == 0) {
+            __threadfence();
+            flags[8] = atomicAdd(counters + 1 + tail, 1) == c.n_eff - 1;
+          }
+          soft_bar();
+          if (flags[8]) {
+            __threadfence();
+            const int64_t p0 = (int64_t)tail * n_ch;
+            // online merge, kMB chunks at a time with every load of a batch
+            // issued before its arithmetic (G * kMB <= 16 loads of each kind
+            // in flight): the running maximum rescales what came before
+            constexpr int kMB = G >= 16 ? 1 : (G >= 8 ? 2 : 4);
+            float mx[G], l[G], acc[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              mx[h] = -INFINITY;
+              l[h] = 0.f;
+              acc[h] = 0.f;
+            }
+            for (int s0 = 0; s0 < c.n_eff; s0 += kMB) {
+              float2 ml[kMB][G];
+              float o[kMB][G];
+#pragma unroll
+              for (int i = 0; i < kMB; ++i)
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                  const bool live = s0 + i < c.n_eff;
+                  const int64_t pi = (p0 + s0 + i) * G + h;
+                  ml[i][h] = live ? __ldcg(&part_ml[pi]) : make_float2(-INFINITY, 0.f);
+                  o[i][h] = live ? __ldcg(&part_o[pi * kDim + r]) : 0.f;
+                }
+#pragma unroll
+              for (int i = 0; i < kMB; ++i)
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                  if (ml[i][h].x == -INFINITY) continue;
+                  const float mn = fmaxf(mx[h], ml[i][h].x);
+                  const float a = exp2f(mx[h] - mn), wgt = exp2f(ml[i][h].x - mn);
+                  l[h] = l[h] * a + wgt * ml[i][h].y;
+                  acc[h] = acc[h] * a + wgt * o[i][h];
+                  mx[h] = mn;
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+              out[(row0 + h) * kDim + r] = __float2bfloat16(l[h] > 0.f ? acc[h] / l[h] : 0.f);
           }
         }
       }
@@ -474,32 +662,38 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     // ------------------------------------------------------------ rotators
     const int rt = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;  // 0 .. 255
     const int ch = rt & 7, r0 = rt >> 3;  // 16-byte chunk, first of four rows
-    float2 cs[4][8];                      // (cos, sin) of delta = r0 + 32 q, pair 8 ch + e
+    // RoPE in the relative form <R(p_q) q, R(p_k) k> = <R(Delta) q, R(delta) k>
+    // for a local tile: a key's rotation by its offset delta in the tile and
+    // the query's by the tile's distance Delta to it.  Thread rt rotates rows
+    // r0 + 32 qq (qq = 0..3), pairs i = 8 ch + e (e = 0..7): their
+    // R(delta w_i) come from fp32 angles delta * w_i < 128 rad (error
+    // <= ~1.5e-5 rad, two orders below the bf16 rounding of the rotated key).
+    float2 cs[4][8];
 #pragma unroll
-    for (int qq = 0; qq < 4; ++qq)
+    for (int e = 0; e < 8; ++e) {
+      const float wi = rope.w[8 * ch + e];
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const float4 t =
-            *reinterpret_cast<const float4*>(cs_tab + (r0 + 32 * qq) * HALF + 8 * ch + e);
-        cs[qq][e] = make_float2(t.x, t.y);
-        cs[qq][e + 1] = make_float2(t.z, t.w);
+      for (int qq = 0; qq < 4; ++qq) {
+        float sn, cn;
+        sincosf((float)(r0 + 32 * qq) * wi, &sn, &cn);
+        cs[qq][e] = make_float2(cn, sn);
       }
-    const int i_q = rt % HALF;  // query pair this thread rotates (every item)
-    const double wq = rope_inv_freq(base, i_q, kDim);
-    const float2 qstep = rope_cs(kTK, wq);
-    const float2 qpos = rope_cs(pos0 + T_loc - 1, wq);  // R(p_q) for memory tiles
+    }
+    const int i_q = rt % HALF;  // query pair this thread rotates (every chunk)
+    const float2 qstep = rope.qstep[i_q];
+    const float2 qpos = rope.qpos[i_q];  // R(p_q) for memory tiles
     float2 qcs = make_float2(1.f, 0.f);
     bool anchored = false;
     Cur c;
     int u = 0;
-    for (bool ok = first(c); ok; ok = next(c), ++u) {
-      const int st = u % kTStages;
-      wait_or_abort(&aux.kfull[st], (u / kTStages) & 1);
-      unsigned char* kt = ring + (size_t)st * kStageBytes;
+    for (bool ok = first(c, 2); ok; ok = next(c, 2), ++u) {
+      const int st = u % kKSt;
+      wait_or_abort(&aux.kfull[st], (u / kKSt) & 1);
+      unsigned char* kt = ring + (size_t)st * kTileBytes;
       __nv_bfloat16* qr = qraw + (c.k & 1) * kNH * kDim;
       if (c.j == 0) {
-        // a new item: its raw query and R(p_q) q go to buffers k&1, whose
-        // last readers (S of item k-2, at or before tile u-1) must be done
+        // a new chunk: its raw query and R(p_q) q go to buffers k&1, whose
+        // last readers (S of chunk k-2, at or before tile u-1) must be done
         if (u >= 1) wait_or_abort(&aux.sfull[(u - 1) & 1], ((u - 1) >> 1) & 1);
         for (int e = rt; e < G * kDim; e += 32 * kRotWarps)
           qr[e] = q[((int64_t)c.b * Hq + c.g * G) * kDim + e];
@@ -518,18 +712,23 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         }
         anchored = false;
       }
-      const int n_valid = tile_valid(c);
       if (!tile_mem(c)) {
         // R(Delta) q into buffer u&1, whose last reader S(u-2) must be done
         if (u >= 2) wait_or_abort(&aux.sfull[u & 1], ((u - 2) >> 1) & 1);
-        const int Delta = T_loc - 1 - tile_key0(c);
         if (!anchored) {
-          qcs = rope_cs(Delta, wq);
+          // Delta = (T_loc - 1) - kTK t for the chunk's first local tile t:
+          // R((T_loc - 1) w) R(kTK w)^(-t), the power by repeated squaring
+          int t = tile_key0(c) / kTK;
+          float2 sq = qstep;
+          qcs = rope.qdelta[i_q];
+          while (t) {
+            if (t & 1) qcs = cmul_conj(qcs, sq);
+            sq = cmul(sq, sq);
+            t >>= 1;
+          }
           anchored = true;
         } else {  // Delta fell by kTK: multiply by e^{-i kTK w}
-          const float cc = qcs.x * qstep.x + qcs.y * qstep.y;
-          qcs.y = qcs.y * qstep.x - qcs.x * qstep.y;
-          qcs.x = cc;
+          qcs = cmul_conj(qcs, qstep);
         }
         unsigned char* qb = qt + (u & 1) * kQBytes;
         for (int e = rt; e < G * HALF; e += 32 * kRotWarps) {
@@ -561,42 +760,6 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           *p1 = Vec16<__nv_bfloat16>::pack(y1);
           *p2 = Vec16<__nv_bfloat16>::pack(y2);
         }
-      } else if (kFused) {
-        // rows of a group past its document's end (and the repeated groups
-        // past the query's last one) are other bank rows: zero their V as
-        // below, so a non-finite bank value cannot turn 0 * V into NaN
-        const int g0 = tile_key0(c) / 8, ng = c.M / 8;
-        const int2* gq = groups + (int64_t)c.b * max_groups;
-        bool partial = false;
-        for (int gi = 0; gi < kTK / 8; ++gi)
-          partial |= g0 + gi >= ng || gq[g0 + gi].y < 8;
-        if (partial) {
-          if (u >= kTStages) wait_or_abort(&aux.vfree[st], ((u / kTStages) - 1) & 1);
-          wait_or_abort(&aux.vfull[st], (u / kTStages) & 1);
-          unsigned char* vt = kt + kTileBytes;
-          for (int e = rt; e < kTK * 16; e += 32 * kRotWarps) {
-            const int rr = e / 16, cc = e % 16, grp = g0 + rr / 8;
-            const int nv = grp < ng ? gq[grp].y : 0;
-            if ((rr & 7) >= nv)
-              *reinterpret_cast<uint4*>(vt + (cc >> 3) * kBlk + rr * 128 + ((cc & 7) << 4)) =
-                  make_uint4(0, 0, 0, 0);
-          }
-        }
-      } else if (n_valid < kTK) {
-        // memory rows past mem_len hold whatever the caller's buffer holds:
-        // zero their V (once it has landed) so that 0 * V stays 0 in P V,
-        // which is issued after S(u) and so after this tile's kready.  The V
-        // stream may trail the K stream by a whole ring, so first wait for
-        // the slot's previous tile (u - 3) to leave it: then the vfull
-        // parity below can only mean tile u.
-        if (u >= kTStages) wait_or_abort(&aux.vfree[st], ((u / kTStages) - 1) & 1);
-        wait_or_abort(&aux.vfull[st], (u / kTStages) & 1);
-        unsigned char* vt = kt + kTileBytes;
-        for (int e = rt; e < (kTK - n_valid) * 16; e += 32 * kRotWarps) {
-          const int rr = n_valid + e / 16, cc = e % 16;
-          *reinterpret_cast<uint4*>(vt + (cc >> 3) * kBlk + rr * 128 + ((cc & 7) << 4)) =
-              make_uint4(0, 0, 0, 0);
-        }
       }
       tc::fence_proxy_async_smem();
       __syncwarp();
@@ -612,44 +775,64 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   }
 }
 
-// (cos, sin) of delta * w_i for delta in [0, 128), i in [0, 64): exact
-// angles (reduced in double), once per call.
-__global__ void decode_cs_table_kernel(double base, float2* __restrict__ tab) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e < kTK * (kDim / 2)) tab[e] = rope_cs(e / (kDim / 2), rope_inv_freq(base, e % (kDim / 2), kDim));
-}
-
 struct DTPlan {
-  int n_split;
-  size_t tab_bytes, po_bytes, ml_bytes, total;
+  int n_whole, n_tail, n_ch;
+  size_t cnt_bytes, po_bytes, ml_bytes, total;
 };
 
-// Key splits: each of min(items, SMs) CTAs walks items round-robin, so the
-// busiest CTA runs ceil(items / CTAs) items of ceil(tiles / splits) tiles;
-// take the split count that makes that smallest, charging a quarter tile per
-// item for its query set-up and output.
+// Items (batch element, KV head) are handed out whole for as many complete
+// rounds of the grid as they fill (a chunk boundary costs the pipeline a few
+// microseconds, so whole items are cheapest); the items of the last, partial
+// round are cut into about grid / n_tail chunks each, so that every CTA
+// takes a share of the tail.  At most one chunk per key tile of the longest
+// item, and at most 64.
 DTPlan dt_plan(int B, int Hq, int H, int T_loc, int m_cap) {
   DTPlan p{};
-  const int64_t base = (int64_t)B * H;
+  const int64_t items = (int64_t)B * H;
   const int64_t tiles = ((int64_t)m_cap + kTK - 1) / kTK + (T_loc + kTK - 1) / kTK;
   const int64_t sms = std::max(1, num_sms());
-  double best = 1e30;
-  int pick = 1;
-  for (int ns = 1; ns <= std::min<int64_t>(tiles, 32); ++ns) {
-    const int64_t items = base * ns, grid = std::min(items, sms);
-    const double cost = (double)((items + grid - 1) / grid) * ((tiles + ns - 1) / ns + 0.25);
-    if (cost < best - 1e-9) {
-      best = cost;
-      pick = ns;
-    }
+  int64_t tail = items % sms;
+  if (const char* e = std::getenv("MSA_DECODE_TAIL")) {  // tuning: cut items (-1 = all)
+    const int v = std::atoi(e);
+    if (v == -1) tail = items;
+    else if (v >= 0 && v <= items) tail = v;
   }
-  p.n_split = pick;
-  p.tab_bytes = round_up((size_t)kTK * (kDim / 2) * sizeof(float2), 256);
-  const size_t rows = (size_t)B * Hq;
-  p.po_bytes = p.n_split > 1 ? round_up(rows * p.n_split * kDim * sizeof(float), 256) : 0;
-  p.ml_bytes = p.n_split > 1 ? round_up(rows * p.n_split * sizeof(float2), 256) : 0;
-  p.total = p.tab_bytes + p.po_bytes + p.ml_bytes;
+  int64_t want = tail > 0 ? (sms + tail - 1) / tail : 1;
+  if (const char* e = std::getenv("MSA_DECODE_CHUNKS")) {  // tuning: chunks per cut item
+    const int v = std::atoi(e);
+    if (v >= 1 && v <= 64) want = v;
+  }
+  p.n_ch = (int)std::max<int64_t>(1, std::min<int64_t>({want, tiles, 64}));
+  if (p.n_ch == 1) tail = 0;  // nothing to cut
+  p.n_tail = (int)tail;
+  p.n_whole = (int)(items - tail);
+  p.cnt_bytes = round_up((size_t)(1 + items) * sizeof(int), 256);
+  const size_t rows = (size_t)tail * (Hq / H);
+  p.po_bytes = tail ? round_up(rows * p.n_ch * kDim * sizeof(float), 256) : 0;
+  p.ml_bytes = tail ? round_up(rows * p.n_ch * sizeof(float2), 256) : 0;
+  p.total = p.cnt_bytes + p.po_bytes + p.ml_bytes;
   return p;
+}
+
+// (cos, sin) of p * w for an integer position p, the angle reduced modulo
+// 2 pi in double on the host.
+float2 host_cs(double p, double w) {
+  const double two_pi = 6.283185307179586;
+  const double th = p * w;
+  const double r = th - std::nearbyint(th / two_pi) * two_pi;
+  return make_float2((float)std::cos(r), (float)std::sin(r));
+}
+
+RopeTab rope_tab(float rope_base, int pos0, int T_loc) {
+  RopeTab t;
+  for (int i = 0; i < kDim / 2; ++i) {
+    const double w = std::pow((double)rope_base, -2.0 * i / kDim);
+    t.w[i] = (float)w;
+    t.qpos[i] = host_cs((double)pos0 + T_loc - 1, w);
+    t.qdelta[i] = host_cs((double)T_loc - 1, w);
+    t.qstep[i] = host_cs((double)kTK, w);
+  }
+  return t;
 }
 
 template <int G>
@@ -661,12 +844,9 @@ int launch_dtc(int B, int T_loc, int Hq, int H, const void* q, const void* k_mem
   const int mem_rows_cap = fm ? 8 * fm->max_groups : m_cap;
   const DTPlan p = dt_plan(B, Hq, H, T_loc, mem_rows_cap);
   unsigned char* w = static_cast<unsigned char*>(ws);
-  float2* tab = reinterpret_cast<float2*>(w);
-  float* part_o = reinterpret_cast<float*>(w + p.tab_bytes);
-  float2* part_ml = reinterpret_cast<float2*>(w + p.tab_bytes + p.po_bytes);
-  decode_cs_table_kernel<<<(kTK * (kDim / 2) + 255) / 256, 256, 0, s>>>((double)rope_base, tab);
-  int rc = check_launch();
-  if (rc) return rc;
+  int* counters = reinterpret_cast<int*>(w);
+  float* part_o = reinterpret_cast<float*>(w + p.cnt_bytes);
+  float2* part_ml = reinterpret_cast<float2*>(w + p.cnt_bytes + p.po_bytes);
   CUtensorMap tkm, tvm, tkl, tvl;
   bool ok;
   if (fm) {  // the bank itself, 8-row boxes (one swizzle atom)
@@ -682,19 +862,21 @@ int launch_dtc(int B, int T_loc, int Hq, int H, const void* q, const void* k_mem
        tma_map_sw128_bf16(&tvl, v_loc, kDim, H, (int64_t)B * T_loc, 1, kTK);
   if (!ok) return note_cuda(cudaErrorInvalidValue);
   auto kern = fm ? attn_decode_tc_kernel<G, true> : attn_decode_tc_kernel<G, false>;
-  rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)DTS::ALLOC);
+  int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)DTS::ALLOC);
   if (rc) return rc;
-  const int64_t n_items = (int64_t)p.n_split * B * H;
-  if (n_items > INT32_MAX) return MSA_ERR_UNSUPPORTED;
-  const int grid = (int)std::min<int64_t>(n_items, num_sms());
+  const int64_t n_chunks = (int64_t)p.n_whole + (int64_t)p.n_tail * p.n_ch;
+  if (n_chunks > INT32_MAX) return MSA_ERR_UNSUPPORTED;
+  // the chunk counter and the arrival counters start at zero on every call
+  rc = note_cuda(cudaMemsetAsync(counters, 0, (size_t)(1 + p.n_tail) * sizeof(int), s));
+  if (rc) return rc;
+  const int grid = (int)std::min<int64_t>(n_chunks, num_sms());
   kern<<<grid, kTThreads, DTS::ALLOC, s>>>(
-      tkm, tvm, tkl, tvl, T_loc, Hq, H, (int)n_items, static_cast<const __nv_bfloat16*>(q),
-      fm ? fm->n_groups : mem_len, m_cap, fm ? fm->groups : nullptr, fm ? fm->max_groups : 0,
-      pos0, (double)rope_base, qscale, p.n_split, tab, static_cast<__nv_bfloat16*>(out), part_o,
-      part_ml, device_status_ptr());
-  rc = check_launch();
-  if (rc || p.n_split == 1) return rc;
-  return attn_combine_bf16(B, 1, Hq, kDim, p.n_split, part_o, part_ml, out, s);
+      tkm, tvm, tkl, tvl, T_loc, Hq, H, p.n_whole, p.n_tail, p.n_ch,
+      static_cast<const __nv_bfloat16*>(q), fm ? fm->n_groups : mem_len, m_cap,
+      fm ? fm->groups : nullptr, fm ? fm->max_groups : 0, rope_tab(rope_base, pos0, T_loc),
+      qscale,
+      counters, static_cast<__nv_bfloat16*>(out), part_o, part_ml, device_status_ptr());
+  return check_launch();
 }
 
 int dispatch_dtc(int B, int T_loc, int Hq, int H, int D, const void* q, const void* k_mem,

@@ -88,6 +88,26 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// Prefetch of a 3-D tile of the tensor map into the L2 cache (no shared
+// memory, no barrier): a later load of the same tile then finds it in L2.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int32_t x, int32_t y,
+                                                   int32_t z) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// 1-D bulk prefetch of `bytes` contiguous bytes into the L2 cache (address
+// 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
+}
+
 // 1-D bulk copy of `bytes` contiguous bytes from global memory into this
 // CTA's shared memory, completing on `bar` (both addresses 16-byte aligned,
 // bytes a multiple of 16).

@@ -563,6 +563,45 @@ def test_attention_prefill_tensor_core_shapes(B, T, T_loc, Hq, H, D, m_cap, mem_
     status_ok()
 
 
+def _prefill_sweep_points():
+    import bench
+    return list(bench.PREFILL_SWEEP)
+
+
+@pytest.mark.parametrize("B,T,M", _prefill_sweep_points())
+def test_attention_prefill_sweep_point_sampled(B, T, M):
+    """Each point of the benchmark's prefill sweep (T = T_loc up to 32K, B up
+    to 16), run at its own size with the inputs the sweep draws, checked on
+    sampled blocks of query rows: rows i0 .. i0+7 of a prefill of T tokens
+    are the last 8 rows of a prefill of i0+8 tokens over the same keys, so
+    the oracle computes them from that prefix (first rows, rows across the
+    first key-tile boundary, the middle and the last rows)."""
+    Hq, H, D, pos0 = 32, 8, 128, 16
+    g = torch.Generator(device="cuda").manual_seed(B * T)
+    dt = torch.bfloat16
+    q = synth.randn((B, T, Hq, D), dt, "cuda", g)
+    km = synth.randn((B, M, H, D), dt, "cuda", g)
+    vm = synth.randn((B, M, H, D), dt, "cuda", g)
+    kl = synth.randn((B, T, H, D), dt, "cuda", g)
+    vl = synth.randn((B, T, H, D), dt, "cuda", g)
+    ml = torch.full((B,), M, dtype=torch.int32, device="cuda")
+    att = pipeline.Attention(dt, B, T, T, Hq, H, D, M, "cuda")
+    out = att(q, km, vm, ml, kl, vl, pos0)
+    torch.cuda.synchronize()
+    worst = 0.0
+    for b in sorted({0, B - 1}):
+        for i0 in (0, 124, T // 2 - 4, T - 8):
+            i1 = i0 + 8
+            want = oracle.sparse_attn(f64(q[b:b + 1, i0:i1]), [f64(km[b])], [f64(vm[b])],
+                                      f64(kl[b:b + 1, :i1]), f64(vl[b:b + 1, :i1]), pos0,
+                                      10000.0)
+            got = f64(out[b:b + 1, i0:i1])
+            assert np.all(np.isfinite(got))
+            worst = max(worst, float(np.max(np.abs(got - want))))
+    assert worst <= ATTN_BF16, worst
+    status_ok()
+
+
 @pytest.mark.parametrize("B,T_loc,Hq,H,m_cap,mem_lens", [
     (3, 1, 32, 8, 70, [70, 0, 65]),         # one local token, ragged memory tile
     (2, 65, 8, 8, 64, [64, 1]),             # G = 1, local tail of one key
