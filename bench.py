@@ -339,6 +339,9 @@ def run_libmsa(args, world, rank, local):
         "roofline": {"bound": "tensor",
                      "kernel": "route_tc_kernel on CTA pairs, prepared bank "
                                "(msa_route_scores_prepared call)",
+                     "bank": "unit rows, the bytes msa_encode_pool_prepared writes when it "
+                             "pools the bank (drawn here at chunk level, prepared by "
+                             "msa_route_prepare_bank: 100M token rows would take 600 GB)",
                      "achieved": round(route_tf, 1), "peak": pk["bf16"], "unit": "TFLOP/s",
                      "frac": round(route_tf / pk["bf16"], 4),
                      "peak_kind": "burst bf16 (the timed region is tens of milliseconds, "
@@ -658,10 +661,13 @@ def bench_bank_1m(steps: int, pk: dict) -> dict:
     coff = pipeline.chunk_offsets(toff)
     coff_h = coff.cpu()
     C = int(coff_h[-1])
-    kb, vb, rb = pipeline.encode_pool(w["k_tok"], w["v_tok"], w["kr_tok"], toff, coff, C)
+    # the memory is built by one pass of msa_encode_pool_prepared: pooled K̄, V̄
+    # and the prepared routing bank, no raw K̄_r and no separate preparation
+    kb, vb, rh, _ = pipeline.encode_pool_prepared(w["k_tok"], w["v_tok"], w["kr_tok"], toff,
+                                                  coff, C)
     for name in ("k_tok", "v_tok", "kr_tok"):
         del w[name]
-    hat = pipeline.prepare_bank(rb[0])
+    hat = rh[0]
     m_cap = w["k"] * int((coff_h[1:] - coff_h[:-1]).max())
     p = pipeline.Pipeline(hat, kb[0], vb[0], coff, B=1, T=w["T"], T_loc=w["T_loc"], Hq=w["Hq"],
                           k=w["k"], m_cap=m_cap, pos0=w["pos0"], prepared=True)
@@ -689,8 +695,9 @@ def bench_bank_1m(steps: int, pk: dict) -> dict:
     attn_flops = attn_flops_per_step(p)
     hbm = lambda b, t: round(b / (t * 1e-3) / 1e9 / pk["hbm"], 4)  # noqa: E731
     res = {"workload": "bank_1m: 1,000 token-level docs of U[256,1792] tokens encoded by "
-                       "msa_encode_pool (16,312 chunks), 4 planted needles; one 128-token "
-                       "prefill query, 128 local tokens, top-16",
+                       "msa_encode_pool_prepared (16,312 chunks; K̄, V̄ and the prepared "
+                       "routing bank in one pass), 4 planted needles; one 128-token prefill "
+                       "query, 128 local tokens, top-16",
            "ms_per_step": round(ms, 4), "gchunks_s": round(C / (ms * 1e-3) / 1e9, 4),
            "l2": "flushed (256 MB write) before every timed call",
            "stages_ms": {"route": round(ms_route, 4), "topk": round(ms_topk, 4),
@@ -712,7 +719,7 @@ def bench_bank_1m(steps: int, pk: dict) -> dict:
                              "frac": round(attn_flops / (ms_attn * 1e-3) / 1e12 / pk["bf16"], 5),
                              "note": "0.4 GFLOP: latency-bound"},
            "n_chunks": C, "mem_rows": rows}
-    del graph, p, w, kb, vb, rb, hat, scratch
+    del graph, p, w, kb, vb, rh, hat, scratch
     torch.cuda.empty_cache()
     return res
 

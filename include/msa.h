@@ -161,6 +161,28 @@ int msa_encode_pool(msa_dtype dt, int L, int64_t n_tok, int n_docs, int H,
                     float rope_base, int chunk, void* k_bar, void* v_bar,
                     void* kr_bar, msa_stream_t stream);
 
+/* Memory encoding that also writes the prepared routing bank -- [HYSEN]
+ * §"Memory must be encoded offline before a query can reach it": the routing
+ * keys' per-row normalisation depends on the bank alone, so it is done in
+ * the same pass that pools them.  As msa_encode_pool (same arguments,
+ * layouts and limits), plus:
+ *   kr_hat  [L][n_chunks][H][D] bf16, written: each (chunk, head) row of
+ *           K̄_r (as rounded to bf16) divided by max(|row|, 1e-12) and
+ *           rounded to bf16 -- byte for byte what msa_route_prepare_bank
+ *           writes from K̄_r, ready for msa_route_scores_prepared;
+ *   kr_bar  may be NULL: then only the prepared bank is kept, so building
+ *           the memory takes one pass and one routing bank (the raw K̄_r is
+ *           needed only by msa_route_backward).
+ * bf16 only (MSA_ERR_UNSUPPORTED otherwise); always runs the bulk-copy
+ * pooling kernel, whatever MSA_ENCODE_TMA says.  kr_hat may not alias any
+ * other argument. */
+int msa_encode_pool_prepared(msa_dtype dt, int L, int64_t n_tok, int n_docs, int H,
+                             int D, const void* k_tok, const void* v_tok,
+                             const void* kr_tok, const int64_t* tok_offsets,
+                             const int64_t* chunk_offsets, int64_t n_chunks,
+                             float rope_base, int chunk, void* k_bar, void* v_bar,
+                             void* kr_bar, void* kr_hat, msa_stream_t stream);
+
 /* Routing -- [HYSEN] §"Routing happens inside attention ...": relevance is
  * the cosine similarity of Q_r and K̄_r, averaged over heads, then the
  * maximum over query tokens; [DEEP] §"五、推理阶段" Step 2.  A document's

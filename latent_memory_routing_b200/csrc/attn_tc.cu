@@ -45,6 +45,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdlib>
 
 #include "attn_tc.cuh"
@@ -529,9 +530,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // with 16-byte loads of an element group and its rotate-half partner.
 constexpr int kPosPerCta = 4;
 
+// Inverse frequencies base^(-2i/D) of a call, computed on the host: the
+// kernel keeps only the one double multiply and reduction per (position,
+// pair) that an exact angle needs (FP64 is slow on this part, and a double
+// pow per thread held the kernel up by microseconds).
+struct FreqTab {
+  double w[64];
+};
+
 template <int D>
 __global__ void __launch_bounds__(256)
-rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0, double base,
+rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0,
+                 const __grid_constant__ FreqTab freq,
                  const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_loc,
                  __nv_bfloat16* __restrict__ q_rot, __nv_bfloat16* __restrict__ k_rot) {
   constexpr int HALF = D / 2;
@@ -541,7 +551,7 @@ rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0, double ba
   const int np = min(kPosPerCta, T_loc - p0);
   for (int e = threadIdx.x; e < np * HALF; e += blockDim.x) {
     const int j = e / HALF, i = e % HALF;
-    cs[j][i] = rope_cs(pos0 + p0 + j, rope_inv_freq(base, i, D));
+    cs[j][i] = rope_cs(pos0 + p0 + j, freq.w[i]);
   }
   __syncthreads();
   // local keys: B x np positions x H heads x UPH units
@@ -690,8 +700,10 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   __nv_bfloat16* k_rot = reinterpret_cast<__nv_bfloat16*>(w + p.q_bytes);
   float* part_o = reinterpret_cast<float*>(w + p.q_bytes + p.k_bytes);
   float2* part_ml = reinterpret_cast<float2*>(w + p.q_bytes + p.k_bytes + p.po_bytes);
+  FreqTab freq;
+  for (int i = 0; i < D / 2; ++i) freq.w[i] = std::pow((double)rope_base, -2.0 * i / D);
   rope_prep_kernel<D><<<(unsigned)((T_loc + kPosPerCta - 1) / kPosPerCta), 256, 0, s>>>(
-      B, T, T_loc, Hq, H, pos0, (double)rope_base, static_cast<const __nv_bfloat16*>(q),
+      B, T, T_loc, Hq, H, pos0, freq, static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k_loc), q_rot, k_rot);
   int rc = check_launch();
   if (rc) return rc;

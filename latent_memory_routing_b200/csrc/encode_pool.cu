@@ -173,7 +173,7 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
                   const T* __restrict__ kr_tok, const int64_t* __restrict__ tok_off,
                   const int64_t* __restrict__ chunk_off, int64_t n_chunks, double base,
                   int chunk, T* __restrict__ k_bar, T* __restrict__ v_bar,
-                  T* __restrict__ kr_bar, int* status) {
+                  T* __restrict__ kr_bar, T* __restrict__ kr_hat, int* status) {
   constexpr int VEC = Vec16<T>::N;
   constexpr int HALF = D / 2;
   constexpr int UPH = HALF / VEC;
@@ -338,15 +338,49 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&empty[st]);
         }
-        if (active) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          a1[e] *= inv_n;
+          a2[e] *= inv_n;
+        }
+        const uint4 p1 = Vec16<T>::pack(a1), p2 = Vec16<T>::pack(a2);
+        const int64_t o_off = ((int64_t)l * n_chunks + c) * row_elems + col_lo;
+        if (active && dst) {
+          st16(dst + o_off, p1);
+          st16(dst + o_off + HALF, p2);
+        }
+        if (t == 2 && kr_hat) {
+          // the prepared routing row: the (chunk, head) row of K̄_r as
+          // rounded above, divided by max(|row|, 1e-12) and rounded again --
+          // the arithmetic of the bank preparation step in the same order
+          // (fp32 squares of each 8-element piece, the pieces v and v + UPH
+          // of this thread added, then a butterfly over the head's UPH
+          // threads, which sit on consecutive lanes), so the bytes are those
+          // msa_route_prepare_bank writes from K̄_r.  Whole warps take part
+          // in the shuffles (an inactive lane holds zeros in its own head
+          // group).
+          float f1[VEC], f2[VEC];
+          Vec16<T>::unpack(p1, f1);
+          Vec16<T>::unpack(p2, f2);
+          float s1 = 0.f, s2 = 0.f;
 #pragma unroll
           for (int e = 0; e < VEC; ++e) {
-            a1[e] *= inv_n;
-            a2[e] *= inv_n;
+            s1 = fmaf(f1[e], f1[e], s1);
+            s2 = fmaf(f2[e], f2[e], s2);
           }
-          T* o = dst + ((int64_t)l * n_chunks + c) * row_elems + col_lo;
-          st16(o, Vec16<T>::pack(a1));
-          st16(o + HALF, Vec16<T>::pack(a2));
+          float ss = s1 + s2;
+#pragma unroll
+          for (int o = UPH / 2; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          const float inv = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            f1[e] *= inv;
+            f2[e] *= inv;
+          }
+          if (active) {
+            st16(kr_hat + o_off, Vec16<T>::pack(f1));
+            st16(kr_hat + o_off + HALF, Vec16<T>::pack(f2));
+          }
         }
       }
     }
@@ -392,14 +426,16 @@ __global__ void chunk_offsets_kernel(int n_docs, const int64_t* __restrict__ tok
   }
 }
 
+// rh (the prepared routing bank) != nullptr: bf16 only, and always on the
+// bulk-copy kernel.
 template <typename T, int D>
 int launch_encode(int L, int64_t n_tok, int n_docs, int H, const void* k,
                   const void* v, const void* kr, const int64_t* toff,
                   const int64_t* coff, int64_t n_chunks, float base, int chunk,
-                  void* kb, void* vb, void* rb, cudaStream_t s) {
+                  void* kb, void* vb, void* rb, void* rh, cudaStream_t s) {
   constexpr int VEC = Vec16<T>::N;
   const int64_t row_bytes = (int64_t)H * D * (int64_t)sizeof(T);
-  if (encode_tma_enabled() && row_bytes % 16 == 0 && row_bytes <= kEncStage) {
+  if ((encode_tma_enabled() || rh) && row_bytes % 16 == 0 && row_bytes <= kEncStage) {
     const int U = H * (D / 2 / VEC);
     const int Ug = (U + 31) / 32 * 32;
     const int RS = (int)std::min<int64_t>(chunk, kEncStage / row_bytes);
@@ -413,9 +449,11 @@ int launch_encode(int L, int64_t n_tok, int n_docs, int H, const void* k,
     kern<<<grid, 32 + 3 * Ug, smem, s>>>(
         L, n_tok, n_docs, H, U, Ug, RS, static_cast<const T*>(k), static_cast<const T*>(v),
         static_cast<const T*>(kr), toff, coff, n_chunks, (double)base, chunk,
-        static_cast<T*>(kb), static_cast<T*>(vb), static_cast<T*>(rb), device_status_ptr());
+        static_cast<T*>(kb), static_cast<T*>(vb), static_cast<T*>(rb), static_cast<T*>(rh),
+        device_status_ptr());
     return check_launch();
   }
+  if (rh) return MSA_ERR_UNSUPPORTED;
   const int U = H * (D / 2 / VEC);
   const int R = U >= kEncThreads ? 1 : kEncThreads / U;
   const int threads = U * R;
@@ -449,6 +487,51 @@ extern "C" int msa_chunk_offsets(int n_docs, const int64_t* tok_offsets,
   return msa::debug_finish(msa::check_launch(), s);
 }
 
+namespace msa {
+namespace {
+
+int encode_pool_impl(msa_dtype dt, int L, int64_t n_tok, int n_docs, int H, int D,
+                     const void* k_tok, const void* v_tok, const void* kr_tok,
+                     const int64_t* tok_offsets, const int64_t* chunk_offsets, int64_t n_chunks,
+                     float rope_base, int chunk, void* k_bar, void* v_bar, void* kr_bar,
+                     void* kr_hat, cudaStream_t s) {
+  if (L <= 0 || n_tok <= 0 || n_docs <= 0 || n_chunks < 0 || H <= 0) return MSA_ERR_INVALID_ARG;
+  if (!k_tok || !v_tok || !kr_tok || !tok_offsets || !chunk_offsets || !k_bar || !v_bar ||
+      (!kr_bar && !kr_hat))
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(k_tok) || !aligned16(v_tok) || !aligned16(kr_tok) || !aligned16(k_bar) ||
+      !aligned16(v_bar) || !aligned16(kr_bar) || !aligned16(kr_hat))
+    return MSA_ERR_INVALID_ARG;
+  if (chunk < 1 || chunk > kMaxChunk || !(rope_base > 0.f)) return MSA_ERR_INVALID_ARG;
+  if (H < 1 || H > 16 || (D != 64 && D != 128)) return MSA_ERR_UNSUPPORTED;
+  if (n_chunks > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
+  if (dt != MSA_F32 && dt != MSA_BF16) return MSA_ERR_INVALID_ARG;
+  if (kr_hat && dt != MSA_BF16) return MSA_ERR_UNSUPPORTED;
+  if (int rc = debug_check_offsets(tok_offsets, n_docs, n_tok, s)) return rc;
+  if (int rc = debug_check_offsets(chunk_offsets, n_docs, n_chunks, s)) return rc;
+  int rc;
+  if (dt == MSA_F32)
+    rc = D == 64 ? launch_encode<float, 64>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
+                                            tok_offsets, chunk_offsets, n_chunks, rope_base,
+                                            chunk, k_bar, v_bar, kr_bar, nullptr, s)
+                 : launch_encode<float, 128>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
+                                             tok_offsets, chunk_offsets, n_chunks, rope_base,
+                                             chunk, k_bar, v_bar, kr_bar, nullptr, s);
+  else
+    rc = D == 64 ? launch_encode<__nv_bfloat16, 64>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
+                                                    tok_offsets, chunk_offsets, n_chunks,
+                                                    rope_base, chunk, k_bar, v_bar, kr_bar,
+                                                    kr_hat, s)
+                 : launch_encode<__nv_bfloat16, 128>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
+                                                     tok_offsets, chunk_offsets, n_chunks,
+                                                     rope_base, chunk, k_bar, v_bar, kr_bar,
+                                                     kr_hat, s);
+  return debug_finish(rc, s);
+}
+
+}  // namespace
+}  // namespace msa
+
 extern "C" int msa_encode_pool(msa_dtype dt, int L, int64_t n_tok, int n_docs,
                                int H, int D, const void* k_tok,
                                const void* v_tok, const void* kr_tok,
@@ -456,35 +539,20 @@ extern "C" int msa_encode_pool(msa_dtype dt, int L, int64_t n_tok, int n_docs,
                                const int64_t* chunk_offsets, int64_t n_chunks,
                                float rope_base, int chunk, void* k_bar,
                                void* v_bar, void* kr_bar, msa_stream_t stream) {
-  using namespace msa;
-  if (L <= 0 || n_tok <= 0 || n_docs <= 0 || n_chunks < 0 || H <= 0) return MSA_ERR_INVALID_ARG;
-  if (!k_tok || !v_tok || !kr_tok || !tok_offsets || !chunk_offsets || !k_bar ||
-      !v_bar || !kr_bar)
-    return MSA_ERR_INVALID_ARG;
-  if (!aligned16(k_tok) || !aligned16(v_tok) || !aligned16(kr_tok) ||
-      !aligned16(k_bar) || !aligned16(v_bar) || !aligned16(kr_bar))
-    return MSA_ERR_INVALID_ARG;
-  if (chunk < 1 || chunk > kMaxChunk || !(rope_base > 0.f)) return MSA_ERR_INVALID_ARG;
-  if (H < 1 || H > 16 || (D != 64 && D != 128)) return MSA_ERR_UNSUPPORTED;
-  if (n_chunks > 0x7fffffffLL) return MSA_ERR_UNSUPPORTED;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dt != MSA_F32 && dt != MSA_BF16) return MSA_ERR_INVALID_ARG;
-  if (int rc = debug_check_offsets(tok_offsets, n_docs, n_tok, s)) return rc;
-  if (int rc = debug_check_offsets(chunk_offsets, n_docs, n_chunks, s)) return rc;
-  int rc;
-  if (dt == MSA_F32)
-    rc = D == 64 ? launch_encode<float, 64>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
-                                            tok_offsets, chunk_offsets, n_chunks, rope_base,
-                                            chunk, k_bar, v_bar, kr_bar, s)
-                 : launch_encode<float, 128>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
-                                             tok_offsets, chunk_offsets, n_chunks, rope_base,
-                                             chunk, k_bar, v_bar, kr_bar, s);
-  else
-    rc = D == 64 ? launch_encode<__nv_bfloat16, 64>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
-                                                    tok_offsets, chunk_offsets, n_chunks,
-                                                    rope_base, chunk, k_bar, v_bar, kr_bar, s)
-                 : launch_encode<__nv_bfloat16, 128>(L, n_tok, n_docs, H, k_tok, v_tok, kr_tok,
-                                                     tok_offsets, chunk_offsets, n_chunks,
-                                                     rope_base, chunk, k_bar, v_bar, kr_bar, s);
-  return debug_finish(rc, s);
+  if (!kr_bar) return MSA_ERR_INVALID_ARG;
+  return msa::encode_pool_impl(dt, L, n_tok, n_docs, H, D, k_tok, v_tok, kr_tok, tok_offsets,
+                               chunk_offsets, n_chunks, rope_base, chunk, k_bar, v_bar, kr_bar,
+                               nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int msa_encode_pool_prepared(msa_dtype dt, int L, int64_t n_tok, int n_docs, int H,
+                                        int D, const void* k_tok, const void* v_tok,
+                                        const void* kr_tok, const int64_t* tok_offsets,
+                                        const int64_t* chunk_offsets, int64_t n_chunks,
+                                        float rope_base, int chunk, void* k_bar, void* v_bar,
+                                        void* kr_bar, void* kr_hat, msa_stream_t stream) {
+  if (!kr_hat) return MSA_ERR_INVALID_ARG;
+  return msa::encode_pool_impl(dt, L, n_tok, n_docs, H, D, k_tok, v_tok, kr_tok, tok_offsets,
+                               chunk_offsets, n_chunks, rope_base, chunk, k_bar, v_bar, kr_bar,
+                               kr_hat, reinterpret_cast<cudaStream_t>(stream));
 }

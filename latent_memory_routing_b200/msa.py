@@ -58,6 +58,8 @@ _SIGS = {
     "msa_chunk_offsets": (c_i, [c_i, c_p, c_i, c_p, c_p]),
     "msa_encode_pool": (c_i, [c_i, c_i, c_i64, c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_p,
                               c_i64, c_f, c_i, c_p, c_p, c_p, c_p]),
+    "msa_encode_pool_prepared": (c_i, [c_i, c_i, c_i64, c_i, c_i, c_i, c_p, c_p, c_p, c_p, c_p,
+                                       c_i64, c_f, c_i, c_p, c_p, c_p, c_p, c_p]),
     "msa_route_workspace_size": (c_sz, [c_i, c_i, c_i, c_i, c_i]),
     "msa_route_scores": (c_i, [c_i, c_i, c_i, c_i, c_i, c_p, c_p, c_i64, c_p, c_i, c_p, c_p,
                                c_p, c_sz, c_p]),
@@ -252,6 +254,21 @@ def msa_encode_pool(dt, L, n_tok, n_docs, H, D, k_tok, v_tok, kr_tok, tok_offset
         dt, L, n_tok, n_docs, H, D, _ptr(k_tok), _ptr(v_tok), _ptr(kr_tok),
         _ptr(tok_offsets), _ptr(chunk_offsets), n_chunks, rope_base, chunk,
         _ptr(k_bar), _ptr(v_bar), _ptr(kr_bar), _stream(stream)))
+
+
+def msa_encode_pool_prepared(dt, L, n_tok, n_docs, H, D, k_tok, v_tok, kr_tok, tok_offsets,
+                             chunk_offsets, n_chunks, rope_base, chunk, k_bar, v_bar, kr_bar,
+                             kr_hat, stream=None):
+    for t, what in ((k_tok, "k_tok"), (v_tok, "v_tok"), (kr_tok, "kr_tok")):
+        _numel_ok(t, L * n_tok * H * D, what, _es(dt))
+    for t, what in ((k_bar, "k_bar"), (v_bar, "v_bar"), (kr_bar, "kr_bar"), (kr_hat, "kr_hat")):
+        _numel_ok(t, L * n_chunks * H * D, what, _es(dt))
+    _numel_ok(tok_offsets, n_docs + 1, "tok_offsets", I64)
+    _numel_ok(chunk_offsets, n_docs + 1, "chunk_offsets", I64)
+    _check("msa_encode_pool_prepared", lib().msa_encode_pool_prepared(
+        dt, L, n_tok, n_docs, H, D, _ptr(k_tok), _ptr(v_tok), _ptr(kr_tok),
+        _ptr(tok_offsets), _ptr(chunk_offsets), n_chunks, rope_base, chunk,
+        _ptr(k_bar), _ptr(v_bar), _ptr(kr_bar), _ptr(kr_hat), _stream(stream)))
 
 
 def msa_route_workspace_size(dt, B, T, H, D) -> int:

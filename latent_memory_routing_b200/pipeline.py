@@ -37,6 +37,25 @@ def encode_pool(k_tok, v_tok, kr_tok, tok_offsets, chunk_offs, n_chunks: int,
     return kb, vb, rb
 
 
+def encode_pool_prepared(k_tok, v_tok, kr_tok, tok_offsets, chunk_offs, n_chunks: int,
+                         rope_base: float = 10000.0, chunk: int = 64, keep_raw: bool = False,
+                         stream=None):
+    """bf16 token-level [L][N][H][D] -> pooled K̄, V̄ and the prepared routing
+    bank K̂_r (unit rows, what ``prepare_bank`` makes from K̄_r) in one pass;
+    with ``keep_raw`` the raw K̄_r too.  Returns (k_bar, v_bar, kr_hat,
+    kr_bar or None)."""
+    L, N, H, D = k_tok.shape
+    n_docs = tok_offsets.numel() - 1
+    mk = lambda: torch.empty((L, n_chunks, H, D), dtype=k_tok.dtype,  # noqa: E731
+                             device=k_tok.device)
+    kb, vb, rh = mk(), mk(), mk()
+    rb = mk() if keep_raw else None
+    _m.msa_encode_pool_prepared(dt_code(k_tok), L, N, n_docs, H, D, k_tok, v_tok, kr_tok,
+                                tok_offsets, chunk_offs, n_chunks, rope_base, chunk, kb, vb, rb,
+                                rh, stream)
+    return kb, vb, rh, rb
+
+
 def prepare_bank(kr_bar, out=None, stream=None):
     """Unit-normalised copy of a bf16 routing bank [C][H][D] (built once per
     bank; see msa_route_prepare_bank)."""

@@ -108,6 +108,44 @@ def test_encode_ragged(dtype, L, H, D, tol):
     status_ok()
 
 
+@pytest.mark.parametrize("L,H,D,keep_raw", [
+    (2, 8, 128, True), (1, 3, 128, False), (1, 4, 64, True), (3, 16, 128, False),
+])
+def test_encode_prepared_bank_equals_the_preparation_step(L, H, D, keep_raw):
+    """msa_encode_pool_prepared writes K̄ and V̄ as msa_encode_pool does and
+    the prepared routing bank byte for byte as msa_route_prepare_bank makes
+    it from K̄_r (H = 3 leaves idle lanes in the pooling kernel's head
+    groups; one document's routing keys are all zero, so its rows hit the
+    1e-12 floor); the prepared rows are the oracle's pooled K_r rows over
+    their norms, within the bf16 tolerance."""
+    lengths = [1, 5, 63, 64, 65, 127, 128, 129, 180, 300, 777, 2, 4000]
+    dtype = torch.bfloat16
+    g = torch.Generator(device="cuda").manual_seed(31 + H)
+    toff_c = synth.tok_offsets(torch.tensor(lengths))
+    N = int(toff_c[-1])
+    k, v, r = (synth.randn((L, N, H, D), dtype, "cuda", g) for _ in range(3))
+    r[:, int(toff_c[4]):int(toff_c[5])] = 0.0  # document 4: zero routing keys
+    toff = toff_c.cuda()
+    coff = pipeline.chunk_offsets(toff)
+    C = int(coff[-1])
+    kb, vb, rb = pipeline.encode_pool(k, v, r, toff, coff, C)
+    kb2, vb2, rh, rb2 = pipeline.encode_pool_prepared(k, v, r, toff, coff, C, keep_raw=keep_raw)
+    torch.cuda.synchronize()
+    assert torch.equal(kb, kb2) and torch.equal(vb, vb2)
+    assert (rb2 is not None) == keep_raw
+    if keep_raw:
+        assert torch.equal(rb, rb2)
+    for l in range(L):
+        assert torch.equal(rh[l], pipeline.prepare_bank(rb[l].contiguous()))
+    _, _, orr, ocoff = oracle.encode_pool(f64(k), f64(v), f64(r), toff_c.numpy(), 10000.0)
+    onorm = np.linalg.norm(orr, axis=-1, keepdims=True)
+    ounit = orr / np.maximum(onorm, 1e-12)
+    c4 = slice(int(ocoff[4]), int(ocoff[5]))
+    assert np.all(f64(rh)[:, c4] == 0.0)
+    assert normwise(f64(rh), ounit) <= RTOL_BF16
+    status_ok()
+
+
 def test_encode_tiny_workload_fp32():
     w = synth.tiny("cuda")
     toff = w["tok_offsets"].cuda()
