@@ -523,13 +523,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
 }
 
-// Global RoPE of the query and the local keys, one launch: CTA i owns local
-// positions [i*kPosPerCta, ...): it builds their (cos, sin) in shared memory
-// (angles reduced in double), then rotates every local K row and every query
-// row at those positions (query token t sits at local position T_loc - T + t)
-// with 16-byte loads of an element group and its rotate-half partner.
-constexpr int kPosPerCta = 4;
-
+// Global RoPE of the query and the local keys, one launch: CTA p owns local
+// position p (query token t sits at local position T_loc - T + t).  The
+// kernel is latency-bound at the sizes a step uses, so each thread issues
+// the loads of its first 16-byte unit (an element group and its rotate-half
+// partner) before the position's (cos, sin) are built in shared memory
+// (angle reduced in double, frequencies from the host), then rotates.
+//
 // Inverse frequencies base^(-2i/D) of a call, computed on the host: the
 // kernel keeps only the one double multiply and reduction per (position,
 // pair) that an exact angle needs (FP64 is slow on this part, and a double
@@ -541,59 +541,68 @@ struct FreqTab {
 template <int D>
 __global__ void __launch_bounds__(256)
 rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0,
-                 const __grid_constant__ FreqTab freq,
-                 const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_loc,
-                 __nv_bfloat16* __restrict__ q_rot, __nv_bfloat16* __restrict__ k_rot) {
+                 const __grid_constant__ FreqTab freq, const __nv_bfloat16* __restrict__ q,
+                 const __nv_bfloat16* __restrict__ k_loc, __nv_bfloat16* __restrict__ q_rot,
+                 __nv_bfloat16* __restrict__ k_rot) {
   constexpr int HALF = D / 2;
   constexpr int UPH = HALF / 8;  // 16-byte pair units per head
-  __shared__ float2 cs[kPosPerCta][HALF];
-  const int p0 = blockIdx.x * kPosPerCta;
-  const int np = min(kPosPerCta, T_loc - p0);
-  for (int e = threadIdx.x; e < np * HALF; e += blockDim.x) {
-    const int j = e / HALF, i = e % HALF;
-    cs[j][i] = rope_cs(pos0 + p0 + j, freq.w[i]);
-  }
-  __syncthreads();
-  // local keys: B x np positions x H heads x UPH units
-  const int nk = B * np * H * UPH;
-  for (int e = threadIdx.x; e < nk; e += blockDim.x) {
-    const int u = e % UPH, h = (e / UPH) % H, j = (e / (UPH * H)) % np, b = e / (UPH * H * np);
-    const int64_t off = (((int64_t)b * T_loc + p0 + j) * H + h) * D + u * 8;
+  __shared__ float2 cs[HALF];
+  const int p = blockIdx.x;
+  const int tq = p - (T_loc - T);  // query token at this position, if >= 0
+  const int nk = B * H * UPH;      // local-key units, then query units
+  const int n = nk + (tq >= 0 ? B * Hq * UPH : 0);
+  // unit e -> (source, destination offset, pair group)
+  auto unit = [&](int e, const __nv_bfloat16*& src, __nv_bfloat16*& dst, int64_t& off, int& u) {
+    if (e < nk) {
+      u = e % UPH;
+      const int h = (e / UPH) % H, b = e / (UPH * H);
+      off = (((int64_t)b * T_loc + p) * H + h) * D + u * 8;
+      src = k_loc;
+      dst = k_rot;
+    } else {
+      const int f = e - nk;
+      u = f % UPH;
+      const int h = (f / UPH) % Hq, b = f / (UPH * Hq);
+      off = (((int64_t)b * T + tq) * Hq + h) * D + u * 8;
+      src = q;
+      dst = q_rot;
+    }
+  };
+  auto rotate = [&](const uint4& a, const uint4& bq, __nv_bfloat16* dst, int64_t off, int u) {
     float x1[8], x2[8], y1[8], y2[8];
-    Vec16<__nv_bfloat16>::unpack(ldg16(k_loc + off), x1);
-    Vec16<__nv_bfloat16>::unpack(ldg16(k_loc + off + HALF), x2);
+    Vec16<__nv_bfloat16>::unpack(a, x1);
+    Vec16<__nv_bfloat16>::unpack(bq, x2);
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
-      const float2 c = cs[j][u * 8 + t];
+      const float2 c = cs[u * 8 + t];
       y1[t] = x1[t] * c.x - x2[t] * c.y;
       y2[t] = x2[t] * c.x + x1[t] * c.y;
     }
-    st16(k_rot + off, Vec16<__nv_bfloat16>::pack(y1));
-    st16(k_rot + off + HALF, Vec16<__nv_bfloat16>::pack(y2));
+    st16(dst + off, Vec16<__nv_bfloat16>::pack(y1));
+    st16(dst + off + HALF, Vec16<__nv_bfloat16>::pack(y2));
+  };
+  // the first unit's loads are in flight while the table is built
+  const int e0 = threadIdx.x;
+  const __nv_bfloat16* src0 = nullptr;
+  __nv_bfloat16* dst0 = nullptr;
+  int64_t off0 = 0;
+  int u0 = 0;
+  uint4 a0 = make_uint4(0, 0, 0, 0), b0 = a0;
+  if (e0 < n) {
+    unit(e0, src0, dst0, off0, u0);
+    a0 = ldg16(src0 + off0);
+    b0 = ldg16(src0 + off0 + HALF);
   }
-  // query tokens at these positions
-  const int first_q = T_loc - T;  // local position of query token 0
-  const int t_lo = max(p0, first_q) - first_q, t_hi = p0 + np - first_q;
-  if (t_hi <= t_lo) return;
-  const int nt = t_hi - t_lo;
-  const int nq = B * nt * Hq * UPH;
-  for (int e = threadIdx.x; e < nq; e += blockDim.x) {
-    const int u = e % UPH, h = (e / UPH) % Hq, tt = (e / (UPH * Hq)) % nt,
-              b = e / (UPH * Hq * nt);
-    const int t = t_lo + tt;
-    const int j = first_q + t - p0;
-    const int64_t off = (((int64_t)b * T + t) * Hq + h) * D + u * 8;
-    float x1[8], x2[8], y1[8], y2[8];
-    Vec16<__nv_bfloat16>::unpack(ldg16(q + off), x1);
-    Vec16<__nv_bfloat16>::unpack(ldg16(q + off + HALF), x2);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float2 c = cs[j][u * 8 + i];
-      y1[i] = x1[i] * c.x - x2[i] * c.y;
-      y2[i] = x2[i] * c.x + x1[i] * c.y;
-    }
-    st16(q_rot + off, Vec16<__nv_bfloat16>::pack(y1));
-    st16(q_rot + off + HALF, Vec16<__nv_bfloat16>::pack(y2));
+  for (int i = threadIdx.x; i < HALF; i += blockDim.x) cs[i] = rope_cs(pos0 + p, freq.w[i]);
+  __syncthreads();
+  if (e0 < n) rotate(a0, b0, dst0, off0, u0);
+  for (int e = e0 + blockDim.x; e < n; e += blockDim.x) {
+    const __nv_bfloat16* src;
+    __nv_bfloat16* dst;
+    int64_t off;
+    int u;
+    unit(e, src, dst, off, u);
+    rotate(ldg16(src + off), ldg16(src + off + HALF), dst, off, u);
   }
 }
 
@@ -702,7 +711,7 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   float2* part_ml = reinterpret_cast<float2*>(w + p.q_bytes + p.k_bytes + p.po_bytes);
   FreqTab freq;
   for (int i = 0; i < D / 2; ++i) freq.w[i] = std::pow((double)rope_base, -2.0 * i / D);
-  rope_prep_kernel<D><<<(unsigned)((T_loc + kPosPerCta - 1) / kPosPerCta), 256, 0, s>>>(
+  rope_prep_kernel<D><<<(unsigned)T_loc, 256, 0, s>>>(
       B, T, T_loc, Hq, H, pos0, freq, static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k_loc), q_rot, k_rot);
   int rc = check_launch();
