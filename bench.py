@@ -67,6 +67,77 @@ def peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
+class NvmlSampler:
+    """SM clock and clock-event reasons of this process's GPU polled through
+    NVML about every millisecond by a background thread between start() and
+    stop(), so that samples land inside a timed region of a few milliseconds
+    (nvidia-smi's 200 ms loop only brackets it).  The GPU is found by its PCI
+    bus id, so a restricted CUDA_VISIBLE_DEVICES does not mislead it."""
+    HW_SLOWDOWN, SW_THERMAL, HW_THERMAL, SW_POWER_CAP = 0x8, 0x20, 0x40, 0x4
+
+    def __init__(self, cuda_index: int):
+        import threading
+        self.samples, self.max_mhz, self.h, self.nvml = [], None, None, None
+        self.index = cuda_index
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(cuda_index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.index = pynvml.nvmlDeviceGetIndex(self.h)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
+        except Exception:
+            self.h = None
+        self.stop_ev = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _reasons(self):
+        f = getattr(self.nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        return f(self.h)
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append((self.nvml.nvmlDeviceGetClockInfo(self.h,
+                                                                      self.nvml.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:
+                return
+            self.stop_ev.wait(0.001)
+
+    def start(self):
+        if self.h is not None:
+            self.thread.start()
+        return self
+
+    def stop(self) -> dict | None:
+        if self.h is None:
+            return None
+        self.stop_ev.set()
+        self.thread.join(timeout=5)
+        if not self.samples:
+            return None
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in ((self.HW_SLOWDOWN, "hw_slowdown"),
+                              (self.HW_THERMAL, "hw_thermal_slowdown"),
+                              (self.SW_THERMAL, "sw_thermal_slowdown"),
+                              (self.SW_POWER_CAP, "sw_power_cap")):
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(x for x, _ in self.samples),
+                "sm_min_mhz": min(x for x, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(reasons), "source": "NVML, ~1 ms polling"}
+
+
 class Clocks:
     """nvidia-smi sampling of SM clocks and throttle reasons during the
     timed region."""
@@ -114,6 +185,17 @@ class Clocks:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "samples": len(sm),
                 "reasons": sorted(reasons)}
+
+
+def merge_clocks(nvml: dict | None, smi: dict) -> dict:
+    """The line's `clocks`: the NVML samples taken inside the timed region
+    when there are any (with nvidia-smi's bracketing samples beside them),
+    else nvidia-smi's; throttle reasons seen by either are reported."""
+    if not nvml:
+        return smi
+    return {**nvml, "reasons": sorted(set(nvml["reasons"]) | set(smi.get("reasons", []))
+                                      - {"nvidia-smi unavailable"}),
+            "nvidia_smi": smi}
 
 
 def dist_setup(n_gpus: int, force_group: bool = False):
@@ -243,15 +325,17 @@ def run_libmsa(args, world, rank, local):
     for _ in range(3):
         graph.replay()
     clocks = Clocks(local)
+    nv = NvmlSampler(local)
     barrier(world)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    nv.start()
     t_start.record()
     for _ in range(args.steps):
         graph.replay()
     t_end.record()
     barrier(world)
-    clk = clocks.stop()
+    clk = merge_clocks(nv.stop(), clocks.stop())
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     ms_step = total_ms / args.steps
     value = C / (ms_step * 1e-3) / 1e9
@@ -472,15 +556,17 @@ def run_memory_parallel(args, world, rank, local):
     seg = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(6)]
 
     clocks = Clocks(local)
+    nv = NvmlSampler(local)
     barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    nv.start()
     t0.record()
     for _ in range(args.steps):
         step()
     t1.record()
     barrier(world)
-    clk = clocks.stop()
+    clk = merge_clocks(nv.stop(), clocks.stop())
     ms_step = max_over_ranks(t0.elapsed_time(t1), world) / args.steps
 
     # end to end: the step's inputs uploaded from pinned host memory and the

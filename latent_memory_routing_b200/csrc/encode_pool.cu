@@ -283,6 +283,11 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
         asm volatile("bar.sync 1, %0;" ::"r"(Ug) : "memory");  // old table no longer read
         // frequency i: an exact anchor at p0 (angle reduced in double), then
         // one rotation by w_i per row, in double
+        // stored transposed within a row, [row][e][v] for frequency
+        // i = v * VEC + e, so that the threads of a head (consecutive v)
+        // read consecutive 8-byte words: no bank conflicts (read in the
+        // row's order [v * VEC + e], neighbouring threads' words sit 64 B
+        // apart and four of a head's eight threads share a bank)
         for (int i = jt; i < HALF; i += Ug) {
           const double w = w_tab[i];
           double sa, ca, sw, cw;
@@ -290,8 +295,9 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
           const double th = (double)p0 * w;
           sincos(fma(-rint(th * (1.0 / two_pi)), two_pi, th), &sa, &ca);
           sincos(w, &sw, &cw);
+          const int slot = (i % VEC) * UPH + i / VEC;
           for (int r = 0; r < rows; ++r) {
-            cs_tab[r * HALF + i] = make_float2((float)ca, (float)sa);
+            cs_tab[r * HALF + slot] = make_float2((float)ca, (float)sa);
             const double cn = ca * cw - sa * sw;
             sa = sa * cw + ca * sw;
             ca = cn;
@@ -310,6 +316,7 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
           const int nr = min(RS, rows - g * RS);
           if (active && !*abort_v) {
             const unsigned char* base_row = ring + (size_t)st * kEncStage;
+#pragma unroll 2
             for (int rr = 0; rr < nr; ++rr) {
               const unsigned char* row = base_row + (size_t)rr * row_bytes;
               const uint4 q1 = *reinterpret_cast<const uint4*>(row + col_lo * sizeof(T));
@@ -319,10 +326,10 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
               Vec16<T>::unpack(q1, x1);
               Vec16<T>::unpack(q2, x2);
               if (t == 0) {
-                const float2* cs = cs_tab + (g * RS + rr) * HALF + v * VEC;
+                const float2* cs = cs_tab + (g * RS + rr) * HALF + v;
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) {
-                  const float2 q = cs[e];
+                  const float2 q = cs[e * UPH];
                   a1[e] += x1[e] * q.x - x2[e] * q.y;
                   a2[e] += x2[e] * q.x + x1[e] * q.y;
                 }

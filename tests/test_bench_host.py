@@ -102,3 +102,19 @@ def test_cpu_baseline_visiting_order_is_a_spread_of_distinct_slices():
             assert order[:2] == [0, n // 2]
         if n in (2, 64):  # a power of two: every slice exactly once
             assert sorted(order) == list(range(n))
+
+
+def test_clock_merge_prefers_timed_region_samples():
+    nvml = {"sm_mhz": 1950.0, "sm_min_mhz": 1900, "sm_max_mhz": 1965, "samples": 12,
+            "reasons": ["sw_power_cap"], "source": "NVML, ~1 ms polling"}
+    smi = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "samples": 2, "reasons": ["hw_slowdown"]}
+    got = bench.merge_clocks(nvml, smi)
+    assert got["sm_mhz"] == 1950.0 and got["samples"] == 12
+    assert got["reasons"] == ["hw_slowdown", "sw_power_cap"]  # either source's reason is kept
+    assert got["nvidia_smi"] == smi
+    assert bench.merge_clocks(None, smi) is smi
+
+
+def test_nvml_sampler_without_a_gpu_reports_nothing():
+    s = bench.NvmlSampler(0).start()
+    assert s.stop() is None
