@@ -320,6 +320,28 @@ def run_libmsa(args, world, rank, local):
             seg[j] += e[j].elapsed_time(e[j + 1])
     seg = [x / args.steps for x in seg]
 
+    # ---- each stage's launches replayed from a graph of their own, the L2
+    # flushed before every replay (the eager times above include launch gaps)
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        scratch.fill_(1)
+
+    stage_fns = [
+        lambda: p.router(w["q_r"], p.kr_bar, p.coff, p.n_docs, p.doc_scores, None),
+        lambda: pipeline.topk_docs(p.doc_scores, p.k, p.idx, p.top, p.topk_ws),
+        lambda: pipeline.gather_kv(p.idx, p.coff, p.k_bar, p.v_bar, p.m_cap, p.k_mem, p.v_mem,
+                                   p.mem_len),
+        lambda: p.attn(w["q"], p.k_mem, p.v_mem, p.mem_len, w["k_loc"], w["v_loc"], p.pos0,
+                       p.rope_base, 0.0, p.out)]
+    seg_graph = []
+    for fn in stage_fns:
+        g = graph_of(fn)
+        seg_graph.append(time_device_flushed(g.replay, args.steps, flush))
+        del g
+    del scratch
+    p(w["q_r"], w["q"], w["k_loc"], w["v_loc"])  # leave the buffers of one whole step
+
     # ---- the step as one CUDA graph (ten launches), inputs resident in HBM
     graph = p.capture(w["q_r"], w["q"], w["k_loc"], w["v_loc"])
     for _ in range(3):
@@ -362,9 +384,34 @@ def run_libmsa(args, world, rank, local):
         graph_e2e.replay()
     e1.record()
     barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    e2e_serial_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
     e2e_same = bool(torch.equal(out_h, p.out.cpu()))
     del graph_e2e
+
+    # the same from host buffers through HostStream: each step's upload and
+    # read-back on their own streams, overlapping the neighbouring steps'
+    # compute (every step's copies stay inside the timed region)
+    hs = pipeline.HostStream(p)
+    outs_h = [torch.empty(p.out.shape, dtype=p.out.dtype).pin_memory() for _ in range(2)]
+    idxs_h = [torch.empty(p.idx.shape, dtype=p.idx.dtype).pin_memory() for _ in range(2)]
+    for i in range(4):
+        hs.step(host["q_r"], host["q"], host["k_loc"], host["v_loc"], outs_h[i % 2],
+                idxs_h[i % 2])
+    hs.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    hs.start_after(e0)
+    for i in range(args.steps):
+        hs.step(host["q_r"], host["q"], host["k_loc"], host["v_loc"], outs_h[i % 2],
+                idxs_h[i % 2])
+    e1.record(hs.down)
+    hs.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    e2e_same = e2e_same and bool(torch.equal(outs_h[(args.steps - 1) % 2], p.out.cpu()))
+    del hs
 
     # the same scan over the raw bank (rows normalised inside the scan)
     raw_router = pipeline.Router(torch.bfloat16, 1, w["T"], p.H, p.D, "cuda")
@@ -441,6 +488,10 @@ def run_libmsa(args, world, rank, local):
                       "gather": round(seg[2], 4), "attn": round(seg[3], 4),
                       "note": "eager launches with events between stages; the step "
                               "(ms_per_step) replays the same launches as one CUDA graph"},
+        "stages_graph_ms": {"route": round(seg_graph[0], 4), "topk": round(seg_graph[1], 4),
+                            "gather": round(seg_graph[2], 4), "attn": round(seg_graph[3], 4),
+                            "note": "each stage's launches replayed from a CUDA graph of their "
+                                    "own, the L2 flushed (256 MB write) before every replay"},
         "route_gchunks_s": round(C / (route_ms * 1e-3) / 1e9, 4),
         "fused_step": {"ms_per_step": round(fused_ms, 4),
                        "gchunks_s": round(C / (fused_ms * 1e-3) / 1e9, 4),
@@ -458,9 +509,16 @@ def run_libmsa(args, world, rank, local):
         "e2e": {"value": round(C / (e2e_ms * 1e-3) / 1e9, 4), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "same_output_as_step": e2e_same,
-                "note": "one CUDA graph per step from pinned host inputs to pinned host "
-                        "output (Pipeline.capture_from_host); Q and the local K/V upload "
-                        "under the routing"},
+                "note": "pipeline.HostStream: every step's inputs uploaded from pinned host "
+                        "memory and its output and selection read back into pinned host "
+                        "memory inside the timed region, on their own streams, overlapping "
+                        "the neighbouring steps' compute (double-buffered device buffers, "
+                        "two CUDA graphs)",
+                "serial": {"value": round(C / (e2e_serial_ms * 1e-3) / 1e9, 4),
+                           "ms_per_step": round(e2e_serial_ms, 4),
+                           "note": "one CUDA graph per step from pinned host inputs to pinned "
+                                   "host output (Pipeline.capture_from_host), steps one after "
+                                   "another: the Q_r upload and the read-back on the path"}},
         "gpu_launches": launches * args.steps,
         "gpu_launches_per_step": launches,
         "device_status": status,
@@ -712,6 +770,21 @@ def time_device(fn, steps: int) -> float:
     e1.record()
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / steps
+
+
+def graph_of(fn):
+    """fn's launches captured once (after an eager warm-up) as a CUDA graph."""
+    import torch
+    fn()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
 
 
 def time_device_flushed(fn, steps: int, flush) -> float:

@@ -319,3 +319,103 @@ class Pipeline:
         self.attn(q, self.k_mem, self.v_mem, self.mem_len, k_loc, v_loc, self.pos0,
                   self.rope_base, 0.0, self.out, stream)
         return self.out
+
+
+class HostStream:
+    """Consecutive steps of a Pipeline from pinned host buffers, with the
+    transfers off the compute stream: step i's inputs are uploaded on an
+    upload stream and its output and selected documents read back on a
+    download stream, so they overlap the compute of steps i-1 and i+1.  The
+    device-side inputs and outputs are double-buffered; each of the two
+    buffer sets has its step captured once as a CUDA graph (the Pipeline's
+    launches only, no copies), replayed on the compute stream.
+
+    ``step(q_r_h, q_h, k_loc_h, v_loc_h, out_h, idx_h)`` enqueues one step and
+    returns at once: the inputs are read from the given pinned host tensors
+    and the results written into ``out_h`` / ``idx_h`` (pinned) when the
+    step's read-back completes -- ``wait(i)`` waits for step i's read-back,
+    ``synchronize()`` for every step enqueued.  A caller may refill an input
+    buffer once ``inputs_consumed(i)`` says that step i's uploads are done.
+    Ordering between buffer sets: step i + 2 reuses step i's device buffers,
+    so its upload waits for step i's compute and its compute for step i's
+    read-back (events, no host wait)."""
+
+    def __init__(self, p: Pipeline):
+        self.p = p
+        dev = p.kr_bar.device
+        shapes = {"q_r": (p.B, p.T, p.H, p.D), "q": (p.B, p.T, p.Hq, p.D),
+                  "k_loc": (p.B, p.T_loc, p.H, p.D), "v_loc": (p.B, p.T_loc, p.H, p.D)}
+        dt = p.kr_bar.dtype
+        self.inputs = [{n: torch.empty(sh, dtype=dt, device=dev) for n, sh in shapes.items()}
+                       for _ in range(2)]
+        self.outs = [torch.empty_like(p.out) for _ in range(2)]
+        self.idxs = [torch.empty_like(p.idx) for _ in range(2)]
+        self.compute = torch.cuda.current_stream()
+        self.up = torch.cuda.Stream()
+        self.down = torch.cuda.Stream()
+        self.graphs = [self._capture(x) for x in range(2)]
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.ev_up, self.ev_comp, self.ev_down = ev(), ev(), ev()
+        self.fresh = [True, True]
+        self.n = 0
+
+    def _run(self, x):
+        p, d = self.p, self.inputs[x]
+        out = p.out
+        p.out = self.outs[x]  # the step's attention writes this set's output
+        try:
+            p(d["q_r"], d["q"], d["k_loc"], d["v_loc"])
+        finally:
+            p.out = out
+        self.idxs[x].copy_(p.idx)
+
+    def _capture(self, x):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self._run(x)
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self._run(x)
+        return g
+
+    def start_after(self, event):
+        """Makes the next step's uploads wait for `event` (e.g. the start of
+        a timed region recorded on the compute stream)."""
+        self.up.wait_event(event)
+
+    def step(self, q_r_h, q_h, k_loc_h, v_loc_h, out_h, idx_h) -> int:
+        x = self.n % 2
+        d = self.inputs[x]
+        with torch.cuda.stream(self.up):
+            if not self.fresh[x]:  # step n-2 has read these device inputs
+                self.up.wait_event(self.ev_comp[x])
+            for name, h in (("q_r", q_r_h), ("q", q_h), ("k_loc", k_loc_h), ("v_loc", v_loc_h)):
+                d[name].copy_(h, non_blocking=True)
+            self.ev_up[x].record(self.up)
+        self.compute.wait_event(self.ev_up[x])
+        if not self.fresh[x]:  # step n-2's outputs have been read back
+            self.compute.wait_event(self.ev_down[x])
+        with torch.cuda.stream(self.compute):
+            self.graphs[x].replay()
+            self.ev_comp[x].record(self.compute)
+        with torch.cuda.stream(self.down):
+            self.down.wait_event(self.ev_comp[x])
+            out_h.copy_(self.outs[x], non_blocking=True)
+            idx_h.copy_(self.idxs[x], non_blocking=True)
+            self.ev_down[x].record(self.down)
+        self.fresh[x] = False
+        self.n += 1
+        return self.n - 1
+
+    def inputs_consumed(self, i: int) -> bool:
+        return self.ev_up[i % 2].query() if i >= self.n - 2 else True
+
+    def wait(self, i: int):
+        if i >= self.n - 2:
+            self.ev_down[i % 2].synchronize()
+
+    def synchronize(self):
+        self.down.synchronize()
+        self.compute.synchronize()

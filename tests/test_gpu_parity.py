@@ -898,6 +898,39 @@ def test_pipeline_step_from_host_graph(fused):
     status_ok()
 
 
+def test_host_stream_steps_match_device_steps():
+    """HostStream runs consecutive steps from pinned host buffers with the
+    uploads and read-backs on their own streams (double-buffered device
+    buffers, two graphs): five steps with different inputs, each read back
+    while the next computes, give the device-resident step's bytes."""
+    H, D, Hq, T, k = 8, 128, 32, 64, 8
+    kr, coff, coff_h = _pooled_bank(300, 1, 900, H, D, torch.bfloat16, 61)
+    g = torch.Generator(device="cuda").manual_seed(62)
+    kb = synth.randn(kr.shape, torch.bfloat16, "cuda", g)
+    vb = synth.randn(kr.shape, torch.bfloat16, "cuda", g)
+    m_cap = k * int(np.diff(coff_h).max())
+    p = pipeline.Pipeline(kr, kb, vb, coff, B=1, T=T, T_loc=T, Hq=Hq, k=k, m_cap=m_cap, pos0=k)
+    shapes = {"q_r": (1, T, H, D), "q": (1, T, Hq, D), "k_loc": (1, T, H, D),
+              "v_loc": (1, T, H, D)}
+    steps = []
+    for i in range(5):
+        dev = {n: synth.randn(sh, torch.bfloat16, "cuda", g) for n, sh in shapes.items()}
+        host = {n: t.cpu().pin_memory() for n, t in dev.items()}
+        out_h = torch.empty((1, T, Hq, D), dtype=torch.bfloat16).pin_memory()
+        idx_h = torch.empty((1, k), dtype=torch.int32).pin_memory()
+        steps.append((dev, host, out_h, idx_h))
+    hs = pipeline.HostStream(p)
+    for dev, host, out_h, idx_h in steps:
+        hs.step(host["q_r"], host["q"], host["k_loc"], host["v_loc"], out_h, idx_h)
+    hs.synchronize()
+    for dev, host, out_h, idx_h in steps:
+        want = p(dev["q_r"], dev["q"], dev["k_loc"], dev["v_loc"])
+        torch.cuda.synchronize()
+        assert torch.equal(idx_h, p.idx.cpu())
+        assert torch.equal(out_h, want.cpu())
+    status_ok()
+
+
 def _oracle_route_bank(q64, bank, rows: int = 32768):
     """The oracle's routing over a device bank, upcast slice by slice (the
     whole bank in float64 would not fit in host memory)."""
