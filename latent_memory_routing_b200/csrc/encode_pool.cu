@@ -157,18 +157,40 @@ encode_pool_kernel(int L, int64_t n_tok, int n_docs, int H, int R,
 }
 
 constexpr int kEncStage = 16384;  // bytes per ring stage
-constexpr int kEncStages = 4;     // stages per tensor: one ring per consumer group
+constexpr int kEncStages = 4;     // stages per tensor stream: one ring per consumer group
+constexpr int kEncRing = 3 * kEncStages;  // stages in all rings
 
-// Threads: one producer warp + three consumer groups of Ug (U rounded up to
-// a warp) threads, U = H * (D/2) / VEC.
+// Streams: in bf16 with L >= 2 layers, K -- whose consumers also rotate, the
+// slowest of the three -- is split into two streams by layer parity, each
+// with its own ring of kEncStages / 2 stages and its own consumer group, so
+// twice the threads work on K and no partial sums have to be combined; V
+// and K_r keep one stream of kEncStages stages each.  Otherwise (one layer,
+// or fp32, whose four groups would not fit a CTA's threads) the three
+// tensors are one stream each.
+struct EncStreams {
+  bool split;
+  __host__ __device__ int count() const { return split ? 4 : 3; }
+  __host__ __device__ int tensor(int s) const { return split ? (s < 2 ? 0 : s - 1) : s; }
+  __host__ __device__ int stages(int s) const {
+    return split && s < 2 ? kEncStages / 2 : kEncStages;
+  }
+  __host__ __device__ int first_stage(int s) const {
+    return split ? (s < 2 ? s * (kEncStages / 2) : (s - 1) * kEncStages) : s * kEncStages;
+  }
+  // stream s carries layer l of its tensor
+  __host__ __device__ bool carries(int s, int l) const { return !split || s >= 2 || (l & 1) == s; }
+};
+
+// Threads: one producer warp + three or four consumer groups of Ug (U
+// rounded up to a warp) threads, U = H * (D/2) / VEC.
 template <typename T, int D>
 constexpr int enc_tma_max_threads() {
-  return 32 + 3 * (16 * (D / 2) / Vec16<T>::N);
+  return 32 + (sizeof(T) == 2 ? 4 : 3) * (16 * (D / 2) / Vec16<T>::N);
 }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(enc_tma_max_threads<T, D>(), 1)
-encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS,
+encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS, int split_k,
                   const T* __restrict__ k_tok, const T* __restrict__ v_tok,
                   const T* __restrict__ kr_tok, const int64_t* __restrict__ tok_off,
                   const int64_t* __restrict__ chunk_off, int64_t n_chunks, double base,
@@ -179,9 +201,10 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
   constexpr int UPH = HALF / VEC;
   extern __shared__ __align__(1024) unsigned char enc_dsm[];
   unsigned char* ring = tc::smem_align<1024>(enc_dsm);
-  // ring of tensor t: stages [t * kEncStages, (t + 1) * kEncStages)
-  float2* cs_tab = reinterpret_cast<float2*>(ring + 3 * kEncStages * kEncStage);  // [64][HALF]
-  __shared__ uint64_t full[3 * kEncStages], empty[3 * kEncStages];
+  // ring of stream s: stages [first_stage(s), first_stage(s) + stages(s))
+  float2* cs_tab = reinterpret_cast<float2*>(ring + kEncRing * kEncStage);  // [64][HALF]
+  __shared__ uint64_t full[kEncRing], empty[kEncRing];
+  const EncStreams S{split_k != 0};
   __shared__ double w_tab[HALF];
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -190,7 +213,7 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
   const int64_t cb = (int64_t)blockIdx.x * n_chunks / gridDim.x;
   const int64_t ce = (int64_t)(blockIdx.x + 1) * n_chunks / gridDim.x;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 3 * kEncStages; ++i) {
+    for (int i = 0; i < kEncRing; ++i) {
       tc::mbar_init(&full[i], 1);
       tc::mbar_init(&empty[i], Ug / 32);
     }
@@ -238,21 +261,23 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // lane t streams tensor t into its own ring, so that no ring waits
+    // lane s streams stream s into its own ring, so that no ring waits
     // behind another's slot
-    if (lane < 3) {
-      const int t = lane;
+    if (lane < S.count()) {
+      const int sidx = lane, t = S.tensor(sidx);
+      const int ns = S.stages(sidx), s0 = S.first_stage(sidx);
       const T* src = t == 0 ? k_tok : (t == 1 ? v_tok : kr_tok);
-      uint32_t u = 0;  // stages issued to this tensor's ring
+      uint32_t u = 0;  // stages issued to this stream's ring
       for (int64_t c = cb; c < ce; ++c) {
         int64_t tok0, p0;
         int rows;
         locate(c, tok0, rows, p0);
         const int nstg = (rows + RS - 1) / RS;
-        for (int l = 0; l < L; ++l)
+        for (int l = 0; l < L; ++l) {
+          if (!S.carries(sidx, l)) continue;
           for (int g = 0; g < nstg; ++g, ++u) {
-            const int st = t * kEncStages + (int)(u % kEncStages);
-            wait(&empty[st], ((u / kEncStages) & 1) ^ 1);
+            const int st = s0 + (int)(u % ns);
+            wait(&empty[st], ((u / ns) & 1) ^ 1);
             if (*abort_v) continue;
             const int nr = min(RS, rows - g * RS);
             tc::mbar_arrive_expect_tx(&full[st], (uint32_t)nr * row_bytes);
@@ -260,15 +285,20 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
                           src + ((int64_t)l * n_tok + tok0 + (int64_t)g * RS) * row_elems,
                           (uint32_t)nr * row_bytes, &full[st]);
           }
+        }
       }
       // every copy issued must land before the CTA exits
-      for (uint32_t v = u > (uint32_t)kEncStages ? u - kEncStages : 0; v < u; ++v)
-        tc::mbar_wait(&full[t * kEncStages + v % kEncStages], (v / kEncStages) & 1);
+      for (uint32_t v = u > (uint32_t)ns ? u - ns : 0; v < u; ++v)
+        tc::mbar_wait(&full[s0 + v % ns], (v / ns) & 1);
     }
   } else {
     // ----------------------------------------------------------- consumers
-    const int t = (warp - 1) / (Ug / 32);         // 0: K, 1: V, 2: K_r
-    const int jt = (int)threadIdx.x - 32 - t * Ug;  // index in the group
+    const int sidx = (warp - 1) / (Ug / 32);         // the group's stream
+    const int t = S.tensor(sidx);                    // 0: K, 1: V, 2: K_r
+    const int ns = S.stages(sidx), s0 = S.first_stage(sidx);
+    const int jt = (int)threadIdx.x - 32 - sidx * Ug;  // index in the group
+    const int nk = S.split ? 2 : 1;                  // groups working on K
+    const int jk = jt + (t == 0 && S.split ? sidx : 0) * Ug;  // index among them
     const bool active = jt < U;
     const int h = jt / UPH, v = jt % UPH;
     const int64_t col_lo = (int64_t)h * D + v * VEC;
@@ -279,8 +309,8 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
       int rows;
       locate(c, tok0, rows, p0);
       const int nstg = (rows + RS - 1) / RS;
-      if (t == 0) {  // the K group rebuilds the chunk's (cos, sin) table
-        asm volatile("bar.sync 1, %0;" ::"r"(Ug) : "memory");  // old table no longer read
+      if (t == 0) {  // the K groups rebuild the chunk's (cos, sin) table
+        asm volatile("bar.sync 1, %0;" ::"r"(nk * Ug) : "memory");  // old table no longer read
         // frequency i: an exact anchor at p0 (angle reduced in double), then
         // one rotation by w_i per row, in double
         // stored transposed within a row, [row][e][v] for frequency
@@ -288,7 +318,7 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
         // read consecutive 8-byte words: no bank conflicts (read in the
         // row's order [v * VEC + e], neighbouring threads' words sit 64 B
         // apart and four of a head's eight threads share a bank)
-        for (int i = jt; i < HALF; i += Ug) {
+        for (int i = jk; i < HALF; i += nk * Ug) {
           const double w = w_tab[i];
           double sa, ca, sw, cw;
           const double two_pi = 6.283185307179586;
@@ -303,16 +333,17 @@ encode_tma_kernel(int L, int64_t n_tok, int n_docs, int H, int U, int Ug, int RS
             ca = cn;
           }
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(Ug) : "memory");
+        asm volatile("bar.sync 1, %0;" ::"r"(nk * Ug) : "memory");
       }
       const float inv_n = rows > 0 ? 1.0f / (float)rows : 0.f;
       for (int l = 0; l < L; ++l) {
+        if (!S.carries(sidx, l)) continue;
         float a1[VEC], a2[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) a1[e] = a2[e] = 0.f;
         for (int g = 0; g < nstg; ++g, ++u) {
-          const int st = t * kEncStages + (int)(u % kEncStages);
-          wait(&full[st], (u / kEncStages) & 1);
+          const int st = s0 + (int)(u % ns);
+          wait(&full[st], (u / ns) & 1);
           const int nr = min(RS, rows - g * RS);
           if (active && !*abort_v) {
             const unsigned char* base_row = ring + (size_t)st * kEncStage;
@@ -447,14 +478,15 @@ int launch_encode(int L, int64_t n_tok, int n_docs, int H, const void* k,
     const int Ug = (U + 31) / 32 * 32;
     const int RS = (int)std::min<int64_t>(chunk, kEncStage / row_bytes);
     const size_t smem =
-        1024 + (size_t)3 * kEncStages * kEncStage + sizeof(float2) * kMaxChunk * (D / 2);
+        1024 + (size_t)kEncRing * kEncStage + sizeof(float2) * kMaxChunk * (D / 2);
     auto kern = encode_tma_kernel<T, D>;
     int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)smem);
     if (rc) return rc;
     if (n_chunks == 0) return MSA_OK;
     const int grid = (int)std::min<int64_t>(n_chunks, num_sms());
-    kern<<<grid, 32 + 3 * Ug, smem, s>>>(
-        L, n_tok, n_docs, H, U, Ug, RS, static_cast<const T*>(k), static_cast<const T*>(v),
+    const bool split = sizeof(T) == 2 && L >= 2;
+    kern<<<grid, 32 + EncStreams{split}.count() * Ug, smem, s>>>(
+        L, n_tok, n_docs, H, U, Ug, RS, split ? 1 : 0, static_cast<const T*>(k), static_cast<const T*>(v),
         static_cast<const T*>(kr), toff, coff, n_chunks, (double)base, chunk,
         static_cast<T*>(kb), static_cast<T*>(vb), static_cast<T*>(rb), static_cast<T*>(rh),
         device_status_ptr());
