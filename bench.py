@@ -1214,19 +1214,20 @@ CASES = {
     "prefill_b1_t256": dict(B=1, T=256, T_loc=256, M=273),  # the bank_100m step's attention
     "route_bank_10m_b64": None,  # routing, not attention: see run_route_case
     "topk_b1_100k": None,        # the bank_100m step's top-16: see run_topk_case
-    "encode_l1_t400k": None,     # the encode_4l recipe cut to 1 layer x 400K tokens: run_encode_case
+    "encode_l2_t200k": None,     # the encode_4l recipe cut to 2 layers x 200K tokens: run_encode_case
 }
 
 
 def run_encode_case():
-    """Chunk pooling over 1 layer x 400,000 tokens of the encode_4l recipe
-    (2.5 GB of token rows, above the L2), three calls."""
+    """Chunk pooling over 2 layers x 200,000 tokens of the encode_4l recipe
+    (2.5 GB of token rows, above the L2; two layers, so the K stream is split
+    by layer parity as in the 4-layer workload), three calls."""
     import torch
 
     from latent_memory_routing_b200 import build as _b
     from latent_memory_routing_b200 import pipeline, synth
     _b.build()
-    w = synth.encode_4l("cuda", L=1, n_tok=400_000)
+    w = synth.encode_4l("cuda", L=2, n_tok=200_000)
     toff = w["tok_offsets"].cuda()
     coff = pipeline.chunk_offsets(toff)
     C = int(coff[-1])
@@ -1234,7 +1235,7 @@ def run_encode_case():
     for _ in range(3):
         out = pipeline.encode_pool(w["k_tok"], w["v_tok"], w["kr_tok"], toff, coff, C, out=out)
     torch.cuda.synchronize()
-    print(json.dumps({"case": "encode_l1_t400k", "n_chunks": C,
+    print(json.dumps({"case": "encode_l2_t200k", "n_chunks": C,
                       "kbar_abs_mean": float(out[0].float().abs().mean())}))
 
 
@@ -1287,7 +1288,7 @@ def run_case(name: str):
         return run_route_case()
     if name == "topk_b1_100k":
         return run_topk_case()
-    if name == "encode_l1_t400k":
+    if name == "encode_l2_t200k":
         return run_encode_case()
     _b.build()
     c = CASES[name]

@@ -9,17 +9,20 @@
 // K -> K̄, V -> V̄, K_r -> K̄_r by mean pooling, 180 tokens -> 3 chunks).
 //
 // Design (HBM-bound stream).  encode_tma_kernel (the default): persistent
-// CTAs, one per SM, each owning a contiguous range of chunks.  Three producer
-// threads stream, per (chunk, layer), the chunk's contiguous token rows of K,
-// V and K_r with 1-D bulk copies (cp.async.bulk, 16 KB stages, a four-stage
-// ring per tensor, so that each ring has one consumer group and a group
-// never waits on a slot another group's stage may still hold) -- the copy
-// engine keeps up to 192 KB in flight per SM without a load instruction per
-// 16 bytes; three consumer groups (one per tensor) each own
-// one 16-byte vector of a head and its rotate-half partner, add every row of
-// their tensor from shared memory into fp32 registers (K rotated by the
-// token's document-wise position from the chunk's (cos, sin) table) and write
-// the chunk's mean row once, so no partial sums cross threads.
+// CTAs, one per SM, each owning a contiguous range of chunks.  Producer
+// threads stream, per (chunk, layer), the chunk's contiguous token rows with
+// 1-D bulk copies (cp.async.bulk, 16 KB stages) into one ring per stream, so
+// that each ring has one consumer group and a group never waits on a slot
+// another group's stage may still hold -- the copy engine keeps 192 KB in
+// flight per SM without a load instruction per 16 bytes.  The streams are K,
+// V and K_r, except that in bf16 with two or more layers K -- whose consumers
+// also rotate -- is split into two streams by layer parity, each with its
+// own consumer group.  A consumer group's threads each own one 16-byte
+// vector of a head and its rotate-half partner, add every row of their
+// tensor from shared memory into fp32 registers (K rotated by the token's
+// document-wise position from the chunk's (cos, sin) table, laid out so that
+// a head's threads read consecutive words) and write the chunk's mean row
+// once, so no partial sums cross threads.
 // encode_pool_kernel (MSA_ENCODE_TMA=0): one CTA per chunk, looping over the
 // L layers so the chunk's RoPE table is built once.  Each thread owns two 16-byte vectors
 // of one head -- elements [v*VEC, v*VEC+VEC) and the rotate-half partners at
