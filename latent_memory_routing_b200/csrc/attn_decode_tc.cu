@@ -119,7 +119,7 @@ struct DTAux {
   // K and V tiles of a stage arrive and leave separately: a K slot is free
   // once S has read it, a V slot once P V has
   uint64_t kfull[kKSt], vfull[kVSt], kready[kKSt], kfree[kKSt], vfree[kVSt];
-  uint64_t sfull[2], pfull[2], pvdone[2], odone;
+  uint64_t sfull[2], sfree[2], pfull[2], pvdone[2], odone;
   uint64_t sched_full[kSched], sched_empty[kSched];
   int sched_id[kSched];
   uint32_t tmem_base;
@@ -341,6 +341,7 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&aux.sfull[i], 1);
+      tc::mbar_init(&aux.sfree[i], kSoftWarps);
       tc::mbar_init(&aux.pfull[i], kSoftWarps);
     }
     tc::mbar_init(&aux.pvdone[0], 1);
@@ -412,15 +413,16 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
   } else if (warp == 1) {
     // ------------------------------------------------------------- S MMA
     // S(u) as soon as its K tile is rotated (kready) and its TMEM buffer
-    // u&1 has been read by the softmax of tile u-2 (pfull of u-2): the P V
-    // stream, issued by its own warp, does not hold it back
+    // u&1 has been read by the softmax of tile u-2 (sfree of u-2, which the
+    // softmax signals as soon as S is in its registers): the P V stream,
+    // issued by its own warp, does not hold it back
     if (lane == 0) {
       Cur cs;
       int us = 0;
       for (bool hs = first(cs, 1); hs; hs = next(cs, 1), ++us) {
         const int st = us % kKSt;
         wait_or_abort(&aux.kready[st], (us / kKSt) & 1);
-        if (us >= 2) wait_or_abort(&aux.pfull[us & 1], ((us - 2) >> 1) & 1);
+        if (us >= 2) wait_or_abort(&aux.sfree[us & 1], ((us - 2) >> 1) & 1);
         tc::tc_fence_after();
         const uint32_t a0 = tc::smem_u32(ring + (size_t)st * kTileBytes);
         const uint32_t b0 =
@@ -479,6 +481,13 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       }
       wait_or_abort(&aux.sfull[u & 1], (u >> 1) & 1);
       tc::tc_fence_after();
+      uint32_t sv[16];
+      tc::tmem_ld16(tmem + lane_addr + (u & 1) * kNH, sv);
+      tc::tmem_ld_wait();
+      // S(u) is in registers: its TMEM buffer may take S(u + 2)
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&aux.sfree[u & 1]);
       bool valid = r < tile_valid(c);
       if (kFused && tile_mem(c)) {  // its group holds the row, and the row its document's
         const int grp = (tile_key0(c) + r) / 8;
@@ -500,9 +509,6 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
           *reinterpret_cast<uint4*>(vt + (cc >> 3) * kBlk + r * 128 + ((cc & 7) << 4)) =
               make_uint4(0, 0, 0, 0);
       }
-      uint32_t sv[16];
-      tc::tmem_ld16(tmem + lane_addr + (u & 1) * kNH, sv);
-      tc::tmem_ld_wait();
       float s[G];
       bool need = false;
 #pragma unroll
