@@ -149,6 +149,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
                float2* __restrict__ part_ml, int* __restrict__ status) {
   using K = ACfg<D>;
+  // launched as a programmatic dependent of the RoPE preparation: wait for
+  // its completion (and the visibility of its writes) before reading
+  // anything; a no-op when launched without that dependency
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ AAux aux;
   unsigned char* base = tc::smem_align<1024>(smem_dyn);
@@ -546,6 +550,9 @@ rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0,
                  __nv_bfloat16* __restrict__ k_rot) {
   constexpr int HALF = D / 2;
   constexpr int UPH = HALF / 8;  // 16-byte pair units per head
+  // the attention grid that follows may be scheduled now; it waits for this
+  // grid's completion before reading what this grid writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float2 cs[HALF];
   const int p = blockIdx.x;
   const int tq = p - (T_loc - T);  // query token at this position, if >= 0
@@ -737,11 +744,27 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   const int n_qb = (T + kQT * TQ - 1) / (kQT * TQ);
   if (n_qb > 65535 || B > 65535) return MSA_ERR_UNSUPPORTED;
   const dim3 grid((unsigned)(p.n_split * H), (unsigned)B, (unsigned)n_qb);
-  kern<<<grid, kThreads, K::SMEM, s>>>(tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G,
-                                       fm ? fm->n_groups : mem_len, m_cap,
-                                       fm ? fm->groups : nullptr, fm ? fm->max_groups : 0,
-                                       qscale, p.n_split, static_cast<__nv_bfloat16*>(out),
-                                       part_o, part_ml, device_status_ptr());
+  // programmatic dependent launch: the attention grid may be scheduled while
+  // the RoPE preparation still runs (its launch latency overlaps it); every
+  // thread waits for the preparation's completion (griddepcontrol.wait)
+  // before it reads anything, and the preparation itself started only after
+  // the work before it in the stream had completed
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = K::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  rc = note_cuda(cudaLaunchKernelEx(&cfg, kern, tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G,
+                                    fm ? fm->n_groups : mem_len, m_cap,
+                                    fm ? fm->groups : nullptr, fm ? fm->max_groups : 0,
+                                    qscale, p.n_split, static_cast<__nv_bfloat16*>(out), part_o,
+                                    part_ml, device_status_ptr()));
+  if (rc) return rc;
   rc = check_launch();
   if (rc || p.n_split == 1) return rc;
   return attn_combine_bf16(B, T, Hq, D, p.n_split, part_o, part_ml, out, s);
