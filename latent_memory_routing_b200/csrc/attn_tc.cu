@@ -152,7 +152,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   // launched as a programmatic dependent of the RoPE preparation: wait for
   // its completion (and the visibility of its writes) before reading
   // anything; a no-op when launched without that dependency
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ AAux aux;
   unsigned char* base = tc::smem_align<1024>(smem_dyn);
@@ -519,6 +519,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (row_ok && n_split > 1) part_ml[row_id * n_split + sp] = make_float2(m_run, l_run);
   }
 
+  pdl_trigger();  // this CTA's work is done: the next kernel may be scheduled
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -551,8 +552,10 @@ rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0,
   constexpr int HALF = D / 2;
   constexpr int UPH = HALF / 8;  // 16-byte pair units per head
   // the attention grid that follows may be scheduled now; it waits for this
-  // grid's completion before reading what this grid writes
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // grid's completion before reading what this grid writes.  This grid is
+  // itself a programmatic dependent of the work before it (pdl_wait)
+  pdl_trigger();
+  pdl_wait();
   __shared__ float2 cs[HALF];
   const int p = blockIdx.x;
   const int tq = p - (T_loc - T);  // query token at this position, if >= 0
@@ -718,10 +721,10 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   float2* part_ml = reinterpret_cast<float2*>(w + p.q_bytes + p.k_bytes + p.po_bytes);
   FreqTab freq;
   for (int i = 0; i < D / 2; ++i) freq.w[i] = std::pow((double)rope_base, -2.0 * i / D);
-  rope_prep_kernel<D><<<(unsigned)T_loc, 256, 0, s>>>(
-      B, T, T_loc, Hq, H, pos0, freq, static_cast<const __nv_bfloat16*>(q),
-      static_cast<const __nv_bfloat16*>(k_loc), q_rot, k_rot);
-  int rc = check_launch();
+  int rc = launch_pdl(rope_prep_kernel<D>, dim3((unsigned)T_loc), dim3(256), 0, s, B, T, T_loc,
+                      Hq, H, (int64_t)pos0, freq, static_cast<const __nv_bfloat16*>(q),
+                      static_cast<const __nv_bfloat16*>(k_loc), q_rot, k_rot);
+  if (!rc) rc = check_launch();
   if (rc) return rc;
 
   CUtensorMap tq, tkm, tvm, tkl, tvl;

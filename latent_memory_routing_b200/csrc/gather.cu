@@ -25,6 +25,8 @@ gather_kernel(int k, int n_docs, int row_vecs, const int32_t* __restrict__ idx,
               const int64_t* __restrict__ coff, const uint4* __restrict__ kb,
               const uint4* __restrict__ vb, int m_cap, uint4* __restrict__ km,
               uint4* __restrict__ vm, int32_t* __restrict__ mem_len, int* status) {
+  pdl_wait();  // see msa_common.cuh: nothing is touched before the previous grid is done
+  pdl_trigger();
   __shared__ int64_t s_off, s_src, s_rows;
   const int r = blockIdx.x / kSplit, part = blockIdx.x % kSplit, b = blockIdx.y;
   const int32_t* ib = idx + (int64_t)b * k;
@@ -101,10 +103,10 @@ extern "C" int msa_gather_kv(msa_dtype dt, int B, int k, int H, int D, const int
   // the bank's row count is not an argument here: offsets are checked for order only
   if (int rc = debug_check_offsets(chunk_offsets, n_docs, INT64_MAX, s)) return rc;
   const dim3 grid((unsigned)(k * kSplit), (unsigned)B);
-  gather_kernel<<<grid, 256, 0, s>>>(k, n_docs, (int)(row_bytes / 16), idx, chunk_offsets,
-                                     static_cast<const uint4*>(k_bar),
-                                     static_cast<const uint4*>(v_bar), m_cap,
-                                     static_cast<uint4*>(k_mem), static_cast<uint4*>(v_mem),
-                                     mem_len, device_status_ptr());
-  return debug_finish(check_launch(), s);
+  const int rc = launch_pdl(gather_kernel, grid, dim3(256), 0, s, k, n_docs,
+                            (int)(row_bytes / 16), idx, chunk_offsets,
+                            static_cast<const uint4*>(k_bar), static_cast<const uint4*>(v_bar),
+                            m_cap, static_cast<uint4*>(k_mem), static_cast<uint4*>(v_mem), mem_len,
+                            device_status_ptr());
+  return debug_finish(rc ? rc : check_launch(), s);
 }

@@ -31,6 +31,38 @@ int num_sms();  // SM count of the current device (cached per device)
 // into a CUDA graph -- only launch.
 int ensure_smem_attr(const void* func, int bytes);
 
+// ------------------------------------------ programmatic dependent launch
+//
+// The kernels of a step are launched as programmatic dependents of the work
+// before them in the stream: a grid may be scheduled as soon as every CTA of
+// the kernel before it has signalled (pdl_trigger) or exited, which overlaps
+// the launch latency with that kernel's tail.  Ordering is unchanged: a
+// kernel launched this way calls pdl_wait() before it reads or writes global
+// memory, which waits for the previous grid's completion and the visibility
+// of its writes (and that grid, if it was launched the same way, had itself
+// waited for its predecessor).  Both are no-ops for a kernel launched
+// without the dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+               Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return note_cuda(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
+}
+
 // ---------------------------------------------------------- device status
 
 // Device address of the current device's status word (first

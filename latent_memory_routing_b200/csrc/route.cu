@@ -37,6 +37,8 @@ __global__ void route_prep_kernel(int NT, int H, int D, int n_pad,
                                   Tout* __restrict__ qhat, uint32_t* doc_u,
                                   int64_t n_doc_u, uint32_t* chunk_u,
                                   int64_t n_chunk_u) {
+  pdl_wait();  // see msa_common.cuh: nothing is touched before the previous grid is done
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_rows = (int64_t)(kHeadMajor ? n_pad : NT) * H;
@@ -121,6 +123,8 @@ route_simt_kernel(int T, int H, const float* __restrict__ qhat,
 
 __global__ void route_finalize_kernel(uint32_t* doc_u, int64_t n_doc_u,
                                       uint32_t* chunk_u, int64_t n_chunk_u) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = gt; i < n_doc_u; i += stride) {
@@ -196,18 +200,20 @@ int route_scores_impl(msa_dtype dt, int B, int T, int H, int D, const void* q_r,
     const int n_pad = (int)route_tc_columns(NT);
     const int64_t rows = (int64_t)n_pad * H;
     const unsigned blocks = (unsigned)std::min<int64_t>((rows * 32 + 255) / 256 + 1, 1 << 20);
-    route_prep_kernel<__nv_bfloat16, __nv_bfloat16, true>
-        <<<std::max<unsigned>(blocks, (unsigned)sms), 256, 0, s>>>(
-            NT, H, D, n_pad, static_cast<const __nv_bfloat16*>(q_r),
-            static_cast<__nv_bfloat16*>(ws), doc_u, n_doc_u, chunk_u, n_chunk_u);
+    if ((rc = launch_pdl(route_prep_kernel<__nv_bfloat16, __nv_bfloat16, true>,
+                         dim3(std::max<unsigned>(blocks, (unsigned)sms)), dim3(256), 0, s, NT, H,
+                         D, n_pad, static_cast<const __nv_bfloat16*>(q_r),
+                         static_cast<__nv_bfloat16*>(ws), doc_u, n_doc_u, chunk_u, n_chunk_u)))
+      return rc;
     if ((rc = check_launch())) return rc;
     rc = route_tc_launch(B, T, H, D, static_cast<const __nv_bfloat16*>(ws), n_pad,
                          static_cast<const __nv_bfloat16*>(kr), n_chunks, chunk_offsets, n_docs,
                          doc_u, chunk_u, device_status_ptr(), prepared, s);
     if (rc) return rc;
   }
-  route_finalize_kernel<<<(unsigned)sms * 4, 256, 0, s>>>(doc_u, n_doc_u, chunk_u, n_chunk_u);
-  return debug_finish(check_launch(), s);
+  rc = launch_pdl(route_finalize_kernel, dim3((unsigned)sms * 4), dim3(256), 0, s, doc_u, n_doc_u,
+                  chunk_u, n_chunk_u);
+  return debug_finish(rc ? rc : check_launch(), s);
 }
 
 }  // namespace

@@ -209,6 +209,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 const int64_t* __restrict__ coff, int n_docs, uint32_t* __restrict__ doc_u,
                 uint32_t* __restrict__ chunk_u, unsigned long long* __restrict__ doc_key,
                 int* __restrict__ status) {
+  pdl_wait();  // launched as a programmatic dependent: nothing is touched before
   using K = Cfg<N, D, kPrep, kPair>;
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ Aux aux;
@@ -688,6 +689,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
   }
 
+  pdl_trigger();  // the scan's work is issued: the next kernel may be scheduled
   tc::tc_fence_before();
   __syncthreads();
   // neither CTA of a pair frees TMEM or leaves while the other may still
@@ -784,20 +786,21 @@ int launch(int B, int T, int H, const __nv_bfloat16* qhat, int n_pad, const __nv
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = K::SMEM;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return note_cuda(cudaLaunchKernelEx(&cfg, kern, tm_k, tm_q, H, NT, T, n_pass, C, n_tiles,
                                         coff, n_docs, doc_u, chunk_u, doc_key, status));
   } else {
     const int grid = (int)std::min<int64_t>(n_tiles, num_sms());
-    kern<<<grid, kThreads, K::SMEM, s>>>(tm_k, tm_q, H, NT, T, n_pass, C, n_tiles, coff, n_docs,
-                                         doc_u, chunk_u, doc_key, status);
-    return check_launch();
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), K::SMEM, s, tm_k, tm_q, H, NT, T, n_pass,
+                      C, n_tiles, coff, n_docs, doc_u, chunk_u, doc_key, status);
   }
 }
 

@@ -341,6 +341,8 @@ __global__ void __launch_bounds__(kSmallThreads)
 topk_small_select_kernel(int n, int k, const float* __restrict__ scores,
                          int32_t* __restrict__ idx_out, float* __restrict__ top_out,
                          unsigned long long* __restrict__ seg_out) {
+  pdl_wait();  // see msa_common.cuh: nothing is touched before the previous grid is done
+  pdl_trigger();
   __shared__ unsigned long long lists[kSmallWarps][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int b = blockIdx.y;
@@ -375,6 +377,8 @@ __global__ void __launch_bounds__(kSmallThreads)
 topk_small_merge_kernel(int n, int k, int n_seg, const unsigned long long* __restrict__ seg_in,
                         const float* __restrict__ scores, int32_t* __restrict__ idx_out,
                         float* __restrict__ top_out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ unsigned long long staged[kMergeSmemLists * 32];
   __shared__ unsigned long long lists[kSmallWarps][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -452,12 +456,12 @@ static int topk_docs_body(int B, int n_docs, int k, const float* scores, int32_t
   const dim3 grid((unsigned)p.n_seg, (unsigned)B);
   int rc;
   if (p.small) {
-    topk_small_select_kernel<<<grid, kSmallThreads, 0, s>>>(n_docs, k, scores, idx, top_scores,
-                                                            cand);
-    if ((rc = check_launch()) || p.n_seg == 1) return rc;
-    topk_small_merge_kernel<<<B, kSmallThreads, 0, s>>>(n_docs, k, p.n_seg, cand, scores, idx,
-                                                        top_scores);
-    return check_launch();
+    rc = launch_pdl(topk_small_select_kernel, grid, dim3(kSmallThreads), 0, s, n_docs, k, scores,
+                    idx, top_scores, cand);
+    if (rc || (rc = check_launch()) || p.n_seg == 1) return rc;
+    rc = launch_pdl(topk_small_merge_kernel, dim3(B), dim3(kSmallThreads), 0, s, n_docs, k,
+                    p.n_seg, cand, scores, idx, top_scores);
+    return rc ? rc : check_launch();
   }
   if (p.smem_keys) {
     const size_t smem = (size_t)p.seg_len * sizeof(uint32_t);
