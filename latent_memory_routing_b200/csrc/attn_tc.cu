@@ -12,9 +12,14 @@
 //   * rope_prep_kernel rotates Q (to pos0 + T_loc - T + i) and the local K
 //     (to pos0 + j) once per call into bf16 workspace copies, one launch,
 //     cos/sin per position built in shared memory (angles reduced in double).
-//   * attn_tc_kernel: one CTA per (two Q tiles of 128 rows, KV head, batch,
-//     key split), query blocks dispatched heaviest first (causal work grows
-//     with the block index).  Up to 3 splits of the key tiles, at most one
+//   * attn_tc_kernel: a persistent grid, one CTA per SM, working through
+//     items of (two Q tiles of 128 rows, KV head, batch, key split), claimed
+//     at run time heaviest first (causal work grows with the query block).
+//     An item's Q tiles and first K/V tiles load while the previous item's
+//     last tiles are still in the tensor core and softmax, and its O is read
+//     out of TMEM before the stores, so the next item's MMAs start at once:
+//     a CTA's setup, first-load latency and epilogue are paid once per SM
+//     instead of once per item.  Up to 3 splits of the key tiles, at most one
 //     per 8 tiles, are merged by the split-KV combine kernel when there are
 //     too few query blocks to fill the SMs.  GQA rows are packed as (token,
 //     head of the group): a TMA box of {64 d, G heads, 128/G tokens} lands as
@@ -61,12 +66,9 @@ constexpr int kKeys = 128;   // keys per tile (MMA N of S, K of P V)
 constexpr int kSoftWarps = 4 * kQT;
 // warpgroup 0: TMA producer (warp 0), MMA issuer (warp 1), two idle warps;
 // warpgroups 1 .. kQT: softmax.  Registers move from warpgroup 0 to the
-// softmax warpgroups: 128 x kRegLow + 256 x kRegHigh = 384 x 168, the
+// softmax warpgroups: 128 x REG_LOW + 256 x REG_HIGH = 384 x 168, the
 // block's launch allocation under __launch_bounds__(384, 1).
 constexpr int kThreads = 128 + 32 * kSoftWarps;
-constexpr int kRegLow = 40;
-constexpr int kRegHigh = 232;
-static_assert(kQT == 2 && 128 * kRegLow + 256 * kRegHigh == 384 * 168, "register split");
 constexpr int kStages = 2;
 
 template <int D>
@@ -85,10 +87,25 @@ struct ACfg {
   static constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(kRows, kKeys);
   // O: M=128, N=D, A (P, TMEM) K-major, B (V) MN-major (bit 16)
   static constexpr uint32_t IDESC_O = tc::idesc_bf16_f32(kRows, D) | (1u << 16);
+  // registers per thread of warpgroup 0 (producer, MMA issuer: the item
+  // bookkeeping of the persistent loop) and of the softmax warpgroups,
+  // chosen where the compiler reports no or few spills for either
+  static constexpr int REG_LOW = D == 128 ? 72 : 88;
+  static constexpr int REG_HIGH = D == 128 ? 216 : 208;
+  static_assert(kQT == 2 && 128 * REG_LOW + 256 * REG_HIGH == 384 * 168, "register split");
 };
 
+// item-id ring between the producer and the other roles
+constexpr int kSched = 4;
+constexpr int kSchedReaders = 1 + kSoftWarps;  // the MMA issuer, each softmax warp
+// the producer claims the next item this many tiles before its current
+// item's last tile load
+constexpr int kClaimAhead = 3;
+
 struct AAux {
-  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[kQT], p_full[kQT], o_full[kQT];
+  uint64_t q_full, q_empty, kv_full[kStages], kv_empty[kStages], s_full[kQT], p_full[kQT],
+      o_full[kQT], o_empty[kQT], sched_full[kSched], sched_empty[kSched];
+  int sched_id[kSched];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -133,25 +150,75 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Work item `idx` of a call, heaviest first: query blocks in descending order
+// (under a causal mask later blocks see more key tiles), then batch, KV head
+// and key split.
+struct Item {
+  int mt, b, g, sp;
+};
+__device__ __forceinline__ Item item_of(int idx, int B, int H, int n_split, int n_qb) {
+  const int per_qb = B * H * n_split;
+  Item it;
+  it.mt = n_qb - 1 - idx / per_qb;
+  const int r = idx % per_qb;
+  it.b = r / (H * n_split);
+  it.g = (r % (H * n_split)) / n_split;
+  it.sp = r % n_split;
+  return it;
+}
+
+// The key tiles of an item: the memory tiles (mem_len rows, clamped), then
+// the local tiles up to the block's last visible key; the split owns
+// [j_lo, j_lo + nt) of them.
+struct Span {
+  int tok0, n_tok, M, n_mt, j_lo, nt;
+};
+template <bool kFused>
+__device__ __forceinline__ Span span_of(const Item& it, int T, int T_loc, int TQ,
+                                        const int32_t* __restrict__ mem_len, int m_cap,
+                                        int max_groups, int n_split) {
+  Span s;
+  s.tok0 = it.mt * kQT * TQ;
+  s.n_tok = min(kQT * TQ, T - s.tok0);
+  const int ml = max(__ldg(mem_len + it.b), 0);
+  s.M = kFused ? 8 * min(ml, max_groups) : min(ml, m_cap);
+  const int lim_max = T_loc - T + s.tok0 + s.n_tok - 1;  // last local key any row sees
+  s.n_mt = (s.M + kKeys - 1) / kKeys;
+  const int nt_all = s.n_mt + (lim_max + 1 + kKeys - 1) / kKeys;
+  s.j_lo = (int)((int64_t)it.sp * nt_all / n_split);
+  s.nt = (int)((int64_t)(it.sp + 1) * nt_all / n_split) - s.j_lo;
+  return s;
+}
+
 // kFused: memory rows read straight from the pooled bank, per query a list
 // of 8-row groups (first bank row, rows of the group inside its document)
 // in rank order; tm_km / tm_vm map the bank with 8-row boxes (one
 // 128B-swizzle atom), a memory tile is 16 groups, and `mem_len` holds the
 // group count.  Rows past a document's end are other bank rows: masked, and
 // their V zeroed in shared memory before P V reads it.
+//
+// Persistent: one CTA per SM (grid = min(items, SMs)); CTA c starts with
+// item c and claims the next one from `next_item` (zeroed by the RoPE
+// preparation) while the loads of its current item's last tile are issued.
+// The producer publishes each item id in a shared-memory ring that the MMA
+// issuer and the softmax warps read.  Every ring, tile and item barrier
+// counts phases over the whole CTA lifetime: the K/V ring by the CTA's
+// running tile count, q_full / q_empty / o_full / o_empty by its running
+// count of non-empty items.
 template <int D, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_km,
                const __grid_constant__ CUtensorMap tm_vm, const __grid_constant__ CUtensorMap tm_kl,
-               const __grid_constant__ CUtensorMap tm_vl, int T, int T_loc, int Hq, int H, int G,
-               const int32_t* __restrict__ mem_len, int m_cap, const int2* __restrict__ groups,
-               int max_groups, float qscale, int n_split,
+               const __grid_constant__ CUtensorMap tm_vl, int B, int T, int T_loc, int Hq, int H,
+               int G, const int32_t* __restrict__ mem_len, int m_cap,
+               const int2* __restrict__ groups, int max_groups, float qscale, int n_split,
+               int n_qb, int n_items, int* __restrict__ next_item,
                __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
                float2* __restrict__ part_ml, int* __restrict__ status) {
   using K = ACfg<D>;
   // launched as a programmatic dependent of the RoPE preparation: wait for
-  // its completion (and the visibility of its writes) before reading
-  // anything; a no-op when launched without that dependency
+  // its completion (and the visibility of its writes, the zeroed item
+  // counter among them) before reading anything
   pdl_wait();
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   __shared__ AAux aux;
@@ -160,39 +227,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   unsigned char* sKV = sQ + kQT * K::Q_BYTES;      // kStages x (K tile, V tile)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid (split x head, batch, query block): z is dispatched slowest and
-  // runs the query blocks in descending order -- under a causal mask later
-  // blocks see more key tiles, so the longest CTAs start first
-  const int mt = (int)(gridDim.z - 1 - blockIdx.z);
-  const int b = blockIdx.y;
-  const int g = blockIdx.x / n_split, sp = blockIdx.x % n_split;
-  const int TQ = kRows / G;          // tokens per Q tile
-  const int tok0 = mt * kQT * TQ;    // first token of the CTA
-  const int n_tok = min(kQT * TQ, T - tok0);
-  const int M =
-      kFused ? 8 * min(max(mem_len[b], 0), max_groups) : min(max(mem_len[b], 0), m_cap);
-  const int2* gq = kFused ? groups + (int64_t)b * max_groups : nullptr;
-  const int lim_max = T_loc - T + tok0 + n_tok - 1;  // last local key any row sees
-  const int n_mt = (M + kKeys - 1) / kKeys;
-  const int n_lt = (lim_max + 1 + kKeys - 1) / kKeys;
-  const int nt_all = n_mt + n_lt;
-  // this CTA's share [j_lo, j_hi) of the key tiles
-  const int j_lo = (int)((int64_t)sp * nt_all / n_split);
-  const int j_hi = (int)((int64_t)(sp + 1) * nt_all / n_split);
-  if (j_lo == j_hi) {  // nothing to attend: an empty partial (uniform exit)
-    for (int r = threadIdx.x; r < kQT * kRows; r += blockDim.x) {
-      if (r / G >= n_tok) continue;
-      const int64_t row_id = ((int64_t)b * Hq + g * G + r % G) * T + tok0 + r / G;
-      float* po = part_o + (row_id * n_split + sp) * D;
-      for (int d = 0; d < D; ++d) po[d] = 0.f;
-      part_ml[row_id * n_split + sp] = make_float2(-INFINITY, 0.f);
-    }
-    return;
-  }
-  const int nt = j_hi - j_lo;  // tiles j_lo + 0 .. j_lo + nt - 1
+  const int TQ = kRows / G;  // tokens per Q tile
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&aux.q_full, 1);
+    tc::mbar_init(&aux.q_empty, 1);
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&aux.kv_full[i], 1);
       tc::mbar_init(&aux.kv_empty[i], 1);
@@ -201,6 +240,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_init(&aux.s_full[i], 1);
       tc::mbar_init(&aux.p_full[i], 4);
       tc::mbar_init(&aux.o_full[i], 1);
+      tc::mbar_init(&aux.o_empty[i], 4);
+    }
+    for (int i = 0; i < kSched; ++i) {
+      tc::mbar_init(&aux.sched_full[i], 1);
+      tc::mbar_init(&aux.sched_empty[i], kSchedReaders);
     }
     aux.abort_flag = 0;
     tc::fence_mbar_init();
@@ -215,121 +259,196 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const uint32_t tmem = aux.tmem_base;
   // TMEM columns: S/P of tile i at i*kKeys, O of tile i at kQT*kKeys + i*D
   volatile int* abort_flag = &aux.abort_flag;
+  auto fail = [&]() {
+    record_error(status, MSA_ERR_TIMEOUT);
+    *abort_flag = 1;
+  };
+  auto span = [&](const Item& it) {
+    return span_of<kFused>(it, T, T_loc, TQ, mem_len, m_cap, max_groups, n_split);
+  };
 
   if (warp < 4) {
-   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegLow));
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(K::REG_LOW));
    if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t issued = 0;
-      tc::mbar_arrive_expect_tx(&aux.q_full, kQT * K::Q_BYTES);
-#pragma unroll
-      for (int i = 0; i < kQT; ++i)
-#pragma unroll
-        for (int kb = 0; kb < K::KB; ++kb)
-          tc::tma_load_3d(sQ + i * K::Q_BYTES + kb * kRows * 128, &tm_q, &aux.q_full, kb * 64,
-                          g * G, b * T + tok0 + i * TQ);
-      for (int j = 0; j < nt; ++j) {
-        const int st = j % kStages;
-        if (*abort_flag || !tc::mbar_wait(&aux.kv_empty[st], ((j / kStages) & 1) ^ 1)) {
-          record_error(status, MSA_ERR_TIMEOUT);
-          *abort_flag = 1;
+      uint32_t tiles = 0, q_loads = 0;  // loads issued over the CTA's items
+      int idx = blockIdx.x;
+      bool ok = true;
+      for (uint32_t n = 0; ok; ++n) {
+        const int slot = n % kSched;
+        if (*abort_flag || !tc::mbar_wait(&aux.sched_empty[slot], ((n / kSched) & 1) ^ 1)) {
+          ok = false;
           break;
         }
-        unsigned char* k_dst = sKV + st * K::STAGE;
-        unsigned char* v_dst = k_dst + K::K_BYTES;
-        tc::mbar_arrive_expect_tx(&aux.kv_full[st], K::STAGE);
-        const int jj = j_lo + j;
-        const bool mem = jj < n_mt;
-        const CUtensorMap* mk = mem ? &tm_km : &tm_kl;
-        const CUtensorMap* mv = mem ? &tm_vm : &tm_vl;
-        if (kFused && mem) {
-          // 16 groups of 8 bank rows; past the last group, repeat it (finite
-          // rows, masked) so every row of the tile is written
-          const int ng = M / 8, g0 = jj * (kKeys / 8);
-          for (int gi = 0; gi < kKeys / 8; ++gi) {
-            const int src = gq[min(g0 + gi, ng - 1)].x;
+        const bool live = idx < n_items;
+        aux.sched_id[slot] = live ? idx : -1;
+        tc::mbar_arrive(&aux.sched_full[slot]);  // release: the id is visible to the waiters
+        if (!live) break;
+        const Item it = item_of(idx, B, H, n_split, n_qb);
+        const Span sp = span(it);
+        int nxt = n_items;
+        if (sp.nt == 0) {
+          idx = atomicAdd(next_item, 1) + (int)gridDim.x;
+          continue;
+        }
+        // the Q tiles are free once the previous item's last S has completed
+        if (q_loads > 0 && (*abort_flag || !tc::mbar_wait(&aux.q_empty, (q_loads - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc::mbar_arrive_expect_tx(&aux.q_full, kQT * K::Q_BYTES);
+#pragma unroll
+        for (int i = 0; i < kQT; ++i)
+#pragma unroll
+          for (int kb = 0; kb < K::KB; ++kb)
+            tc::tma_load_3d(sQ + i * K::Q_BYTES + kb * kRows * 128, &tm_q, &aux.q_full, kb * 64,
+                            it.g * G, it.b * T + sp.tok0 + i * TQ);
+        ++q_loads;
+        const int2* gq = kFused ? groups + (int64_t)it.b * max_groups : nullptr;
+        const int j_claim = max(sp.nt - kClaimAhead, 0);
+        for (int j = 0; j < sp.nt; ++j) {
+          // claim the next item a few tiles before this one's loads end
+          if (j == j_claim) nxt = atomicAdd(next_item, 1) + (int)gridDim.x;
+          const int st = tiles % kStages;
+          if (*abort_flag || !tc::mbar_wait(&aux.kv_empty[st], ((tiles / kStages) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          if (j == j_claim && nxt < n_items) {
+            // its Q tiles into L2: the Q buffer frees only when this item's
+            // last S completes, and from L2 the reload is short
+            const Item ni = item_of(nxt, B, H, n_split, n_qb);
+#pragma unroll
+            for (int i = 0; i < kQT; ++i)
+#pragma unroll
+              for (int kb = 0; kb < K::KB; ++kb)
+                tc::tma_prefetch_l2_3d(&tm_q, kb * 64, ni.g * G,
+                                       ni.b * T + ni.mt * kQT * TQ + i * TQ);
+          }
+          unsigned char* k_dst = sKV + st * K::STAGE;
+          unsigned char* v_dst = k_dst + K::K_BYTES;
+          tc::mbar_arrive_expect_tx(&aux.kv_full[st], K::STAGE);
+          const int jj = sp.j_lo + j;
+          const bool mem = jj < sp.n_mt;
+          const CUtensorMap* mk = mem ? &tm_km : &tm_kl;
+          const CUtensorMap* mv = mem ? &tm_vm : &tm_vl;
+          if (kFused && mem) {
+            // 16 groups of 8 bank rows; past the last group, repeat it
+            // (finite rows, masked) so every row of the tile is written
+            const int ng = sp.M / 8, g0 = jj * (kKeys / 8);
+            for (int gi = 0; gi < kKeys / 8; ++gi) {
+              const int src = gq[min(g0 + gi, ng - 1)].x;
+#pragma unroll
+              for (int kb = 0; kb < K::KB; ++kb) {
+                tc::tma_load_3d(k_dst + kb * kKeys * 128 + gi * 1024, mk, &aux.kv_full[st],
+                                kb * 64, it.g, src);
+                tc::tma_load_3d(v_dst + kb * kKeys * 128 + gi * 1024, mv, &aux.kv_full[st],
+                                kb * 64, it.g, src);
+              }
+            }
+          } else {
+            const int row =
+                mem ? it.b * m_cap + jj * kKeys : it.b * T_loc + (jj - sp.n_mt) * kKeys;
 #pragma unroll
             for (int kb = 0; kb < K::KB; ++kb) {
-              tc::tma_load_3d(k_dst + kb * kKeys * 128 + gi * 1024, mk, &aux.kv_full[st],
-                              kb * 64, g, src);
-              tc::tma_load_3d(v_dst + kb * kKeys * 128 + gi * 1024, mv, &aux.kv_full[st],
-                              kb * 64, g, src);
+              tc::tma_load_3d(k_dst + kb * kKeys * 128, mk, &aux.kv_full[st], kb * 64, it.g,
+                              row);
+              tc::tma_load_3d(v_dst + kb * kKeys * 128, mv, &aux.kv_full[st], kb * 64, it.g,
+                              row);
             }
           }
-        } else {
-          const int row = mem ? b * m_cap + jj * kKeys : b * T_loc + (jj - n_mt) * kKeys;
-#pragma unroll
-          for (int kb = 0; kb < K::KB; ++kb) {
-            tc::tma_load_3d(k_dst + kb * kKeys * 128, mk, &aux.kv_full[st], kb * 64, g, row);
-            tc::tma_load_3d(v_dst + kb * kKeys * 128, mv, &aux.kv_full[st], kb * 64, g, row);
-          }
+          ++tiles;
         }
-        ++issued;
+        idx = nxt;
       }
+      if (!ok) fail();
       // every load issued must land before the CTA exits
-      tc::mbar_wait(&aux.q_full, 0);
-      for (uint32_t v = issued > (uint32_t)kStages ? issued - kStages : 0; v < issued; ++v)
+      if (q_loads > 0) tc::mbar_wait(&aux.q_full, (q_loads - 1) & 1);
+      for (uint32_t v = tiles > (uint32_t)kStages ? tiles - kStages : 0; v < tiles; ++v)
         tc::mbar_wait(&aux.kv_full[v % kStages], (v / kStages) & 1);
     }
    } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    // order: S_0(0) S_1(0) | P_0V(0) S_0(1) P_1V(0) S_1(1) | ... so each
-    // softmax warpgroup works while the tensor core serves the other one;
-    // S_i(j) is issued after P_iV(j-1), which makes the TMEM columns that
-    // held P_i(j-1) safe to overwrite and lets s_full_i(j) imply that
-    // P_iV(j-1) has completed.
+    // order within an item: S_0(0) S_1(0) | P_0V(0) S_0(1) P_1V(0) S_1(1) |
+    // ... so each softmax warpgroup works while the tensor core serves the
+    // other one; S_i(j) is issued after P_iV(j-1), which makes the TMEM
+    // columns that held P_i(j-1) safe to overwrite and lets s_full_i(j)
+    // imply that P_iV(j-1) has completed.  The next item's S_i(0) follows
+    // this item's last P_iV the same way; its first P_iV (which overwrites
+    // O_i) waits until softmax group i has read this item's O_i out.
     if (lane == 0) {
-      bool ok = tc::mbar_wait(&aux.q_full, 0);
-      auto issue_s = [&](int i, int j) -> bool {
-        const int st = j % kStages;
-        if (*abort_flag || !tc::mbar_wait(&aux.kv_full[st], (j / kStages) & 1)) return false;
-        // S_i(j) overwrites P_i(j-1); the P V that reads it was issued
-        // (after its p_full wait) before this MMA, and the tensor core runs
-        // one thread's MMAs in issue order
-        tc::tc_fence_after();
-        const uint32_t q0 = tc::smem_u32(sQ + i * K::Q_BYTES);
-        const uint32_t k0 = tc::smem_u32(sKV + st * K::STAGE);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
-          const uint32_t koff = (kk >> 2) * (kKeys * 128) + (kk & 3) * 32;
-          tc::mma_bf16_ss(tmem + i * kKeys, tc::sdesc_kmajor_sw128(q0 + off),
-                          tc::sdesc_kmajor_sw128(k0 + koff), K::IDESC_S, kk > 0 ? 1u : 0u);
+      uint32_t tiles = 0, ne = 0;  // tiles and non-empty items so far
+      bool ok = true;
+      for (uint32_t n = 0; ok; ++n) {
+        const int slot = n % kSched;
+        if (*abort_flag || !tc::mbar_wait(&aux.sched_full[slot], (n / kSched) & 1)) {
+          ok = false;
+          break;
         }
-        tc::mma_commit(&aux.s_full[i]);
-        return true;
-      };
-      auto issue_pv = [&](int i, int j) -> bool {
-        const int st = j % kStages;
-        // P_i(j) written (and any rescale of O_i done) by softmax group i
-        if (*abort_flag || !tc::mbar_wait(&aux.p_full[i], j & 1)) return false;
-        tc::tc_fence_after();
-        const uint32_t v0 = tc::smem_u32(sKV + st * K::STAGE + K::K_BYTES);
+        const int idx = aux.sched_id[slot];
+        tc::mbar_arrive(&aux.sched_empty[slot]);
+        if (idx < 0) break;
+        const int nt = span(item_of(idx, B, H, n_split, n_qb)).nt;
+        if (nt == 0) continue;
+        ok = !*abort_flag && tc::mbar_wait(&aux.q_full, ne & 1);
+        auto issue_s = [&](int i, int j) -> bool {
+          const uint32_t v = tiles + j;
+          const int st = v % kStages;
+          if (*abort_flag || !tc::mbar_wait(&aux.kv_full[st], (v / kStages) & 1)) return false;
+          // S_i(j) overwrites P_i(j-1); the P V that reads it was issued
+          // (after its p_full wait) before this MMA, and the tensor core runs
+          // one thread's MMAs in issue order
+          tc::tc_fence_after();
+          const uint32_t q0 = tc::smem_u32(sQ + i * K::Q_BYTES);
+          const uint32_t k0 = tc::smem_u32(sKV + st * K::STAGE);
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk)
-          mma_bf16_ts(tmem + kQT * kKeys + i * D, tmem + i * kKeys + kk * 8,
-                      sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kKeys * 128), K::IDESC_O,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        if (j == nt - 1) tc::mma_commit(&aux.o_full[i]);  // one phase: O_i final
-        if (i == kQT - 1) tc::mma_commit(&aux.kv_empty[st]);
-        return true;
-      };
-      for (int i = 0; ok && i < kQT; ++i) ok = issue_s(i, 0);
-      for (int j = 0; ok && j < nt; ++j)
-        for (int i = 0; ok && i < kQT; ++i) {
-          ok = issue_pv(i, j);
-          if (ok && j + 1 < nt) ok = issue_s(i, j + 1);
-        }
-      if (!ok) {
-        record_error(status, MSA_ERR_TIMEOUT);
-        *abort_flag = 1;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+            const uint32_t koff = (kk >> 2) * (kKeys * 128) + (kk & 3) * 32;
+            tc::mma_bf16_ss(tmem + i * kKeys, tc::sdesc_kmajor_sw128(q0 + off),
+                            tc::sdesc_kmajor_sw128(k0 + koff), K::IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&aux.s_full[i]);
+          // the item's last S: its Q tiles may be overwritten once it completes
+          if (i == kQT - 1 && j == nt - 1) tc::mma_commit(&aux.q_empty);
+          return true;
+        };
+        auto issue_pv = [&](int i, int j) -> bool {
+          const uint32_t v = tiles + j;
+          const int st = v % kStages;
+          // O_i of the previous item read out of TMEM by softmax group i
+          if (j == 0 && ne > 0 &&
+              (*abort_flag || !tc::mbar_wait(&aux.o_empty[i], (ne - 1) & 1)))
+            return false;
+          // P_i(j) written (and any rescale of O_i done) by softmax group i
+          if (*abort_flag || !tc::mbar_wait(&aux.p_full[i], v & 1)) return false;
+          tc::tc_fence_after();
+          const uint32_t v0 = tc::smem_u32(sKV + st * K::STAGE + K::K_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk)
+            mma_bf16_ts(tmem + kQT * kKeys + i * D, tmem + i * kKeys + kk * 8,
+                        sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kKeys * 128), K::IDESC_O,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          if (j == nt - 1) tc::mma_commit(&aux.o_full[i]);  // O_i of the item final
+          if (i == kQT - 1) tc::mma_commit(&aux.kv_empty[st]);
+          return true;
+        };
+        for (int i = 0; ok && i < kQT; ++i) ok = issue_s(i, 0);
+        for (int j = 0; ok && j < nt; ++j)
+          for (int i = 0; ok && i < kQT; ++i) {
+            ok = issue_pv(i, j);
+            if (ok && j + 1 < nt) ok = issue_s(i, j + 1);
+          }
+        tiles += nt;
+        ++ne;
       }
+      if (!ok) fail();
     }
    }
   } else {
     // ------------------------------------------------------------- softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegHigh));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(K::REG_HIGH));
     // Warpgroup i owns Q tile i, one thread per query row.  O_i accumulates
     // in TMEM; the row's reference maximum m_run only moves when a tile's
     // maximum exceeds it by more than 2^kRescaleLog2 -- then O_i (in TMEM)
@@ -344,179 +463,210 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const uint32_t tSP = tmem + qt * kKeys + lane_addr;
     const uint32_t tOi = tmem + kQT * kKeys + qt * D + lane_addr;
-    const int tok_local = qt * TQ + r / G;
-    const int tok = tok0 + tok_local;
-    const int lim = T_loc - T + tok;  // last visible local key
-    float m_run = -INFINITY, l_run = 0.f;
-    for (int j = 0; j < nt; ++j) {
-      if (!*abort_flag && !tc::mbar_wait(&aux.s_full[qt], j & 1)) {
-        record_error(status, MSA_ERR_TIMEOUT);
-        *abort_flag = 1;
+    uint32_t tiles = 0, ne = 0;  // tiles and non-empty items so far
+    for (uint32_t n = 0;; ++n) {
+      const int slot = n % kSched;
+      if (*abort_flag) break;
+      if (!tc::mbar_wait(&aux.sched_full[slot], (n / kSched) & 1)) {
+        fail();
+        break;
       }
-      tc::tc_fence_after();
-      const int jj = j_lo + j;
-      const bool mem = jj < n_mt;
-      const int key0 = mem ? jj * kKeys : (jj - n_mt) * kKeys;
-      const int n_vis = mem ? min(kKeys, M - key0) : max(0, min(kKeys, lim - key0 + 1));
-      uint32_t sv[kKeys];
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c)
-        tc::tmem_ld32(tSP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
-      tc::tmem_ld_wait();
-      // keys a row may not see read as -inf (also hides whatever S holds
-      // there: rows past mem_len, keys past the causal limit)
-      bool all8 = true;  // fused memory tile: every row belongs to its document
-      if (kFused && mem) {
-        // valid rows of each of the tile's 16 groups (0 past the last
-        // group), read as the columns reach each group
-        for (int gi = 0; gi < kKeys / 8; ++gi) {
-          const int grp = key0 / 8 + gi;
-          all8 &= grp < M / 8 && gq[grp].y == 8;
+      const int idx = aux.sched_id[slot];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&aux.sched_empty[slot]);
+      if (idx < 0) break;
+      const Item it = item_of(idx, B, H, n_split, n_qb);
+      const Span sp = span(it);
+      const int tok_local = qt * TQ + r / G;
+      const int tok = sp.tok0 + tok_local;
+      const bool row_ok = tok_local < sp.n_tok;
+      const int64_t row_id = ((int64_t)it.b * Hq + it.g * G + r % G) * T + tok;
+      if (sp.nt == 0) {  // nothing to attend: an empty partial
+        if (row_ok) {
+          float* po = part_o + (row_id * n_split + it.sp) * D;
+          for (int d = 0; d < D; d += 4)
+            *reinterpret_cast<float4*>(po + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+          part_ml[row_id * n_split + it.sp] = make_float2(-INFINITY, 0.f);
         }
-        if (!all8) {
-          int nvg = 0;
+        continue;
+      }
+      const int nt = sp.nt, M = sp.M, n_mt = sp.n_mt;
+      const int lim = T_loc - T + tok;  // last visible local key
+      const int2* gq = kFused ? groups + (int64_t)it.b * max_groups : nullptr;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        const uint32_t v = tiles + j;
+        if (!*abort_flag && !tc::mbar_wait(&aux.s_full[qt], v & 1)) fail();
+        tc::tc_fence_after();
+        const int jj = sp.j_lo + j;
+        const bool mem = jj < n_mt;
+        const int key0 = mem ? jj * kKeys : (jj - n_mt) * kKeys;
+        const int n_vis = mem ? min(kKeys, M - key0) : max(0, min(kKeys, lim - key0 + 1));
+        uint32_t sv[kKeys];
 #pragma unroll
-          for (int c = 0; c < kKeys; ++c) {
-            if ((c & 7) == 0) {
-              const int grp = key0 / 8 + (c >> 3);
-              nvg = grp < M / 8 ? gq[grp].y : 0;
+        for (int c = 0; c < kKeys / 32; ++c)
+          tc::tmem_ld32(tSP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + c * 32));
+        tc::tmem_ld_wait();
+        // keys a row may not see read as -inf (also hides whatever S holds
+        // there: rows past mem_len, keys past the causal limit)
+        bool all8 = true;  // fused memory tile: every row belongs to its document
+        if (kFused && mem) {
+          // valid rows of each of the tile's 16 groups (0 past the last
+          // group), read as the columns reach each group
+          for (int gi = 0; gi < kKeys / 8; ++gi) {
+            const int grp = key0 / 8 + gi;
+            all8 &= grp < M / 8 && gq[grp].y == 8;
+          }
+          if (!all8) {
+            int nvg = 0;
+#pragma unroll
+            for (int c = 0; c < kKeys; ++c) {
+              if ((c & 7) == 0) {
+                const int grp = key0 / 8 + (c >> 3);
+                nvg = grp < M / 8 ? gq[grp].y : 0;
+              }
+              if ((c & 7) >= nvg) sv[c] = 0xff800000u;
             }
-            if ((c & 7) >= nvg) sv[c] = 0xff800000u;
+          }
+        } else if (!__all_sync(0xffffffffu, n_vis == kKeys)) {
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c)
+            if (c >= n_vis) sv[c] = 0xff800000u;
+        }
+        // row maximum: 8 independent chains of 3-input max
+        float mx[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(sv[c]);
+#pragma unroll
+        for (int c = 8; c + 16 <= kKeys; c += 16)
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            mx[u] = fmax3(mx[u], __uint_as_float(sv[c + u]), __uint_as_float(sv[c + 8 + u]));
+        if ((kKeys - 8) % 16)  // the last 8 keys
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], __uint_as_float(sv[kKeys - 8 + u]));
+        const float mraw = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7]));
+        const float mt = mraw * qscale;  // qscale > 0 keeps the order
+        const bool grow = mt > m_run + kRescaleLog2;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = m_run == -INFINITY ? 0.f : ex2_approx(m_run - mt);
+          m_run = mt;
+        }
+        if (__any_sync(0xffffffffu, grow && alpha != 0.f) && j > 0) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tc::tmem_ld32(tOi + c * 32, o);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tOi + c * 32, o);
           }
         }
-      } else if (!__all_sync(0xffffffffu, n_vis == kKeys)) {
+        unsigned char* v_tile = sKV + (v % kStages) * K::STAGE + K::K_BYTES;
+        if (!kFused && mem && M - key0 < kKeys) {
+          // rows past mem_len in the last memory tile hold whatever the
+          // caller's buffer holds there; zero their V so that 0 * V stays 0
+          const int vrow = quad * 32 + lane;  // one V row per thread of group 0
+          if (qt == 0 && vrow >= M - key0) {
+            unsigned char* vp = v_tile + vrow * 128;
 #pragma unroll
-        for (int c = 0; c < kKeys; ++c)
-          if (c >= n_vis) sv[c] = 0xff800000u;
-      }
-      // row maximum: 8 independent chains of 3-input max
-      float mx[8];
+            for (int kb = 0; kb < K::KB; ++kb)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(sv[c]);
-#pragma unroll
-      for (int c = 8; c + 16 <= kKeys; c += 16)
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          mx[u] = fmax3(mx[u], __uint_as_float(sv[c + u]), __uint_as_float(sv[c + 8 + u]));
-      if ((kKeys - 8) % 16)  // the last 8 keys
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], __uint_as_float(sv[kKeys - 8 + u]));
-      const float mraw = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                               fmaxf(mx[6], mx[7]));
-      const float mt = mraw * qscale;  // qscale > 0 keeps the order
-      const bool grow = mt > m_run + kRescaleLog2;
-      float alpha = 1.f;
-      if (grow) {
-        alpha = m_run == -INFINITY ? 0.f : ex2_approx(m_run - mt);
-        m_run = mt;
-      }
-      if (__any_sync(0xffffffffu, grow && alpha != 0.f) && j > 0) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tc::tmem_ld32(tOi + c * 32, v);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-          tmem_st32(tOi + c * 32, v);
+              for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<uint4*>(vp + kb * (kKeys * 128) + q * 16) =
+                    make_uint4(0, 0, 0, 0);
+          }
+          tc::fence_proxy_async_smem();
         }
-      }
-      l_run *= alpha;
-      const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-      // p = 2^(s * qscale - m_run): the affine step on pairs (f32x2), one
-      // ex2 per key, packed to bf16 pairs; the row sum in pairs too
-      const unsigned long long sc2 = f2_pack(qscale, qscale), nm2 = f2_pack(neg_m, neg_m);
-      unsigned long long ls2[2] = {0ull, 0ull};
+        if (kFused && mem && !all8) {
+          // rows of a group past its document's end (and the repeated groups
+          // past the query's last one) are other bank rows: their p is 0, and
+          // their V is zeroed so that a non-finite bank value cannot turn
+          // 0 * V into NaN
+          const int vrow = quad * 32 + lane;  // one V row per thread of group 0
+          const int grp = key0 / 8 + vrow / 8;
+          const int nv = grp < M / 8 ? gq[grp].y : 0;
+          if (qt == 0 && (vrow & 7) >= nv) {
+            unsigned char* vp = v_tile + vrow * 128;
 #pragma unroll
-      for (int c = 0; c < kKeys / 64; ++c) {
-        uint32_t w[32];
+            for (int kb = 0; kb < K::KB; ++kb)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int k0 = c * 64 + 2 * e;
-          unsigned long long x2 = (unsigned long long)sv[k0] | ((unsigned long long)sv[k0 + 1] << 32);
-          asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(x2) : "l"(sc2), "l"(nm2));
-          const float p0 = ex2_approx(__uint_as_float((uint32_t)x2));
-          const float p1 = ex2_approx(__uint_as_float((uint32_t)(x2 >> 32)));
-          const unsigned long long p2 = f2_pack(p0, p1);
-          asm("add.rn.f32x2 %0, %0, %1;" : "+l"(ls2[e & 1]) : "l"(p2));
-          w[e] = pack_bf16(p0, p1);
+              for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<uint4*>(vp + kb * (kKeys * 128) + q * 16) =
+                    make_uint4(0, 0, 0, 0);
+          }
+          tc::fence_proxy_async_smem();
         }
-        tmem_st32(tSP + c * 32, w);  // keys 64c .. 64c+63 -> columns 32c .. 32c+31
-      }
-      asm("add.rn.f32x2 %0, %0, %1;" : "+l"(ls2[0]) : "l"(ls2[1]));
-      const float ls = __uint_as_float((uint32_t)ls2[0]) + __uint_as_float((uint32_t)(ls2[0] >> 32));
-      l_run += ls;
-      if (!kFused && mem && M - key0 < kKeys) {
-        // rows past mem_len in the last memory tile hold whatever the
-        // caller's buffer holds there; zero their V so that 0 * V stays 0
-        const int vrow = quad * 32 + lane;  // one V row per thread of group 0
-        if (qt == 0 && vrow >= M - key0) {
-          unsigned char* vp = sKV + (j % kStages) * K::STAGE + K::K_BYTES + vrow * 128;
+        l_run *= alpha;
+        const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+        // p = 2^(s * qscale - m_run): the affine step on pairs (f32x2), one
+        // ex2 per key, packed to bf16 pairs; the row sum in pairs too
+        const unsigned long long sc2 = f2_pack(qscale, qscale), nm2 = f2_pack(neg_m, neg_m);
+        unsigned long long ls2[2] = {0ull, 0ull};
 #pragma unroll
-          for (int kb = 0; kb < K::KB; ++kb)
+        for (int c = 0; c < kKeys / 64; ++c) {
+          uint32_t w[32];
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              *reinterpret_cast<uint4*>(vp + kb * (kKeys * 128) + q * 16) = make_uint4(0, 0, 0, 0);
+          for (int e = 0; e < 32; ++e) {
+            const int k0 = c * 64 + 2 * e;
+            unsigned long long x2 =
+                (unsigned long long)sv[k0] | ((unsigned long long)sv[k0 + 1] << 32);
+            asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(x2) : "l"(sc2), "l"(nm2));
+            const float p0 = ex2_approx(__uint_as_float((uint32_t)x2));
+            const float p1 = ex2_approx(__uint_as_float((uint32_t)(x2 >> 32)));
+            const unsigned long long p2 = f2_pack(p0, p1);
+            asm("add.rn.f32x2 %0, %0, %1;" : "+l"(ls2[e & 1]) : "l"(p2));
+            w[e] = pack_bf16(p0, p1);
+          }
+          tmem_st32(tSP + c * 32, w);  // keys 64c .. 64c+63 -> columns 32c .. 32c+31
         }
-        tc::fence_proxy_async_smem();
+        asm("add.rn.f32x2 %0, %0, %1;" : "+l"(ls2[0]) : "l"(ls2[1]));
+        const float ls =
+            __uint_as_float((uint32_t)ls2[0]) + __uint_as_float((uint32_t)(ls2[0] >> 32));
+        l_run += ls;
+        tmem_st_wait();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&aux.p_full[qt]);
       }
-      if (kFused && mem && !all8) {
-        // rows of a group past its document's end (and the repeated groups
-        // past the query's last one) are other bank rows: their p is 0, and
-        // their V is zeroed so that a non-finite bank value cannot turn
-        // 0 * V into NaN
-        const int vrow = quad * 32 + lane;  // one V row per thread of group 0
-        const int grp = key0 / 8 + vrow / 8;
-        const int nv = grp < M / 8 ? gq[grp].y : 0;
-        if (qt == 0 && (vrow & 7) >= nv) {
-          unsigned char* vp = sKV + (j % kStages) * K::STAGE + K::K_BYTES + vrow * 128;
+      // O_i is final once the item's last P V completes; read it out of
+      // TMEM, release the columns to the next item's P V, then store
+      if (!*abort_flag && !tc::mbar_wait(&aux.o_full[qt], ne & 1)) fail();
+      tc::tc_fence_after();
+      uint32_t o[D];
 #pragma unroll
-          for (int kb = 0; kb < K::KB; ++kb)
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              *reinterpret_cast<uint4*>(vp + kb * (kKeys * 128) + q * 16) = make_uint4(0, 0, 0, 0);
-        }
-        tc::fence_proxy_async_smem();
-      }
-      tmem_st_wait();
+      for (int c = 0; c < D / 32; ++c)
+        tc::tmem_ld32(tOi + c * 32, *reinterpret_cast<uint32_t(*)[32]>(o + c * 32));
+      tc::tmem_ld_wait();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&aux.p_full[qt]);
-    }
-    // O_i is final once the last P V completes (o_full has one phase)
-    if (!*abort_flag && !tc::mbar_wait(&aux.o_full[qt], 0)) {
-      record_error(status, MSA_ERR_TIMEOUT);
-      *abort_flag = 1;
-    }
-    tc::tc_fence_after();
-    const bool row_ok = tok_local < n_tok;
-    const int64_t row_id = ((int64_t)b * Hq + g * G + r % G) * T + tok;
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t v[32];
-      tc::tmem_ld32(tOi + c * 32, v);
-      tc::tmem_ld_wait();
+      if (lane == 0) tc::mbar_arrive(&aux.o_empty[qt]);
+      tiles += nt;
+      ++ne;
       if (!row_ok) continue;
       if (n_split > 1) {
-        float* po = part_o + (row_id * n_split + sp) * D + c * 32;
+        float* po = part_o + (row_id * n_split + it.sp) * D;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
+        for (int e = 0; e < D; e += 4)
           *reinterpret_cast<float4*>(po + e) =
-              make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                          __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+              make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
+                          __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+        part_ml[row_id * n_split + it.sp] = make_float2(m_run, l_run);
       } else {
-        __nv_bfloat16* op = out + (((int64_t)b * T + tok) * Hq + g * G + r % G) * D + c * 32;
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        __nv_bfloat16* op = out + (((int64_t)it.b * T + tok) * Hq + it.g * G + r % G) * D;
 #pragma unroll
-        for (int e = 0; e < 32; e += 8)
+        for (int e = 0; e < D; e += 8)
           *reinterpret_cast<uint4*>(op + e) = make_uint4(
-              pack_bf16(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv),
-              pack_bf16(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv),
-              pack_bf16(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv),
-              pack_bf16(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv));
+              pack_bf16(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv),
+              pack_bf16(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv),
+              pack_bf16(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv),
+              pack_bf16(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv));
       }
     }
-    if (row_ok && n_split > 1) part_ml[row_id * n_split + sp] = make_float2(m_run, l_run);
   }
 
   pdl_trigger();  // this CTA's work is done: the next kernel may be scheduled
@@ -548,7 +698,7 @@ __global__ void __launch_bounds__(256)
 rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0,
                  const __grid_constant__ FreqTab freq, const __nv_bfloat16* __restrict__ q,
                  const __nv_bfloat16* __restrict__ k_loc, __nv_bfloat16* __restrict__ q_rot,
-                 __nv_bfloat16* __restrict__ k_rot) {
+                 __nv_bfloat16* __restrict__ k_rot, int* __restrict__ next_item) {
   constexpr int HALF = D / 2;
   constexpr int UPH = HALF / 8;  // 16-byte pair units per head
   // the attention grid that follows may be scheduled now; it waits for this
@@ -556,6 +706,9 @@ rope_prep_kernel(int B, int T, int T_loc, int Hq, int H, int64_t pos0,
   // itself a programmatic dependent of the work before it (pdl_wait)
   pdl_trigger();
   pdl_wait();
+  // the attention grid's item counter: zero once the work before this grid
+  // (an earlier attention call that claimed items from it) has completed
+  if (blockIdx.x == 0 && threadIdx.x == 0) *next_item = 0;
   __shared__ float2 cs[HALF];
   const int p = blockIdx.x;
   const int tq = p - (T_loc - T);  // query token at this position, if >= 0
@@ -667,7 +820,7 @@ namespace {
 
 struct TcPlan {
   int n_split;
-  size_t q_bytes, k_bytes, po_bytes, ml_bytes, total;
+  size_t q_bytes, k_bytes, po_bytes, ml_bytes, cnt_bytes, total;
 };
 
 // Upper bound on key-tile splits: 3, or MSA_ATTN_SPLITS (1..16) from the
@@ -701,7 +854,8 @@ TcPlan tc_plan(int B, int T, int T_loc, int Hq, int H, int D, int m_cap) {
   const size_t rows = (size_t)B * Hq * T;
   p.po_bytes = p.n_split > 1 ? round_up(rows * p.n_split * D * sizeof(float), 256) : 0;
   p.ml_bytes = p.n_split > 1 ? round_up(rows * p.n_split * sizeof(float2), 256) : 0;
-  p.total = p.q_bytes + p.k_bytes + p.po_bytes + p.ml_bytes;
+  p.cnt_bytes = 256;  // the persistent grid's item counter
+  p.total = p.q_bytes + p.k_bytes + p.po_bytes + p.ml_bytes + p.cnt_bytes;
   return p;
 }
 
@@ -719,11 +873,12 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   __nv_bfloat16* k_rot = reinterpret_cast<__nv_bfloat16*>(w + p.q_bytes);
   float* part_o = reinterpret_cast<float*>(w + p.q_bytes + p.k_bytes);
   float2* part_ml = reinterpret_cast<float2*>(w + p.q_bytes + p.k_bytes + p.po_bytes);
+  int* next_item = reinterpret_cast<int*>(w + p.q_bytes + p.k_bytes + p.po_bytes + p.ml_bytes);
   FreqTab freq;
   for (int i = 0; i < D / 2; ++i) freq.w[i] = std::pow((double)rope_base, -2.0 * i / D);
   int rc = launch_pdl(rope_prep_kernel<D>, dim3((unsigned)T_loc), dim3(256), 0, s, B, T, T_loc,
                       Hq, H, (int64_t)pos0, freq, static_cast<const __nv_bfloat16*>(q),
-                      static_cast<const __nv_bfloat16*>(k_loc), q_rot, k_rot);
+                      static_cast<const __nv_bfloat16*>(k_loc), q_rot, k_rot, next_item);
   if (!rc) rc = check_launch();
   if (rc) return rc;
 
@@ -745,8 +900,11 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), (int)K::SMEM);
   if (rc) return rc;
   const int n_qb = (T + kQT * TQ - 1) / (kQT * TQ);
-  if (n_qb > 65535 || B > 65535) return MSA_ERR_UNSUPPORTED;
-  const dim3 grid((unsigned)(p.n_split * H), (unsigned)B, (unsigned)n_qb);
+  const int64_t n_items = (int64_t)n_qb * B * H * p.n_split;
+  if (n_items > INT32_MAX / 2) return MSA_ERR_UNSUPPORTED;
+  // persistent: one CTA per SM (the shared memory admits one), items claimed
+  // at run time
+  const dim3 grid((unsigned)std::min<int64_t>(n_items, num_sms()));
   // programmatic dependent launch: the attention grid may be scheduled while
   // the RoPE preparation still runs (its launch latency overlaps it); every
   // thread waits for the preparation's completion (griddepcontrol.wait)
@@ -762,11 +920,12 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  rc = note_cuda(cudaLaunchKernelEx(&cfg, kern, tq, tkm, tvm, tkl, tvl, T, T_loc, Hq, H, G,
+  rc = note_cuda(cudaLaunchKernelEx(&cfg, kern, tq, tkm, tvm, tkl, tvl, B, T, T_loc, Hq, H, G,
                                     fm ? fm->n_groups : mem_len, m_cap,
                                     fm ? fm->groups : nullptr, fm ? fm->max_groups : 0,
-                                    qscale, p.n_split, static_cast<__nv_bfloat16*>(out), part_o,
-                                    part_ml, device_status_ptr()));
+                                    qscale, p.n_split, n_qb, (int)n_items, next_item,
+                                    static_cast<__nv_bfloat16*>(out), part_o, part_ml,
+                                    device_status_ptr()));
   if (rc) return rc;
   rc = check_launch();
   if (rc || p.n_split == 1) return rc;
@@ -780,10 +939,10 @@ bool attn_tc_supported(int B, int T, int T_loc, int Hq, int H, int D, int m_cap)
   const int G = Hq / H;
   if (G > 16 || (G & (G - 1))) return false;
   if ((int64_t)B * T > (1LL << 30) || (int64_t)B * T_loc > (1LL << 30) ||
-      (int64_t)B * m_cap > (1LL << 30) || B > 65535 || H > 65535)
+      (int64_t)B * m_cap > (1LL << 30))
     return false;
-  // grid (3 splits x H, B, query blocks of kQT * 128 / G tokens)
-  if ((int64_t)3 * H > INT32_MAX || (T + kQT * (kRows / G) - 1) / (kQT * (kRows / G)) > 65535)
+  // items: up to 16 splits x H x B x query blocks of kQT * 128 / G tokens
+  if ((int64_t)16 * H * B * ((T + kQT * (kRows / G) - 1) / (kQT * (kRows / G))) > INT32_MAX / 2)
     return false;
   return true;
 }
