@@ -424,15 +424,14 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         wait_or_abort(&aux.kready[st], (us / kKSt) & 1);
         if (us >= 2) wait_or_abort(&aux.sfree[us & 1], ((us - 2) >> 1) & 1);
         tc::tc_fence_after();
-        const uint32_t a0 = tc::smem_u32(ring + (size_t)st * kTileBytes);
-        const uint32_t b0 =
-            tc::smem_u32(tile_mem(cs) ? qmem + (cs.k & 1) * kQBytes : qt + (us & 1) * kQBytes);
+        const uint64_t ad = tc::sdesc_kmajor_sw128(tc::smem_u32(ring + (size_t)st * kTileBytes));
+        const uint64_t bd = tc::sdesc_kmajor_sw128(
+            tc::smem_u32(tile_mem(cs) ? qmem + (cs.k & 1) * kQBytes : qt + (us & 1) * kQBytes));
 #pragma unroll
         for (int kk = 0; kk < kDim / 16; ++kk) {
           const uint32_t koff = (kk & 3) * 32;
-          tc::mma_bf16_ss(tmem + (us & 1) * kNH,
-                          tc::sdesc_kmajor_sw128(a0 + (kk >> 2) * kBlk + koff),
-                          tc::sdesc_kmajor_sw128(b0 + (kk >> 2) * (kNH * 128) + koff), kIdescS,
+          tc::mma_bf16_ss(tmem + (us & 1) * kNH, tc::desc_add(ad, (kk >> 2) * kBlk + koff),
+                          tc::desc_add(bd, (kk >> 2) * (kNH * 128) + koff), kIdescS,
                           kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&aux.sfull[us & 1]);
@@ -450,14 +449,15 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
         wait_or_abort(&aux.pfull[up & 1], (up >> 1) & 1);
         wait_or_abort(&aux.vfull[st], (up / kVSt) & 1);
         tc::tc_fence_after();
-        const uint32_t v0 = tc::smem_u32(vring + (size_t)st * kTileBytes);
-        const uint32_t p0 = tc::smem_u32(pbuf + (up & 1) * kPBytes);
+        const uint64_t vd =
+            tc::sdesc_mnmajor_sw128(tc::smem_u32(vring + (size_t)st * kTileBytes), kBlk);
+        const uint64_t pd = tc::sdesc_kmajor_sw128(tc::smem_u32(pbuf + (up & 1) * kPBytes));
         const bool first_tile = cp.j == 0, last_tile = cp.j == cp.nt - 1;
 #pragma unroll
         for (int kk = 0; kk < kTK / 16; ++kk)
-          tc::mma_bf16_ss(tmem + 2 * kNH, tc::sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kBlk),
-                          tc::sdesc_kmajor_sw128(p0 + (kk >> 2) * (kNH * 128) + (kk & 3) * 32),
-                          kIdescO, (!first_tile || kk > 0) ? 1u : 0u);
+          tc::mma_bf16_ss(tmem + 2 * kNH, tc::desc_add(vd, kk * 16 * 128),
+                          tc::desc_add(pd, (kk >> 2) * (kNH * 128) + (kk & 3) * 32), kIdescO,
+                          (!first_tile || kk > 0) ? 1u : 0u);
         tc::mma_commit(&aux.vfree[st]);        // P V has read the V slot
         tc::mma_commit(&aux.pvdone[up & 1]);   // ... and the P buffer up&1
         if (last_tile) tc::mma_commit(&aux.odone);  // this chunk's O^T is final

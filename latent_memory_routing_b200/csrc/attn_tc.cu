@@ -400,14 +400,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           // (after its p_full wait) before this MMA, and the tensor core runs
           // one thread's MMAs in issue order
           tc::tc_fence_after();
-          const uint32_t q0 = tc::smem_u32(sQ + i * K::Q_BYTES);
-          const uint32_t k0 = tc::smem_u32(sKV + st * K::STAGE);
+          const uint64_t qd = tc::sdesc_kmajor_sw128(tc::smem_u32(sQ + i * K::Q_BYTES));
+          const uint64_t kd = tc::sdesc_kmajor_sw128(tc::smem_u32(sKV + st * K::STAGE));
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
             const uint32_t koff = (kk >> 2) * (kKeys * 128) + (kk & 3) * 32;
-            tc::mma_bf16_ss(tmem + i * kKeys, tc::sdesc_kmajor_sw128(q0 + off),
-                            tc::sdesc_kmajor_sw128(k0 + koff), K::IDESC_S, kk > 0 ? 1u : 0u);
+            tc::mma_bf16_ss(tmem + i * kKeys, tc::desc_add(qd, off), tc::desc_add(kd, koff),
+                            K::IDESC_S, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&aux.s_full[i]);
           // the item's last S: its Q tiles may be overwritten once it completes
@@ -424,12 +424,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           // P_i(j) written (and any rescale of O_i done) by softmax group i
           if (*abort_flag || !tc::mbar_wait(&aux.p_full[i], v & 1)) return false;
           tc::tc_fence_after();
-          const uint32_t v0 = tc::smem_u32(sKV + st * K::STAGE + K::K_BYTES);
+          const uint64_t vd =
+              sdesc_mnmajor_sw128(tc::smem_u32(sKV + st * K::STAGE + K::K_BYTES), kKeys * 128);
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk)
             mma_bf16_ts(tmem + kQT * kKeys + i * D, tmem + i * kKeys + kk * 8,
-                        sdesc_mnmajor_sw128(v0 + kk * 16 * 128, kKeys * 128), K::IDESC_O,
-                        (j > 0 || kk > 0) ? 1u : 0u);
+                        tc::desc_add(vd, kk * 16 * 128), K::IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
           if (j == nt - 1) tc::mma_commit(&aux.o_full[i]);  // O_i of the item final
           if (i == kQT - 1) tc::mma_commit(&aux.kv_empty[st]);
           return true;

@@ -338,14 +338,13 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 break;
               }
               tc::tc_fence_after();
-              const uint32_t a0 = tc::smem_u32(ring + st * K::STAGE);
-              const uint32_t b0 = a0 + K::A_BYTES;
+              const uint64_t a_d = tc::sdesc_kmajor_sw128(tc::smem_u32(ring + st * K::STAGE));
+              const uint64_t b_d = tc::desc_add(a_d, K::A_BYTES);
 #pragma unroll
               for (int kk = 0; kk < K::SKB * 4; ++kk) {
                 const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside the swizzle atom
-                const uint64_t ad = tc::sdesc_kmajor_sw128(a0 + (kk >> 2) * (kTile * 128) + koff);
-                const uint64_t bd =
-                    tc::sdesc_kmajor_sw128(b0 + (kk >> 2) * (K::NB * 128) + koff);
+                const uint64_t ad = tc::desc_add(a_d, (kk >> 2) * (kTile * 128) + koff);
+                const uint64_t bd = tc::desc_add(b_d, (kk >> 2) * (K::NB * 128) + koff);
                 const uint32_t acc = (h > 0 || s > 0 || kk > 0) ? 1u : 0u;
                 if constexpr (kPair) tc::mma_bf16_ss_pair(d_tmem, ad, bd, K::IDESC, acc);
                 else tc::mma_bf16_ss(d_tmem, ad, bd, K::IDESC, acc);

@@ -301,6 +301,16 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// A descriptor moved on by `bytes` (a multiple of 16): only the 14-bit
+// start-address field changes, which an address below 256 KB cannot carry
+// out of.  One 32-bit add: an MMA issue loop that rebuilt each descriptor
+// from its address spent more time in that one thread's integer chain than
+// the tensor core spends on an N = 128 instruction.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+  const uint32_t lo = (uint32_t)desc + (bytes >> 4);
+  return ((desc >> 32) << 32) | lo;
+}
+
 // UMMA descriptor of an MN-major, 128B-swizzled operand whose MN extent is
 // split in 64-element (128 B) column blocks `lbo` bytes apart and whose K
 // rows are 128 B apart (8-row swizzle atoms 1024 B apart): the layout of a
