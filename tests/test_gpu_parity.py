@@ -601,6 +601,65 @@ def test_attention_prefill_tensor_core_shapes(B, T, T_loc, Hq, H, D, m_cap, mem_
     status_ok()
 
 
+@pytest.mark.parametrize("B,T,Hq,H,m_cap,mem_lens", [
+    (16, 512, 32, 8, 384, [384] * 8 + [0, 1, 127, 128, 129, 255, 256, 383]),  # ~7 items per CTA
+    (2, 64, 32, 8, 3072, [3072, 0]),  # 3 key splits; batch 1's splits past its one tile are empty
+])
+def test_attention_prefill_persistent_items_repeat_bit_exactly(B, T, Hq, H, m_cap, mem_lens):
+    """The prefill's persistent CTAs claim their items at run time from a
+    counter that the RoPE preparation zeroes: on one workspace, two more
+    eager calls and three replays of a CUDA graph of the call reproduce the
+    first call bit for bit (each item is computed whole by one CTA, in a
+    fixed order, whatever CTA claims it), and the first call matches the
+    oracle on sampled rows of the first and last batch element."""
+    D, pos0 = 128, 16
+    g = torch.Generator(device="cuda").manual_seed(B * T + m_cap)
+    dt = torch.bfloat16
+    q = synth.randn((B, T, Hq, D), dt, "cuda", g)
+    km = synth.randn((B, m_cap, H, D), dt, "cuda", g)
+    vm = synth.randn((B, m_cap, H, D), dt, "cuda", g)
+    for b, n in enumerate(mem_lens):
+        km[b, n:] = float("nan")
+        vm[b, n:] = float("nan")
+    kl = synth.randn((B, T, H, D), dt, "cuda", g)
+    vl = synth.randn((B, T, H, D), dt, "cuda", g)
+    ml = torch.tensor(mem_lens, dtype=torch.int32, device="cuda")
+    att = pipeline.Attention(dt, B, T, T, Hq, H, D, m_cap, "cuda")
+    first = att(q, km, vm, ml, kl, vl, pos0).clone()
+    out = torch.empty_like(first)
+    for _ in range(2):
+        att(q, km, vm, ml, kl, vl, pos0, out=out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, first)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up on the capture stream
+        att(q, km, vm, ml, kl, vl, pos0, out=out)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        att(q, km, vm, ml, kl, vl, pos0, out=out)
+    for _ in range(3):
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, first)
+    del graph
+    worst = 0.0
+    for b in sorted({0, B - 1}):
+        n = mem_lens[b]
+        for i0 in sorted({0, T // 2 - 4, T - 8}):
+            i1 = i0 + 8
+            want = oracle.sparse_attn(f64(q[b:b + 1, i0:i1]), [f64(km[b, :n])], [f64(vm[b, :n])],
+                                      f64(kl[b:b + 1, :i1]), f64(vl[b:b + 1, :i1]), pos0,
+                                      10000.0)
+            got = f64(first[b:b + 1, i0:i1])
+            assert np.all(np.isfinite(got))
+            worst = max(worst, float(np.max(np.abs(got - want))))
+    assert worst <= ATTN_BF16, worst
+    status_ok()
+
+
 def _prefill_sweep_points():
     import bench
     return list(bench.PREFILL_SWEEP)
