@@ -30,6 +30,10 @@
  *     arguments are host values.  The library keeps no pointer after a call
  *     returns and allocates no device memory: scratch comes from the
  *     caller's workspace (sizes from the *_workspace_size functions).
+ *     A workspace holds a call's state while its kernels run (rotated
+ *     copies, split partials, the tensor-core prefill's work-item counter),
+ *     so calls that share one must run in order: on one stream, or ordered
+ *     by events.
  *   - `dt` selects the element type of every floating-point tensor of the
  *     call (MSA_F32 = float, MSA_BF16 = __nv_bfloat16); arithmetic is fp32.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
