@@ -51,8 +51,9 @@
 // them to finish merges them into the output (an arrival counter), so no
 // second launch combines them; a lone chunk writes the output directly.  The
 // RoPE constants come from the host (no double-precision arithmetic on the
-// device), so nothing precedes the kernel but the reset of its counters.  Every wait is bounded; after a timeout every role walks its
-// loop without waiting.
+// device), so nothing precedes the kernel but the reset of its counters.
+// Every wait is bounded; after a timeout every role walks its loop without
+// waiting.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -383,22 +384,31 @@ attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_km,
       for (bool ok = first(c, role); ok; ok = next(c, role), ++u) {
         const int st = u % nst;
         if (!isv && c.j == c.nt - 1) ahead = atomicAdd(counters, 1);  // the next chunk
+        const bool mem = tile_mem(c);
+        // fused memory tile: its 16 groups' first bank rows, all read before
+        // the slot wait (one round trip, overlapping it; the TMA issue below
+        // is ordered after every memory access, so a read between two issues
+        // would cost a round trip per group); past the query's last group,
+        // the last one again (masked, V zeroed) so every row of the tile is
+        // written
+        int src[kTK / 8];
+        if (kFused && mem) {
+          const int ng = c.M / 8, g0 = tile_key0(c) / 8;
+          const int2* gq = groups + (int64_t)c.b * max_groups;
+#pragma unroll
+          for (int gi = 0; gi < kTK / 8; ++gi) src[gi] = __ldg(&gq[min(g0 + gi, ng - 1)].x);
+        }
         wait_or_abort(&freeb[st], ((u / nst) & 1) ^ 1);
         if (*abort_flag) break;
         unsigned char* d = (isv ? vring : ring) + (size_t)st * kTileBytes;
-        const bool mem = tile_mem(c);
         const CUtensorMap* m = mem ? (isv ? &tm_vm : &tm_km) : (isv ? &tm_vl : &tm_kl);
         tc::mbar_arrive_expect_tx(&fullb[st], kTileBytes);
         if (kFused && mem) {
-          // 16 groups of 8 bank rows; past the query's last group, repeat it
-          // (masked, V zeroed) so every row of the tile is written
-          const int ng = c.M / 8, g0 = tile_key0(c) / 8;
-          const int2* gq = groups + (int64_t)c.b * max_groups;
-#pragma unroll 4
+          // 16 groups of 8 bank rows
+#pragma unroll
           for (int gi = 0; gi < kTK / 8; ++gi) {
-            const int src = gq[min(g0 + gi, ng - 1)].x;
-            tc::tma_load_3d(d + gi * 1024, m, &fullb[st], 0, c.g, src);
-            tc::tma_load_3d(d + kBlk + gi * 1024, m, &fullb[st], 64, c.g, src);
+            tc::tma_load_3d(d + gi * 1024, m, &fullb[st], 0, c.g, src[gi]);
+            tc::tma_load_3d(d + kBlk + gi * 1024, m, &fullb[st], 64, c.g, src[gi]);
           }
         } else {
           const int row0 = (mem ? c.b * m_cap : c.b * T_loc) + tile_key0(c);

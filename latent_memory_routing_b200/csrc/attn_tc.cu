@@ -92,7 +92,11 @@ struct ACfg {
   // chosen where the compiler reports no or few spills for either
   static constexpr int REG_LOW = D == 128 ? 72 : 88;
   static constexpr int REG_HIGH = D == 128 ? 216 : 208;
+  // the fused form's producer also holds a memory tile's 16 group rows
+  static constexpr int REG_LOW_FUSED = 88;
+  static constexpr int REG_HIGH_FUSED = 208;
   static_assert(kQT == 2 && 128 * REG_LOW + 256 * REG_HIGH == 384 * 168, "register split");
+  static_assert(128 * REG_LOW_FUSED + 256 * REG_HIGH_FUSED == 384 * 168, "register split");
 };
 
 // item-id ring between the producer and the other roles
@@ -268,7 +272,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   };
 
   if (warp < 4) {
-   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(K::REG_LOW));
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n"
+                ::"n"(kFused ? K::REG_LOW_FUSED : K::REG_LOW));
    if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -311,6 +316,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           // claim the next item a few tiles before this one's loads end
           if (j == j_claim) nxt = atomicAdd(next_item, 1) + (int)gridDim.x;
           const int st = tiles % kStages;
+          const int jj = sp.j_lo + j;
+          const bool mem = jj < sp.n_mt;
+          // fused memory tile: its 16 groups' first bank rows, all read before
+          // the slot wait (one round trip, overlapping it; the TMA issue below
+          // is ordered after every memory access, so a read between two issues
+          // would cost a round trip per group); past the last group, the last
+          // one again (finite rows, masked) so every row of the tile is written
+          int src[kKeys / 8];
+          if (kFused && mem) {
+            const int ng = sp.M / 8, g0 = jj * (kKeys / 8);
+#pragma unroll
+            for (int gi = 0; gi < kKeys / 8; ++gi) src[gi] = __ldg(&gq[min(g0 + gi, ng - 1)].x);
+          }
           if (*abort_flag || !tc::mbar_wait(&aux.kv_empty[st], ((tiles / kStages) & 1) ^ 1)) {
             ok = false;
             break;
@@ -329,24 +347,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           unsigned char* k_dst = sKV + st * K::STAGE;
           unsigned char* v_dst = k_dst + K::K_BYTES;
           tc::mbar_arrive_expect_tx(&aux.kv_full[st], K::STAGE);
-          const int jj = sp.j_lo + j;
-          const bool mem = jj < sp.n_mt;
           const CUtensorMap* mk = mem ? &tm_km : &tm_kl;
           const CUtensorMap* mv = mem ? &tm_vm : &tm_vl;
           if (kFused && mem) {
-            // 16 groups of 8 bank rows; past the last group, repeat it
-            // (finite rows, masked) so every row of the tile is written
-            const int ng = sp.M / 8, g0 = jj * (kKeys / 8);
-            for (int gi = 0; gi < kKeys / 8; ++gi) {
-              const int src = gq[min(g0 + gi, ng - 1)].x;
+            // 16 groups of 8 bank rows
+#pragma unroll
+            for (int gi = 0; gi < kKeys / 8; ++gi)
 #pragma unroll
               for (int kb = 0; kb < K::KB; ++kb) {
                 tc::tma_load_3d(k_dst + kb * kKeys * 128 + gi * 1024, mk, &aux.kv_full[st],
-                                kb * 64, it.g, src);
+                                kb * 64, it.g, src[gi]);
                 tc::tma_load_3d(v_dst + kb * kKeys * 128 + gi * 1024, mv, &aux.kv_full[st],
-                                kb * 64, it.g, src);
+                                kb * 64, it.g, src[gi]);
               }
-            }
           } else {
             const int row =
                 mem ? it.b * m_cap + jj * kKeys : it.b * T_loc + (jj - sp.n_mt) * kKeys;
@@ -448,7 +461,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
    }
   } else {
     // ------------------------------------------------------------- softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(K::REG_HIGH));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n"
+                 ::"n"(kFused ? K::REG_HIGH_FUSED : K::REG_HIGH));
     // Warpgroup i owns Q tile i, one thread per query row.  O_i accumulates
     // in TMEM; the row's reference maximum m_run only moves when a tile's
     // maximum exceeds it by more than 2^kRescaleLog2 -- then O_i (in TMEM)
