@@ -14,7 +14,9 @@
 //     cos/sin per position built in shared memory (angles reduced in double).
 //   * attn_tc_kernel: a persistent grid, one CTA per SM, working through
 //     items of (two Q tiles of 128 rows, KV head, batch, key split), claimed
-//     at run time heaviest first (causal work grows with the query block).
+//     at run time in groups of (batch, KV head) pairs whose keys and values
+//     fit a share of the L2, heaviest first within a group (causal work
+//     grows with the query block).
 //     An item's Q tiles and first K/V tiles load while the previous item's
 //     last tiles are still in the tensor core and softmax, and its O is read
 //     out of TMEM before the stores, so the next item's MMAs start at once:
@@ -99,6 +101,10 @@ struct ACfg {
   static_assert(128 * REG_LOW_FUSED + 256 * REG_HIGH_FUSED == 384 * 168, "register split");
 };
 
+// L2 budget of a group of (batch, KV head) pairs' key/value rows (of the
+// 126 MB L2; the query tiles stream beside them)
+constexpr int64_t kL2GroupBytes = 48ll << 20;
+
 // item-id ring between the producer and the other roles
 constexpr int kSched = 4;
 constexpr int kSchedReaders = 1 + kSoftWarps;  // the MMA issuer, each softmax warp
@@ -154,20 +160,26 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Work item `idx` of a call, heaviest first: query blocks in descending order
-// (under a causal mask later blocks see more key tiles), then batch, KV head
-// and key split.
+// Work item `idx` of a call: the (batch, KV head) pairs in groups of `pg`
+// consecutive pairs, group after group; within a group heaviest first --
+// query blocks in descending order (under a causal mask later blocks see
+// more key tiles) -- then pair and key split.
 struct Item {
   int mt, b, g, sp;
 };
-__device__ __forceinline__ Item item_of(int idx, int B, int H, int n_split, int n_qb) {
-  const int per_qb = B * H * n_split;
+__device__ __forceinline__ Item item_of(int idx, int B, int H, int n_split, int n_qb, int pg) {
+  const int P = B * H;                        // (batch, KV head) pairs
+  const int per_group = n_qb * pg * n_split;  // items of a full group of pg pairs
+  const int k = min(idx / per_group, P / pg);
+  const int r = idx - k * per_group;
+  const int per_qb = min(pg, P - k * pg) * n_split;
   Item it;
-  it.mt = n_qb - 1 - idx / per_qb;
-  const int r = idx % per_qb;
-  it.b = r / (H * n_split);
-  it.g = (r % (H * n_split)) / n_split;
-  it.sp = r % n_split;
+  it.mt = n_qb - 1 - r / per_qb;
+  const int rem = r % per_qb;
+  const int pair = k * pg + rem / n_split;
+  it.b = pair / H;
+  it.g = pair % H;
+  it.sp = rem % n_split;
   return it;
 }
 
@@ -216,7 +228,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_vl, int B, int T, int T_loc, int Hq, int H,
                int G, const int32_t* __restrict__ mem_len, int m_cap,
                const int2* __restrict__ groups, int max_groups, float qscale, int n_split,
-               int n_qb, int n_items, int* __restrict__ next_item,
+               int n_qb, int n_items, int pairs_per_group, int* __restrict__ next_item,
                __nv_bfloat16* __restrict__ out, float* __restrict__ part_o,
                float2* __restrict__ part_ml, int* __restrict__ status) {
   using K = ACfg<D>;
@@ -290,7 +302,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         aux.sched_id[slot] = live ? idx : -1;
         tc::mbar_arrive(&aux.sched_full[slot]);  // release: the id is visible to the waiters
         if (!live) break;
-        const Item it = item_of(idx, B, H, n_split, n_qb);
+        const Item it = item_of(idx, B, H, n_split, n_qb, pairs_per_group);
         const Span sp = span(it);
         int nxt = n_items;
         if (sp.nt == 0) {
@@ -336,7 +348,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (j == j_claim && nxt < n_items) {
             // its Q tiles into L2: the Q buffer frees only when this item's
             // last S completes, and from L2 the reload is short
-            const Item ni = item_of(nxt, B, H, n_split, n_qb);
+            const Item ni = item_of(nxt, B, H, n_split, n_qb, pairs_per_group);
 #pragma unroll
             for (int i = 0; i < kQT; ++i)
 #pragma unroll
@@ -402,7 +414,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int idx = aux.sched_id[slot];
         tc::mbar_arrive(&aux.sched_empty[slot]);
         if (idx < 0) break;
-        const int nt = span(item_of(idx, B, H, n_split, n_qb)).nt;
+        const int nt = span(item_of(idx, B, H, n_split, n_qb, pairs_per_group)).nt;
         if (nt == 0) continue;
         ok = !*abort_flag && tc::mbar_wait(&aux.q_full, ne & 1);
         auto issue_s = [&](int i, int j) -> bool {
@@ -489,7 +501,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&aux.sched_empty[slot]);
       if (idx < 0) break;
-      const Item it = item_of(idx, B, H, n_split, n_qb);
+      const Item it = item_of(idx, B, H, n_split, n_qb, pairs_per_group);
       const Span sp = span(it);
       const int tok_local = qt * TQ + r / G;
       const int tok = sp.tok0 + tok_local;
@@ -915,6 +927,13 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   if (rc) return rc;
   const int n_qb = (T + kQT * TQ - 1) / (kQT * TQ);
   const int64_t n_items = (int64_t)n_qb * B * H * p.n_split;
+  // items in groups of (batch, KV head) pairs whose key and value rows fit
+  // kL2GroupBytes, heaviest first within a group: the CTAs then work on few
+  // pairs at a time, and the tiles every query block of a pair re-reads stay
+  // in the L2
+  const int64_t pair_bytes = (int64_t)(m_cap + T_loc) * D * 2 * 2;
+  const int pg =
+      (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)B * H, kL2GroupBytes / pair_bytes));
   if (n_items > INT32_MAX / 2) return MSA_ERR_UNSUPPORTED;
   // persistent: one CTA per SM (the shared memory admits one), items claimed
   // at run time
@@ -937,7 +956,7 @@ int launch_tc(int B, int T, int T_loc, int Hq, int H, const void* q, const void*
   rc = note_cuda(cudaLaunchKernelEx(&cfg, kern, tq, tkm, tvm, tkl, tvl, B, T, T_loc, Hq, H, G,
                                     fm ? fm->n_groups : mem_len, m_cap,
                                     fm ? fm->groups : nullptr, fm ? fm->max_groups : 0,
-                                    qscale, p.n_split, n_qb, (int)n_items, next_item,
+                                    qscale, p.n_split, n_qb, (int)n_items, pg, next_item,
                                     static_cast<__nv_bfloat16*>(out), part_o, part_ml,
                                     device_status_ptr()));
   if (rc) return rc;
