@@ -1210,6 +1210,7 @@ def run_reference(args, world, rank):
 CASES = {
     "prefill_b1_t4096": dict(B=1, T=4096, T_loc=4096, M=384),
     "prefill_b2_t8192": dict(B=2, T=8192, T_loc=8192, M=384),
+    "prefill_b16_t2048": dict(B=16, T=2048, T_loc=2048, M=384),  # 128 (batch, head) pairs
     "decode_b64_t2048": dict(B=64, T=1, T_loc=2048, M=250),
     "prefill_b1_t256": dict(B=1, T=256, T_loc=256, M=273),  # the bank_100m step's attention
     "route_bank_10m_b64": None,  # routing, not attention: see run_route_case
